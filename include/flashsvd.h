@@ -1,0 +1,292 @@
+/*
+ * flashsvd.h — C ABI of libflashsvd.so, the B200 (sm_100a) hot path of
+ * SVD-compressed ("low-rank") transformer inference.
+ *
+ * Sources, cited by page title and section:
+ *   [v1.5] "FlashSVD v1.5: Making Low-Rank Transformers Inference Actually
+ *          Fast" (gist.science explainer, English), Technical Summary:
+ *          Problem Statement; Methodology 1 (Unified Runtime Abstraction),
+ *          2 (Dense-KV Attention, Decode Phase), 3 (Packed MLP Execution),
+ *          4 (Per-Layer CUDA Graph Replay).
+ *   [v1]   "FlashSVD: Memory-Efficient Inference with Streaming for
+ *          Low-Rank Models" (abstract).
+ *
+ * Conventions for every call
+ *   - Tensors are caller-owned DEVICE pointers unless stated otherwise,
+ *     row-major with the last dimension contiguous, base addresses 16-byte
+ *     aligned.  Matrix widths d, r, n, f, H*D must be multiples of 8 (one
+ *     16-byte vector = 8 bf16).  Violations return FLASHSVD_ERR_MISALIGNED
+ *     or FLASHSVD_ERR_UNSUPPORTED_SHAPE and launch nothing.
+ *   - flashsvd_bf16 is the bfloat16 bit pattern.  Arithmetic is fp32
+ *     (accumulation, softmax, norms); storage between kernels is bf16.
+ *   - Calls are asynchronous on the given stream (a cudaStream_t; NULL is
+ *     the legacy default stream).  Device-side errors surface at the
+ *     caller's next synchronisation, or through
+ *     flashsvd_check_device_status().
+ *   - Compute calls allocate nothing, never synchronise and copy nothing
+ *     between host and device, so they may be captured in a CUDA graph.
+ *     They use the library workspace made by flashsvd_init(): calls that
+ *     share it must be ordered on one stream (overlapping calls race).
+ *   - Read-only factor pointers may alias each other (shared bases,
+ *     [v1.5] Methodology 1, Basis Sharing).  Outputs must not alias inputs
+ *     except where a call says "in place".
+ *   - Every call returns a status (enum flashsvd_status); nothing aborts.
+ */
+#ifndef FLASHSVD_H
+#define FLASHSVD_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define FLASHSVD_API __attribute__((visibility("default")))
+#else
+#define FLASHSVD_API
+#endif
+
+typedef uint16_t flashsvd_bf16;                 /* bfloat16 bit pattern */
+struct CUstream_st;
+typedef struct CUstream_st* flashsvd_stream;    /* same as cudaStream_t */
+
+enum flashsvd_status {
+  FLASHSVD_OK = 0,
+  FLASHSVD_ERR_INVALID_ARG = 1,       /* null pointer, bad enum, size < 0 */
+  FLASHSVD_ERR_MISALIGNED = 2,        /* pointer not 16-byte aligned       */
+  FLASHSVD_ERR_UNSUPPORTED_SHAPE = 3, /* width not a multiple of 8, or a
+                                         size beyond the workspace limits  */
+  FLASHSVD_ERR_NOT_INITIALIZED = 4,   /* flashsvd_init() not called        */
+  FLASHSVD_ERR_CAPTURE_UNSAFE = 5,    /* call would allocate or sync while
+                                         the stream is being captured      */
+  FLASHSVD_ERR_CUDA = 6,              /* a CUDA runtime call failed; see
+                                         flashsvd_last_cuda_error()        */
+  FLASHSVD_ERR_TIMEOUT = 7,           /* a bounded device wait expired     */
+  FLASHSVD_ERR_NO_MEMORY = 8          /* workspace allocation failed       */
+};
+
+/* Text for a status code (static storage). */
+FLASHSVD_API const char* flashsvd_status_string(int status);
+/* The cudaError_t of the last call that returned FLASHSVD_ERR_CUDA. */
+FLASHSVD_API int flashsvd_last_cuda_error(void);
+/* Library version, major*10000 + minor*100 + patch. */
+FLASHSVD_API int flashsvd_version(void);
+
+/* ---------------------------------------------------------------- setup --
+ * flashsvd_init: make `device` current and allocate the library workspace on
+ * it: the fp32 rank-activation exchange and split-K partial sums of the
+ * decode linears, the split-sequence partials of decode attention, a device
+ * status word, and per-layer activation scratch for up to `max_tokens` rows
+ * of width `max_hidden` and FFN width `max_ffn` (prefill and encoder
+ * layers).  `max_rank` bounds every factor rank.  Calling it again with the
+ * same or smaller limits is a no-op; larger limits re-allocate (not allowed
+ * during stream capture: FLASHSVD_ERR_CAPTURE_UNSAFE).
+ * flashsvd_shutdown frees the workspace (after a device synchronise).
+ */
+FLASHSVD_API int flashsvd_init(int device, int max_tokens, int max_rank, int max_hidden,
+                  int max_ffn);
+FLASHSVD_API int flashsvd_shutdown(void);
+
+/* Synchronise `stream`, then read and clear the device status word written
+ * by kernels whose bounded waits expired.  Returns FLASHSVD_OK or
+ * FLASHSVD_ERR_TIMEOUT (or FLASHSVD_ERR_CUDA if the stream reports an
+ * error). */
+FLASHSVD_API int flashsvd_check_device_status(flashsvd_stream stream);
+
+/* Number of kernels this library has launched since load: eager launches
+ * plus the kernel nodes of every replayed graph. */
+FLASHSVD_API int64_t flashsvd_launch_count(void);
+
+/* ------------------------------------------------------ factorized linear --
+ * y[M x n] = (x[M x d] . U[d x r]) . V[r x n] + bias[n]           (bias may be NULL)
+ *
+ * [v1] abstract (truncated factors applied as two chained products whose
+ * rank-r intermediate is reduced on the fly, never materialised as a
+ * full-size activation); [v1.5] Problem Statement (prefill and decode have
+ * different bottlenecks, so each phase has its own kernel).
+ *   M <= 32 (decode): split-K GEMV over U, then over V; the intermediate
+ *     z = x.U [M x r] stays fp32 in a small L2-resident workspace.
+ *   M > 32 (prefill): tcgen05 tensor-core kernel; each 128-row tile of z is
+ *     computed into tensor memory, rounded to bf16 into shared memory and
+ *     multiplied by V on chip; z never reaches global memory.
+ * Sizes: 1 <= M <= max_tokens; d, r, n multiples of 8 (prefill: d, r
+ * multiples of 64 as well); r <= max_rank.
+ */
+FLASHSVD_API int flashsvd_lowrank_linear(const flashsvd_bf16* x, const flashsvd_bf16* U,
+                            const flashsvd_bf16* V, const flashsvd_bf16* bias,
+                            flashsvd_bf16* y, int M, int d, int r, int n,
+                            flashsvd_stream stream);
+
+/* Dense y[M x n] = x[M x d] . W[d x n] (the output head, which is not
+ * factorized), fp32 result.  Same size rules as flashsvd_lowrank_linear. */
+FLASHSVD_API int flashsvd_dense_linear_f32(const flashsvd_bf16* x, const flashsvd_bf16* W,
+                              float* y, int M, int d, int n,
+                              flashsvd_stream stream);
+
+/* -------------------------------------------------- packed gate|up MLP --
+ * [v1.5] Methodology 3 (Packed MLP Execution): the input-side gate and up
+ * factors are packed offline into one tensor, U_gu[d x 2r_f] = [U_g | U_u]
+ * (gate columns first); one wide projection z = x.U_gu [M x 2r_f] is taken
+ * and split; V_gu[2r_f x f] holds V_g (rows 0..r_f-1) stacked on V_u.
+ *   h = SiLU(z_g . V_g) * (z_u . V_u)                 [M x f]
+ *   y = (h . U_dn[f x r_dn]) . V_dn[r_dn x d]         [M x d]
+ * flashsvd_gateup_swiglu stops at h (the first two stages).
+ */
+FLASHSVD_API int flashsvd_packed_gateup_mlp(const flashsvd_bf16* x,
+                               const flashsvd_bf16* U_gu,
+                               const flashsvd_bf16* V_gu,
+                               const flashsvd_bf16* U_dn,
+                               const flashsvd_bf16* V_dn, flashsvd_bf16* y,
+                               int M, int d, int r_f, int f, int r_dn,
+                               flashsvd_stream stream);
+FLASHSVD_API int flashsvd_gateup_swiglu(const flashsvd_bf16* x, const flashsvd_bf16* U_gu,
+                           const flashsvd_bf16* V_gu, flashsvd_bf16* h, int M,
+                           int d, int r_f, int f, flashsvd_stream stream);
+
+/* ------------------------------------------------ dense-KV decode attention --
+ * [v1.5] Methodology 2 ("reconstruct the present, read the past
+ * contiguously"): the history lives in a dense contiguous KV cache laid out
+ * like flash_attn_with_kvcache's, k_cache/v_cache [B, S_max, H, D] bf16, with
+ * cache_seqlens a DEVICE int32[B].  If k_new and v_new (each [B x H x D]) are
+ * non-NULL they are written at index cache_seqlens[b]; either way the query
+ * q[B x H x D] then attends over keys 0..cache_seqlens[b] inclusive:
+ *   out[b,h] = softmax(q.K^T * scale) . V               [B x H x D] bf16
+ * cache_seqlens is not incremented (see flashsvd_advance_seqlens).
+ * Requires cache_seqlens[b] < S_max (entries at or beyond S_max are clamped
+ * to S_max-1 on the device), D in {64, 128}.
+ */
+FLASHSVD_API int flashsvd_dense_kv_decode_attn(const flashsvd_bf16* q,
+                                  const flashsvd_bf16* k_new,
+                                  const flashsvd_bf16* v_new,
+                                  flashsvd_bf16* k_cache,
+                                  flashsvd_bf16* v_cache,
+                                  const int32_t* cache_seqlens,
+                                  flashsvd_bf16* out, int B, int H, int D,
+                                  int S_max, float scale,
+                                  flashsvd_stream stream);
+
+/* Full-sequence (prefill / encoder) attention, [v1.5] Methodology 2,
+ * "Prefill": q and out [B, S, H, D]; keys and values are rows 0..S-1 of
+ * k_cache/v_cache [B, S_max, H, D].  causal != 0 masks key j > query i.
+ * D in {64, 128}. */
+FLASHSVD_API int flashsvd_prefill_attn(const flashsvd_bf16* q, const flashsvd_bf16* k_cache,
+                          const flashsvd_bf16* v_cache, flashsvd_bf16* out,
+                          int B, int S, int H, int D, int S_max, int causal,
+                          float scale, flashsvd_stream stream);
+
+/* --------------------------------------------------------------- glue ----
+ * RMSNorm y = x * g / sqrt(mean(x^2) + eps); LayerNorm
+ * y = (x - mean) / sqrt(var + eps) * g + b (population variance).  Rows of
+ * width d, M rows; y may equal x (in place).
+ * Rotary table: cos_tab/sin_tab [S_max x D/2] fp32 with
+ * angle(p, i) = p * base^(-2i/D), computed in double on the device.
+ * Embedding gather: x[b] = emb[tokens[b]] for b < B (tokens on the device;
+ * ids outside [0, vocab) are clamped).
+ * Greedy: next[m] = argmax_j logits[m, j] (ties to the lowest index).
+ * advance: cache_seqlens[b] += 1 for b < B.
+ */
+FLASHSVD_API int flashsvd_rmsnorm(const flashsvd_bf16* x, const flashsvd_bf16* g,
+                     flashsvd_bf16* y, int M, int d, float eps,
+                     flashsvd_stream stream);
+FLASHSVD_API int flashsvd_layernorm(const flashsvd_bf16* x, const flashsvd_bf16* g,
+                       const flashsvd_bf16* b, flashsvd_bf16* y, int M, int d,
+                       float eps, flashsvd_stream stream);
+FLASHSVD_API int flashsvd_rope_table(float* cos_tab, float* sin_tab, int S_max, int D,
+                        float base, flashsvd_stream stream);
+FLASHSVD_API int flashsvd_embed(const int32_t* tokens, const flashsvd_bf16* emb,
+                   flashsvd_bf16* x, int B, int d, int vocab,
+                   flashsvd_stream stream);
+FLASHSVD_API int flashsvd_greedy(const float* logits, int32_t* next_tokens, int M,
+                    int vocab, flashsvd_stream stream);
+FLASHSVD_API int flashsvd_advance_seqlens(int32_t* cache_seqlens, int B,
+                             flashsvd_stream stream);
+
+/* -------------------------------------------------------------- layers ---
+ * One transformer layer as caller-owned factor pointers.
+ * kind = FLASHSVD_DECODER: pre-norm RMSNorm, RoPE, causal attention,
+ *   packed gate|up SwiGLU MLP (U_gu, V_gu, r_f) and factorized down
+ *   projection (down), no biases:
+ *     h = x + o(attn(rope(q(n1)), rope(k(n1)), v(n1))),  n1 = rmsnorm(x, norm1_g)
+ *     y = h + down(SiLU(gate) * up)(rmsnorm(h, norm2_g))
+ * kind = FLASHSVD_ENCODER: post-LN, bidirectional attention, GELU FFN (up,
+ *   down), every linear with its bias:
+ *     h = LN1(x + o(attn(q(x), k(x), v(x))));  y = LN2(h + down(GELU(up(h))))
+ * Heads are contiguous D-slices of the hidden width (d = H * D).
+ */
+typedef struct flashsvd_factor {
+  const flashsvd_bf16* U;      /* [d_in x r]  */
+  const flashsvd_bf16* V;      /* [r x d_out] */
+  const flashsvd_bf16* bias;   /* [d_out] or NULL */
+  int r;
+} flashsvd_factor;
+
+enum flashsvd_layer_kind { FLASHSVD_DECODER = 0, FLASHSVD_ENCODER = 1 };
+enum flashsvd_mode {
+  FLASHSVD_PREFILL_CAUSAL = 0,  /* decoder, whole prompt, fills cache [0,S) */
+  FLASHSVD_DECODE = 1,          /* decoder, one token per sequence (S = 1)  */
+  FLASHSVD_ENCODER_BIDIR = 2    /* encoder, whole sequence                  */
+};
+
+typedef struct flashsvd_layer {
+  int kind;                     /* enum flashsvd_layer_kind */
+  int d, H, D, f;               /* hidden, heads, head dim, FFN width */
+  float norm_eps;
+  const flashsvd_bf16* norm1_g; const flashsvd_bf16* norm1_b;  /* b: encoder */
+  const flashsvd_bf16* norm2_g; const flashsvd_bf16* norm2_b;
+  flashsvd_factor q, k, v, o;
+  const flashsvd_bf16* U_gu;    /* decoder: [d x 2 r_f] packed gate|up */
+  const flashsvd_bf16* V_gu;    /* decoder: [2 r_f x f] */
+  int r_f;
+  flashsvd_factor up;           /* encoder: [d -> f] */
+  flashsvd_factor down;         /* [f -> d] */
+  const float* rope_cos;        /* decoder: [S_max x D/2] (flashsvd_rope_table) */
+  const float* rope_sin;
+} flashsvd_layer;
+
+/* Run one layer in place on x_inout ([B*S x d] bf16, token-major).
+ * PREFILL_CAUSAL: positions 0..S-1; rotated keys and values are written to
+ *   cache rows [0, S) of every batch entry; cache_seqlens is not read.
+ * DECODE: S must be 1; positions are cache_seqlens[b] (device); the new key
+ *   and value are appended there ([v1.5] Methodology 2); cache_seqlens is not
+ *   incremented.
+ * ENCODER_BIDIR: k_cache/v_cache are [B, S_max >= S, H, D] scratch the
+ *   caller provides; cache_seqlens may be NULL.
+ * B*S <= max_tokens of flashsvd_init (DECODE: B <= 32). */
+FLASHSVD_API int flashsvd_layer_forward(const flashsvd_layer* L, flashsvd_bf16* x_inout,
+                           flashsvd_bf16* k_cache, flashsvd_bf16* v_cache,
+                           const int32_t* cache_seqlens, int B, int S,
+                           int S_max, int mode, flashsvd_stream stream);
+
+/* -------------------------------------------------------------- graphs ---
+ * [v1.5] Methodology 4 (Per-Layer CUDA Graph Replay): the stable decode body
+ * of one layer is captured once and replayed every step.  Buffers, B and
+ * S_max are fixed at capture; positions come from cache_seqlens in device
+ * memory, so one graph serves every step.
+ * flashsvd_capture_begin/end capture any sequence of library calls issued on
+ * `stream` between them (e.g. embedding, output head, greedy pick and
+ * advance) into a replayable graph.  A graph may also be a composition of
+ * other graphs (flashsvd_graph_compose), replayed as one launch.
+ */
+typedef struct flashsvd_graph flashsvd_graph;
+
+FLASHSVD_API int flashsvd_decode_graph_capture(const flashsvd_layer* L,
+                                  flashsvd_bf16* x_inout,
+                                  flashsvd_bf16* k_cache,
+                                  flashsvd_bf16* v_cache,
+                                  const int32_t* cache_seqlens, int B,
+                                  int S_max, flashsvd_stream stream,
+                                  flashsvd_graph** graph);
+FLASHSVD_API int flashsvd_capture_begin(flashsvd_stream stream);
+FLASHSVD_API int flashsvd_capture_end(flashsvd_stream stream, flashsvd_graph** graph);
+FLASHSVD_API int flashsvd_graph_compose(flashsvd_graph* const* parts, int n_parts,
+                           flashsvd_graph** graph);
+FLASHSVD_API int flashsvd_graph_replay(flashsvd_graph* graph, flashsvd_stream stream);
+/* Kernel nodes in the graph (used for launch accounting). */
+FLASHSVD_API int flashsvd_graph_kernel_count(const flashsvd_graph* graph);
+FLASHSVD_API int flashsvd_graph_destroy(flashsvd_graph* graph);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FLASHSVD_H */

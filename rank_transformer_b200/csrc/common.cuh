@@ -1,0 +1,112 @@
+// Shared device helpers of libflashsvd (sm_100a only).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "../../include/flashsvd.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "libflashsvd is built for sm_100a only"
+#endif
+
+namespace fsvd {
+
+typedef __nv_bfloat16 bf16;
+
+// ------------------------------------------------------------ host side --
+
+// Host-side count of kernel launches (eager) and replayed kernel nodes.
+extern std::atomic<int64_t> g_launches;
+// Last CUDA error seen by an entry point.
+extern int g_last_cuda_error;
+
+inline int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return FLASHSVD_OK;
+  g_last_cuda_error = (int)e;
+  return FLASHSVD_ERR_CUDA;
+}
+
+#define FSVD_TRY(expr)                     \
+  do {                                     \
+    int _st = (expr);                      \
+    if (_st != FLASHSVD_OK) return _st;    \
+  } while (0)
+
+#define FSVD_CUDA(expr) FSVD_TRY(::fsvd::cuda_status(expr))
+
+// Launch `kernel` with programmatic dependent launch enabled, so that its
+// prologue (weight loads) can overlap the tail of the previous kernel on the
+// stream; the kernel orders itself after that kernel with
+// griddepcontrol.wait before it touches anything the previous kernel wrote.
+template <typename... KArgs, typename... Args>
+inline int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block,
+                      size_t smem, cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess) return cuda_status(e);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return FLASHSVD_OK;
+}
+
+inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+inline int round_up(int a, int b) { return ceil_div(a, b) * b; }
+inline bool aligned16(const void* p) { return (((uintptr_t)p) & 15u) == 0; }
+
+// ---------------------------------------------------------- device side --
+
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// 16-byte streaming load of read-once data (weights): no L1 allocation.
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// bf16x2 packed in a 32-bit word -> two floats (exact).
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ float bf2f(bf16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ bf16 f2bf(float v) { return __float2bfloat16_rn(v); }
+
+__device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
+  __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&t);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Device status word codes (written by kernels whose bounded waits expire).
+enum : int { DEV_STATUS_OK = 0, DEV_STATUS_TIMEOUT = 1 };
+
+}  // namespace fsvd

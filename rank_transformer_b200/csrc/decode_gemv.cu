@@ -1,0 +1,358 @@
+// Decode-regime (M <= 32 rows) factorized linear: split-K GEMV kernels.
+//
+// FlashSVD v1.5 (gist.science explainer), Technical Summary, Problem
+// Statement: decode is memory-bound, so each stage of y = (x U) V is a
+// stream over one factor matrix.  One launch handles one stage for up to
+// three factor matrices that share the same activation rows:
+//   stage 1:  z[m, :]  = A[m, :] . U        (A = x, optionally RMS-normalised)
+//   stage 2:  y[m, :]  = z[m, :] . V        (+ fused epilogue)
+// The grid is (column tiles x K splits).  Each CTA streams a [KC x 64]
+// block of the factor with 16-byte loads (no L1 allocation), multiplies it
+// by the matching activation slice held in shared memory (fp32), reduces
+// over its 8 warps and writes a partial tile; the last CTA to finish a
+// column tile (atomic counter, no waiting) sums the partials in split order
+// -- deterministic -- and applies the epilogue.  The intermediate z stays
+// in fp32 in a small L2-resident workspace.
+#include <cstdio>
+
+#include "kernels.h"
+
+namespace fsvd {
+
+namespace {
+
+constexpr int GV_THREADS = 256;
+constexpr int GV_BATCH = 8;  // 16-byte weight vectors in flight per thread
+
+__device__ __forceinline__ void unpack8(const uint4& v, float* w) {
+  w[0] = bf_lo(v.x); w[1] = bf_hi(v.x); w[2] = bf_lo(v.y); w[3] = bf_hi(v.y);
+  w[4] = bf_lo(v.z); w[5] = bf_hi(v.z); w[6] = bf_lo(v.w); w[7] = bf_hi(v.w);
+}
+
+// Global output column of tile column c (0..63) for the column map.
+template <int MAP>
+__device__ __forceinline__ int tile_col(int t, int c, int D) {
+  if (MAP == MAP_PLAIN) return t * 64 + c;
+  if (MAP == MAP_ROPE) {
+    const int tph = D >> 6, h = t / tph, j = t - h * tph;
+    return h * D + j * 32 + (c & 31) + (c >> 5) * (D >> 1);
+  }
+  return t * 32 + (c & 31);  // SWIGLU: c < 32 gate, c >= 32 up, same column
+}
+
+template <int MT, int PRO, int EPI, int MAP>
+__global__ void __launch_bounds__(GV_THREADS)
+gemv_splitk_kernel(const __grid_constant__ GvParams p) {
+  constexpr int NSEG = (MAP == MAP_SWIGLU) ? 2 : 1;
+  extern __shared__ __align__(16) float sm[];
+  float* As = sm;                           // [NSEG][MT][KC]
+  float* red = sm + NSEG * MT * p.KC;       // [8][MT][64]
+  __shared__ float s_rstd[MT];
+  __shared__ int s_last;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int cg = tid & 7, rr = tid >> 3;
+  const int tile = blockIdx.x, split = blockIdx.y;
+
+  int pi = 0;
+#pragma unroll
+  for (int i = 1; i < 3; ++i)
+    if (i < p.nprob && tile >= p.tile_start[i]) pi = i;
+  const GvProblem P = p.prob[pi];
+  const int t = tile - p.tile_start[pi];
+  const int hi = cg >> 2;
+  const int col = tile_col<MAP>(t, cg * 8, p.D);
+  const long long wrow = (MAP == MAP_SWIGLU && hi) ? P.w_row2 : 0;
+  const bool colok = col < P.N;
+  const int k0 = split * p.KC;
+  const int kn = min(p.K - k0, p.KC);
+  const int niter = (kn + 31) >> 5;  // <= KC/32
+
+  pdl_launch_dependents();
+
+  // Factor loads do not depend on the previous kernel: issue the first
+  // batch before waiting for it.
+  const bf16* wp = P.W + (wrow + k0 + rr) * P.ldw + col;
+  uint4 wv[GV_BATCH];
+#pragma unroll
+  for (int i = 0; i < GV_BATCH; ++i) {
+    const int kk = rr + 32 * i;
+    wv[i] = (i < niter && kk < kn && colok)
+                ? ldg_stream(wp + (long long)(32 * i) * P.ldw)
+                : make_uint4(0u, 0u, 0u, 0u);
+  }
+
+  pdl_wait();
+
+  // ---- stage the activation slice A[m0+m, acol + k0 .. + KC) in fp32 ----
+  if (PRO == PRO_RMSNORM) {
+    for (int m = warp; m < MT; m += GV_THREADS / 32) {
+      float ss = 0.f;
+      if (m < p.M) {
+        const bf16* xr = p.x + (long long)(p.m0 + m) * p.ldx;
+        for (int c = lane * 8; c < p.K; c += 256) {
+          float w[8];
+          unpack8(*reinterpret_cast<const uint4*>(xr + c), w);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) ss = fmaf(w[j], w[j], ss);
+        }
+      }
+      ss = warp_sum(ss);
+      if (lane == 0) s_rstd[m] = rsqrtf(ss / (float)p.K + p.eps);
+    }
+    __syncthreads();
+  }
+  {
+    const int kc8 = p.KC >> 3;
+    const int items = NSEG * MT * kc8;
+    for (int it = tid; it < items; it += GV_THREADS) {
+      const int seg = it / (MT * kc8);
+      const int rem = it - seg * MT * kc8;
+      const int m = rem / kc8;
+      const int kk = (rem - m * kc8) * 8;
+      float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (m < p.M && kk < kn) {
+        const int acol = (seg ? P.a_col2 : P.a_col) + k0 + kk;
+        const long long row = p.m0 + m;
+        if (PRO == PRO_F32) {
+          const float4* src = reinterpret_cast<const float4*>(p.a32 + row * p.lda + acol);
+          const float4 u0 = src[0], u1 = src[1];
+          a[0] = u0.x; a[1] = u0.y; a[2] = u0.z; a[3] = u0.w;
+          a[4] = u1.x; a[5] = u1.y; a[6] = u1.z; a[7] = u1.w;
+        } else {
+          unpack8(*reinterpret_cast<const uint4*>(p.x + row * p.ldx + acol), a);
+          if (PRO == PRO_RMSNORM) {
+            float g[8];
+            unpack8(*reinterpret_cast<const uint4*>(p.norm_g + acol), g);
+            const float rs = s_rstd[m];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) a[j] = a[j] * rs * g[j];
+          }
+        }
+      }
+      float4* dst = reinterpret_cast<float4*>(As + (seg * MT + m) * p.KC + kk);
+      dst[0] = make_float4(a[0], a[1], a[2], a[3]);
+      dst[1] = make_float4(a[4], a[5], a[6], a[7]);
+    }
+  }
+  __syncthreads();
+
+  // ---- multiply-accumulate ----
+  float acc[MT][8];
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[m][j] = 0.f;
+
+  const float* Aseg = As + (NSEG == 2 ? hi : 0) * MT * p.KC;
+  for (int base = 0; base < niter; base += GV_BATCH) {
+    if (base > 0) {
+#pragma unroll
+      for (int i = 0; i < GV_BATCH; ++i) {
+        const int kk = rr + 32 * (base + i);
+        wv[i] = (base + i < niter && kk < kn && colok)
+                    ? ldg_stream(wp + (long long)(32 * (base + i)) * P.ldw)
+                    : make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < GV_BATCH; ++i) {
+      if (base + i < niter) {
+        const int kk = rr + 32 * (base + i);
+        float w[8];
+        unpack8(wv[i], w);
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          const float a = Aseg[m * p.KC + kk];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[m][j] = fmaf(a, w[j], acc[m][j]);
+        }
+      }
+    }
+  }
+
+  // ---- reduce the 32 row lanes: 4 per warp by shuffles, 8 warps in smem ----
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float v = acc[m][j];
+      v += __shfl_xor_sync(0xffffffffu, v, 8);
+      v += __shfl_xor_sync(0xffffffffu, v, 16);
+      acc[m][j] = v;
+    }
+  if (lane < 8) {
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) red[(warp * MT + m) * 64 + lane * 8 + j] = acc[m][j];
+  }
+  __syncthreads();
+
+  constexpr int NOUT = MT * 64;
+  constexpr int PER = (NOUT + GV_THREADS - 1) / GV_THREADS;
+  float val[PER];
+#pragma unroll
+  for (int q = 0; q < PER; ++q) {
+    const int o = tid + q * GV_THREADS;
+    float s = 0.f;
+    if (o < NOUT) {
+      const int m = o >> 6, c = o & 63;
+#pragma unroll
+      for (int w = 0; w < GV_THREADS / 32; ++w) s += red[(w * MT + m) * 64 + c];
+    }
+    val[q] = s;
+  }
+
+  if (p.splits > 1) {
+    float* mypart = p.part + ((long long)tile * p.splits + split) * NOUT;
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+      const int o = tid + q * GV_THREADS;
+      if (o < NOUT) __stcg(mypart + o, val[q]);
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = (atomicAdd(p.counters + tile, 1) == p.splits - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    const float* tp = p.part + (long long)tile * p.splits * NOUT;
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+      const int o = tid + q * GV_THREADS;
+      float s = 0.f;
+      if (o < NOUT)
+        for (int sp = 0; sp < p.splits; ++sp) s += __ldcg(tp + (long long)sp * NOUT + o);
+      val[q] = s;
+    }
+    if (tid == 0) p.counters[tile] = 0;  // ready for the next launch
+  }
+
+  // ---- epilogue on the finished [MT x 64] tile ----
+  __syncthreads();  // red is reused as the finished tile
+  float* fin = red;
+#pragma unroll
+  for (int q = 0; q < PER; ++q) {
+    const int o = tid + q * GV_THREADS;
+    if (o < NOUT) fin[o] = val[q];
+  }
+  __syncthreads();
+
+  if (EPI == EPI_F32 || EPI == EPI_BF16) {
+    for (int o = tid; o < NOUT; o += GV_THREADS) {
+      const int m = o >> 6, c = o & 63;
+      const int gc = tile_col<MAP>(t, c, p.D);
+      if (m >= p.M || gc >= P.N) continue;
+      const long long row = p.m0 + m;
+      float v = fin[o];
+      if (EPI == EPI_F32) {
+        p.out32[row * p.ldo32 + P.out_col + gc] = v;
+      } else {
+        if (p.bias) v += bf2f(p.bias[gc]);
+        if (p.resid) v += bf2f(p.resid[row * p.ldr + gc]);
+        p.out16[row * p.ldo16 + gc] = f2bf(v);
+      }
+    }
+  } else if (EPI == EPI_QKV) {
+    const int half = p.D >> 1;
+    for (int o = tid; o < MT * 32; o += GV_THREADS) {
+      const int m = o >> 5, c = o & 31;
+      if (m >= p.M) continue;
+      const int b = p.m0 + m;
+      int pos = p.seqlens[b];
+      pos = pos < 0 ? 0 : (pos >= p.S_max ? p.S_max - 1 : pos);
+      const int glo = tile_col<MAP>(t, c, p.D);
+      const int i = glo % p.D;  // rotation index in [0, D/2)
+      float lo = fin[m * 64 + c], hv = fin[m * 64 + c + 32];
+      if (P.kind < 2) {
+        const float cs = p.rope_cos[(long long)pos * half + i];
+        const float sn = p.rope_sin[(long long)pos * half + i];
+        const float l2 = lo * cs - hv * sn;
+        hv = hv * cs + lo * sn;
+        lo = l2;
+      }
+      bf16* dst;
+      if (P.kind == 0) dst = p.out16 + (long long)b * p.ldo16;
+      else dst = (P.kind == 1 ? p.k_cache : p.v_cache) + ((long long)b * p.S_max + pos) * p.HD;
+      dst[glo] = f2bf(lo);
+      dst[glo + half] = f2bf(hv);
+    }
+  } else {  // EPI_SWIGLU
+    for (int o = tid; o < MT * 32; o += GV_THREADS) {
+      const int m = o >> 5, c = o & 31;
+      const int fc = t * 32 + c;
+      if (m >= p.M || fc >= P.N) continue;
+      const float g = fin[m * 64 + c], u = fin[m * 64 + c + 32];
+      const float h = g / (1.f + expf(-g)) * u;
+      p.out16[(long long)(p.m0 + m) * p.ldo16 + fc] = f2bf(h);
+    }
+  }
+}
+
+template <int MT, int PRO, int EPI, int MAP>
+int launch_one(const GvParams& p, int total_tiles, cudaStream_t stream) {
+  constexpr int NSEG = (MAP == MAP_SWIGLU) ? 2 : 1;
+  const size_t smem = (size_t)(NSEG * MT * p.KC + 8 * MT * 64) * sizeof(float);
+  auto kern = gemv_splitk_kernel<MT, PRO, EPI, MAP>;
+  static bool configured = false;  // once per instantiation
+  if (!configured) {
+    FSVD_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024));
+    configured = true;
+  }
+  if (smem > 160 * 1024) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  return launch_pdl(kern, dim3(total_tiles, p.splits), dim3(GV_THREADS), smem, stream, p);
+}
+
+template <int PRO, int EPI, int MAP>
+int launch_mt(const GvParams& p, int total_tiles, cudaStream_t stream) {
+  if (p.M <= 1) return launch_one<1, PRO, EPI, MAP>(p, total_tiles, stream);
+  if (p.M <= 2) return launch_one<2, PRO, EPI, MAP>(p, total_tiles, stream);
+  if (p.M <= 4) return launch_one<4, PRO, EPI, MAP>(p, total_tiles, stream);
+  return launch_one<8, PRO, EPI, MAP>(p, total_tiles, stream);
+}
+
+}  // namespace
+
+int gemv_tiles_for(int map, int N, int D) {
+  if (map == MAP_SWIGLU) return ceil_div(N, 32);
+  if (map == MAP_ROPE) return (N / D) * (D / 64);
+  return ceil_div(N, 64);
+}
+
+int gemv_launch(GvParams p, int pro, int epi, int map, int total_rows,
+                int target_ctas, cudaStream_t stream) {
+  int tiles = 0;
+  for (int i = 0; i < p.nprob; ++i) {
+    p.tile_start[i] = tiles;
+    tiles += gemv_tiles_for(map, p.prob[i].N, p.D);
+  }
+  for (int i = p.nprob; i < 4; ++i) p.tile_start[i] = tiles;
+  // Split K so the grid fills the GPU; at most 512 rows per CTA.
+  int splits = target_ctas / (tiles > 0 ? tiles : 1);
+  splits = splits < 1 ? 1 : splits;
+  const int max_splits = ceil_div(p.K, 32);
+  splits = splits > max_splits ? max_splits : splits;
+  const int min_splits = ceil_div(p.K, 512);
+  splits = splits < min_splits ? min_splits : splits;
+  p.KC = round_up(ceil_div(p.K, splits), 32);
+  p.splits = ceil_div(p.K, p.KC);
+
+  for (int m0 = 0; m0 < total_rows; m0 += 8) {
+    p.m0 = m0;
+    p.M = total_rows - m0 < 8 ? total_rows - m0 : 8;
+    int st = FLASHSVD_ERR_INVALID_ARG;
+#define FSVD_GV(PRO_, EPI_, MAP_) \
+    if (pro == PRO_ && epi == EPI_ && map == MAP_) st = launch_mt<PRO_, EPI_, MAP_>(p, tiles, stream);
+    FSVD_GV(PRO_RMSNORM, EPI_F32, MAP_PLAIN)
+    FSVD_GV(PRO_BF16, EPI_F32, MAP_PLAIN)
+    FSVD_GV(PRO_F32, EPI_BF16, MAP_PLAIN)
+    FSVD_GV(PRO_F32, EPI_QKV, MAP_ROPE)
+    FSVD_GV(PRO_F32, EPI_SWIGLU, MAP_SWIGLU)
+#undef FSVD_GV
+    if (st != FLASHSVD_OK) return st;
+  }
+  return FLASHSVD_OK;
+}
+
+}  // namespace fsvd

@@ -1,0 +1,214 @@
+// Row-wise glue around the factorized linears: RMSNorm, LayerNorm, rotary
+// table, embedding gather, greedy pick and sequence-length advance.  All
+// are memory-bound one-pass kernels with 16-byte vector access.
+#include "kernels.h"
+
+namespace fsvd {
+
+namespace {
+
+constexpr int NT = 256;
+
+__device__ __forceinline__ float block_sum(float v, float* sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = warp_sum(v);
+  __syncthreads();
+  if (lane == 0) sh[warp] = v;
+  __syncthreads();
+  float t = 0.f;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += sh[w];
+  return t;
+}
+
+__device__ __forceinline__ void ld8(const bf16* p, float* v) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  v[0] = bf_lo(u.x); v[1] = bf_hi(u.x); v[2] = bf_lo(u.y); v[3] = bf_hi(u.y);
+  v[4] = bf_lo(u.z); v[5] = bf_hi(u.z); v[6] = bf_lo(u.w); v[7] = bf_hi(u.w);
+}
+__device__ __forceinline__ void st8(bf16* p, const float* v) {
+  uint4 u;
+  u.x = pack_bf2(v[0], v[1]); u.y = pack_bf2(v[2], v[3]);
+  u.z = pack_bf2(v[4], v[5]); u.w = pack_bf2(v[6], v[7]);
+  *reinterpret_cast<uint4*>(p) = u;
+}
+
+// Rows of up to 32 * 256 = 8192 elements are held in registers.
+constexpr int ROW_VEC = 4;  // 16-byte vectors per thread
+
+__global__ void __launch_bounds__(NT)
+rmsnorm_kernel(const bf16* x, const bf16* g, bf16* y, int d, float eps) {
+  __shared__ float sh[NT / 32];
+  pdl_launch_dependents();
+  pdl_wait();
+  const long long row = blockIdx.x;
+  float v[ROW_VEC][8];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < ROW_VEC; ++i) {
+    const int c = (threadIdx.x + i * NT) * 8;
+    if (c < d) {
+      ld8(x + row * d + c, v[i]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) ss = fmaf(v[i][j], v[i][j], ss);
+    }
+  }
+  const float rs = rsqrtf(block_sum(ss, sh) / (float)d + eps);
+#pragma unroll
+  for (int i = 0; i < ROW_VEC; ++i) {
+    const int c = (threadIdx.x + i * NT) * 8;
+    if (c < d) {
+      float gg[8], o[8];
+      ld8(g + c, gg);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) o[j] = v[i][j] * rs * gg[j];
+      st8(y + row * d + c, o);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(NT)
+layernorm_kernel(const bf16* x, const bf16* g, const bf16* b, bf16* y, int d,
+                 float eps) {
+  __shared__ float sh[NT / 32];
+  pdl_launch_dependents();
+  pdl_wait();
+  const long long row = blockIdx.x;
+  float v[ROW_VEC][8];
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < ROW_VEC; ++i) {
+    const int c = (threadIdx.x + i * NT) * 8;
+    if (c < d) {
+      ld8(x + row * d + c, v[i]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) s += v[i][j];
+    }
+  }
+  const float mean = block_sum(s, sh) / (float)d;
+  float q = 0.f;
+#pragma unroll
+  for (int i = 0; i < ROW_VEC; ++i) {
+    const int c = (threadIdx.x + i * NT) * 8;
+    if (c < d) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float t = v[i][j] - mean;
+        q = fmaf(t, t, q);
+      }
+    }
+  }
+  const float rs = rsqrtf(block_sum(q, sh) / (float)d + eps);
+#pragma unroll
+  for (int i = 0; i < ROW_VEC; ++i) {
+    const int c = (threadIdx.x + i * NT) * 8;
+    if (c < d) {
+      float gg[8], bb[8], o[8];
+      ld8(g + c, gg);
+      ld8(b + c, bb);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) o[j] = (v[i][j] - mean) * rs * gg[j] + bb[j];
+      st8(y + row * d + c, o);
+    }
+  }
+}
+
+__global__ void rope_table_kernel(float* cs, float* sn, int S_max, int D,
+                                  double base) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int half = D / 2;
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)S_max * half) return;
+  const int p = (int)(idx / half), i = (int)(idx - (long long)p * half);
+  const double ang = (double)p * pow(base, -2.0 * (double)i / (double)D);
+  cs[idx] = (float)cos(ang);
+  sn[idx] = (float)sin(ang);
+}
+
+__global__ void __launch_bounds__(NT)
+embed_kernel(const int* tokens, const bf16* emb, bf16* x, int d, int vocab) {
+  pdl_launch_dependents();
+  pdl_wait();
+  int t = tokens[blockIdx.x];
+  t = t < 0 ? 0 : (t >= vocab ? vocab - 1 : t);
+  const uint4* src = reinterpret_cast<const uint4*>(emb + (long long)t * d);
+  uint4* dst = reinterpret_cast<uint4*>(x + (long long)blockIdx.x * d);
+  for (int c = threadIdx.x; c < d / 8; c += NT) dst[c] = src[c];
+}
+
+__global__ void __launch_bounds__(1024)
+greedy_kernel(const float* logits, int* next, int vocab) {
+  __shared__ float sv[32];
+  __shared__ int si[32];
+  pdl_launch_dependents();
+  pdl_wait();
+  const float* row = logits + (long long)blockIdx.x * vocab;
+  float bv = -INFINITY;
+  int bi = 0x7fffffff;
+  for (int j = threadIdx.x; j < vocab; j += blockDim.x) {
+    const float v = row[j];
+    if (v > bv) { bv = v; bi = j; }  // j increases: ties keep the lower index
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) { sv[warp] = bv; si[warp] = bi; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w)
+      if (sv[w] > bv || (sv[w] == bv && si[w] < bi)) { bv = sv[w]; bi = si[w]; }
+    next[blockIdx.x] = bi == 0x7fffffff ? 0 : bi;
+  }
+}
+
+__global__ void advance_kernel(int* seqlens, int B) {
+  pdl_launch_dependents();
+  pdl_wait();
+  for (int b = threadIdx.x; b < B; b += blockDim.x) seqlens[b] += 1;
+}
+
+}  // namespace
+
+int rmsnorm_launch(const bf16* x, const bf16* g, bf16* y, int M, int d,
+                   float eps, cudaStream_t s) {
+  if (d > NT * ROW_VEC * 8) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return FLASHSVD_OK;
+  return launch_pdl(rmsnorm_kernel, dim3(M), dim3(NT), 0, s, x, g, y, d, eps);
+}
+
+int layernorm_launch(const bf16* x, const bf16* g, const bf16* b, bf16* y,
+                     int M, int d, float eps, cudaStream_t s) {
+  if (d > NT * ROW_VEC * 8) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return FLASHSVD_OK;
+  return launch_pdl(layernorm_kernel, dim3(M), dim3(NT), 0, s, x, g, b, y, d, eps);
+}
+
+int rope_table_launch(float* c, float* sn, int S_max, int D, float base,
+                      cudaStream_t s) {
+  const long long n = (long long)S_max * (D / 2);
+  if (n == 0) return FLASHSVD_OK;
+  return launch_pdl(rope_table_kernel, dim3((unsigned)((n + NT - 1) / NT)), dim3(NT), 0, s,
+                    c, sn, S_max, D, (double)base);
+}
+
+int embed_launch(const int* tokens, const bf16* emb, bf16* x, int B, int d,
+                 int vocab, cudaStream_t s) {
+  if (B == 0) return FLASHSVD_OK;
+  return launch_pdl(embed_kernel, dim3(B), dim3(NT), 0, s, tokens, emb, x, d, vocab);
+}
+
+int greedy_launch(const float* logits, int* next, int M, int vocab,
+                  cudaStream_t s) {
+  if (M == 0) return FLASHSVD_OK;
+  return launch_pdl(greedy_kernel, dim3(M), dim3(1024), 0, s, logits, next, vocab);
+}
+
+int advance_launch(int* seqlens, int B, cudaStream_t s) {
+  return launch_pdl(advance_kernel, dim3(1), dim3(32), 0, s, seqlens, B);
+}
+
+}  // namespace fsvd

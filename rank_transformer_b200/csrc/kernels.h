@@ -1,0 +1,109 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include "common.cuh"
+
+namespace fsvd {
+
+// ------------------------------------------------ decode split-K GEMV ----
+// One launch computes, for up to three "problems" that share the same
+// activation rows and the same reduction length K,
+//     out[m, cols] = A[m, a_col + k] . W[k, cols]      (k < K)
+// for rows m in [m0, m0+M), M <= 8, with the reduction split over CTAs and
+// finished deterministically by the last CTA of each column tile.
+
+enum GvPro { PRO_F32 = 0, PRO_BF16 = 1, PRO_RMSNORM = 2 };
+enum GvEpi { EPI_F32 = 0, EPI_BF16 = 1, EPI_QKV = 2, EPI_SWIGLU = 3 };
+
+struct GvProblem {
+  const bf16* W;     // [K x N] (row stride ldw)
+  long long ldw;
+  long long w_row2;  // SWIGLU: first W row of the "up" half
+  int a_col;         // first A column read
+  int a_col2;        // SWIGLU: first A column of the "up" half
+  int N;             // output columns
+  int out_col;       // EPI_F32: column offset of this problem in out32
+  int kind;          // EPI_QKV: 0 = q, 1 = k, 2 = v
+};
+
+struct GvParams {
+  int M, m0, K, KC, splits, nprob;
+  int tile_start[4];
+  GvProblem prob[3];
+  // A operand
+  const float* a32; long long lda;                  // PRO_F32
+  const bf16* x; long long ldx;                     // PRO_BF16 / PRO_RMSNORM
+  const bf16* norm_g; float eps;                    // PRO_RMSNORM (row width K)
+  // epilogue
+  float* out32; long long ldo32;                    // EPI_F32
+  bf16* out16; long long ldo16;                     // EPI_BF16 / QKV(q) / SWIGLU
+  const bf16* bias;                                 // EPI_BF16 (may be null)
+  const bf16* resid; long long ldr;                 // EPI_BF16 (may be null)
+  bf16* k_cache; bf16* v_cache; const int* seqlens; // EPI_QKV
+  int S_max, HD, D;
+  const float* rope_cos; const float* rope_sin;     // [S_max x D/2]
+  // workspace
+  float* part; int* counters;
+};
+
+enum GvMap { MAP_PLAIN = 0, MAP_ROPE = 1, MAP_SWIGLU = 2 };
+
+// Host launcher: fills tile_start/splits/KC, picks the row-tile variant and
+// launches once per group of 8 rows.
+int gemv_launch(GvParams p, int pro, int epi, int map, int total_rows,
+                int target_ctas, cudaStream_t stream);
+int gemv_tiles_for(int map, int N, int D);
+
+// ---------------------------------------------- dense-KV decode attention --
+struct AttnDecParams {
+  const bf16* q; const bf16* k_new; const bf16* v_new;
+  bf16* k_cache; bf16* v_cache; const int* seqlens; bf16* out;
+  int B, H, D, S_max, nsplit, chunk;
+  float scale_log2;              // scale * log2(e)
+  float* part; int* counters;
+};
+int attn_decode_launch(AttnDecParams p, int target_ctas, cudaStream_t stream);
+
+// ----------------------------------------------------------------- glue --
+int rmsnorm_launch(const bf16* x, const bf16* g, bf16* y, int M, int d,
+                   float eps, cudaStream_t s);
+int layernorm_launch(const bf16* x, const bf16* g, const bf16* b, bf16* y,
+                     int M, int d, float eps, cudaStream_t s);
+int rope_table_launch(float* c, float* sn, int S_max, int D, float base,
+                      cudaStream_t s);
+int embed_launch(const int* tokens, const bf16* emb, bf16* x, int B, int d,
+                 int vocab, cudaStream_t s);
+int greedy_launch(const float* logits, int* next, int M, int vocab,
+                  cudaStream_t s);
+int advance_launch(int* seqlens, int B, cudaStream_t s);
+
+// ------------------------------------------ prefill (tcgen05) linears ----
+enum PfEpi { PF_EPI_BF16 = 0, PF_EPI_QKV = 1, PF_EPI_SWIGLU = 2, PF_EPI_GELU = 3,
+             PF_EPI_F32 = 4 };
+
+struct PfLinear {
+  const bf16* x; long long ldx;      // A rows [M x d]
+  const bf16* U; const bf16* V;      // [d x r], [r x n] (SWIGLU: V rows 0..r/2-1 gate, r/2.. up)
+  const bf16* bias;                  // [n] or null
+  const bf16* resid; long long ldr;  // [M x n] or null (added after bias/activation)
+  bf16* y; long long ldy;            // output
+  float* y32;                        // PF_EPI_F32 output (ld = ldy)
+  int M, d, r, n;
+  int epi;
+  // QKV epilogue: y is the q buffer for kind 0; k/v rows go to the caches.
+  int kind; bf16* cache; int S, S_max, HD, D;
+  const float* rope_cos; const float* rope_sin;
+  int* status;
+};
+int prefill_linear_launch(const PfLinear& p, cudaStream_t stream);
+int prefill_dense_launch(const PfLinear& p, cudaStream_t stream);
+
+// ------------------------------------------------ prefill attention -------
+struct AttnPfParams {
+  const bf16* q; const bf16* k; const bf16* v; bf16* out;
+  int B, S, H, D, S_max, causal;
+  float scale_log2;
+};
+int attn_prefill_launch(const AttnPfParams& p, cudaStream_t stream);
+
+}  // namespace fsvd

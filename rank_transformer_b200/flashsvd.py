@@ -1,0 +1,260 @@
+"""ctypes binding of libflashsvd.so (argument marshalling only).
+
+Every function here forwards to the C entry point of the same name in
+``include/flashsvd.h``; tensors are passed as raw device pointers
+(``tensor.data_ptr()``), streams as ``cudaStream_t`` handles.  All compute
+runs in the library's CUDA kernels; there is no CPU fallback.  Importing this
+module fails loudly if the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libflashsvd.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m rank_transformer_b200.build` "
+        "(the CUDA library is required; there is no fallback path)")
+
+lib = C.CDLL(LIB_PATH)
+
+OK = 0
+STATUS_NAMES = {
+    0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_MISALIGNED", 3: "ERR_UNSUPPORTED_SHAPE",
+    4: "ERR_NOT_INITIALIZED", 5: "ERR_CAPTURE_UNSAFE", 6: "ERR_CUDA",
+    7: "ERR_TIMEOUT", 8: "ERR_NO_MEMORY",
+}
+DECODER, ENCODER = 0, 1
+PREFILL_CAUSAL, DECODE, ENCODER_BIDIR = 0, 1, 2
+
+_p = C.c_void_p
+_i = C.c_int
+_f = C.c_float
+
+
+class FlashSVDError(RuntimeError):
+    def __init__(self, fn, status):
+        msg = lib.flashsvd_status_string(status).decode()
+        if status == 6:
+            msg += f" (cudaError {lib.flashsvd_last_cuda_error()})"
+        super().__init__(f"{fn}: {STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+class Factor(C.Structure):
+    _fields_ = [("U", _p), ("V", _p), ("bias", _p), ("r", _i)]
+
+
+class Layer(C.Structure):
+    _fields_ = [
+        ("kind", _i), ("d", _i), ("H", _i), ("D", _i), ("f", _i),
+        ("norm_eps", _f),
+        ("norm1_g", _p), ("norm1_b", _p), ("norm2_g", _p), ("norm2_b", _p),
+        ("q", Factor), ("k", Factor), ("v", Factor), ("o", Factor),
+        ("U_gu", _p), ("V_gu", _p), ("r_f", _i),
+        ("up", Factor), ("down", Factor),
+        ("rope_cos", _p), ("rope_sin", _p),
+    ]
+
+
+_SIGS = {
+    "flashsvd_status_string": ([_i], C.c_char_p),
+    "flashsvd_last_cuda_error": ([], _i),
+    "flashsvd_version": ([], _i),
+    "flashsvd_init": ([_i, _i, _i, _i, _i], _i),
+    "flashsvd_shutdown": ([], _i),
+    "flashsvd_check_device_status": ([_p], _i),
+    "flashsvd_launch_count": ([], C.c_int64),
+    "flashsvd_lowrank_linear": ([_p, _p, _p, _p, _p, _i, _i, _i, _i, _p], _i),
+    "flashsvd_dense_linear_f32": ([_p, _p, _p, _i, _i, _i, _p], _i),
+    "flashsvd_packed_gateup_mlp": ([_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p], _i),
+    "flashsvd_gateup_swiglu": ([_p, _p, _p, _p, _i, _i, _i, _i, _p], _i),
+    "flashsvd_dense_kv_decode_attn": ([_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _f, _p], _i),
+    "flashsvd_prefill_attn": ([_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p], _i),
+    "flashsvd_rmsnorm": ([_p, _p, _p, _i, _i, _f, _p], _i),
+    "flashsvd_layernorm": ([_p, _p, _p, _p, _i, _i, _f, _p], _i),
+    "flashsvd_rope_table": ([_p, _p, _i, _i, _f, _p], _i),
+    "flashsvd_embed": ([_p, _p, _p, _i, _i, _i, _p], _i),
+    "flashsvd_greedy": ([_p, _p, _i, _i, _p], _i),
+    "flashsvd_advance_seqlens": ([_p, _i, _p], _i),
+    "flashsvd_layer_forward": ([C.POINTER(Layer), _p, _p, _p, _p, _i, _i, _i, _i, _p], _i),
+    "flashsvd_decode_graph_capture": ([C.POINTER(Layer), _p, _p, _p, _p, _i, _i, _p,
+                                       C.POINTER(_p)], _i),
+    "flashsvd_capture_begin": ([_p], _i),
+    "flashsvd_capture_end": ([_p, C.POINTER(_p)], _i),
+    "flashsvd_graph_compose": ([C.POINTER(_p), _i, C.POINTER(_p)], _i),
+    "flashsvd_graph_replay": ([_p, _p], _i),
+    "flashsvd_graph_kernel_count": ([_p], _i),
+    "flashsvd_graph_destroy": ([_p], _i),
+}
+
+for _name, (_args, _ret) in _SIGS.items():
+    _fn = getattr(lib, _name)  # AttributeError here means the build is stale
+    _fn.argtypes = _args
+    _fn.restype = _ret
+
+EXPORTED = tuple(_SIGS)
+
+
+def check(fn_name: str, status: int) -> None:
+    if status != OK:
+        raise FlashSVDError(fn_name, status)
+
+
+def ptr(t) -> int | None:
+    """Device pointer of a tensor (None passes NULL)."""
+    return None if t is None else t.data_ptr()
+
+
+def stream_handle(stream=None) -> int | None:
+    """cudaStream_t of a torch stream (default: torch's current stream)."""
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _call(name, *args):
+    check(name, getattr(lib, name)(*args))
+
+
+# ---------------------------------------------------------------- setup --
+
+def init(device: int = 0, max_tokens: int = 8192, max_rank: int = 4096,
+         max_hidden: int = 4096, max_ffn: int = 11008) -> None:
+    _call("flashsvd_init", device, max_tokens, max_rank, max_hidden, max_ffn)
+
+
+def shutdown() -> None:
+    _call("flashsvd_shutdown")
+
+
+def check_device_status(stream=None) -> None:
+    _call("flashsvd_check_device_status", stream_handle(stream))
+
+
+def launch_count() -> int:
+    return int(lib.flashsvd_launch_count())
+
+
+# -------------------------------------------------------------- compute --
+
+def lowrank_linear(x, U, V, bias, y, M, d, r, n, stream=None):
+    _call("flashsvd_lowrank_linear", ptr(x), ptr(U), ptr(V), ptr(bias), ptr(y),
+          M, d, r, n, stream_handle(stream))
+
+
+def dense_linear_f32(x, W, y, M, d, n, stream=None):
+    _call("flashsvd_dense_linear_f32", ptr(x), ptr(W), ptr(y), M, d, n,
+          stream_handle(stream))
+
+
+def packed_gateup_mlp(x, U_gu, V_gu, U_dn, V_dn, y, M, d, r_f, f, r_dn, stream=None):
+    _call("flashsvd_packed_gateup_mlp", ptr(x), ptr(U_gu), ptr(V_gu), ptr(U_dn),
+          ptr(V_dn), ptr(y), M, d, r_f, f, r_dn, stream_handle(stream))
+
+
+def gateup_swiglu(x, U_gu, V_gu, h, M, d, r_f, f, stream=None):
+    _call("flashsvd_gateup_swiglu", ptr(x), ptr(U_gu), ptr(V_gu), ptr(h), M, d,
+          r_f, f, stream_handle(stream))
+
+
+def dense_kv_decode_attn(q, k_new, v_new, k_cache, v_cache, cache_seqlens, out,
+                         B, H, D, S_max, scale, stream=None):
+    _call("flashsvd_dense_kv_decode_attn", ptr(q), ptr(k_new), ptr(v_new),
+          ptr(k_cache), ptr(v_cache), ptr(cache_seqlens), ptr(out), B, H, D,
+          S_max, scale, stream_handle(stream))
+
+
+def prefill_attn(q, k_cache, v_cache, out, B, S, H, D, S_max, causal, scale,
+                 stream=None):
+    _call("flashsvd_prefill_attn", ptr(q), ptr(k_cache), ptr(v_cache), ptr(out),
+          B, S, H, D, S_max, int(causal), scale, stream_handle(stream))
+
+
+def rmsnorm(x, g, y, M, d, eps, stream=None):
+    _call("flashsvd_rmsnorm", ptr(x), ptr(g), ptr(y), M, d, eps, stream_handle(stream))
+
+
+def layernorm(x, g, b, y, M, d, eps, stream=None):
+    _call("flashsvd_layernorm", ptr(x), ptr(g), ptr(b), ptr(y), M, d, eps,
+          stream_handle(stream))
+
+
+def rope_table(cos_tab, sin_tab, S_max, D, base=10000.0, stream=None):
+    _call("flashsvd_rope_table", ptr(cos_tab), ptr(sin_tab), S_max, D, base,
+          stream_handle(stream))
+
+
+def embed(tokens, emb, x, B, d, vocab, stream=None):
+    _call("flashsvd_embed", ptr(tokens), ptr(emb), ptr(x), B, d, vocab,
+          stream_handle(stream))
+
+
+def greedy(logits, next_tokens, M, vocab, stream=None):
+    _call("flashsvd_greedy", ptr(logits), ptr(next_tokens), M, vocab,
+          stream_handle(stream))
+
+
+def advance_seqlens(cache_seqlens, B, stream=None):
+    _call("flashsvd_advance_seqlens", ptr(cache_seqlens), B, stream_handle(stream))
+
+
+def layer_forward(layer: Layer, x, k_cache, v_cache, cache_seqlens, B, S, S_max,
+                  mode, stream=None):
+    _call("flashsvd_layer_forward", C.byref(layer), ptr(x), ptr(k_cache),
+          ptr(v_cache), ptr(cache_seqlens), B, S, S_max, mode, stream_handle(stream))
+
+
+# --------------------------------------------------------------- graphs --
+
+class Graph:
+    """Owner of a flashsvd_graph handle."""
+
+    def __init__(self, handle: int):
+        self.handle = handle
+
+    @property
+    def kernels(self) -> int:
+        return int(lib.flashsvd_graph_kernel_count(self.handle))
+
+    def replay(self, stream=None) -> None:
+        _call("flashsvd_graph_replay", self.handle, stream_handle(stream))
+
+    def destroy(self) -> None:
+        if self.handle:
+            _call("flashsvd_graph_destroy", self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+
+def decode_graph_capture(layer: Layer, x, k_cache, v_cache, cache_seqlens, B,
+                         S_max, stream) -> Graph:
+    h = _p()
+    _call("flashsvd_decode_graph_capture", C.byref(layer), ptr(x), ptr(k_cache),
+          ptr(v_cache), ptr(cache_seqlens), B, S_max, stream_handle(stream), C.byref(h))
+    return Graph(h.value)
+
+
+def capture_begin(stream) -> None:
+    _call("flashsvd_capture_begin", stream_handle(stream))
+
+
+def capture_end(stream) -> Graph:
+    h = _p()
+    _call("flashsvd_capture_end", stream_handle(stream), C.byref(h))
+    return Graph(h.value)
+
+
+def graph_compose(parts) -> Graph:
+    arr = (_p * len(parts))(*[g.handle for g in parts])
+    h = _p()
+    _call("flashsvd_graph_compose", arr, len(parts), C.byref(h))
+    return Graph(h.value)

@@ -1,0 +1,254 @@
+"""GPU parity of the decode path (M <= 32) against the CPU oracle, called
+through the C ABI."""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import flashsvd_oracle as oracle
+from rank_transformer_b200 import synth
+from tests.gpu_util import assert_parity, dev_bf16, host_bits, host_f64
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def fs():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from rank_transformer_b200 import flashsvd
+    flashsvd.init(0, max_tokens=4096, max_rank=4096, max_hidden=4096, max_ffn=11008)
+    return flashsvd
+
+
+def _rand_factors(rng, d, r, n):
+    return (synth.normal_bf16(rng, (d, r), d ** -0.5),
+            synth.normal_bf16(rng, (r, n), r ** -0.5))
+
+
+LINEAR_CASES = [
+    (1, 256, 64, 688), (1, 688, 64, 256), (2, 256, 64, 256), (7, 256, 64, 688),
+    (8, 4096, 512, 4096), (32, 4096, 1024, 4096), (1, 4096, 2048, 4096),
+    (31, 4096, 1216, 4096), (3, 11008, 1792, 4096), (1, 4096, 1792, 11008),
+]
+
+
+@pytest.mark.parametrize("M,d,r,n", LINEAR_CASES)
+def test_lowrank_linear_decode(fs, M, d, r, n):
+    rng = synth.rng_for(1000 + M + d + r + n)
+    U, V = _rand_factors(rng, d, r, n)
+    x = synth.normal_bf16(rng, (M, d))
+    bias = synth.normal_bf16(rng, (n,), 0.02) if (M % 2) else None
+    y = torch.empty((M, n), dtype=torch.bfloat16, device="cuda")
+    b_dev = dev_bf16(bias) if bias is not None else None
+    fs.lowrank_linear(dev_bf16(x), dev_bf16(U), dev_bf16(V), b_dev, y, M, d, r, n)
+    torch.cuda.synchronize()
+    ref = oracle.lowrank_linear(oracle.from_bf16(x), oracle.from_bf16(U), oracle.from_bf16(V),
+                                None if bias is None else oracle.from_bf16(bias))
+    assert_parity(host_f64(y), ref, f"lowrank M={M} d={d} r={r} n={n}")
+
+
+def test_lowrank_linear_svd_factors(fs):
+    # Factors from the truncated SVD of W = P diag(i^-0.5) Q^T (square 4096).
+    rng = synth.rng_for(7)
+    U, V, _ = synth.svd_factors(rng, 4096, 4096, 512, full_rank=512)
+    for M in (1, 8, 32):
+        x = synth.normal_bf16(rng, (M, 4096))
+        y = torch.empty((M, 4096), dtype=torch.bfloat16, device="cuda")
+        fs.lowrank_linear(dev_bf16(x), dev_bf16(U), dev_bf16(V), None, y, M, 4096, 512, 4096)
+        torch.cuda.synchronize()
+        ref = oracle.lowrank_linear(oracle.from_bf16(x), oracle.from_bf16(U), oracle.from_bf16(V))
+        assert_parity(host_f64(y), ref, f"svd M={M}")
+
+
+@pytest.mark.parametrize("M,d,r_f,f,r_dn", [(1, 256, 64, 688, 64), (5, 256, 64, 688, 64),
+                                           (1, 4096, 1792, 11008, 1792),
+                                           (8, 4096, 512, 11008, 1024)])
+def test_packed_mlp_decode(fs, M, d, r_f, f, r_dn):
+    rng = synth.rng_for(2000 + M + r_f)
+    U_gu = synth.normal_bf16(rng, (d, 2 * r_f), d ** -0.5)
+    V_gu = synth.normal_bf16(rng, (2 * r_f, f), r_f ** -0.5)
+    U_dn, V_dn = _rand_factors(rng, f, r_dn, d)
+    x = synth.normal_bf16(rng, (M, d))
+    h = torch.empty((M, f), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((M, d), dtype=torch.bfloat16, device="cuda")
+    xs, ugs, vgs = dev_bf16(x), dev_bf16(U_gu), dev_bf16(V_gu)
+    fs.gateup_swiglu(xs, ugs, vgs, h, M, d, r_f, f)
+    fs.packed_gateup_mlp(xs, ugs, vgs, dev_bf16(U_dn), dev_bf16(V_dn), y, M, d, r_f, f, r_dn)
+    torch.cuda.synchronize()
+    X = oracle.from_bf16(x)
+    w = [oracle.from_bf16(a) for a in (U_gu, V_gu, U_dn, V_dn)]
+    assert_parity(host_f64(h), oracle.gateup_swiglu(X, w[0], w[1], r_f), "gate|up h")
+    assert_parity(host_f64(y), oracle.packed_gateup_mlp(X, *w, r_f), "packed mlp y")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("append", [False, True])
+def test_dense_kv_decode_attention(fs, D, append):
+    rng = synth.rng_for(3000 + D + append)
+    B, H, S_max = 3, 4, 300
+    seqlens = np.array([0, 131, 299], dtype=np.int32)
+    kc = synth.normal_bf16(rng, (B, S_max, H, D))
+    vc = synth.normal_bf16(rng, (B, S_max, H, D))
+    q = synth.normal_bf16(rng, (B, H, D))
+    kn = synth.normal_bf16(rng, (B, H, D))
+    vn = synth.normal_bf16(rng, (B, H, D))
+    kcd, vcd = dev_bf16(kc), dev_bf16(vc)
+    out = torch.empty((B, H, D), dtype=torch.bfloat16, device="cuda")
+    sl = torch.from_numpy(seqlens).cuda()
+    scale = 1.0 / math.sqrt(D)
+    fs.dense_kv_decode_attn(dev_bf16(q), dev_bf16(kn) if append else None,
+                            dev_bf16(vn) if append else None, kcd, vcd, sl, out, B, H, D,
+                            S_max, scale)
+    torch.cuda.synchronize()
+    K, Vv = oracle.from_bf16(kc), oracle.from_bf16(vc)
+    if append:
+        for b in range(B):
+            K[b, seqlens[b]] = oracle.from_bf16(kn[b])
+            Vv[b, seqlens[b]] = oracle.from_bf16(vn[b])
+        # the cache row at the current position now holds the new entries
+        assert np.array_equal(host_bits(kcd)[np.arange(B), seqlens], kn)
+        assert np.array_equal(host_bits(vcd)[np.arange(B), seqlens], vn)
+    Q = oracle.from_bf16(q)
+    ref = np.zeros((B, H, D))
+    for b in range(B):
+        L = seqlens[b] + 1
+        for h in range(H):
+            ref[b, h] = oracle.attention(Q[b, h][None], K[b, :L, h], Vv[b, :L, h])[0]
+    assert_parity(host_f64(out), ref, f"decode attn D={D} append={append}")
+
+
+def test_glue_kernels(fs):
+    rng = synth.rng_for(4000)
+    M, d = 5, 768
+    x = synth.normal_bf16(rng, (M, d))
+    g = synth.normal_bf16(rng, (d,), 0.1, 1.0)
+    b = synth.normal_bf16(rng, (d,), 0.1)
+    y = torch.empty((M, d), dtype=torch.bfloat16, device="cuda")
+    fs.rmsnorm(dev_bf16(x), dev_bf16(g), y, M, d, 1e-5)
+    torch.cuda.synchronize()
+    assert_parity(host_f64(y), oracle.rmsnorm(oracle.from_bf16(x), oracle.from_bf16(g), 1e-5), "rmsnorm")
+    fs.layernorm(dev_bf16(x), dev_bf16(g), dev_bf16(b), y, M, d, 1e-12)
+    torch.cuda.synchronize()
+    assert_parity(host_f64(y), oracle.layernorm(oracle.from_bf16(x), oracle.from_bf16(g),
+                                                oracle.from_bf16(b), 1e-12), "layernorm")
+    # rotary table
+    S_max, D = 4096, 128
+    c = torch.empty((S_max, D // 2), dtype=torch.float32, device="cuda")
+    s = torch.empty_like(c)
+    fs.rope_table(c, s, S_max, D, 10000.0)
+    torch.cuda.synchronize()
+    ang = np.arange(S_max)[:, None] * (10000.0 ** (-2.0 * np.arange(D // 2) / D))[None, :]
+    assert np.max(np.abs(c.cpu().numpy() - np.cos(ang))) < 1e-6
+    assert np.max(np.abs(s.cpu().numpy() - np.sin(ang))) < 1e-6
+    # embedding gather, greedy pick, advance
+    vocab = 1000
+    emb = synth.normal_bf16(rng, (vocab, d))
+    toks = np.array([3, 999, 0, 512], dtype=np.int32)
+    xe = torch.empty((4, d), dtype=torch.bfloat16, device="cuda")
+    fs.embed(torch.from_numpy(toks).cuda(), dev_bf16(emb), xe, 4, d, vocab)
+    logits = rng.standard_normal((3, vocab)).astype(np.float32)
+    logits[1, 10] = logits[1, 700] = 50.0  # tie -> lowest index
+    nxt = torch.empty(3, dtype=torch.int32, device="cuda")
+    fs.greedy(torch.from_numpy(logits).cuda(), nxt, 3, vocab)
+    sl = torch.tensor([5, 7], dtype=torch.int32, device="cuda")
+    fs.advance_seqlens(sl, 2)
+    torch.cuda.synchronize()
+    assert np.array_equal(host_bits(xe), emb[toks])
+    assert list(nxt.cpu().numpy()) == list(oracle.greedy(logits))
+    assert list(sl.cpu().numpy()) == [6, 8]
+
+
+def _layer_struct(fs, w, d, H, D, f, r, r_f, cos_t, sin_t):
+    dev = {k: dev_bf16(v) for k, v in w.items() if isinstance(v, np.ndarray)}
+    L = fs.Layer()
+    L.kind = fs.DECODER
+    L.d, L.H, L.D, L.f = d, H, D, f
+    L.norm_eps = 1e-5
+    L.norm1_g, L.norm2_g = dev["g1"].data_ptr(), dev["g2"].data_ptr()
+    for name in ("q", "k", "v", "o"):
+        F = getattr(L, name)
+        F.U, F.V, F.bias, F.r = dev["U_" + name].data_ptr(), dev["V_" + name].data_ptr(), None, r
+    L.U_gu, L.V_gu, L.r_f = dev["U_gu"].data_ptr(), dev["V_gu"].data_ptr(), r_f
+    L.down.U, L.down.V, L.down.bias, L.down.r = dev["U_dn"].data_ptr(), dev["V_dn"].data_ptr(), None, r_f
+    L.rope_cos, L.rope_sin = cos_t.data_ptr(), sin_t.data_ptr()
+    return L, dev
+
+
+@pytest.mark.parametrize("B", [1, 3])
+def test_decoder_layer_decode_steps(fs, B):
+    """Tiny decoder layer (hidden 256, 4 heads of 64, SwiGLU 688, rank 64):
+    16 decode steps after a 128-token history; each step is compared with
+    the oracle's decode of the same layer over the GPU's cache contents
+    (teacher forcing)."""
+    d, H, D, f, r, steps, P = 256, 4, 64, 688, 64, 16, 128
+    S_max = P + steps
+    rng = synth.rng_for(0)
+    w = synth.decoder_layer_weights(rng, d, f, r, r, gain_jitter=0.1)
+    cos_t = torch.empty((S_max, D // 2), dtype=torch.float32, device="cuda")
+    sin_t = torch.empty_like(cos_t)
+    fs.rope_table(cos_t, sin_t, S_max, D, 10000.0)
+    L, dev = _layer_struct(fs, w, d, H, D, f, r, r, cos_t, sin_t)
+    kc = dev_bf16(synth.normal_bf16(rng, (B, S_max, H, D)))
+    vc = dev_bf16(synth.normal_bf16(rng, (B, S_max, H, D)))
+    seq = torch.full((B,), P, dtype=torch.int32, device="cuda")
+    wf = oracle.widen_layer(w)
+    for t in range(steps):
+        xt = synth.normal_bf16(rng, (B, d))
+        hist_k, hist_v = host_f64(kc), host_f64(vc)
+        x = dev_bf16(xt)
+        fs.layer_forward(L, x, kc, vc, seq, B, 1, S_max, fs.DECODE)
+        fs.advance_seqlens(seq, B)
+        torch.cuda.synchronize()
+        y, kn, vn = oracle.decoder_layer_decode(oracle.from_bf16(xt), wf, H, hist_k, hist_v,
+                                                [P + t] * B)
+        assert_parity(host_f64(x), y, f"layer decode step {t}")
+        assert_parity(host_f64(kc)[:, P + t], kn, f"appended k step {t}")
+        assert_parity(host_f64(vc)[:, P + t], vn, f"appended v step {t}")
+    assert list(seq.cpu().numpy()) == [P + steps] * B
+
+
+def test_decode_graph_replay_bitwise(fs):
+    d, H, D, f, r, P, B = 256, 4, 64, 688, 64, 100, 2
+    S_max = P + 8
+    rng = synth.rng_for(5)
+    w = synth.decoder_layer_weights(rng, d, f, r, r, gain_jitter=0.1)
+    cos_t = torch.empty((S_max, D // 2), dtype=torch.float32, device="cuda")
+    sin_t = torch.empty_like(cos_t)
+    fs.rope_table(cos_t, sin_t, S_max, D, 10000.0)
+    L, dev = _layer_struct(fs, w, d, H, D, f, r, r, cos_t, sin_t)
+    kc0 = synth.normal_bf16(rng, (B, S_max, H, D))
+    vc0 = synth.normal_bf16(rng, (B, S_max, H, D))
+    xs = [synth.normal_bf16(rng, (B, d)) for _ in range(6)]
+
+    def run(use_graph):
+        kc, vc = dev_bf16(kc0), dev_bf16(vc0)
+        seq = torch.full((B,), P, dtype=torch.int32, device="cuda")
+        x = torch.empty((B, d), dtype=torch.bfloat16, device="cuda")
+        stream = torch.cuda.Stream()
+        outs = []
+        with torch.cuda.stream(stream):
+            g = fs.decode_graph_capture(L, x, kc, vc, seq, B, S_max, stream) if use_graph else None
+            for xt in xs:
+                x.copy_(dev_bf16(xt))
+                if use_graph:
+                    g.replay(stream)
+                else:
+                    fs.layer_forward(L, x, kc, vc, seq, B, 1, S_max, fs.DECODE, stream)
+                fs.advance_seqlens(seq, B, stream)
+                outs.append(x.clone())
+        stream.synchronize()
+        if g is not None:
+            assert g.kernels >= 9
+            g.destroy()
+        return [host_bits(o) for o in outs], host_bits(kc)
+
+    eager, kc_e = run(False)
+    graph, kc_g = run(True)
+    eager2, _ = run(False)
+    for a, b, c in zip(eager, graph, eager2):
+        assert np.array_equal(a, b)
+        assert np.array_equal(a, c)
+    assert np.array_equal(kc_e, kc_g)
