@@ -98,6 +98,16 @@ FLASHSVD_API int flashsvd_check_device_status(flashsvd_stream stream);
  * plus the kernel nodes of every replayed graph. */
 FLASHSVD_API int64_t flashsvd_launch_count(void);
 
+/* Profiler.  flashsvd_profile_enable(1) brackets every EAGER launch of this
+ * library with CUDA events on its stream (graph replays and launches made
+ * during capture are not instrumented; the events serialise the launches).
+ * flashsvd_profile_report synchronises the device and writes one line per
+ * operation, "name launches total_ms algorithmic_bytes flops\n", into buf
+ * (NUL-terminated, truncated to buflen); reset != 0 clears the totals.  With
+ * buf == NULL it returns the buffer size needed. */
+FLASHSVD_API int flashsvd_profile_enable(int on);
+FLASHSVD_API int flashsvd_profile_report(char* buf, int buflen, int reset);
+
 /* ------------------------------------------------------ factorized linear --
  * y[M x n] = (x[M x d] . U[d x r]) . V[r x n] + bias[n]           (bias may be NULL)
  *

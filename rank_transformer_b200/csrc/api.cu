@@ -66,7 +66,17 @@ int check_w8(int v) {
   return (v % 8) ? FLASHSVD_ERR_UNSUPPORTED_SHAPE : FLASHSVD_OK;
 }
 
-int target_ctas() { return g_ctx.sm_count * 4; }
+int target_ctas() { return g_ctx.sm_count * 3; }
+
+// Capacity guard for decode attention: one partial of D + 2 floats per
+// (batch, head, 64-key chunk).
+int attn_fits(int B, int H, int D, int S_max) {
+  const size_t chunks = (size_t)ceil_div(S_max, 64);
+  if (chunks > 1024 || (size_t)B * H > (size_t)kCountersN ||
+      (size_t)B * H * chunks * (D + 2) > g_ctx.apart_elems)
+    return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  return FLASHSVD_OK;
+}
 
 GvParams gv_base() {
   GvParams p;
@@ -226,6 +236,7 @@ int layer_decode(const flashsvd_layer* L, bf16* x, bf16* kc, bf16* vc,
     FSVD_TRY(gemv_launch(p, PRO_F32, EPI_QKV, MAP_ROPE, B, target_ctas(), s));
   }
   // 3) dense-KV attention over 0..pos
+  FSVD_TRY(attn_fits(B, L->H, L->D, S_max));
   {
     AttnDecParams a;
     memset(&a, 0, sizeof(a));
@@ -414,7 +425,7 @@ int flashsvd_init(int device, int max_tokens, int max_rank, int max_hidden,
   const int wide = max_ffn > max_hidden ? max_ffn : max_hidden;
   c.z_elems = (size_t)DECODE_MAX_ROWS * 3 * (max_rank > wide / 2 ? max_rank : wide / 2) + 4096;
   c.part_elems = (size_t)16 << 20;
-  c.apart_elems = (size_t)DECODE_MAX_ROWS * 64 * (max_hidden + 2 * (max_hidden / 64 + 1));
+  c.apart_elems = (size_t)16 << 20;  // split-sequence partials of decode attention
   cudaError_t e = cudaSuccess;
 #define FSVD_ALLOC(ptr, bytes) \
   if (e == cudaSuccess) e = cudaMalloc((void**)&(ptr), (bytes));
@@ -567,8 +578,7 @@ int flashsvd_dense_kv_decode_attn(const flashsvd_bf16* q,
   if (B < 0 || H <= 0 || S_max <= 0 || !(scale > 0.f)) return FLASHSVD_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   if (B == 0) return FLASHSVD_OK;
-  if ((size_t)B * H * 64 * (D + 2) > g_ctx.apart_elems || B * H > kCountersN)
-    return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  FSVD_TRY(attn_fits(B, H, D, S_max));
   AttnDecParams a;
   memset(&a, 0, sizeof(a));
   a.q = (const bf16*)q; a.k_new = (const bf16*)k_new; a.v_new = (const bf16*)v_new;

@@ -38,13 +38,28 @@ inline int cuda_status(cudaError_t e) {
 
 #define FSVD_CUDA(expr) FSVD_TRY(::fsvd::cuda_status(expr))
 
+// Name and algorithmic work of one launch (for the optional profiler).
+struct LaunchTag {
+  const char* name;
+  double bytes;   // bytes the operation must move to or from HBM
+  double flops;
+};
+
+// Profiler hooks (prof.cu): when enabled, eager launches are bracketed by
+// CUDA events on their stream; launches being captured are not.
+bool prof_active(cudaStream_t s);
+void prof_begin(cudaStream_t s);
+void prof_end(const LaunchTag& tag, cudaStream_t s);
+
 // Launch `kernel` with programmatic dependent launch enabled, so that its
 // prologue (weight loads) can overlap the tail of the previous kernel on the
 // stream; the kernel orders itself after that kernel with
 // griddepcontrol.wait before it touches anything the previous kernel wrote.
 template <typename... KArgs, typename... Args>
-inline int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block,
-                      size_t smem, cudaStream_t stream, Args&&... args) {
+inline int launch_pdl(const LaunchTag& tag, void (*kernel)(KArgs...), dim3 grid,
+                      dim3 block, size_t smem, cudaStream_t stream, Args&&... args) {
+  const bool prof = prof_active(stream);
+  if (prof) prof_begin(stream);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -58,6 +73,7 @@ inline int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block,
   cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
   if (e != cudaSuccess) return cuda_status(e);
   g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (prof) prof_end(tag, stream);
   return FLASHSVD_OK;
 }
 

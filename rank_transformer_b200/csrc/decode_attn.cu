@@ -16,42 +16,33 @@ namespace {
 
 constexpr int AD_THREADS = 128;
 constexpr int AD_WARPS = AD_THREADS / 32;
-constexpr int AD_KB = 8;  // keys per warp per batch
+constexpr int AD_CHUNK = 64;  // keys per CTA (two per lane in the score pass)
 
-template <int EPL>
-__device__ __forceinline__ void load_row(const bf16* p, float* v) {
-  if (EPL == 4) {
-    const uint2 u = *reinterpret_cast<const uint2*>(p);
-    v[0] = bf_lo(u.x); v[1] = bf_hi(u.x); v[2] = bf_lo(u.y); v[3] = bf_hi(u.y);
-  } else {
-    const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
-    v[0] = bf_lo(u); v[1] = bf_hi(u);
-  }
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const uint32_t sa = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global.L2::128B [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
 }
 
-template <int EPL>
-__device__ __forceinline__ void store_row(bf16* p, const float* v) {
-  if (EPL == 4) {
-    uint2 u;
-    u.x = pack_bf2(v[0], v[1]);
-    u.y = pack_bf2(v[2], v[3]);
-    *reinterpret_cast<uint2*>(p) = u;
-  } else {
-    *reinterpret_cast<uint32_t*>(p) = pack_bf2(v[0], v[1]);
-  }
-}
-
+// K/V rows of the chunk live in shared memory with a row pitch of D + 8
+// elements, so that 32 lanes reading 16 bytes of 32 different rows hit
+// distinct banks.
 template <int D>
 __global__ void __launch_bounds__(AD_THREADS)
 attn_decode_kernel(const __grid_constant__ AttnDecParams p) {
-  constexpr int EPL = D / 32;
-  __shared__ float s_m[AD_WARPS], s_l[AD_WARPS];
-  __shared__ float s_o[AD_WARPS][D];
+  constexpr int PITCH = D + 8;
+  constexpr int VPR = D / 8;  // 16-byte vectors per row
+  __shared__ __align__(16) bf16 Ks[AD_CHUNK * PITCH];
+  __shared__ __align__(16) bf16 Vs[AD_CHUNK * PITCH];
+  __shared__ __align__(16) float qs[D];
+  __shared__ float ps[AD_CHUNK];
+  __shared__ float s_red[AD_WARPS];
+  __shared__ float s_o[AD_THREADS / D > 1 ? AD_THREADS / D : 1][D];
   __shared__ int s_last;
 
   const int bh = blockIdx.x, s = blockIdx.y;
   const int b = bh / p.H, h = bh - b * p.H;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long HD = (long long)p.H * D;
 
   pdl_launch_dependents();
   pdl_wait();
@@ -59,114 +50,101 @@ attn_decode_kernel(const __grid_constant__ AttnDecParams p) {
   int pos = p.seqlens[b];
   pos = pos < 0 ? 0 : (pos >= p.S_max ? p.S_max - 1 : pos);
   const int L = pos + 1;
-  const int start = s * p.chunk;
-  const int end = min(L, start + p.chunk);
-
-  const long long HD = (long long)p.H * D;
-  const long long head_off = ((long long)b * p.H + h) * D + lane * EPL;
-  float qv[EPL];
-  load_row<EPL>(p.q + head_off, qv);
-#pragma unroll
-  for (int e = 0; e < EPL; ++e) qv[e] *= p.scale_log2;
-
-  const bf16* kbase = p.k_cache + (long long)b * p.S_max * HD + (long long)h * D + lane * EPL;
-  const bf16* vbase = p.v_cache + (long long)b * p.S_max * HD + (long long)h * D + lane * EPL;
-
-  // The CTA whose slice holds the current position writes the new key and
-  // value into the cache and uses them directly (no other CTA reads them).
-  const bool has_new = p.k_new != nullptr && pos >= start && pos < end;
-  float kn[EPL], vn[EPL];
-  if (has_new) {
-    load_row<EPL>(p.k_new + head_off, kn);
-    load_row<EPL>(p.v_new + head_off, vn);
-    if (warp == 0) {
-      store_row<EPL>(p.k_cache + ((long long)b * p.S_max + pos) * HD + (long long)h * D + lane * EPL, kn);
-      store_row<EPL>(p.v_cache + ((long long)b * p.S_max + pos) * HD + (long long)h * D + lane * EPL, vn);
-    }
-  }
-
-  float m = -INFINITY, l = 0.f, acc[EPL];
-#pragma unroll
-  for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
-
-  for (int j0 = start + warp * AD_KB; j0 < end; j0 += AD_WARPS * AD_KB) {
-    float kv[AD_KB][EPL], vv[AD_KB][EPL];
-#pragma unroll
-    for (int i = 0; i < AD_KB; ++i) {
-      const int j = j0 + i;
-      if (j < end) {
-        if (has_new && j == pos) {
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) { kv[i][e] = kn[e]; vv[i][e] = vn[e]; }
-        } else {
-          load_row<EPL>(kbase + (long long)j * HD, kv[i]);
-          load_row<EPL>(vbase + (long long)j * HD, vv[i]);
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) { kv[i][e] = 0.f; vv[i][e] = 0.f; }
-      }
-    }
-    float sc[AD_KB];
-    float mb = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < AD_KB; ++i) {
-      float dot = 0.f;
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) dot = fmaf(qv[e], kv[i][e], dot);
-      dot = warp_sum(dot);
-      sc[i] = (j0 + i < end) ? dot : -INFINITY;
-      mb = fmaxf(mb, sc[i]);
-    }
-    const float mn = fmaxf(m, mb);
-    const float corr = exp2f(m - mn);
-    l *= corr;
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) acc[e] *= corr;
-#pragma unroll
-    for (int i = 0; i < AD_KB; ++i) {
-      const float pe = exp2f(sc[i] - mn);
-      l += pe;
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) acc[e] = fmaf(pe, vv[i][e], acc[e]);
-    }
-    m = mn;
-  }
-
-  // ---- merge the warps of this CTA ----
-  if (lane == 0) { s_m[warp] = m; s_l[warp] = l; }
-#pragma unroll
-  for (int e = 0; e < EPL; ++e) s_o[warp][lane * EPL + e] = acc[e];
-  __syncthreads();
-  float M = -INFINITY;
-#pragma unroll
-  for (int w = 0; w < AD_WARPS; ++w) M = fmaxf(M, s_m[w]);
-  float Lc = 0.f;
-  float wgt[AD_WARPS];
-#pragma unroll
-  for (int w = 0; w < AD_WARPS; ++w) {
-    wgt[w] = (M == -INFINITY) ? 0.f : exp2f(s_m[w] - M);
-    Lc += s_l[w] * wgt[w];
-  }
-
-  if (p.nsplit == 1) {
-    for (int dd = tid; dd < D; dd += AD_THREADS) {
-      float o = 0.f;
-#pragma unroll
-      for (int w = 0; w < AD_WARPS; ++w) o += s_o[w][dd] * wgt[w];
-      p.out[((long long)b * p.H + h) * D + dd] = f2bf(o / Lc);
-    }
-    return;
-  }
+  const int start = s * AD_CHUNK;
+  const int n = min(L - start, AD_CHUNK);  // keys in this CTA (may be <= 0)
 
   float* mypart = p.part + ((long long)bh * p.nsplit + s) * (D + 2);
-  for (int dd = tid; dd < D; dd += AD_THREADS) {
-    float o = 0.f;
+  if (n > 0) {
+    // ---- all K/V rows of the chunk in flight at once ----
+    const bf16* kg = p.k_cache + ((long long)b * p.S_max + start) * HD + (long long)h * D;
+    const bf16* vg = p.v_cache + ((long long)b * p.S_max + start) * HD + (long long)h * D;
+    const bool has_new = p.k_new != nullptr && pos >= start && pos < start + n;
+    for (int idx = tid; idx < n * VPR; idx += AD_THREADS) {
+      const int j = idx / VPR, c = (idx - j * VPR) * 8;
+      if (has_new && start + j == pos) continue;
+      cp_async16(Ks + j * PITCH + c, kg + (long long)j * HD + c);
+      cp_async16(Vs + j * PITCH + c, vg + (long long)j * HD + c);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    const long long qoff = ((long long)b * p.H + h) * D;
+    for (int c = tid; c < D; c += AD_THREADS) qs[c] = bf2f(p.q[qoff + c]) * p.scale_log2;
+    if (has_new) {
+      // The new key/value: written to the cache and used from shared memory.
+      const int j = pos - start;
+      const long long goff = ((long long)b * p.S_max + pos) * HD + (long long)h * D;
+      for (int c = tid * 8; c < D; c += AD_THREADS * 8) {
+        const uint4 kv = *reinterpret_cast<const uint4*>(p.k_new + qoff + c);
+        const uint4 vv = *reinterpret_cast<const uint4*>(p.v_new + qoff + c);
+        *reinterpret_cast<uint4*>(Ks + j * PITCH + c) = kv;
+        *reinterpret_cast<uint4*>(Vs + j * PITCH + c) = vv;
+        *reinterpret_cast<uint4*>(p.k_cache + goff + c) = kv;
+        *reinterpret_cast<uint4*>(p.v_cache + goff + c) = vv;
+      }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+
+    // ---- scores: one key per lane (two lanes' worth per warp pass) ----
+    float mloc = -INFINITY;
+    for (int j = tid; j < n; j += AD_THREADS) {
+      float dot = 0.f;
 #pragma unroll
-    for (int w = 0; w < AD_WARPS; ++w) o += s_o[w][dd] * wgt[w];
-    __stcg(mypart + 2 + dd, o);
+      for (int c = 0; c < D; c += 8) {
+        const uint4 u = *reinterpret_cast<const uint4*>(Ks + j * PITCH + c);
+        const float4 q0 = *reinterpret_cast<const float4*>(qs + c);
+        const float4 q1 = *reinterpret_cast<const float4*>(qs + c + 4);
+        dot = fmaf(q0.x, bf_lo(u.x), dot); dot = fmaf(q0.y, bf_hi(u.x), dot);
+        dot = fmaf(q0.z, bf_lo(u.y), dot); dot = fmaf(q0.w, bf_hi(u.y), dot);
+        dot = fmaf(q1.x, bf_lo(u.z), dot); dot = fmaf(q1.y, bf_hi(u.z), dot);
+        dot = fmaf(q1.z, bf_lo(u.w), dot); dot = fmaf(q1.w, bf_hi(u.w), dot);
+      }
+      ps[j] = dot;
+      mloc = fmaxf(mloc, dot);
+    }
+    mloc = warp_max(mloc);
+    if (lane == 0) s_red[warp] = mloc;
+    __syncthreads();
+    float M = s_red[0];
+#pragma unroll
+    for (int w = 1; w < AD_WARPS; ++w) M = fmaxf(M, s_red[w]);
+    __syncthreads();
+    float lsum = 0.f;
+    for (int j = tid; j < n; j += AD_THREADS) {
+      const float e = exp2f(ps[j] - M);
+      ps[j] = e;
+      lsum += e;
+    }
+    lsum = warp_sum(lsum);
+    if (lane == 0) s_red[warp] = lsum;
+    __syncthreads();
+    float Lc = 0.f;
+#pragma unroll
+    for (int w = 0; w < AD_WARPS; ++w) Lc += s_red[w];
+
+    // ---- o = sum_j p_j v_j: thread owns one dimension and a key stripe ----
+    constexpr int STRIPES = AD_THREADS / D > 1 ? AD_THREADS / D : 1;
+    const int dim = tid % D, stripe = tid / D;
+    float o = 0.f;
+    if (stripe < STRIPES) {
+      for (int j = stripe; j < n; j += STRIPES) o = fmaf(ps[j], bf2f(Vs[j * PITCH + dim]), o);
+      s_o[stripe][dim] = o;
+    }
+    __syncthreads();
+    if (tid < D) {
+      o = 0.f;
+#pragma unroll
+      for (int st = 0; st < STRIPES; ++st) o += s_o[st][tid];
+      if (p.nsplit == 1) {
+        p.out[((long long)b * p.H + h) * D + tid] = f2bf(o / Lc);
+        return;
+      }
+      __stcg(mypart + 2 + tid, o);
+      if (tid == 0) { __stcg(mypart, M); __stcg(mypart + 1, Lc); }
+    }
+  } else {
+    if (tid == 0) { __stcg(mypart, -INFINITY); __stcg(mypart + 1, 0.f); }
   }
-  if (tid == 0) { __stcg(mypart, M); __stcg(mypart + 1, Lc); }
+  if (p.nsplit == 1) return;
   __threadfence();
   __syncthreads();
   if (tid == 0) s_last = (atomicAdd(p.counters + bh, 1) == p.nsplit - 1);
@@ -196,16 +174,17 @@ attn_decode_kernel(const __grid_constant__ AttnDecParams p) {
 }  // namespace
 
 int attn_decode_launch(AttnDecParams p, int target_ctas, cudaStream_t stream) {
+  (void)target_ctas;
   const int pairs = p.B * p.H;
-  int nsplit = target_ctas / pairs;
-  const int max_split = ceil_div(p.S_max, 64);
-  nsplit = nsplit < 1 ? 1 : (nsplit > max_split ? max_split : nsplit);
-  nsplit = nsplit > 64 ? 64 : nsplit;
-  p.chunk = round_up(ceil_div(p.S_max, nsplit), AD_WARPS * AD_KB);
-  p.nsplit = ceil_div(p.S_max, p.chunk);
+  p.chunk = AD_CHUNK;
+  p.nsplit = ceil_div(p.S_max, AD_CHUNK);
+  if (p.nsplit > 1024) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   const dim3 grid(pairs, p.nsplit);
-  if (p.D == 128) return launch_pdl(attn_decode_kernel<128>, grid, dim3(AD_THREADS), 0, stream, p);
-  if (p.D == 64) return launch_pdl(attn_decode_kernel<64>, grid, dim3(AD_THREADS), 0, stream, p);
+  // History K and V once (cache length is only known on the device; the
+  // tag counts the full capacity), plus q, out and the new rows.
+  const LaunchTag tag{"attn_decode", 2.0 * 2.0 * pairs * (double)p.S_max * p.D, 0.0};
+  if (p.D == 128) return launch_pdl(tag, attn_decode_kernel<128>, grid, dim3(AD_THREADS), 0, stream, p);
+  if (p.D == 64) return launch_pdl(tag, attn_decode_kernel<64>, grid, dim3(AD_THREADS), 0, stream, p);
   return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
 }
 

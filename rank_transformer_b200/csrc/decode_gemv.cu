@@ -40,13 +40,21 @@ __device__ __forceinline__ int tile_col(int t, int c, int D) {
   return t * 32 + (c & 31);  // SWIGLU: c < 32 gate, c >= 32 up, same column
 }
 
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const uint32_t sa = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global.L2::128B [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 template <int MT, int PRO, int EPI, int MAP>
 __global__ void __launch_bounds__(GV_THREADS)
 gemv_splitk_kernel(const __grid_constant__ GvParams p) {
   constexpr int NSEG = (MAP == MAP_SWIGLU) ? 2 : 1;
   extern __shared__ __align__(16) float sm[];
-  float* As = sm;                           // [NSEG][MT][KC]
-  float* red = sm + NSEG * MT * p.KC;       // [8][MT][64]
+  float* As = sm;                                   // [NSEG][MT][KC] fp32
+  float* red = As + NSEG * MT * p.KC;               // [8][MT][64] fp32
+  bf16* Ws = reinterpret_cast<bf16*>(red + 8 * MT * 64);  // [KC][64] bf16
   __shared__ float s_rstd[MT];
   __shared__ int s_last;
 
@@ -70,27 +78,29 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
 
   pdl_launch_dependents();
 
-  // Factor loads do not depend on the previous kernel: issue the first
-  // batch before waiting for it.
-  const bf16* wp = P.W + (wrow + k0 + rr) * P.ldw + col;
-  uint4 wv[GV_BATCH];
-#pragma unroll
-  for (int i = 0; i < GV_BATCH; ++i) {
-    const int kk = rr + 32 * i;
-    wv[i] = (i < niter && kk < kn && colok)
-                ? ldg_stream(wp + (long long)(32 * i) * P.ldw)
-                : make_uint4(0u, 0u, 0u, 0u);
+  // The whole [kn x 64] factor block of this CTA is copied into shared
+  // memory with asynchronous 16-byte copies issued before waiting for the
+  // previous kernel: factors never depend on it, so these bytes stream
+  // while that kernel drains.
+  if (colok) {
+    const bf16* wp = P.W + (wrow + k0 + rr) * P.ldw + col;
+    for (int i = 0; i < niter; ++i) {
+      const int kk = rr + 32 * i;
+      if (kk < kn) cp_async16(Ws + kk * 64 + cg * 8, wp + (long long)(32 * i) * P.ldw);
+    }
   }
+  cp_async_commit();
 
   pdl_wait();
-
   // ---- stage the activation slice A[m0+m, acol + k0 .. + KC) in fp32 ----
   if (PRO == PRO_RMSNORM) {
-    for (int m = warp; m < MT; m += GV_THREADS / 32) {
+    // Sum of squares of each row: all 256 threads read the row at once.
+    float* ssq = red;  // [8 warps][MT] scratch, reused below
+    for (int m = 0; m < MT; ++m) {
       float ss = 0.f;
       if (m < p.M) {
         const bf16* xr = p.x + (long long)(p.m0 + m) * p.ldx;
-        for (int c = lane * 8; c < p.K; c += 256) {
+        for (int c = tid * 8; c < p.K; c += GV_THREADS * 8) {
           float w[8];
           unpack8(*reinterpret_cast<const uint4*>(xr + c), w);
 #pragma unroll
@@ -98,7 +108,14 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
         }
       }
       ss = warp_sum(ss);
-      if (lane == 0) s_rstd[m] = rsqrtf(ss / (float)p.K + p.eps);
+      if (lane == 0) ssq[warp * MT + m] = ss;
+    }
+    __syncthreads();
+    if (tid < MT) {
+      float ss = 0.f;
+#pragma unroll
+      for (int w = 0; w < GV_THREADS / 32; ++w) ss += ssq[w * MT + tid];
+      s_rstd[tid] = rsqrtf(ss / (float)p.K + p.eps);
     }
     __syncthreads();
   }
@@ -137,7 +154,9 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
   }
   __syncthreads();
 
-  // ---- multiply-accumulate ----
+  // ---- multiply-accumulate from shared memory ----
+  cp_async_wait_all();
+  __syncthreads();
   float acc[MT][8];
 #pragma unroll
   for (int m = 0; m < MT; ++m)
@@ -145,28 +164,17 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
     for (int j = 0; j < 8; ++j) acc[m][j] = 0.f;
 
   const float* Aseg = As + (NSEG == 2 ? hi : 0) * MT * p.KC;
-  for (int base = 0; base < niter; base += GV_BATCH) {
-    if (base > 0) {
+#pragma unroll 4
+  for (int i = 0; i < niter; ++i) {
+    const int kk = rr + 32 * i;
+    if (kk < kn) {
+      float w[8];
+      unpack8(*reinterpret_cast<const uint4*>(Ws + kk * 64 + cg * 8), w);
 #pragma unroll
-      for (int i = 0; i < GV_BATCH; ++i) {
-        const int kk = rr + 32 * (base + i);
-        wv[i] = (base + i < niter && kk < kn && colok)
-                    ? ldg_stream(wp + (long long)(32 * (base + i)) * P.ldw)
-                    : make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
+      for (int m = 0; m < MT; ++m) {
+        const float a = Aseg[m * p.KC + kk];
 #pragma unroll
-    for (int i = 0; i < GV_BATCH; ++i) {
-      if (base + i < niter) {
-        const int kk = rr + 32 * (base + i);
-        float w[8];
-        unpack8(wv[i], w);
-#pragma unroll
-        for (int m = 0; m < MT; ++m) {
-          const float a = Aseg[m * p.KC + kk];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) acc[m][j] = fmaf(a, w[j], acc[m][j]);
-        }
+        for (int j = 0; j < 8; ++j) acc[m][j] = fmaf(a, w[j], acc[m][j]);
       }
     }
   }
@@ -290,18 +298,46 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
   }
 }
 
+const char* gv_name(int pro, int epi) {
+  if (epi == EPI_QKV) return "gemv_qkv_rope_append";
+  if (epi == EPI_SWIGLU) return "gemv_gateup_swiglu";
+  if (epi == EPI_BF16) return "gemv_stage2";
+  return pro == PRO_RMSNORM ? "gemv_stage1_rmsnorm" : "gemv_stage1";
+}
+
+// Bytes one launch must move: every factor element once, the activation
+// rows once, the outputs once (a residual is read once more).
+double gv_bytes(const GvParams& p, int pro, int epi) {
+  double b = 0.0;
+  for (int i = 0; i < p.nprob; ++i) {
+    const double kn = (double)p.K * p.prob[i].N;
+    b += 2.0 * kn * (epi == EPI_SWIGLU ? 2.0 : 1.0);
+    b += (double)p.M * p.prob[i].N * (epi == EPI_F32 ? 4.0 : 2.0);
+  }
+  const double a_elems = (double)p.M * p.K * (epi == EPI_SWIGLU ? 2.0 : 1.0) *
+                         (pro == PRO_F32 ? (epi == EPI_QKV ? 3.0 : 1.0) : 1.0);
+  b += a_elems * (pro == PRO_F32 ? 4.0 : 2.0);
+  if (p.resid) b += 2.0 * p.M * p.prob[0].N;
+  return b;
+}
+
 template <int MT, int PRO, int EPI, int MAP>
 int launch_one(const GvParams& p, int total_tiles, cudaStream_t stream) {
   constexpr int NSEG = (MAP == MAP_SWIGLU) ? 2 : 1;
-  const size_t smem = (size_t)(NSEG * MT * p.KC + 8 * MT * 64) * sizeof(float);
+  const size_t smem = (size_t)(NSEG * MT * p.KC + 8 * MT * 64) * sizeof(float) +
+                      (size_t)p.KC * 64 * sizeof(bf16);
   auto kern = gemv_splitk_kernel<MT, PRO, EPI, MAP>;
   static bool configured = false;  // once per instantiation
   if (!configured) {
-    FSVD_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024));
+    FSVD_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
     configured = true;
   }
-  if (smem > 160 * 1024) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
-  return launch_pdl(kern, dim3(total_tiles, p.splits), dim3(GV_THREADS), smem, stream, p);
+  if (smem > 200 * 1024) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  double flops = 0.0;
+  for (int i = 0; i < p.nprob; ++i)
+    flops += 2.0 * p.M * (double)p.K * p.prob[i].N * (EPI == EPI_SWIGLU ? 2.0 : 1.0);
+  const LaunchTag tag{gv_name(PRO, EPI), gv_bytes(p, PRO, EPI), flops};
+  return launch_pdl(tag, kern, dim3(total_tiles, p.splits), dim3(GV_THREADS), smem, stream, p);
 }
 
 template <int PRO, int EPI, int MAP>
@@ -328,14 +364,14 @@ int gemv_launch(GvParams p, int pro, int epi, int map, int total_rows,
     tiles += gemv_tiles_for(map, p.prob[i].N, p.D);
   }
   for (int i = p.nprob; i < 4; ++i) p.tile_start[i] = tiles;
-  // Split K so the grid fills the GPU; at most 512 rows per CTA.
+  // Split K so that about `target_ctas` CTAs (one resident wave) cover the
+  // launch, with at most 512 factor rows (64 KB) per CTA.
   int splits = target_ctas / (tiles > 0 ? tiles : 1);
   splits = splits < 1 ? 1 : splits;
   const int max_splits = ceil_div(p.K, 32);
   splits = splits > max_splits ? max_splits : splits;
-  const int min_splits = ceil_div(p.K, 512);
-  splits = splits < min_splits ? min_splits : splits;
   p.KC = round_up(ceil_div(p.K, splits), 32);
+  p.KC = p.KC > 512 ? 512 : p.KC;
   p.splits = ceil_div(p.K, p.KC);
 
   for (int m0 = 0; m0 < total_rows; m0 += 8) {

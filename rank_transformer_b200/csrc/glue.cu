@@ -177,38 +177,38 @@ int rmsnorm_launch(const bf16* x, const bf16* g, bf16* y, int M, int d,
                    float eps, cudaStream_t s) {
   if (d > NT * ROW_VEC * 8) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return FLASHSVD_OK;
-  return launch_pdl(rmsnorm_kernel, dim3(M), dim3(NT), 0, s, x, g, y, d, eps);
+  return launch_pdl(LaunchTag{"rmsnorm", 4.0 * M * d, 0.0}, rmsnorm_kernel, dim3(M), dim3(NT), 0, s, x, g, y, d, eps);
 }
 
 int layernorm_launch(const bf16* x, const bf16* g, const bf16* b, bf16* y,
                      int M, int d, float eps, cudaStream_t s) {
   if (d > NT * ROW_VEC * 8) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return FLASHSVD_OK;
-  return launch_pdl(layernorm_kernel, dim3(M), dim3(NT), 0, s, x, g, b, y, d, eps);
+  return launch_pdl(LaunchTag{"layernorm", 4.0 * M * d, 0.0}, layernorm_kernel, dim3(M), dim3(NT), 0, s, x, g, b, y, d, eps);
 }
 
 int rope_table_launch(float* c, float* sn, int S_max, int D, float base,
                       cudaStream_t s) {
   const long long n = (long long)S_max * (D / 2);
   if (n == 0) return FLASHSVD_OK;
-  return launch_pdl(rope_table_kernel, dim3((unsigned)((n + NT - 1) / NT)), dim3(NT), 0, s,
+  return launch_pdl(LaunchTag{"rope_table", 8.0 * n, 0.0}, rope_table_kernel, dim3((unsigned)((n + NT - 1) / NT)), dim3(NT), 0, s,
                     c, sn, S_max, D, (double)base);
 }
 
 int embed_launch(const int* tokens, const bf16* emb, bf16* x, int B, int d,
                  int vocab, cudaStream_t s) {
   if (B == 0) return FLASHSVD_OK;
-  return launch_pdl(embed_kernel, dim3(B), dim3(NT), 0, s, tokens, emb, x, d, vocab);
+  return launch_pdl(LaunchTag{"embed", 4.0 * B * d, 0.0}, embed_kernel, dim3(B), dim3(NT), 0, s, tokens, emb, x, d, vocab);
 }
 
 int greedy_launch(const float* logits, int* next, int M, int vocab,
                   cudaStream_t s) {
   if (M == 0) return FLASHSVD_OK;
-  return launch_pdl(greedy_kernel, dim3(M), dim3(1024), 0, s, logits, next, vocab);
+  return launch_pdl(LaunchTag{"greedy", 4.0 * M * vocab, 0.0}, greedy_kernel, dim3(M), dim3(1024), 0, s, logits, next, vocab);
 }
 
 int advance_launch(int* seqlens, int B, cudaStream_t s) {
-  return launch_pdl(advance_kernel, dim3(1), dim3(32), 0, s, seqlens, B);
+  return launch_pdl(LaunchTag{"advance", 8.0 * B, 0.0}, advance_kernel, dim3(1), dim3(32), 0, s, seqlens, B);
 }
 
 }  // namespace fsvd

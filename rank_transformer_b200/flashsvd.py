@@ -68,6 +68,8 @@ _SIGS = {
     "flashsvd_shutdown": ([], _i),
     "flashsvd_check_device_status": ([_p], _i),
     "flashsvd_launch_count": ([], C.c_int64),
+    "flashsvd_profile_enable": ([_i], _i),
+    "flashsvd_profile_report": ([C.c_char_p, _i, _i], _i),
     "flashsvd_lowrank_linear": ([_p, _p, _p, _p, _p, _i, _i, _i, _i, _p], _i),
     "flashsvd_dense_linear_f32": ([_p, _p, _p, _i, _i, _i, _p], _i),
     "flashsvd_packed_gateup_mlp": ([_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p], _i),
@@ -137,6 +139,23 @@ def check_device_status(stream=None) -> None:
 
 def launch_count() -> int:
     return int(lib.flashsvd_launch_count())
+
+
+def profile_enable(on: bool = True) -> None:
+    _call("flashsvd_profile_enable", int(on))
+
+
+def profile_report(reset: bool = True) -> dict:
+    """{name: dict(launches, ms, bytes, flops)} of eager launches since the
+    last reset (synchronises the device)."""
+    n = lib.flashsvd_profile_report(None, 0, 0)
+    buf = C.create_string_buffer(max(n, 1) + 64)
+    _call("flashsvd_profile_report", buf, len(buf), int(reset))
+    out = {}
+    for line in buf.value.decode().splitlines():
+        name, cnt, ms, by, fl = line.split()
+        out[name] = dict(launches=int(cnt), ms=float(ms), bytes=float(by), flops=float(fl))
+    return out
 
 
 # -------------------------------------------------------------- compute --
