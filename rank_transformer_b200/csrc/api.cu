@@ -31,6 +31,7 @@ struct Ctx {
   bf16* q = nullptr;           // [rows x max_hidden]
   bf16* att = nullptr;         // [rows x max_hidden]
   bf16* h = nullptr;           // [rows x max_ffn]
+  bf16* zb = nullptr;          // [rows x 2*max_rank] prefill rank activations
   int rows = 0;                // rows of the scratch above
 };
 
@@ -39,7 +40,7 @@ std::mutex g_mu;
 
 void free_ctx(Ctx& c) {
   void* ptrs[] = {c.z, c.part, c.counters, c.apart, c.acounters, c.status,
-                  c.xn, c.q, c.att, c.h};
+                  c.xn, c.q, c.att, c.h, c.zb};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   c = Ctx();
@@ -203,6 +204,7 @@ PfLinear pf_base(const bf16* x, long long ldx, const flashsvd_factor& F, int M,
   p.x = x; p.ldx = ldx; p.U = cb(F.U); p.V = cb(F.V); p.bias = cb(F.bias);
   p.y = y; p.ldy = ldy; p.M = M; p.d = d; p.r = F.r; p.n = n;
   p.epi = PF_EPI_BF16;
+  p.z = g_ctx.zb;
   p.status = g_ctx.status;
   return p;
 }
@@ -439,6 +441,7 @@ int flashsvd_init(int device, int max_tokens, int max_rank, int max_hidden,
   FSVD_ALLOC(c.q, (size_t)c.rows * max_hidden * sizeof(bf16));
   FSVD_ALLOC(c.att, (size_t)c.rows * max_hidden * sizeof(bf16));
   FSVD_ALLOC(c.h, (size_t)c.rows * max_ffn * sizeof(bf16));
+  FSVD_ALLOC(c.zb, (size_t)c.rows * 2 * max_rank * sizeof(bf16));
 #undef FSVD_ALLOC
   if (e == cudaSuccess) e = cudaMemset(c.counters, 0, kCountersN * sizeof(int));
   if (e == cudaSuccess) e = cudaMemset(c.acounters, 0, kCountersN * sizeof(int));

@@ -93,6 +93,7 @@ struct PfLinear {
   // QKV epilogue: y is the q buffer for kind 0; k/v rows go to the caches.
   int kind; bf16* cache; int S, S_max, HD, D;
   const float* rope_cos; const float* rope_sin;
+  bf16* z;                           // [M x r] bf16 scratch for the rank activations
   int* status;
 };
 int prefill_linear_launch(const PfLinear& p, cudaStream_t stream);

@@ -1,8 +1,447 @@
-// Prefill-regime factorized linear (tcgen05).  Placeholder until the
-// tensor-core kernel lands.
+// Prefill-regime (M > 32) factorized linear on the 5th-generation tensor
+// cores.
+//
+// FlashSVD v1.5 (gist.science explainer), Technical Summary, Problem
+// Statement: prefill is arithmetic-bound and benefits from the reduced FLOPs
+// of y = (x U) V, so both stages are dense tensor-core contractions.
+//
+// tc_gemm_kernel: persistent, warp-specialised C = A . B, A [M x K] bf16
+// K-major, B [K x N] bf16 MN-major (row-major factors as stored), fp32
+// accumulation in tensor memory.
+//   warp 0      one thread issues TMA loads of A [128 x 64] and B [64 x BN]
+//               tiles (128-byte swizzle) into a STAGES-deep ring;
+//   warp 1      allocates tensor memory; one thread issues tcgen05.mma
+//               (M=128, N=BN, K=16) into one of two accumulator buffers and
+//               frees ring slots / publishes finished tiles with
+//               tcgen05.commit;
+//   warps 2..5  read the accumulator with tcgen05.ld (one TMEM lane
+//               quadrant each), apply the fused epilogue and store.
+// Every wait is bounded: on expiry the CTA raises the device status word
+// and winds down (waits for its own copies, frees tensor memory).
+#include <cstring>
+
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace fsvd {
-int prefill_linear_launch(const PfLinear&, cudaStream_t) { return FLASHSVD_ERR_UNSUPPORTED_SHAPE; }
-int prefill_dense_launch(const PfLinear&, cudaStream_t) { return FLASHSVD_ERR_UNSUPPORTED_SHAPE; }
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int TC_THREADS = 192;
+
+struct TcArgs {
+  int M, N, K;          // per half for the dual (SwiGLU) form
+  int tiles_m, tiles_n;
+  int a2, b2;           // dual: A column / B row offset of the second half
+  const bf16* bias;
+  const bf16* resid; long long ldr;
+  bf16* y; long long ldy;
+  float* y32;
+  int kind; bf16* cache; int S, S_max, HD, D;
+  const float* rope_cos; const float* rope_sin;
+  int* status;
+};
+
+__device__ __forceinline__ void store8(bf16* p, const float* v) {
+  uint4 u;
+  u.x = pack_bf2(v[0], v[1]); u.y = pack_bf2(v[2], v[3]);
+  u.z = pack_bf2(v[4], v[5]); u.w = pack_bf2(v[6], v[7]);
+  *reinterpret_cast<uint4*>(p) = u;
+}
+__device__ __forceinline__ void load8(const bf16* p, float* v) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  v[0] = bf_lo(u.x); v[1] = bf_hi(u.x); v[2] = bf_lo(u.y); v[3] = bf_hi(u.y);
+  v[4] = bf_lo(u.z); v[5] = bf_hi(u.z); v[6] = bf_lo(u.w); v[7] = bf_hi(u.w);
+}
+
+template <int BN, int STAGES, bool DUAL>
+struct Layout {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BK * BN * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  static constexpr int SMEM = 1024 + BAR_OFF + 256;  // + alignment slack
+  static constexpr int ACC_COLS = DUAL ? 2 * BN : BN;
+  static constexpr int TMEM_COLS = 2 * ACC_COLS;
+  static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "tensor memory allocation must be a power of 2");
+};
+
+template <int BN, int STAGES, bool DUAL, int EPI>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const __grid_constant__ TcArgs a) {
+  using L = Layout<BN, STAGES, DUAL>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles = a.tiles_m * a.tiles_n;
+  const int nkb = (a.K + BK - 1) / BK;
+  const int kb_total = DUAL ? 2 * nkb : nkb;
+  constexpr uint32_t IDESC = tc::idesc_bf16(BN, true);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      tc::mbar_init(full + s, 1);
+      tc::mbar_init(empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(tfull + b, 1);
+      tc::mbar_init(tempty + b, 4);
+    }
+    tc::mbar_init(drain, 1);
+    *abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tc::tma_prefetch_desc(&tmA);
+    tc::tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_holder, L::TMEM_COLS);
+    tc::tmem_relinquish();
+    tc::fence_before_sync();
+  }
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem_base = *tmem_holder;
+
+  pdl_launch_dependents();
+  pdl_wait();
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer --
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+        const int m0 = (t % a.tiles_m) * BM, n0 = (t / a.tiles_m) * BN;
+        for (int kb = 0; kb < kb_total; ++kb) {
+          if (!tc::mbar_wait(empty + stage, phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
+          tc::mbar_expect_tx(full + stage, L::STAGE_BYTES);
+          const bool second = DUAL && kb >= nkb;
+          const int kk = second ? kb - nkb : kb;
+          const int ka = (second ? a.a2 : 0) + kk * BK;
+          const int kr = (second ? a.b2 : 0) + kk * BK;
+          uint8_t* sA = smem + stage * L::STAGE_BYTES;
+          uint8_t* sB = sA + L::A_BYTES;
+          tc::tma_load_2d(sA, &tmA, full + stage, ka, m0);
+#pragma unroll
+          for (int j = 0; j < BN / 64; ++j) tc::tma_load_2d(sB + j * 8192, &tmB, full + stage, n0 + 64 * j, kr);
+          ++issued;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        // Winding down: let this CTA's copies that are still in flight land
+        // before shared memory is released (bounded, ignores the flag).
+        const int outstanding = issued < STAGES ? issued : STAGES;
+        for (int i = 1; i <= outstanding; ++i) {
+          int s = stage - i;
+          uint32_t ph = phase;
+          if (s < 0) { s += STAGES; ph ^= 1u; }
+          const long long t0 = clock64();
+          while (!tc::mbar_try_wait(full + s, ph) && clock64() - t0 < tc::kWaitCycles) {}
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++it) {
+        const int buf = it & 1;
+        const uint32_t tph = (uint32_t)(it >> 1) & 1u;
+        if (!tc::mbar_wait(tempty + buf, tph ^ 1u, abort_flag, a.status)) { ok = false; break; }
+        tc::fence_after_sync();
+        const uint32_t d0 = tmem_base + (uint32_t)(buf * L::ACC_COLS);
+        for (int kb = 0; kb < kb_total; ++kb) {
+          if (!tc::mbar_wait(full + stage, phase, abort_flag, a.status)) { ok = false; break; }
+          tc::fence_after_sync();
+          const bool second = DUAL && kb >= nkb;
+          const uint32_t d = second ? d0 + BN : d0;
+          const bool first = (kb == 0) || (DUAL && kb == nkb);
+          const uint32_t sa = tc::smem_u32(smem + stage * L::STAGE_BYTES);
+          const uint32_t sb = sa + L::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = tc::sdesc_sw128(sa + k * 32, 16, 1024);
+            const uint64_t bd = tc::sdesc_sw128(sb + k * 2048, 8192, 1024);
+            tc::mma_bf16(d, ad, bd, IDESC, (first && k == 0) ? 0u : 1u);
+          }
+          tc::mma_commit(empty + stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (ok) tc::mma_commit(tfull + buf);
+      }
+      // Every MMA this thread issued has completed once `drain` fires.
+      tc::mma_commit(drain);
+      const long long t0 = clock64();
+      while (!tc::mbar_try_wait(drain, 0) && clock64() - t0 < tc::kWaitCycles) {}
+    }
+  } else {
+    // --------------------------------------------------------- epilogue --
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    int it = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
+      const int buf = it & 1;
+      const uint32_t tph = (uint32_t)(it >> 1) & 1u;
+      if (!tc::mbar_wait(tfull + buf, tph, abort_flag, a.status)) break;
+      tc::fence_after_sync();
+      const int m0 = (t % a.tiles_m) * BM, n0 = (t / a.tiles_m) * BN;
+      const int m = m0 + row;
+      const bool mok = m < a.M;
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * L::ACC_COLS);
+
+      if (EPI == PF_EPI_QKV) {
+        // RoPE pairs columns i and i + D/2 of a head: process a first-half
+        // chunk of 32 columns together with its partner chunk.
+        const int half = a.D >> 1;
+        const int hc = half >> 5;  // chunks per half head
+        const int bq = mok ? m / a.S : 0, tq = mok ? m - bq * a.S : 0;
+        for (int c = 0; c < BN / 32; ++c) {
+          if ((c % (2 * hc)) >= hc) continue;  // second-half chunks ride along
+          uint32_t r0[32], r1[32];
+          tc::tmem_ld32(tb + c * 32, r0);
+          tc::tmem_ld32(tb + (c + hc) * 32, r1);
+          tc::tmem_ld_wait();
+          const int n = n0 + c * 32;
+          if (!mok || n >= a.N) continue;
+          float lo[32], hi[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) { lo[j] = __uint_as_float(r0[j]); hi[j] = __uint_as_float(r1[j]); }
+          if (a.bias) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              float b0[8], b1[8];
+              load8(a.bias + n + 8 * g, b0);
+              load8(a.bias + n + half + 8 * g, b1);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) { lo[8 * g + j] += b0[j]; hi[8 * g + j] += b1[j]; }
+            }
+          }
+          if (a.rope_cos) {
+            const int i0 = n % a.D;
+            const float* cs = a.rope_cos + (long long)tq * half + i0;
+            const float* sn = a.rope_sin + (long long)tq * half + i0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float cj = cs[j], sj = sn[j];
+              const float l2 = lo[j] * cj - hi[j] * sj;
+              hi[j] = hi[j] * cj + lo[j] * sj;
+              lo[j] = l2;
+            }
+          }
+          bf16* dst = a.kind == 0 ? a.y + (long long)m * a.ldy
+                                  : a.cache + ((long long)bq * a.S_max + tq) * a.HD;
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            store8(dst + n + 8 * g, lo + 8 * g);
+            store8(dst + n + half + 8 * g, hi + 8 * g);
+          }
+        }
+      } else {
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r0[32];
+          uint32_t r1[DUAL ? 32 : 1];
+          tc::tmem_ld32(tb + c * 32, r0);
+          if (DUAL) tc::tmem_ld32(tb + BN + c * 32, r1);
+          tc::tmem_ld_wait();
+          const int n = n0 + c * 32;
+          if (!mok) continue;
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int ng = n + 8 * g;
+            if (ng >= a.N) break;
+            float v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = __uint_as_float(r0[8 * g + j]);
+            if (EPI == PF_EPI_F32) {
+              float4* dst = reinterpret_cast<float4*>(a.y32 + (long long)m * a.ldy + ng);
+              dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+              dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+              continue;
+            }
+            if (DUAL) {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const float u = __uint_as_float(r1[8 * g + j]);
+                v[j] = v[j] / (1.f + expf(-v[j])) * u;
+              }
+            } else {
+              if (a.bias) {
+                float b[8];
+                load8(a.bias + ng, b);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] += b[j];
+              }
+              if (EPI == PF_EPI_GELU) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = 0.5f * v[j] * (1.f + erff(v[j] * 0.70710678118654752f));
+              }
+              if (a.resid) {
+                float rr[8];
+                load8(a.resid + (long long)m * a.ldr + ng, rr);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] += rr[j];
+              }
+            }
+            store8(a.y + (long long)m * a.ldy + ng, v);
+          }
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(tempty + buf);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem_base, L::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------- host ----
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// bf16 matrix [rows x cols], row stride ld elements; box = 64 columns x box_rows rows.
+int make_map(CUtensorMap* map, const void* base, long long rows, long long cols, long long ld,
+             int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return FLASHSVD_ERR_CUDA;
+  if (!aligned16(base) || (ld * 2) % 16 != 0) return FLASHSVD_ERR_MISALIGNED;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1u, 1u};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                        box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FLASHSVD_OK : FLASHSVD_ERR_INVALID_ARG;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+double gemm_bytes(const TcArgs& a, bool dual) {
+  const double halves = dual ? 2.0 : 1.0;
+  return 2.0 * ((double)a.M * a.K * halves + (double)a.K * a.N * halves + (double)a.M * a.N);
+}
+
+template <int BN, int STAGES, bool DUAL, int EPI>
+int launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, TcArgs a, const char* name,
+              cudaStream_t stream) {
+  using L = Layout<BN, STAGES, DUAL>;
+  auto kern = tc_gemm_kernel<BN, STAGES, DUAL, EPI>;
+  static bool configured = false;
+  if (!configured) {
+    FSVD_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM));
+    configured = true;
+  }
+  a.tiles_m = ceil_div(a.M, BM);
+  a.tiles_n = ceil_div(a.N, BN);
+  const int tiles = a.tiles_m * a.tiles_n;
+  const int grid = tiles < sm_count() ? tiles : sm_count();
+  const double flops = 2.0 * a.M * (double)a.N * a.K * (DUAL ? 2.0 : 1.0);
+  const LaunchTag tag{name, gemm_bytes(a, DUAL), flops};
+  return launch_pdl(tag, kern, dim3(grid), dim3(TC_THREADS), (size_t)L::SMEM, stream, ma, mb, a);
+}
+
+// One tensor-core GEMM C = A . B with the given epilogue.
+int gemm(const bf16* A, long long lda, long long a_cols, const bf16* B, long long ldb, long long b_rows,
+         TcArgs a, int epi, bool dual, const char* name, cudaStream_t stream) {
+  CUtensorMap ma, mb;
+  FSVD_TRY(make_map(&ma, A, a.M, a_cols, lda, BM));
+  if (dual) {
+    FSVD_TRY(make_map(&mb, B, b_rows, a.N, ldb, BK));
+    return launch_tc<128, 6, true, PF_EPI_SWIGLU>(ma, mb, a, name, stream);
+  }
+  FSVD_TRY(make_map(&mb, B, b_rows, a.N, ldb, BK));
+  switch (epi) {
+    case PF_EPI_BF16: return launch_tc<256, 4, false, PF_EPI_BF16>(ma, mb, a, name, stream);
+    case PF_EPI_GELU: return launch_tc<256, 4, false, PF_EPI_GELU>(ma, mb, a, name, stream);
+    case PF_EPI_QKV: return launch_tc<256, 4, false, PF_EPI_QKV>(ma, mb, a, name, stream);
+    case PF_EPI_F32: return launch_tc<256, 4, false, PF_EPI_F32>(ma, mb, a, name, stream);
+    default: return FLASHSVD_ERR_INVALID_ARG;
+  }
+}
+
+}  // namespace
+
+int prefill_linear_launch(const PfLinear& p, cudaStream_t stream) {
+  if (!p.z) return FLASHSVD_ERR_NOT_INITIALIZED;
+  const bool dual = p.epi == PF_EPI_SWIGLU;
+  if (dual && (p.r % 128) != 0) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;  // r = 2 r_f, r_f % 64 == 0
+  if (p.epi == PF_EPI_QKV && (p.D % 64 != 0 || 256 % p.D != 0)) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  // Stage 1: z = x . U  [M x r], rounded to bf16.
+  TcArgs a1;
+  memset(&a1, 0, sizeof(a1));
+  a1.M = p.M; a1.N = p.r; a1.K = p.d;
+  a1.y = p.z; a1.ldy = p.r;
+  a1.status = p.status;
+  FSVD_TRY(gemm(p.x, p.ldx, p.d, p.U, p.r, p.d, a1, PF_EPI_BF16, false, "tc_stage1_xu", stream));
+  // Stage 2: y = epilogue(z . V).
+  TcArgs a2;
+  memset(&a2, 0, sizeof(a2));
+  a2.M = p.M; a2.N = p.n; a2.K = dual ? p.r / 2 : p.r;
+  a2.a2 = p.r / 2; a2.b2 = p.r / 2;
+  a2.bias = p.bias; a2.resid = p.resid; a2.ldr = p.ldr;
+  a2.y = p.y; a2.ldy = p.ldy; a2.y32 = p.y32;
+  a2.kind = p.kind; a2.cache = p.cache; a2.S = p.S; a2.S_max = p.S_max; a2.HD = p.HD; a2.D = p.D;
+  a2.rope_cos = p.rope_cos; a2.rope_sin = p.rope_sin;
+  a2.status = p.status;
+  return gemm(p.z, p.r, p.r, p.V, p.n, p.r, a2, p.epi, dual, dual ? "tc_stage2_swiglu" : "tc_stage2_zv",
+              stream);
+}
+
+int prefill_dense_launch(const PfLinear& p, cudaStream_t stream) {
+  TcArgs a;
+  memset(&a, 0, sizeof(a));
+  a.M = p.M; a.N = p.n; a.K = p.d;
+  a.y32 = p.y32; a.ldy = p.ldy;
+  a.status = p.status;
+  return gemm(p.x, p.ldx, p.d, p.V, p.n, p.d, a, PF_EPI_F32, false, "tc_dense_f32", stream);
+}
+
 }  // namespace fsvd
