@@ -41,6 +41,9 @@ def parse():
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-step", action="store_true",
+                    help="after warm-up, run one prefill and two decode steps inside an NVTX "
+                         "range 'profile_step' (for an ncu launch list) and exit")
     return ap.parse_args()
 
 
@@ -231,6 +234,20 @@ def run_ours(args):
             one_step()
     stream.synchronize()
 
+    if args.profile_step:
+        torch.cuda.synchronize()
+        torch.cuda.nvtx.range_push("profile_step")
+        with torch.cuda.stream(stream):
+            model.prefill(prompt, stream)
+            model.decode_step(stream)
+            model.decode_step(stream)
+        stream.synchronize()
+        torch.cuda.nvtx.range_pop()
+        per_step = model.step_kernels()
+        model.release_graphs()
+        print(json.dumps({"profile_step": "done", "launches_per_decode_step": per_step}))
+        return 0
+
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
@@ -240,10 +257,12 @@ def run_ours(args):
     launches0 = fs.launch_count()
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     t_wall = time.perf_counter()
+    torch.cuda.nvtx.range_push("timed_steps")
     with torch.cuda.stream(stream):
         for k in range(args.steps):
             one_step(events[k])
     stream.synchronize()
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     t_wall = time.perf_counter() - t_wall
     if world > 1:

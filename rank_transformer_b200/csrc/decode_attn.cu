@@ -142,6 +142,8 @@ attn_decode_kernel(const __grid_constant__ AttnDecParams p) {
       if (tid == 0) { __stcg(mypart, M); __stcg(mypart + 1, Lc); }
     }
   } else {
+    // Empty slice (beyond the current length): a neutral partial.
+    for (int dd = tid; dd < D; dd += AD_THREADS) __stcg(mypart + 2 + dd, 0.f);
     if (tid == 0) { __stcg(mypart, -INFINITY); __stcg(mypart + 1, 0.f); }
   }
   if (p.nsplit == 1) return;
@@ -152,22 +154,51 @@ attn_decode_kernel(const __grid_constant__ AttnDecParams p) {
   if (!s_last) return;
   __threadfence();
 
+  // Merge the split partials: per-split weights exp2(M_s - M) computed once
+  // into shared memory, then every thread sums its dimension over splits
+  // with independent loads (fixed split order: deterministic).
   const float* base = p.part + (long long)bh * p.nsplit * (D + 2);
+  float* wts = ps;  // AD_CHUNK floats, reused (nsplit <= 1024 handled in passes)
   float Mg = -INFINITY;
-  for (int sp = 0; sp < p.nsplit; ++sp) Mg = fmaxf(Mg, __ldcg(base + sp * (D + 2)));
-  float Lg = 0.f;
-  for (int sp = 0; sp < p.nsplit; ++sp) {
-    const float ms = __ldcg(base + sp * (D + 2));
-    if (ms != -INFINITY) Lg += __ldcg(base + sp * (D + 2) + 1) * exp2f(ms - Mg);
-  }
-  for (int dd = tid; dd < D; dd += AD_THREADS) {
-    float o = 0.f;
-    for (int sp = 0; sp < p.nsplit; ++sp) {
-      const float ms = __ldcg(base + sp * (D + 2));
-      if (ms != -INFINITY) o += __ldcg(base + sp * (D + 2) + 2 + dd) * exp2f(ms - Mg);
+  for (int sp = tid; sp < p.nsplit; sp += AD_THREADS) Mg = fmaxf(Mg, __ldcg(base + (long long)sp * (D + 2)));
+  Mg = warp_max(Mg);
+  if (lane == 0) s_red[warp] = Mg;
+  __syncthreads();
+  Mg = s_red[0];
+#pragma unroll
+  for (int w = 1; w < AD_WARPS; ++w) Mg = fmaxf(Mg, s_red[w]);
+  __syncthreads();
+  float Lg = 0.f, acc = 0.f;
+  for (int s0 = 0; s0 < p.nsplit; s0 += AD_CHUNK) {
+    const int ns = min(AD_CHUNK, p.nsplit - s0);
+    if (tid < ns) {
+      const float ms = __ldcg(base + (long long)(s0 + tid) * (D + 2));
+      const float w = (ms == -INFINITY) ? 0.f : exp2f(ms - Mg);
+      wts[tid] = w;
+      Lg += w * __ldcg(base + (long long)(s0 + tid) * (D + 2) + 1);
     }
-    p.out[((long long)b * p.H + h) * D + dd] = f2bf(o / Lg);
+    __syncthreads();
+    if (tid < D) {
+      const float* ob = base + (long long)s0 * (D + 2) + 2 + tid;
+      int sp = 0;
+      for (; sp + 4 <= ns; sp += 4) {
+        const float o0 = __ldcg(ob + (long long)sp * (D + 2));
+        const float o1 = __ldcg(ob + (long long)(sp + 1) * (D + 2));
+        const float o2 = __ldcg(ob + (long long)(sp + 2) * (D + 2));
+        const float o3 = __ldcg(ob + (long long)(sp + 3) * (D + 2));
+        acc += (o0 * wts[sp] + o1 * wts[sp + 1]) + (o2 * wts[sp + 2] + o3 * wts[sp + 3]);
+      }
+      for (; sp < ns; ++sp) acc += __ldcg(ob + (long long)sp * (D + 2)) * wts[sp];
+    }
+    __syncthreads();
   }
+  Lg = warp_sum(Lg);
+  if (lane == 0) s_red[warp] = Lg;
+  __syncthreads();
+  Lg = 0.f;
+#pragma unroll
+  for (int w = 0; w < AD_WARPS; ++w) Lg += s_red[w];
+  if (tid < D) p.out[((long long)b * p.H + h) * D + tid] = f2bf(acc / Lg);
   if (tid == 0) p.counters[bh] = 0;
 }
 

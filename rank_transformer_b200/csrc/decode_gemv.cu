@@ -225,13 +225,28 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
     __syncthreads();
     if (!s_last) return;
     __threadfence();
+    // Sum the split partials: LPO threads per output, each a fixed stride
+    // of splits, combined by a fixed shuffle tree (deterministic order).
     const float* tp = p.part + (long long)tile * p.splits * NOUT;
+    constexpr int LPO = NOUT >= GV_THREADS ? 1 : GV_THREADS / NOUT;
 #pragma unroll
     for (int q = 0; q < PER; ++q) {
-      const int o = tid + q * GV_THREADS;
+      const int o = (LPO == 1) ? tid + q * GV_THREADS : tid / LPO;
+      const int sub = (LPO == 1) ? 0 : tid % LPO;
       float s = 0.f;
-      if (o < NOUT)
-        for (int sp = 0; sp < p.splits; ++sp) s += __ldcg(tp + (long long)sp * NOUT + o);
+      if (o < NOUT) {
+        int sp = sub;
+        for (; sp + 3 * LPO < p.splits; sp += 4 * LPO) {
+          const float v0 = __ldcg(tp + (long long)sp * NOUT + o);
+          const float v1 = __ldcg(tp + (long long)(sp + LPO) * NOUT + o);
+          const float v2 = __ldcg(tp + (long long)(sp + 2 * LPO) * NOUT + o);
+          const float v3 = __ldcg(tp + (long long)(sp + 3 * LPO) * NOUT + o);
+          s += ((v0 + v1) + (v2 + v3));
+        }
+        for (; sp < p.splits; sp += LPO) s += __ldcg(tp + (long long)sp * NOUT + o);
+      }
+#pragma unroll
+      for (int w = 1; w < LPO; w <<= 1) s += __shfl_xor_sync(0xffffffffu, s, w);
       val[q] = s;
     }
     if (tid == 0) p.counters[tile] = 0;  // ready for the next launch
@@ -240,10 +255,15 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
   // ---- epilogue on the finished [MT x 64] tile ----
   __syncthreads();  // red is reused as the finished tile
   float* fin = red;
+  {
+    constexpr int LPO = NOUT >= GV_THREADS ? 1 : GV_THREADS / NOUT;
+    const bool reduced_layout = p.splits > 1 && LPO > 1;
 #pragma unroll
-  for (int q = 0; q < PER; ++q) {
-    const int o = tid + q * GV_THREADS;
-    if (o < NOUT) fin[o] = val[q];
+    for (int q = 0; q < PER; ++q) {
+      const int o = reduced_layout ? tid / LPO : tid + q * GV_THREADS;
+      const bool writer = reduced_layout ? (tid % LPO) == 0 : true;
+      if (o < NOUT && writer) fin[o] = val[q];
+    }
   }
   __syncthreads();
 

@@ -236,15 +236,21 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             }
           }
           if (a.rope_cos) {
+            // 32 consecutive angles of this row's position: 16-byte loads.
             const int i0 = n % a.D;
-            const float* cs = a.rope_cos + (long long)tq * half + i0;
-            const float* sn = a.rope_sin + (long long)tq * half + i0;
+            const float4* cs = reinterpret_cast<const float4*>(a.rope_cos + (long long)tq * half + i0);
+            const float4* sn = reinterpret_cast<const float4*>(a.rope_sin + (long long)tq * half + i0);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float cj = cs[j], sj = sn[j];
-              const float l2 = lo[j] * cj - hi[j] * sj;
-              hi[j] = hi[j] * cj + lo[j] * sj;
-              lo[j] = l2;
+            for (int j4 = 0; j4 < 8; ++j4) {
+              const float4 c4 = __ldg(cs + j4), s4 = __ldg(sn + j4);
+              const float cj[4] = {c4.x, c4.y, c4.z, c4.w}, sj[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int j = 4 * j4 + e;
+                const float l2 = lo[j] * cj[e] - hi[j] * sj[e];
+                hi[j] = hi[j] * cj[e] + lo[j] * sj[e];
+                lo[j] = l2;
+              }
             }
           }
           bf16* dst = a.kind == 0 ? a.y + (long long)m * a.ldy
