@@ -212,6 +212,35 @@ FLASHSVD_API int flashsvd_greedy(const float* logits, int32_t* next_tokens, int 
 FLASHSVD_API int flashsvd_advance_seqlens(int32_t* cache_seqlens, int B,
                              flashsvd_stream stream);
 
+/* ------------------------------------------------ no-allocation variant --
+ * No counterpart in the pages.  Same result as flashsvd_lowrank_linear,
+ * y[M x n] = (x[M x d] . U[d x r]) . V[r x n] + bias[n] (bias may be NULL),
+ * with the decode kernels, for callers that cannot allocate device memory:
+ * flashsvd_init obtains its workspace with cudaMalloc, which a plugin inside
+ * a framework whose allocator owns all device memory, or a serving process
+ * that must not allocate after start-up, cannot do.  This call needs no
+ * flashsvd_init and calls no cudaMalloc, cudaFree or allocating routine; its
+ * scratch (rank activations, split partial sums, tile counters) is one fixed
+ * array of about 2.2 MiB in device memory that every GPU which loads the
+ * library holds until the process exits.
+ * Limits: 1 <= M <= 8, r <= 4096, d and n <= 16384 (all multiples of 8) and
+ * the split partial sums must fit the array; anything larger returns
+ * FLASHSVD_ERR_UNSUPPORTED_SHAPE and launches nothing.
+ * The first call on each device looks up the array's device address with
+ * that device current; make that first call before any stream capture.
+ * All calls share the one array and each overwrites it (the tile counters
+ * are cleared by a memset on `stream` at the start of every call), so calls
+ * that overlap on the GPU -- on different streams or from different host
+ * threads -- race: order them on one stream.
+ */
+FLASHSVD_API int flashsvd_lowrank_linear_noalloc(const flashsvd_bf16* x,
+                                                 const flashsvd_bf16* U,
+                                                 const flashsvd_bf16* V,
+                                                 const flashsvd_bf16* bias,
+                                                 flashsvd_bf16* y, int M, int d,
+                                                 int r, int n,
+                                                 flashsvd_stream stream);
+
 /* -------------------------------------------------------------- layers ---
  * One transformer layer as caller-owned factor pointers.
  * kind = FLASHSVD_DECODER: pre-norm RMSNorm, RoPE, causal attention,

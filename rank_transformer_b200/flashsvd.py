@@ -71,6 +71,7 @@ _SIGS = {
     "flashsvd_profile_enable": ([_i], _i),
     "flashsvd_profile_report": ([C.c_char_p, _i, _i], _i),
     "flashsvd_lowrank_linear": ([_p, _p, _p, _p, _p, _i, _i, _i, _i, _p], _i),
+    "flashsvd_lowrank_linear_noalloc": ([_p, _p, _p, _p, _p, _i, _i, _i, _i, _p], _i),
     "flashsvd_dense_linear_f32": ([_p, _p, _p, _i, _i, _i, _p], _i),
     "flashsvd_packed_gateup_mlp": ([_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p], _i),
     "flashsvd_gateup_swiglu": ([_p, _p, _p, _p, _i, _i, _i, _i, _p], _i),
@@ -162,6 +163,13 @@ def profile_report(reset: bool = True) -> dict:
 
 def lowrank_linear(x, U, V, bias, y, M, d, r, n, stream=None):
     _call("flashsvd_lowrank_linear", ptr(x), ptr(U), ptr(V), ptr(bias), ptr(y),
+          M, d, r, n, stream_handle(stream))
+
+
+def lowrank_linear_noalloc(x, U, V, bias, y, M, d, r, n, stream=None):
+    """Decode-size factorized linear that allocates nothing (fixed device
+    scratch; see include/flashsvd.h for its limits)."""
+    _call("flashsvd_lowrank_linear_noalloc", ptr(x), ptr(U), ptr(V), ptr(bias), ptr(y),
           M, d, r, n, stream_handle(stream))
 
 
