@@ -94,6 +94,13 @@ FLASHSVD_API int flashsvd_shutdown(void);
  * error). */
 FLASHSVD_API int flashsvd_check_device_status(flashsvd_stream stream);
 
+/* Decode implementation used by flashsvd_layer_forward(DECODE): fused != 0
+ * (default) runs the whole layer as one persistent kernel (one CTA per SM,
+ * factor tiles streamed through a TMA ring across all nine stages, stages
+ * separated by bounded grid barriers) when B <= 8; fused == 0 runs one
+ * launch per stage.  Both give the same result within rounding. */
+FLASHSVD_API int flashsvd_set_decode_path(int fused);
+
 /* Number of kernels this library has launched since load: eager launches
  * plus the kernel nodes of every replayed graph. */
 FLASHSVD_API int64_t flashsvd_launch_count(void);
@@ -281,7 +288,33 @@ typedef struct flashsvd_layer {
   flashsvd_factor down;         /* [f -> d] */
   const float* rope_cos;        /* decoder: [S_max x D/2] (flashsvd_rope_table) */
   const float* rope_sin;
+  const void* decode_pack;      /* decoder: flashsvd_decode_pack output, or NULL */
 } flashsvd_layer;
+
+/* ---------------------------------------------------------- decode pack ---
+ * Decode is bound by reading the factors (FlashSVD v1.5 Technical Summary,
+ * Problem Statement).  The fused decode-layer kernel reads a decoder layer's
+ * factors from a "decode pack": a copy of q/k/v/o U and V, U_gu, V_gu and
+ * down U/V re-tiled so that every 256-row x 64-output-column block the kernel
+ * consumes is one contiguous run of device memory, stored in the order the
+ * kernel consumes them.  It is a pure layout change: no value is altered.
+ * Whole contiguous blocks stream at close to the HBM copy rate; 64- or
+ * 128-byte row pieces spaced at the matrix pitch do not.
+ *
+ * flashsvd_decode_pack_bytes: size of L's pack (host only, no device work).
+ * flashsvd_decode_pack: writes L's pack into dst (device memory, 16-byte
+ *   aligned, at least the size above, owned by the caller), asynchronously
+ *   on `stream`.  Then set L->decode_pack = dst: DECODE-mode
+ *   flashsvd_layer_forward runs the fused single-kernel layer from it; with
+ *   decode_pack NULL it runs the per-stage kernels.  The pack must outlive
+ *   its use and be rebuilt whenever a factor changes.
+ * Errors: INVALID_ARG (null argument, dst too small, not a decoder layer),
+ *   MISALIGNED, UNSUPPORTED_SHAPE (ranks of q, k, v differ, down rank !=
+ *   r_f, D not 64 or 128, d not a multiple of 64, a rank or f not a multiple
+ *   of 8). */
+FLASHSVD_API int flashsvd_decode_pack_bytes(const flashsvd_layer* L, size_t* bytes);
+FLASHSVD_API int flashsvd_decode_pack(const flashsvd_layer* L, void* dst, size_t bytes,
+                                      flashsvd_stream stream);
 
 /* Run one layer in place on x_inout ([B*S x d] bf16, token-major).
  * PREFILL_CAUSAL: positions 0..S-1; rotated keys and values are written to

@@ -32,6 +32,8 @@ struct Ctx {
   bf16* att = nullptr;         // [rows x max_hidden]
   bf16* h = nullptr;           // [rows x max_ffn]
   bf16* zb = nullptr;          // [rows x 2*max_rank] prefill rank activations
+  float* df_part = nullptr;    // fused decode: per-CTA partial slots
+  int* df_cnt = nullptr;       // fused decode: tile counters, stage barriers, done counter
   int rows = 0;                // rows of the scratch above
 };
 
@@ -40,7 +42,7 @@ std::mutex g_mu;
 
 void free_ctx(Ctx& c) {
   void* ptrs[] = {c.z, c.part, c.counters, c.apart, c.acounters, c.status,
-                  c.xn, c.q, c.att, c.h, c.zb};
+                  c.xn, c.q, c.att, c.h, c.zb, c.df_part, c.df_cnt};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   c = Ctx();
@@ -209,11 +211,43 @@ PfLinear pf_base(const bf16* x, long long ldx, const flashsvd_factor& F, int M,
   return p;
 }
 
+bool g_fused_decode = true;
+
+// Whether the fused decode layer (and hence a decode pack) covers L's shapes.
+bool pack_shapes_ok(const flashsvd_layer* L) {
+  const int r = L->q.r;
+  return L->k.r == r && L->v.r == r && L->down.r == L->r_f && L->f % 8 == 0 &&
+         decode_fused_supported(1, L->d, L->D, r, L->r_f);
+}
+
+DecodeLayerDesc decode_desc(const flashsvd_layer* L) {
+  DecodeLayerDesc D;
+  memset(&D, 0, sizeof(D));
+  D.U[0] = cb(L->q.U); D.U[1] = cb(L->k.U); D.U[2] = cb(L->v.U);
+  D.V[0] = cb(L->q.V); D.V[1] = cb(L->k.V); D.V[2] = cb(L->v.V);
+  D.U_o = cb(L->o.U); D.V_o = cb(L->o.V);
+  D.U_gu = cb(L->U_gu); D.V_gu = cb(L->V_gu);
+  D.U_dn = cb(L->down.U); D.V_dn = cb(L->down.V);
+  D.g1 = cb(L->norm1_g); D.g2 = cb(L->norm2_g);
+  D.d = L->d; D.H = L->H; D.D = L->D; D.f = L->f; D.r = L->q.r; D.r_f = L->r_f;
+  D.eps = L->norm_eps; D.rope_cos = L->rope_cos; D.rope_sin = L->rope_sin;
+  D.pack = L->decode_pack;
+  return D;
+}
+
 // ------------------------------------------------------- layer: decode ----
 int layer_decode(const flashsvd_layer* L, bf16* x, bf16* kc, bf16* vc,
                  const int* seqlens, int B, int S_max, cudaStream_t s) {
   const int d = L->d, r = L->q.r;
   const bool same_r = L->k.r == r && L->v.r == r;
+  if (g_fused_decode && L->decode_pack && pack_shapes_ok(L) && g_ctx.sm_count <= 148 &&
+      decode_fused_supported(B, d, L->D, r, L->r_f)) {
+    const DecodeLayerDesc D = decode_desc(L);
+    const int st = decode_fused_launch(D, x, kc, vc, seqlens, B, S_max, g_ctx.q, g_ctx.att, g_ctx.h,
+                                       g_ctx.z, g_ctx.df_part, g_ctx.df_cnt, g_ctx.df_cnt + 4096,
+                                       g_ctx.df_cnt + 4096 + 32, g_ctx.status, g_ctx.sm_count, s);
+    if (st != FLASHSVD_ERR_UNSUPPORTED_SHAPE) return st;
+  }
   // 1) z_qkv = rmsnorm(x) . [U_q | U_k | U_v]
   if (!same_r) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   {
@@ -402,7 +436,37 @@ const char* flashsvd_status_string(int status) {
 
 int flashsvd_last_cuda_error(void) { return g_last_cuda_error; }
 int flashsvd_version(void) { return 100; }
+
+int flashsvd_set_decode_path(int fused) {
+  g_fused_decode = fused != 0;
+  return FLASHSVD_OK;
+}
 int64_t flashsvd_launch_count(void) { return g_launches.load(); }
+
+int flashsvd_decode_pack_bytes(const flashsvd_layer* L, size_t* bytes) {
+  if (!L || !bytes) return FLASHSVD_ERR_INVALID_ARG;
+  if (L->kind != FLASHSVD_DECODER) return FLASHSVD_ERR_INVALID_ARG;
+  if (!pack_shapes_ok(L)) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  *bytes = (size_t)decode_pack_bytes(decode_desc(L));
+  return FLASHSVD_OK;
+}
+
+int flashsvd_decode_pack(const flashsvd_layer* L, void* dst, size_t bytes, flashsvd_stream stream) {
+  size_t need = 0;
+  FSVD_TRY(flashsvd_decode_pack_bytes(L, &need));
+  if (!dst || bytes < need) return FLASHSVD_ERR_INVALID_ARG;
+  if (!aligned16(dst)) return FLASHSVD_ERR_MISALIGNED;
+  const flashsvd_bf16* ptrs[] = {L->q.U, L->k.U, L->v.U, L->q.V, L->k.V, L->v.V, L->o.U, L->o.V,
+                                 L->U_gu, L->V_gu, L->down.U, L->down.V};
+  for (const flashsvd_bf16* q : ptrs) {
+    if (!q) return FLASHSVD_ERR_INVALID_ARG;
+    if (!aligned16(q)) return FLASHSVD_ERR_MISALIGNED;
+  }
+  int sms = 148, dev = 0;
+  FSVD_CUDA(cudaGetDevice(&dev));
+  FSVD_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  return decode_pack_launch(decode_desc(L), dst, (long long)bytes, sms, (cudaStream_t)stream);
+}
 
 int flashsvd_init(int device, int max_tokens, int max_rank, int max_hidden,
                   int max_ffn) {
@@ -442,10 +506,13 @@ int flashsvd_init(int device, int max_tokens, int max_rank, int max_hidden,
   FSVD_ALLOC(c.att, (size_t)c.rows * max_hidden * sizeof(bf16));
   FSVD_ALLOC(c.h, (size_t)c.rows * max_ffn * sizeof(bf16));
   FSVD_ALLOC(c.zb, (size_t)c.rows * 2 * max_rank * sizeof(bf16));
+  FSVD_ALLOC(c.df_part, (size_t)kFusedPartFloats * sizeof(float));
+  FSVD_ALLOC(c.df_cnt, (size_t)(4096 + 64) * sizeof(int));
 #undef FSVD_ALLOC
   if (e == cudaSuccess) e = cudaMemset(c.counters, 0, kCountersN * sizeof(int));
   if (e == cudaSuccess) e = cudaMemset(c.acounters, 0, kCountersN * sizeof(int));
   if (e == cudaSuccess) e = cudaMemset(c.status, 0, 64 * sizeof(int));
+  if (e == cudaSuccess) e = cudaMemset(c.df_cnt, 0, (4096 + 64) * sizeof(int));
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
     free_ctx(c);
@@ -473,6 +540,9 @@ int flashsvd_check_device_status(flashsvd_stream stream) {
   FSVD_CUDA(cudaMemcpy(&word, g_ctx.status, sizeof(int), cudaMemcpyDeviceToHost));
   if (word != DEV_STATUS_OK) {
     FSVD_CUDA(cudaMemset(g_ctx.status, 0, sizeof(int)));
+    FSVD_CUDA(cudaMemset(g_ctx.df_cnt, 0, (4096 + 64) * sizeof(int)));
+    FSVD_CUDA(cudaMemset(g_ctx.counters, 0, kCountersN * sizeof(int)));
+    FSVD_CUDA(cudaMemset(g_ctx.acounters, 0, kCountersN * sizeof(int)));
     return FLASHSVD_ERR_TIMEOUT;
   }
   return FLASHSVD_OK;

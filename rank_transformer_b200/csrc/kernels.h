@@ -1,6 +1,8 @@
 // Internal launch interface between the C-ABI layer (api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace fsvd {
@@ -98,6 +100,27 @@ struct PfLinear {
 };
 int prefill_linear_launch(const PfLinear& p, cudaStream_t stream);
 int prefill_dense_launch(const PfLinear& p, cudaStream_t stream);
+
+// --------------------------------------------- fused decode layer ---------
+struct DecodeLayerDesc {
+  const bf16 *U[3], *V[3], *U_o, *V_o, *U_gu, *V_gu, *U_dn, *V_dn;
+  const bf16 *g1, *g2;
+  int d, H, D, f, r, r_f;
+  float eps;
+  const float *rope_cos, *rope_sin;
+  const void* pack;  // the layer's decode pack (decode_pack_launch), or null
+};
+int decode_fused_supported(int B, int d, int D, int r, int r_f);
+long long decode_pack_bytes(const DecodeLayerDesc& L);
+int decode_pack_launch(const DecodeLayerDesc& L, void* dst, long long bytes, int sm_count,
+                       cudaStream_t stream);
+int decode_fused_launch(const DecodeLayerDesc& L, bf16* x, bf16* kc, bf16* vc, const int* seqlens,
+                        int B, int S_max, bf16* qbuf, bf16* att, bf16* hbuf, float* z, float* part,
+                        int* tilecnt, int* bar, int* done, int* status, int sm_count,
+                        cudaStream_t stream);
+int encode_map(CUtensorMap* map, const void* base, long long rows, long long cols, long long ld,
+               int box_cols, int box_rows, bool swizzle128);
+constexpr int kFusedPartFloats = 148 * 16 * 640;  // per SM: 16 partial slots of 640 floats
 
 // ------------------------------------------------ prefill attention -------
 struct AttnPfParams {

@@ -57,6 +57,7 @@ class Layer(C.Structure):
         ("U_gu", _p), ("V_gu", _p), ("r_f", _i),
         ("up", Factor), ("down", Factor),
         ("rope_cos", _p), ("rope_sin", _p),
+        ("decode_pack", _p),
     ]
 
 
@@ -68,6 +69,9 @@ _SIGS = {
     "flashsvd_shutdown": ([], _i),
     "flashsvd_check_device_status": ([_p], _i),
     "flashsvd_launch_count": ([], C.c_int64),
+    "flashsvd_set_decode_path": ([_i], _i),
+    "flashsvd_decode_pack_bytes": ([_p, C.POINTER(C.c_size_t)], _i),
+    "flashsvd_decode_pack": ([_p, _p, C.c_size_t, _p], _i),
     "flashsvd_profile_enable": ([_i], _i),
     "flashsvd_profile_report": ([C.c_char_p, _i, _i], _i),
     "flashsvd_lowrank_linear": ([_p, _p, _p, _p, _p, _i, _i, _i, _i, _p], _i),
@@ -136,6 +140,24 @@ def shutdown() -> None:
 
 def check_device_status(stream=None) -> None:
     _call("flashsvd_check_device_status", stream_handle(stream))
+
+
+def set_decode_path(fused: bool) -> None:
+    _call("flashsvd_set_decode_path", int(fused))
+
+
+def decode_pack_bytes(L: "Layer") -> int:
+    n = C.c_size_t(0)
+    _call("flashsvd_decode_pack_bytes", C.byref(L), C.byref(n))
+    return int(n.value)
+
+
+def decode_pack(L: "Layer", dst, stream=None) -> None:
+    """Write L's decode pack into the device buffer dst (a torch tensor of
+    at least decode_pack_bytes(L) bytes) and point L.decode_pack at it."""
+    nbytes = dst.numel() * dst.element_size()
+    _call("flashsvd_decode_pack", C.byref(L), ptr(dst), nbytes, stream_handle(stream))
+    L.decode_pack = ptr(dst)
 
 
 def launch_count() -> int:

@@ -55,7 +55,7 @@ def _bf16_normal(shape, std, gen, device):
 
 class DecoderModel:
     def __init__(self, cfg: DecoderConfig, B: int, S_max: int, seed: int = 0,
-                 device: str = "cuda", weights=None):
+                 device: str = "cuda", weights=None, decode_pack: bool = False):
         self.cfg, self.B, self.S_max, self.device = cfg, B, S_max, device
         gen = torch.Generator(device=device)
         gen.manual_seed(seed)
@@ -95,6 +95,20 @@ class DecoderModel:
         self.tokens = torch.zeros(B, dtype=torch.int32, device=device)
         self.logits = torch.zeros((B, cfg.vocab), dtype=torch.float32, device=device)
         self.structs = [self._struct(w) for w in self.layers]
+        # Decode packs: each layer's factors re-tiled for the fused decode
+        # kernel (layers whose shapes it does not cover keep the per-stage
+        # decode path).
+        self.packs = []
+        if decode_pack:
+            for L in self.structs:
+                try:
+                    n = fs.decode_pack_bytes(L)
+                except fs.FlashSVDError:
+                    self.packs.append(None)
+                    continue
+                buf = torch.empty(n, dtype=torch.uint8, device=device)
+                fs.decode_pack(L, buf)
+                self.packs.append(buf)
         self.graphs = None
         self.step_graph = None
 
