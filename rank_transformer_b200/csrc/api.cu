@@ -243,9 +243,9 @@ int layer_decode(const flashsvd_layer* L, bf16* x, bf16* kc, bf16* vc,
   if (g_fused_decode && L->decode_pack && pack_shapes_ok(L) && g_ctx.sm_count <= 148 &&
       decode_fused_supported(B, d, L->D, r, L->r_f)) {
     const DecodeLayerDesc D = decode_desc(L);
-    const int st = decode_fused_launch(D, x, kc, vc, seqlens, B, S_max, g_ctx.q, g_ctx.att, g_ctx.h,
-                                       g_ctx.z, g_ctx.df_part, g_ctx.df_cnt, g_ctx.df_cnt + 4096,
-                                       g_ctx.df_cnt + 4096 + 32, g_ctx.status, g_ctx.sm_count, s);
+    const int st = decode_fused_launch(D, x, kc, vc, seqlens, B, S_max, g_ctx.xn, g_ctx.df_part,
+                                       kFusedPartFloats, g_ctx.df_cnt, g_ctx.df_cnt + 32, g_ctx.status,
+                                       g_ctx.sm_count, s);
     if (st != FLASHSVD_ERR_UNSUPPORTED_SHAPE) return st;
   }
   // 1) z_qkv = rmsnorm(x) . [U_q | U_k | U_v]
@@ -447,7 +447,10 @@ int flashsvd_decode_pack_bytes(const flashsvd_layer* L, size_t* bytes) {
   if (!L || !bytes) return FLASHSVD_ERR_INVALID_ARG;
   if (L->kind != FLASHSVD_DECODER) return FLASHSVD_ERR_INVALID_ARG;
   if (!pack_shapes_ok(L)) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
-  *bytes = (size_t)decode_pack_bytes(decode_desc(L));
+  int sms = 148, dev = 0;
+  FSVD_CUDA(cudaGetDevice(&dev));
+  FSVD_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  *bytes = (size_t)decode_pack_bytes(decode_desc(L), sms);
   return FLASHSVD_OK;
 }
 
@@ -456,6 +459,7 @@ int flashsvd_decode_pack(const flashsvd_layer* L, void* dst, size_t bytes, flash
   FSVD_TRY(flashsvd_decode_pack_bytes(L, &need));
   if (!dst || bytes < need) return FLASHSVD_ERR_INVALID_ARG;
   if (!aligned16(dst)) return FLASHSVD_ERR_MISALIGNED;
+  if (capturing((cudaStream_t)stream)) return FLASHSVD_ERR_CAPTURE_UNSAFE;
   const flashsvd_bf16* ptrs[] = {L->q.U, L->k.U, L->v.U, L->q.V, L->k.V, L->v.V, L->o.U, L->o.V,
                                  L->U_gu, L->V_gu, L->down.U, L->down.V};
   for (const flashsvd_bf16* q : ptrs) {
@@ -543,7 +547,7 @@ int flashsvd_check_device_status(flashsvd_stream stream) {
     FSVD_CUDA(cudaMemset(g_ctx.df_cnt, 0, (4096 + 64) * sizeof(int)));
     FSVD_CUDA(cudaMemset(g_ctx.counters, 0, kCountersN * sizeof(int)));
     FSVD_CUDA(cudaMemset(g_ctx.acounters, 0, kCountersN * sizeof(int)));
-    return FLASHSVD_ERR_TIMEOUT;
+    return word == DEV_STATUS_SCHEDULE ? FLASHSVD_ERR_UNSUPPORTED_SHAPE : FLASHSVD_ERR_TIMEOUT;
   }
   return FLASHSVD_OK;
 }

@@ -123,6 +123,8 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 // Device status word codes (written by kernels whose bounded waits expire).
-enum : int { DEV_STATUS_OK = 0, DEV_STATUS_TIMEOUT = 1 };
+// DEV_STATUS_SCHEDULE: a kernel met a work split beyond its fixed limits
+// (e.g. very unequal sequence lengths) and skipped that work.
+enum : int { DEV_STATUS_OK = 0, DEV_STATUS_TIMEOUT = 1, DEV_STATUS_SCHEDULE = 2 };
 
 }  // namespace fsvd

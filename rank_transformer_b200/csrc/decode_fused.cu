@@ -6,36 +6,47 @@
 // through the low-rank projections and the history is read from a dense KV
 // cache (Methodology 2), gate and up share one packed projection
 // (Methodology 3), and the per-layer decode body is one replay unit
-// (Methodology 4).  Here that replay unit is a single kernel whose nine
-// stages (z = rmsnorm(x) U_qkv; q,k,v = z V (+RoPE, KV append); attention;
-// z = a U_o; x += z V_o; z = rmsnorm(x) U_gu; h = SiLU(z_g V_g) (z_u V_u);
-// z = h U_dn; x += z V_dn) are separated by grid barriers, while the bytes
-// that do not depend on any stage -- every factor tile -- stream without
-// pause.
+// (Methodology 4).  Here that replay unit is a single kernel with nine
+// stages separated by grid barriers:
+//   0  z = rmsnorm(x) [U_q | U_k | U_v]      5  z = rmsnorm(x') U_gu
+//   1  q, k, v = z V (+RoPE)                 6  h = SiLU(z_g V_g) (z_u V_u)
+//   2  attention over the dense cache        7  z = h U_dn
+//   3  z = a U_o                             8  x'' = x' + z V_dn
+//   4  x' = x + z V_o
+// followed by a short final pass that writes x'' back over x.
 //
-// The factors are read from the layer's decode pack: every factor matrix
-// re-tiled once, at load time, so that each ring entry (256 rows x 64
-// output columns, as two [rows x 32] boxes) is one contiguous block of HBM,
-// stored in the order the stages consume them.  Streaming whole blocks
-// instead of 64- or 128-byte row pieces scattered at the matrix's row pitch
-// is what lets the factor stream run near the HBM roofline.
+// Factors.  They are read from the layer's decode pack: every factor matrix
+// re-tiled once, at load time, so that each ring entry (256 rows x 64 output
+// columns, as two [rows x 32] boxes) is one contiguous block of HBM, stored
+// in consumption order.  Whole blocks stream near the HBM copy rate; 64- or
+// 128-byte row pieces spaced at the matrix pitch do not.
+//
+// Reduction ("reduce on read").  A CTA's share of a stage is a contiguous
+// range of (tile, 256-row chunk) entries, so a column tile's K range is
+// split over a few CTAs.  A CTA writes one fp32 partial per tile it touched
+// and nothing else: no atomics, no last-arriver combine.  After the grid
+// barrier, each CTA builds the stage input it needs by summing those
+// partials (in CTA order, so every reader gets the same bits) and applying
+// the previous stage's epilogue as it reads: RoPE and bf16 rounding of q/k/v,
+// residual add and RMSNorm, SwiGLU, and the softmax merge of attention
+// partials.  The new key and value enter attention from these sums; the CTA
+// that owns a sequence's last cache chunk also appends them to the cache.
+// Hence the K/V chunks themselves depend on no stage and are loaded as soon
+// as ring slots free up.
 //
 // Roles per CTA (CW consumer warps + 2 producer warps):
-//   warp CW   factor producer: walks this CTA's schedule across all stages and
-//             bulk-copies each entry of the pack into a ring slot as soon as
-//             the slot is free (and prefetches the next entries into L2); it
-//             never waits for activations.
-//   warp CW+1 activation producer: after each stage's grid barrier, bulk-copies
-//           the activation rows each ring entry needs (and, for attention,
-//           the K/V chunk) into the same slot.
-//   warps 0..CW-1 consumers: multiply, keep whole K ranges in registers, and
-//           finish a column tile either directly (sole owner) or through a
-//           last-arriver combine of per-CTA partials (fixed order).
-// A CTA's share of a stage is a contiguous range of (tile, 256-row chunk)
-// entries, so partial sums are written once per tile touched (1-4 per stage)
-// instead of once per chunk.  All waits are bounded.
+//   warp CW   producer: fills every ring entry in order -- bulk copies of
+//             pack entries for the GEMV stages (prefetched ahead into L2),
+//             TMA loads of 64-key cache chunks for attention; it never waits
+//             for activations.
+//   warp CW+1 prefetches this CTA's cache chunks into L2 at kernel start.
+//   consumers multiply-accumulate ring entries against the stage input
+//             built in shared memory, and run attention with per-warp
+//             online-softmax state.
+// All waits are bounded; a timeout sets the device status word.
 #include <algorithm>
 #include <cstring>
+#include <vector>
 
 #include "kernels.h"
 #include "tc.cuh"
@@ -44,52 +55,64 @@ namespace fsvd {
 
 namespace {
 
-constexpr int DF_KC = 256;
-constexpr int DF_MAX_SU = 16;
-constexpr int DF_PART_STRIDE = 640;
+constexpr int DF_KC = 256;            // rows per ring entry
+constexpr int DF_MAX_SU = 16;         // tiles (or attention pairs) per CTA and stage
+constexpr int DF_PART_STRIDE = 640;   // floats per partial slot (>= 4 x 64, >= 4 + 128)
 constexpr int DF_NPHASE = 9;
 constexpr int DF_NMAPS = 2;
+constexpr int DF_ABUF_COLS = 4096;    // floats per row of the stage-input buffer
+constexpr int DF_MAX_PAIRS = 8;       // attention (batch, head) pairs per CTA
+constexpr int DF_MAX_NK = 64;         // 256-row chunks per factor (K <= 16384)
+constexpr int DF_CMAX = 15;           // contributing CTAs per tile (or pair) read
+constexpr int DF_MAX_UNITS = 96;      // tiles (or pairs) read per stage and CTA
 
 enum { DF_GEMV = 0, DF_ATTN = 1 };
+// How a stage's input is built from what the previous stage left.
+enum { SRC_X = 0, SRC_PART = 1, SRC_ATT = 2, SRC_XMID = 3, SRC_SWIGLU = 4 };
 
 struct DfPhase {
-  int type, pro, epi, map;
+  int type, map, src, norm;
   int nprob;
   int tile_start[4];
   int T, K, nk;
-  long long pack_off;  // byte offset of this stage's entries in the pack
   int N[3];
-  int a_col[3];
-  int a_col2;
-  int w_row2;
-  int out_col[3];
-  int kind[3];
-  const void* a;
-  int a_f32;
-  long long lda;
+  int a_col2;          // SwiGLU stage: offset of the up half in the previous output
+  long long pack_off;  // byte offset of this stage's entries in the pack
   const bf16* norm_g;
-  float* out32; long long ldo32;
-  bf16* out16; long long ldo16;
-  const bf16* resid; long long ldr;
 };
+
+// Per (stage, CTA) schedule record, built on the host with the pack: the
+// input chunks (problem << 8 | 256-row chunk) of the CTA's entries in
+// first-use order, the chunk of each entry, and the contributor table of the
+// previous-stage tiles those chunks draw on.  Records 0..8 follow the
+// stages (attention-dependent tables are filled on the device); record 9
+// serves the final pass.
+constexpr int DF_NREC = DF_NPHASE + 1;
+constexpr int DF_MAX_E = 48;  // entries per CTA and stage
+struct SchedRec {
+  int n, nunits, pad0, pad1;
+  int clist[16];
+  uint8_t chunk_of[DF_MAX_E];
+  short utab[DF_MAX_UNITS][16];
+};
+static_assert(sizeof(SchedRec) % 128 == 0, "schedule records stay 128-byte aligned");
 
 struct DfParams {
   CUtensorMap maps[DF_NMAPS];  // the K and V cache views [B * S_max x H * D]
   const uint8_t* pack;
+  const SchedRec* sched;       // [DF_NREC][G], inside the pack
   DfPhase ph[DF_NPHASE];
-  int nphase;
-  int B, H, D, S_max;
+  int B, H, D, S_max, d;
   float eps, scale_log2;
   const int* seqlens;
+  bf16* x;        // layer input and output [B x d]
+  bf16* xm;       // x' (after the attention block) [B x d]
   bf16* k_cache;
   bf16* v_cache;
   const float* rope_cos;
   const float* rope_sin;
-  const bf16* q;
-  bf16* att;
-  float* part;
-  int* tilecnt;
-  int* bar;
+  float* part;    // [2][G][DF_MAX_SU][DF_PART_STRIDE]: stage s writes half s & 1
+  int* bar;       // [DF_NPHASE] arrivals per stage
   int* done;
   int* status;
 };
@@ -98,16 +121,17 @@ template <int MT>
 struct DfCfg {
   static constexpr int CW = MT <= 2 ? 16 : 8;        // consumer warps
   static constexpr int CT = CW * 32;                 // consumer threads
-  static constexpr int THREADS = CT + 64;            // + factor and activation producers
-  static constexpr int W_BYTES = 32768;
-  static constexpr int A_BYTES = 2 * MT * DF_KC * 4;
-  static constexpr int SLOT = W_BYTES + A_BYTES;
-  static constexpr int NSLOT = MT == 1 ? 6 : (MT == 8 ? 4 : 5);
+  static constexpr int THREADS = CT + 64;            // + producer and prefetch warps
+  static constexpr int SLOT = 32768;
+  static constexpr int NSLOT = MT == 1 ? 6 : (MT == 2 ? 5 : 4);
+  static constexpr int ABUF_BYTES = MT * DF_ABUF_COLS * 4;
   static constexpr int RED_BYTES = CW * MT * 64 * 4 > 2048 ? CW * MT * 64 * 4 : 2048;
-  static constexpr int SCR_BYTES = (64 + CW * 128 + 128) * 4;
-  static constexpr int BAR_BYTES = 1024;
-  static constexpr int PH_BYTES = 2048;  // copy of the stage table
-  static constexpr int SMEM = 1024 + NSLOT * SLOT + RED_BYTES + SCR_BYTES + BAR_BYTES + PH_BYTES;
+  static constexpr int SCR_BYTES = (64 + CW * 128) * 4;
+  static constexpr int MISC_BYTES = 4608;  // chunk map and list, rstd, contributor table
+  static constexpr int BAR_BYTES = 512;
+  static constexpr int PH_BYTES = 768;     // copy of the stage table
+  static constexpr int SMEM = 1024 + NSLOT * SLOT + ABUF_BYTES + RED_BYTES + SCR_BYTES + MISC_BYTES +
+                              BAR_BYTES + PH_BYTES;
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -116,16 +140,12 @@ __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;"
 __device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
-
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
           tc::smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(tc::smem_u32(bar))
       : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect(uint64_t* bar, uint32_t bytes) {
-  tc::mbar_expect_tx(bar, bytes);  // arrive (count 1) + expect bytes
 }
 __device__ __forceinline__ int ld_acquire(const int* p) {
   int v;
@@ -135,6 +155,21 @@ __device__ __forceinline__ int ld_acquire(const int* p) {
 __device__ __forceinline__ void red_release_add(int* p, int v) {
   asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+__device__ __forceinline__ float bf_round(float v) { return bf2f(f2bf(v)); }
+
+// Bounded wait until every CTA has arrived at stage counter *bar.
+__device__ __forceinline__ void grid_wait(const int* bar, int G, volatile int* abort_flag, int* status) {
+  const long long t0 = clock64();
+  while (ld_acquire(bar) < G) {
+    if (*abort_flag) return;
+    if (clock64() - t0 > tc::kWaitCycles) {
+      *abort_flag = 1;
+      atomicExch(status, DEV_STATUS_TIMEOUT);
+      return;
+    }
+    __nanosleep(32);
+  }
+}
 
 // Contiguous share [c0, c1) of C entries for CTA g of G; owner of entry c.
 // (32-bit: C * G stays below 2^31 for every stage the host accepts.)
@@ -142,26 +177,13 @@ __device__ __forceinline__ void share(int C, int G, int g, int& c0, int& c1) {
   c0 = g * C / G;
   c1 = (g + 1) * C / G;
 }
-__device__ __forceinline__ int owner_of(int c, int C, int G) {
-  return ((c + 1) * G - 1) / C;
-}
-
-// Whether CTA g has at least one of the C entries.
-__device__ __forceinline__ bool share_nonempty(int C, int G, int g) {
+__host__ __device__ __forceinline__ int owner_of(int c, int C, int G) { return ((c + 1) * G - 1) / C; }
+__host__ __device__ __forceinline__ bool share_nonempty(int C, int G, int g) {
   return (g + 1) * C / G > g * C / G;
-}
-// Number of distinct CTAs owning entries first..last: every CTA between the
-// two owners when each CTA has entries (C >= G), else only the non-empty ones.
-__device__ __forceinline__ int count_owners(int first, int last, int C, int G) {
-  const int gf = owner_of(first, C, G), gl = owner_of(last, C, G);
-  if (C >= G) return gl - gf + 1;
-  int n = 0;
-  for (int gg = gf; gg <= gl; ++gg) n += share_nonempty(C, G, gg);
-  return n;
 }
 
 // Attention entry layout: for each batch row b, H heads x nk_b chunks of 64
-// keys (nk_b from the current length).
+// keys (nk_b from the current length L_b = position + 1).
 struct AttnSched {
   int nk[8];
   int pre[9];
@@ -190,38 +212,133 @@ __device__ __forceinline__ void attn_entry(const AttnSched& s, int c, int& b, in
   kc = r - h * s.nk[b];
 }
 
-// Global output column of tile column c (0..63).
-__device__ __forceinline__ int out_col(const DfPhase& ph, int D, int tl, int c) {
-  const int box = c >> 5, cc = c & 31;
-  if (ph.map == MAP_PLAIN) return 64 * tl + c;
-  if (ph.map == MAP_ROPE) {
-    const int tph = D >> 6, hh = tl / tph, j = tl - hh * tph;
-    return hh * D + 32 * j + cc + box * (D >> 1);
+// Contributors of a tile (or attention pair) are the CTAs whose shares hold
+// its entries: a contiguous CTA range.  A unit of the contributor table is
+// u[0] = count, u[1..] = partial slot indices (gg * DF_MAX_SU + su).
+
+// Tile t of GEMV stage q.  False if the slots do not fit the table.
+__host__ __device__ __forceinline__ bool tile_slots(const DfPhase& q, int t, int G, short* u) {
+  const int Ctot = q.T * q.nk;
+  const int gf = owner_of(t * q.nk, Ctot, G), gl = owner_of(t * q.nk + q.nk - 1, Ctot, G);
+  int n = 0;
+  bool ok = true;
+  for (int gg = gf; gg <= gl; ++gg) {
+    if (Ctot < G && !share_nonempty(Ctot, G, gg)) continue;
+    const int su = t - (gg * Ctot / G) / q.nk;
+    if (su < 0 || su >= DF_MAX_SU || n >= DF_CMAX) { ok = false; continue; }
+    u[1 + n++] = (short)(gg * DF_MAX_SU + su);
   }
-  return 32 * tl + cc;
+  u[0] = (short)n;
+  return ok;
 }
 
-// acc[m][0..7] += A[m][kk] * W[kk][8 columns] over this thread's 8 rows of
-// a 256-row entry.  NORM: A is bf16 x scaled by rstd[m] * g[kk]; AF32: A is
-// fp32 (rank activations), else bf16.
-template <int MT, int NORM, int AF32, int RSTEP>
-__device__ __forceinline__ void entry_mac(float (&acc)[MT][8], const uint8_t* w, const uint8_t* a_s,
-                                          int seg, int kn, int row0, const bf16* g,
-                                          const float* rstd) {
+// Attention pair (b, h).
+__device__ __forceinline__ bool pair_slots(const AttnSched& s, int H, int G, int b, int h, short* u) {
+  const int Ctot = s.pre[8];
+  const int e0 = s.pre[b] + h * s.nk[b];
+  const int gf = owner_of(e0, Ctot, G), gl = owner_of(e0 + s.nk[b] - 1, Ctot, G);
+  int n = 0;
+  bool ok = true;
+  for (int gg = gf; gg <= gl; ++gg) {
+    if (Ctot < G && !share_nonempty(Ctot, G, gg)) continue;
+    int b2, h2, k2;
+    attn_entry(s, gg * Ctot / G, b2, h2, k2);
+    const int su = b * H + h - (b2 * H + h2);
+    if (su < 0 || su >= DF_MAX_SU || n >= DF_CMAX) { ok = false; continue; }
+    u[1 + n++] = (short)(gg * DF_MAX_SU + su);
+  }
+  u[0] = (short)n;
+  return ok;
+}
+
+__device__ __forceinline__ void add4(float4& a, const float4& b, float w = 1.f) {
+  a.x = fmaf(w, b.x, a.x); a.y = fmaf(w, b.y, a.y); a.z = fmaf(w, b.z, a.z); a.w = fmaf(w, b.w, a.w);
+}
+// Sums of 4 consecutive floats over two units' partial slots (s0 at idx0
+// over u0; s1 at idx1 over u1 when has1), weighted by w0 / w1 when given.
+// Slots are added in CTA order, so every reader gets the same bits; the
+// loads of both sums are issued before any add, four slots at a time.
+__device__ __forceinline__ void gather4x2(const float* buf, const short* u0, int idx0, const float* w0,
+                                          const short* u1, int idx1, const float* w1, bool has1,
+                                          float4& s0, float4& s1) {
+  s0 = make_float4(0.f, 0.f, 0.f, 0.f);
+  s1 = s0;
+  const int n0 = u0[0], n1 = has1 ? u1[0] : 0;
+  const int n = n0 > n1 ? n0 : n1;
+  for (int c0 = 0; c0 < n; c0 += 4) {
+    float4 a[4], b[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      a[c] = c0 + c < n0
+                 ? __ldcg(reinterpret_cast<const float4*>(buf + (long long)u0[1 + c0 + c] * DF_PART_STRIDE + idx0))
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+      b[c] = c0 + c < n1
+                 ? __ldcg(reinterpret_cast<const float4*>(buf + (long long)u1[1 + c0 + c] * DF_PART_STRIDE + idx1))
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (c0 + c < n0) add4(s0, a[c], w0 ? w0[c0 + c] : 1.f);
+      if (c0 + c < n1) add4(s1, b[c], w1 ? w1[c0 + c] : 1.f);
+    }
+  }
+}
+// Softmax merge of one attention pair's (m, l, o) partials for dims
+// [dim, dim + 4): an online merge in contributor (CTA) order, so every reader
+// gets the same bits; loads four contributors at a time.
+__device__ __forceinline__ float4 attn_gather4(const float* buf, const short* u, int dim) {
+  const int n = u[0];
+  float M = -INFINITY, Ls = 0.f;
+  float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int c0 = 0; c0 < n; c0 += 4) {
+    float mc[4], lc[4];
+    float4 oc[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      mc[c] = -INFINITY;
+      lc[c] = 0.f;
+      oc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (c0 + c < n) {
+        const float* ps = buf + (long long)u[1 + c0 + c] * DF_PART_STRIDE;
+        mc[c] = __ldcg(ps);
+        lc[c] = __ldcg(ps + 1);
+        oc[c] = __ldcg(reinterpret_cast<const float4*>(ps + 4 + dim));
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (mc[c] == -INFINITY) continue;
+      const float Mn = fmaxf(M, mc[c]);
+      const float a = M == -INFINITY ? 0.f : exp2f(M - Mn), b = exp2f(mc[c] - Mn);
+      Ls = Ls * a + lc[c] * b;
+      O = make_float4(O.x * a + oc[c].x * b, O.y * a + oc[c].y * b, O.z * a + oc[c].z * b, O.w * a + oc[c].w * b);
+      M = Mn;
+    }
+  }
+  const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+  return make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
+}
+
+__device__ __forceinline__ float4 round4(float4 v) {
+  return make_float4(bf_round(v.x), bf_round(v.y), bf_round(v.z), bf_round(v.w));
+}
+
+// acc[m][0..7] += A[m][kk] * W[kk][8 columns] over this thread's rows of a
+// 256-row entry.  a points at the entry's input chunk (row m at
+// m * DF_ABUF_COLS); NORM scales it by rstd[m] * g[kk].  Rows at or beyond kn
+// are masked (their shared memory holds stale data).
+template <int MT, int NORM, int RSTEP>
+__device__ __forceinline__ void entry_mac(float (&acc)[MT][8], const uint8_t* w, const float* a, int kn,
+                                          int row0, const bf16* g, const float* rstd) {
   constexpr int IT = DF_KC / RSTEP;
-  // All shared-memory loads of this thread's rows first (slots are always
-  // fully allocated), then the arithmetic; rows at or beyond kn are masked.
   uint4 u[IT];
-  float a[IT][MT];
+  float av[IT][MT];
 #pragma unroll
   for (int i = 0; i < IT; ++i) {
     const int kk = row0 + RSTEP * i;
     u[i] = *reinterpret_cast<const uint4*>(w + kk * 64);
 #pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      if (AF32) a[i][m] = reinterpret_cast<const float*>(a_s)[(seg * MT + m) * DF_KC + kk];
-      else a[i][m] = bf2f(reinterpret_cast<const bf16*>(a_s)[(seg * MT + m) * DF_KC + kk]);
-    }
+    for (int m = 0; m < MT; ++m) av[i][m] = a[m * DF_ABUF_COLS + kk];
   }
   float gk[IT];
 #pragma unroll
@@ -236,12 +353,17 @@ __device__ __forceinline__ void entry_mac(float (&acc)[MT][8], const uint8_t* w,
                          bf_lo(u[i].z), bf_hi(u[i].z), bf_lo(u[i].w), bf_hi(u[i].w)};
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
-      float av = NORM ? a[i][m] * (rstd[m] * gk[i]) : a[i][m];
-      av = valid ? av : 0.f;
+      float x = NORM ? av[i][m] * (rstd[m] * gk[i]) : av[i][m];
+      x = valid ? x : 0.f;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) acc[m][j] = fmaf(av, valid ? wv[j] : 0.f, acc[m][j]);
+      for (int j = 0; j < 8; ++j) acc[m][j] = fmaf(x, valid ? wv[j] : 0.f, acc[m][j]);
     }
   }
+}
+
+__device__ __forceinline__ void prefetch_l2_2d(const CUtensorMap* tm, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(tm), "r"(c0), "r"(c1)
+               : "memory");
 }
 
 template <int MT>
@@ -251,19 +373,24 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* slots = smem;
-  float* red = reinterpret_cast<float*>(smem + C::NSLOT * C::SLOT);
-  float* scr = reinterpret_cast<float*>(smem + C::NSLOT * C::SLOT + C::RED_BYTES);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::NSLOT * C::SLOT + C::RED_BYTES + C::SCR_BYTES);
+  float* abuf = reinterpret_cast<float*>(smem + C::NSLOT * C::SLOT);   // [MT][DF_ABUF_COLS]
+  float* red = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(abuf) + C::ABUF_BYTES);
+  float* scr = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(red) + C::RED_BYTES);
+  uint8_t* misc = reinterpret_cast<uint8_t*>(scr) + C::SCR_BYTES;
+  SchedRec* srec = reinterpret_cast<SchedRec*>(misc);    // this CTA's record of the current stage
+  int* clist = srec->clist;
+  short* utab = &srec->utab[0][0];
+  float* s_rstd = reinterpret_cast<float*>(misc + sizeof(SchedRec));  // [8]
+  static_assert(sizeof(SchedRec) + 32 <= C::MISC_BYTES, "schedule record exceeds its shared copy");
+  uint64_t* full = reinterpret_cast<uint64_t*>(misc + C::MISC_BYTES);
   uint64_t* empty = full + C::NSLOT;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + C::NSLOT);
-  int* s_flag = const_cast<int*>(abort_flag) + 1;
-  float* s_rstd = reinterpret_cast<float*>(s_flag + 4);  // [8]
-  DfPhase* s_ph = reinterpret_cast<DfPhase*>(smem + C::NSLOT * C::SLOT + C::RED_BYTES + C::SCR_BYTES +
-                                             C::BAR_BYTES);
-  static_assert(sizeof(DfPhase) * DF_NPHASE <= 2048, "stage table exceeds its shared-memory copy");
+  DfPhase* s_ph = reinterpret_cast<DfPhase*>(reinterpret_cast<uint8_t*>(full) + C::BAR_BYTES);
+  static_assert(sizeof(DfPhase) * DF_NPHASE <= C::PH_BYTES, "stage table exceeds its shared copy");
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, g = blockIdx.x;
+  const long long half = (long long)G * DF_MAX_SU * DF_PART_STRIDE;
 
   {
     // Stage descriptors are read in every inner loop: keep a shared copy.
@@ -273,7 +400,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
   }
   if (tid == 0) {
     for (int s = 0; s < C::NSLOT; ++s) {
-      tc::mbar_init(full + s, 2);
+      tc::mbar_init(full + s, 1);
       tc::mbar_init(empty + s, C::CW);
     }
     *abort_flag = 0;
@@ -283,16 +410,16 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
   pdl_launch_dependents();
 
   if (warp == C::CW) {
-    // ============================================ factor producer ==========
+    // =================================================== producer ==========
     if (lane == 0) {
-      // L2 prefetch cursor over this CTA's factor entries, PF entries ahead
-      // of the loads, so that the loads into the ring hit L2.
-      constexpr int PF = 12;
+      // L2 prefetch cursor over this CTA's pack entries, PF entries ahead of
+      // the copies into the ring.
+      constexpr int PF = 2;
       int pf_ph = -1, pf_c = 0, pf_c1 = 0;
       auto pf_step = [&]() {
         while (pf_c >= pf_c1) {
-          if (pf_ph >= p.nphase) return;
-          if (++pf_ph >= p.nphase) return;
+          if (pf_ph >= DF_NPHASE) return;
+          if (++pf_ph >= DF_NPHASE) return;
           const DfPhase& q = s_ph[pf_ph];
           if (q.type != DF_GEMV) { pf_c = pf_c1 = 0; continue; }
           share(q.T * q.nk, G, g, pf_c, pf_c1);
@@ -306,116 +433,73 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
       };
       for (int i = 0; i < PF; ++i) pf_step();
       int seq = 0;
-      bool waited = false;
-      for (int ph_i = 0; ph_i < p.nphase && !*abort_flag; ++ph_i) {
+      bool waited = false, ok = true;
+      for (int ph_i = 0; ph_i < DF_NPHASE && ok && !*abort_flag; ++ph_i) {
         const DfPhase& ph = s_ph[ph_i];
-        int Ctot, c0, c1;
+        int c0, c1;
         if (ph.type == DF_ATTN) {
+          // K/V chunks of the dense cache (rows before the current position
+          // are fixed for this step; the current row is taken from q/k/v)
           if (!waited) { pdl_wait(); waited = true; }
           AttnSched s;
           attn_sched(p, s);
-          Ctot = s.pre[8];
-        } else {
-          Ctot = ph.T * ph.nk;
-        }
-        if (Ctot == 0) continue;
-        share(Ctot, G, g, c0, c1);
-        for (int c = c0; c < c1; ++c, ++seq) {
-          const int slot = seq % C::NSLOT;
-          const uint32_t par = (uint32_t)(seq / C::NSLOT) & 1u;
-          if (!tc::mbar_wait_sleep(empty + slot, par ^ 1u, abort_flag, p.status)) break;
-          if (ph.type == DF_ATTN) {
-            tc::mbar_arrive(full + slot);  // the K/V chunk comes from the other producer
-          } else {
-            const int t = c / ph.nk, kc = c - t * ph.nk;
-            const uint32_t box = (uint32_t)min(DF_KC, ph.K - kc * DF_KC) * 64u;
-            const uint8_t* e = p.pack + ph.pack_off + (long long)t * ph.K * 128 + (long long)kc * 32768;
-            uint8_t* w = slots + slot * C::SLOT;
-            mbar_arrive_expect(full + slot, 2u * box);
-            bulk_g2s(w, e, box, full + slot);
-            bulk_g2s(w + 16384, e + box, box, full + slot);
-            pf_step();
-          }
-        }
-      }
-      if (*abort_flag) {
-        const long long t0 = clock64();
-        while (clock64() - t0 < 2000000) {}
-      }
-    }
-  } else if (warp == C::CW + 1) {
-    // ======================================== activation producer ==========
-    if (lane == 0) {
-      for (int i = 0; i < DF_NMAPS; ++i) tc::tma_prefetch_desc(&p.maps[i]);
-      pdl_wait();
-      int seq = 0;
-      for (int ph_i = 0; ph_i < p.nphase && !*abort_flag; ++ph_i) {
-        const DfPhase& ph = s_ph[ph_i];
-        if (ph_i > 0) {
-          // grid barrier: every CTA has finished stage ph_i - 1
-          const long long t0 = clock64();
-          while (ld_acquire(p.bar + ph_i - 1) < G) {
-            if (*abort_flag) break;
-            if (clock64() - t0 > tc::kWaitCycles) {
-              *abort_flag = 1;
-              atomicExch(p.status, DEV_STATUS_TIMEOUT);
-              break;
-            }
-            __nanosleep(64);
-          }
-          if (*abort_flag) break;
-        }
-        int Ctot, c0, c1;
-        AttnSched s;
-        if (ph.type == DF_ATTN) {
-          attn_sched(p, s);
-          Ctot = s.pre[8];
-        } else {
-          Ctot = ph.T * ph.nk;
-        }
-        if (Ctot == 0) continue;
-        share(Ctot, G, g, c0, c1);
-        for (int c = c0; c < c1; ++c, ++seq) {
-          const int slot = seq % C::NSLOT;
-          const uint32_t par = (uint32_t)(seq / C::NSLOT) & 1u;
-          if (!tc::mbar_wait_sleep(empty + slot, par ^ 1u, abort_flag, p.status)) break;
-          uint8_t* base = slots + slot * C::SLOT;
-          if (ph.type == DF_ATTN) {
+          share(s.pre[8], G, g, c0, c1);
+          const int NB = p.D >> 6;
+          for (int c = c0; c < c1; ++c, ++seq) {
+            const int slot = seq % C::NSLOT;
+            const uint32_t par = (uint32_t)(seq / C::NSLOT) & 1u;
+            if (!tc::mbar_wait_sleep(empty + slot, par ^ 1u, abort_flag, p.status)) { ok = false; break; }
+            uint8_t* base = slots + slot * C::SLOT;
             int b, h, kc;
             attn_entry(s, c, b, h, kc);
-            const int NB = p.D >> 6;
-            mbar_arrive_expect(full + slot, (uint32_t)(2 * NB * 8192));
+            tc::mbar_expect_tx(full + slot, (uint32_t)(2 * NB * 8192));
             const int row = b * p.S_max + kc * 64;
             for (int bx = 0; bx < NB; ++bx) {
               tc::tma_load_2d(base + bx * 8192, &p.maps[0], full + slot, h * p.D + 64 * bx, row);
               tc::tma_load_2d(base + 16384 + bx * 8192, &p.maps[1], full + slot, h * p.D + 64 * bx, row);
             }
-          } else {
-            const int t = c / ph.nk, kc = c - t * ph.nk;
-            const int k0 = kc * DF_KC;
-            const int kn = min(DF_KC, ph.K - k0);
-            int pi = 0;
-            for (int i = 1; i < 3; ++i)
-              if (i < ph.nprob && t >= ph.tile_start[i]) pi = i;
-            const int esz = ph.a_f32 ? 4 : 2;
-            const int nseg = ph.map == MAP_SWIGLU ? 2 : 1;
-            const uint32_t rowbytes = (uint32_t)(kn * esz);
-            mbar_arrive_expect(full + slot, rowbytes * (uint32_t)(nseg * p.B));
-            uint8_t* a_s = base + C::W_BYTES;
-            for (int sg = 0; sg < nseg; ++sg) {
-              const int acol = (sg ? ph.a_col2 : ph.a_col[pi]) + k0;
-              for (int m = 0; m < p.B; ++m) {
-                const uint8_t* src = reinterpret_cast<const uint8_t*>(ph.a) +
-                                     ((long long)m * ph.lda + acol) * esz;
-                bulk_g2s(a_s + (sg * MT + m) * DF_KC * esz, src, rowbytes, full + slot);
-              }
-            }
           }
+          continue;
+        }
+        share(ph.T * ph.nk, G, g, c0, c1);
+        for (int c = c0; c < c1; ++c, ++seq) {
+          const int slot = seq % C::NSLOT;
+          const uint32_t par = (uint32_t)(seq / C::NSLOT) & 1u;
+          if (!tc::mbar_wait_sleep(empty + slot, par ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          const int t = c / ph.nk, kc = c - t * ph.nk;
+          const uint32_t box = (uint32_t)min(DF_KC, ph.K - kc * DF_KC) * 64u;
+          const uint8_t* e = p.pack + ph.pack_off + (long long)t * ph.K * 128 + (long long)kc * 32768;
+          uint8_t* w = slots + slot * C::SLOT;
+          tc::mbar_expect_tx(full + slot, 2u * box);
+          bulk_g2s(w, e, box, full + slot);
+          bulk_g2s(w + 16384, e + box, box, full + slot);
+          pf_step();
         }
       }
       if (*abort_flag) {
-        const long long t0 = clock64();
+        const long long t0 = clock64();  // let copies in flight land
         while (clock64() - t0 < 2000000) {}
+      }
+    }
+  } else if (warp == C::CW + 1) {
+    // ================================================ K/V prefetch ==========
+    // History rows are fixed for this step: pull this CTA's chunks of the
+    // cache into L2 while the first stages stream their factors.
+    if (lane == 0) {
+      for (int i = 0; i < DF_NMAPS; ++i) tc::tma_prefetch_desc(&p.maps[i]);
+      pdl_wait();
+      AttnSched s;
+      attn_sched(p, s);
+      const int NB = p.D >> 6;
+      int a0, a1;
+      share(s.pre[8], G, g, a0, a1);
+      for (int c = a0; c < a1; ++c) {
+        int b, h, kc;
+        attn_entry(s, c, b, h, kc);
+        for (int bx = 0; bx < NB; ++bx) {
+          prefetch_l2_2d(&p.maps[0], h * p.D + 64 * bx, b * p.S_max + kc * 64);
+          prefetch_l2_2d(&p.maps[1], h * p.D + 64 * bx, b * p.S_max + kc * 64);
+        }
       }
     }
   } else {
@@ -428,20 +512,208 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
     const int row0 = 2 * rowlane + rsub;
     constexpr int RSTEP = C::CT / 8;
     int seq = 0;
-    for (int ph_i = 0; ph_i < p.nphase; ++ph_i) {
+    for (int ph_i = 0; ph_i < DF_NPHASE; ++ph_i) {
       const DfPhase& ph = s_ph[ph_i];
+      float* part_cur = p.part + (ph_i & 1) * half;
+      const float* part_prev = p.part + ((ph_i + 1) & 1) * half;
       if (ph.type == DF_GEMV) {
         const int Ctot = ph.T * ph.nk;
         int c0, c1;
         share(Ctot, G, g, c0, c1);
-        const int hi = box;
+        const int nseg = ph.map == MAP_SWIGLU ? 2 : 1;
+        const bool xin = ph.src == SRC_X || ph.src == SRC_XMID;
+        // this CTA's schedule record of the stage (static: from the pack)
+        {
+          const int4* src = reinterpret_cast<const int4*>(p.sched + (long long)ph_i * G + g);
+          int4* dst = reinterpret_cast<int4*>(srec);
+          for (int w = tid; w < (int)(sizeof(SchedRec) / 16); w += C::CT) dst[w] = __ldg(src + w);
+        }
+        consumer_sync<C::CT>();
+
+        // ---- the stage input, built from what the previous stage left ----
+        // (1) contributor table: one unit per previous-stage tile (or
+        // attention pair) that this CTA's input chunks draw on; static ones
+        // come with the record, attention pairs depend on the lengths.
+        const int n = srec->n;
+        const int hpc = DF_KC / p.D;  // heads per 256-column chunk
+        int nunits = srec->nunits;
+        if (ph.src == SRC_ATT) {
+          nunits = n * MT * hpc;
+          if (nunits > DF_MAX_UNITS) {
+            if (tid == 0) atomicExch(p.status, DEV_STATUS_SCHEDULE);
+            nunits = 0;
+          }
+          AttnSched s;
+          attn_sched(p, s);
+          for (int ui = tid; ui < nunits; ui += C::CT) {
+            short* u = utab + ui * 16;
+            u[0] = 0;
+            const int j = ui % hpc, r2 = ui / hpc, m = r2 % MT, ci = r2 / MT;
+            const int hh = (clist[ci] & 255) * DF_KC / p.D + j;
+            if (m < p.B && hh < p.H && !pair_slots(s, p.H, G, m, hh, u)) atomicExch(p.status, DEV_STATUS_SCHEDULE);
+          }
+        }
+        if (ph.norm) {
+          // the norm gains, into L1 for the scaling after the barrier
+          for (int o = tid * 64; o < p.d; o += C::CT * 64)
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(ph.norm_g + o));
+        }
+        // ---- wait for the previous stage on every CTA ----
+        if (ph_i > 0 && tid == 0) grid_wait(p.bar + ph_i - 1, G, abort_flag, p.status);
+        consumer_sync<C::CT>();
+        // (2) the input itself, 4 consecutive values per group, two groups
+        // per thread and step (their loads in flight together)
+        if (xin) {
+          // x (stage 0) or x' = x + (z V_o) (stage 5), whole rows, for RMSNorm
+          const int d4 = p.d >> 2, tot = MT * d4;
+          for (int e0 = tid; e0 < tot; e0 += 2 * C::CT) {
+            int ee[2] = {e0, e0 + C::CT};
+            float4 v[2], sp[2];
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+              v[k2] = make_float4(0.f, 0.f, 0.f, 0.f);
+              const int m = ee[k2] / d4, j = (ee[k2] - m * d4) * 4;
+              if (ee[k2] < tot && m < p.B) {
+                const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(p.x + (long long)m * p.d + j));
+                v[k2] = make_float4(bf_lo(raw.x), bf_hi(raw.x), bf_lo(raw.y), bf_hi(raw.y));
+              }
+            }
+            if (ph.src == SRC_XMID && nunits) {
+              const int m0 = ee[0] / d4, j0 = (ee[0] - m0 * d4) * 4;
+              const int m1 = ee[1] / d4, j1 = (ee[1] - m1 * d4) * 4;
+              const bool h0 = m0 < p.B, h1 = ee[1] < tot && m1 < p.B;
+              gather4x2(part_prev, utab + (h0 ? (j0 >> 6) : 0) * 16, m0 * 64 + (j0 & 63), nullptr,
+                        utab + (h1 ? (j1 >> 6) : 0) * 16, m1 * 64 + (j1 & 63), nullptr, h1, sp[0], sp[1]);
+  #pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+                const int m = ee[k2] / d4, j = (ee[k2] - m * d4) * 4;
+                if (ee[k2] >= tot || m >= p.B) continue;
+                add4(v[k2], sp[k2]);
+                v[k2] = round4(v[k2]);
+                if ((j >> 6) % G == g) {
+                  uint2 o;
+                  o.x = pack_bf2(v[k2].x, v[k2].y);
+                  o.y = pack_bf2(v[k2].z, v[k2].w);
+                  *reinterpret_cast<uint2*>(p.xm + (long long)m * p.d + j) = o;
+                }
+              }
+            }
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+              if (ee[k2] >= tot) continue;
+              const int m = ee[k2] / d4, j = (ee[k2] - m * d4) * 4;
+              *reinterpret_cast<float4*>(abuf + m * DF_ABUF_COLS + j) = v[k2];
+            }
+          }
+        } else if (ph.src == SRC_SWIGLU) {
+          // h = SiLU(gate) * up; a SwiGLU tile holds 32 gate then 32 up columns
+          const int tot = n * MT * 64;
+          for (int e = tid; e < tot; e += C::CT) {
+            const int i = (e & 63) * 4, m = (e >> 6) % MT, ci = (e >> 6) / MT;
+            const int k = (clist[ci] & 255) * DF_KC + i;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (m < p.B && k < ph.K && nunits) {
+              const short* u = utab + (ci * 8 + (i >> 5)) * 16;
+              float4 gv, uv;
+              gather4x2(part_prev, u, m * 64 + (k & 31), nullptr, u, m * 64 + (k & 31) + 32, nullptr, true, gv,
+                        uv);
+              v = round4(make_float4(gv.x / (1.f + expf(-gv.x)) * uv.x, gv.y / (1.f + expf(-gv.y)) * uv.y,
+                                     gv.z / (1.f + expf(-gv.z)) * uv.z, gv.w / (1.f + expf(-gv.w)) * uv.w));
+            }
+            *reinterpret_cast<float4*>(abuf + m * DF_ABUF_COLS + ci * 256 + i) = v;
+          }
+        } else if (ph.src == SRC_ATT) {
+          // attention output: dims k % D .. + 3 of head k / D of row m
+          const int tot = n * MT * 64;
+          for (int e = tid; e < tot; e += C::CT) {
+            const int i = (e & 63) * 4, m = (e >> 6) % MT, ci = (e >> 6) / MT;
+            const int k = (clist[ci] & 255) * DF_KC + i;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (m < p.B && k < ph.K && nunits)
+              v = round4(attn_gather4(part_prev, utab + ((ci * MT + m) * hpc + i / p.D) * 16, k % p.D));
+            *reinterpret_cast<float4*>(abuf + m * DF_ABUF_COLS + ci * 256 + i) = v;
+          }
+        } else {
+          // SRC_PART: fp32 rank activations z (plain column tiles of 64)
+          const int tot = n * nseg * MT * 64;
+          for (int e0 = tid; e0 < tot; e0 += 2 * C::CT) {
+            const short* uu[2];
+            const float* ww[2];
+            int idx[2], dst[2];
+            bool ok[2];
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+              const int e = e0 + k2 * C::CT;
+              const int i = (e & 63) * 4;
+              int rest = e >> 6;
+              const int m = rest % MT;
+              rest /= MT;
+              const int seg = rest % nseg, ci = rest / nseg;
+              const int kc = clist[ci < n ? ci : 0] & 255;
+              const int k = kc * DF_KC + i;
+              ok[k2] = e < tot && m < p.B && k < ph.K && nunits;
+              dst[k2] = e < tot ? m * DF_ABUF_COLS + ci * 256 * nseg + seg * 256 + i : -1;
+              uu[k2] = utab;
+              ww[k2] = nullptr;
+              idx[k2] = 0;
+              if (!ok[k2]) continue;
+              const int col = seg * ph.a_col2 + k, col0 = seg * ph.a_col2 + kc * DF_KC;
+              uu[k2] = utab + ((ci * nseg + seg) * 5 + (col >> 6) - (col0 >> 6)) * 16;
+              idx[k2] = m * 64 + (col & 63);
+            }
+            float4 sv[2];
+            if (ok[0] || ok[1]) {
+              const bool sw = !ok[0];  // keep the live group first
+              gather4x2(part_prev, uu[sw ? 1 : 0], idx[sw ? 1 : 0], ww[sw ? 1 : 0], uu[1], idx[1], ww[1],
+                        ok[0] && ok[1], sv[sw ? 1 : 0], sv[1]);
+            }
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+              if (dst[k2] < 0) continue;
+              *reinterpret_cast<float4*>(abuf + dst[k2]) = ok[k2] ? sv[k2] : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+          }
+        }
+        consumer_sync<C::CT>();
+        if (ph.norm) {
+          // rstd of each row of the stage input
+          for (int m = 0; m < MT; ++m) {
+            float ss = 0.f;
+            for (int j = tid; j < p.d; j += C::CT) {
+              const float v = abuf[m * DF_ABUF_COLS + j];
+              ss = fmaf(v, v, ss);
+            }
+            ss = warp_sum(ss);
+            if (lane == 0) red[warp * MT + m] = ss;
+          }
+          consumer_sync<C::CT>();
+          if (tid < MT) {
+            float ss = 0.f;
+#pragma unroll
+            for (int w = 0; w < C::CW; ++w) ss += red[w * MT + tid];
+            s_rstd[tid] = rsqrtf(ss / (float)p.d + p.eps);
+          }
+          consumer_sync<C::CT>();
+          // the normalized input x * (rstd * g), once for all entries
+          for (int e = tid; e < MT * (p.d >> 2); e += C::CT) {
+            const int m = e / (p.d >> 2), j = (e - m * (p.d >> 2)) * 4;
+            const uint2 gr = __ldg(reinterpret_cast<const uint2*>(ph.norm_g + j));
+            const float r = s_rstd[m];
+            float4* a4 = reinterpret_cast<float4*>(abuf + m * DF_ABUF_COLS + j);
+            float4 v = *a4;
+            v.x *= r * bf_lo(gr.x); v.y *= r * bf_hi(gr.x); v.z *= r * bf_lo(gr.y); v.w *= r * bf_hi(gr.y);
+            *a4 = v;
+          }
+          consumer_sync<C::CT>();
+        }
+
+        // ---- entries ----
         float acc[MT][8];
 #pragma unroll
         for (int m = 0; m < MT; ++m)
 #pragma unroll
           for (int j = 0; j < 8; ++j) acc[m][j] = 0.f;
         int su = 0;
-        const int t_first = c0 / (ph.nk > 0 ? ph.nk : 1);
         for (int c = c0; c < c1; ++c, ++seq) {
           const int slot = seq % C::NSLOT;
           const uint32_t par = (uint32_t)(seq / C::NSLOT) & 1u;
@@ -449,47 +721,19 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
           const int t = c / ph.nk, kc = c - t * ph.nk;
           const int k0 = kc * DF_KC;
           const int kn = min(DF_KC, ph.K - k0);
-          if (ph.pro == PRO_RMSNORM && c == c0) {
-            // rstd of each row of x (the stage's input, complete after the barrier)
-            const bf16* xb = reinterpret_cast<const bf16*>(ph.a);
-            for (int m = 0; m < MT; ++m) {
-              float ss = 0.f;
-              if (m < p.B)
-                for (int col = tid * 8; col < ph.K; col += C::CT * 8) {
-                  const uint4 u = __ldcg(reinterpret_cast<const uint4*>(xb + (long long)m * ph.lda + col));
-                  const float v[8] = {bf_lo(u.x), bf_hi(u.x), bf_lo(u.y), bf_hi(u.y),
-                                      bf_lo(u.z), bf_hi(u.z), bf_lo(u.w), bf_hi(u.w)};
-#pragma unroll
-                  for (int j = 0; j < 8; ++j) ss = fmaf(v[j], v[j], ss);
-                }
-              ss = warp_sum(ss);
-              if (lane == 0) red[warp * MT + m] = ss;
-            }
-            consumer_sync<C::CT>();
-            if (tid < MT) {
-              float ss = 0.f;
-#pragma unroll
-              for (int w = 0; w < C::CW; ++w) ss += red[w * MT + tid];
-              s_rstd[tid] = rsqrtf(ss / (float)ph.K + p.eps);
-            }
-            consumer_sync<C::CT>();
+          const uint8_t* w = slots + slot * C::SLOT + box * 16384 + chunk * 16;
+          if (ph.norm) {
+            entry_mac<MT, 0, RSTEP>(acc, w, abuf + k0, kn, row0, nullptr, s_rstd);
+          } else {
+            const int off = srec->chunk_of[c - c0] * 256 * nseg + (nseg == 2 ? box * 256 : 0);
+            entry_mac<MT, 0, RSTEP>(acc, w, abuf + off, kn, row0, nullptr, s_rstd);
           }
-          const uint8_t* w = slots + slot * C::SLOT + hi * 16384 + (cg & 3) * 16;
-          const uint8_t* a_s = slots + slot * C::SLOT + C::W_BYTES;
-          if (ph.pro == PRO_RMSNORM)
-            entry_mac<MT, 1, 0, RSTEP>(acc, w, a_s, 0, kn, row0, ph.norm_g + k0, s_rstd);
-          else if (!ph.a_f32)
-            entry_mac<MT, 0, 0, RSTEP>(acc, w, a_s, 0, kn, row0, nullptr, s_rstd);
-          else
-            entry_mac<MT, 0, 1, RSTEP>(acc, w, a_s, (ph.map == MAP_SWIGLU) ? hi : 0, kn, row0, nullptr,
-                                       s_rstd);
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(empty + slot);
 
           const bool tile_end = (c == c1 - 1) || (kc == ph.nk - 1);
           if (!tile_end) continue;
-
-          // ---- finish this CTA's part of tile t ----
+          // ---- this CTA's partial of tile t ----
 #pragma unroll
           for (int m = 0; m < MT; ++m)
 #pragma unroll
@@ -501,143 +745,98 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
               if ((lane & 20) == 0) red[(warp * MT + m) * 64 + cg * 8 + j] = v;
             }
           consumer_sync<C::CT>();
-          constexpr int NOUT = MT * 64;
-          const int e_first = t * ph.nk, e_last = min(Ctot - 1, t * ph.nk + ph.nk - 1);
-          const int gf = owner_of(e_first, Ctot, G);
-          const int gl = owner_of(e_last, Ctot, G);
-          (void)gl;
-          float* mypart = p.part + ((long long)g * DF_MAX_SU + (su < DF_MAX_SU ? su : DF_MAX_SU - 1)) *
-                                       DF_PART_STRIDE;
-          for (int o = tid; o < NOUT; o += C::CT) {
-            float s = 0.f;
+          float* ps = su < DF_MAX_SU ? part_cur + ((long long)g * DF_MAX_SU + su) * DF_PART_STRIDE : nullptr;
+          if (!ps && tid == 0) atomicExch(p.status, DEV_STATUS_SCHEDULE);
+          for (int o = tid; o < MT * 64; o += C::CT) {
+            float v = 0.f;
 #pragma unroll
-            for (int w8 = 0; w8 < C::CW; ++w8) s += red[(w8 * MT + (o >> 6)) * 64 + (o & 63)];
-            if (gf == gl) scr[o] = s;
-            else __stcg(mypart + o, s);
-          }
-          bool run_epi = true;
-          if (gf != gl) {
-            __threadfence();
-            consumer_sync<C::CT>();
-            if (tid == 0)
-              *s_flag = (atomicAdd(p.tilecnt + t, 1) == count_owners(e_first, e_last, Ctot, G) - 1);
-            consumer_sync<C::CT>();
-            run_epi = *s_flag != 0;
-            if (run_epi) {
-              __threadfence();
-              // SPL threads per output each sum a fixed stride of the
-              // contributing CTAs; the SPL sums are added in fixed order.
-              constexpr int SPL = C::CT / NOUT > 1 ? C::CT / NOUT : 1;
-              const int o = tid % NOUT, sub = tid / NOUT;
-              float sacc = 0.f;
-              if (sub < SPL)
-                for (int gg = gf + sub; gg <= gl; gg += SPL) {
-                  if (Ctot < G && !share_nonempty(Ctot, G, gg)) continue;
-                  const int c0g = gg * Ctot / G;
-                  int sug = t - c0g / ph.nk;
-                  sug = sug < DF_MAX_SU ? sug : DF_MAX_SU - 1;
-                  sacc += __ldcg(p.part + ((long long)gg * DF_MAX_SU + sug) * DF_PART_STRIDE + o);
-                }
-              if (SPL > 1) {
-                if (sub < SPL) red[sub * NOUT + o] = sacc;
-                consumer_sync<C::CT>();
-                if (tid < NOUT) {
-                  float tot = 0.f;
-#pragma unroll
-                  for (int k2 = 0; k2 < SPL; ++k2) tot += red[k2 * NOUT + tid];
-                  scr[tid] = tot;
-                }
-              } else {
-                for (int o2 = tid; o2 < NOUT; o2 += C::CT) {
-                  float tot = 0.f;
-                  for (int gg = gf; gg <= gl; ++gg) {
-                    if (Ctot < G && !share_nonempty(Ctot, G, gg)) continue;
-                    const int c0g = gg * Ctot / G;
-                    int sug = t - c0g / ph.nk;
-                    sug = sug < DF_MAX_SU ? sug : DF_MAX_SU - 1;
-                    tot += __ldcg(p.part + ((long long)gg * DF_MAX_SU + sug) * DF_PART_STRIDE + o2);
-                  }
-                  scr[o2] = tot;
-                }
-              }
-              if (tid == 0) p.tilecnt[t] = 0;
-            }
-          }
-          consumer_sync<C::CT>();
-          if (run_epi) {
-            int pi = 0;
-            for (int i = 1; i < 3; ++i)
-              if (i < ph.nprob && t >= ph.tile_start[i]) pi = i;
-            const int tl = t - ph.tile_start[pi];
-            const int Np = ph.N[pi];
-            if (ph.epi == EPI_F32 || ph.epi == EPI_BF16) {
-              for (int o = tid; o < NOUT; o += C::CT) {
-                const int m = o >> 6, cc = o & 63;
-                const int gc = out_col(ph, p.D, tl, cc);
-                if (m >= p.B || gc >= Np) continue;
-                float v = scr[o];
-                if (ph.epi == EPI_F32) {
-                  ph.out32[(long long)m * ph.ldo32 + ph.out_col[pi] + gc] = v;
-                } else {
-                  if (ph.resid) v += bf2f(__ldcg(ph.resid + (long long)m * ph.ldr + gc));
-                  ph.out16[(long long)m * ph.ldo16 + gc] = f2bf(v);
-                }
-              }
-            } else if (ph.epi == EPI_QKV) {
-              const int half = p.D >> 1;
-              const int kind = ph.kind[pi];
-              for (int o = tid; o < MT * 32; o += C::CT) {
-                const int m = o >> 5, cc = o & 31;
-                if (m >= p.B) continue;
-                int pos = p.seqlens[m];
-                pos = pos < 0 ? 0 : (pos >= p.S_max ? p.S_max - 1 : pos);
-                const int glo = out_col(ph, p.D, tl, cc);
-                const int i = glo % p.D;
-                float lo = scr[m * 64 + cc], hv = scr[m * 64 + cc + 32];
-                if (kind < 2) {
-                  const float cs = p.rope_cos[(long long)pos * half + i];
-                  const float sn = p.rope_sin[(long long)pos * half + i];
-                  const float l2 = lo * cs - hv * sn;
-                  hv = hv * cs + lo * sn;
-                  lo = l2;
-                }
-                bf16* dst;
-                if (kind == 0) dst = ph.out16 + (long long)m * ph.ldo16;
-                else dst = (kind == 1 ? p.k_cache : p.v_cache) + ((long long)m * p.S_max + pos) * (p.H * p.D);
-                dst[glo] = f2bf(lo);
-                dst[glo + half] = f2bf(hv);
-              }
-            } else {  // EPI_SWIGLU
-              for (int o = tid; o < MT * 32; o += C::CT) {
-                const int m = o >> 5, cc = o & 31;
-                const int fc = 32 * tl + cc;
-                if (m >= p.B || fc >= Np) continue;
-                const float gv = scr[m * 64 + cc], uv = scr[m * 64 + cc + 32];
-                ph.out16[(long long)m * ph.ldo16 + fc] = f2bf(gv / (1.f + expf(-gv)) * uv);
-              }
-            }
+            for (int w8 = 0; w8 < C::CW; ++w8) v += red[(w8 * MT + (o >> 6)) * 64 + (o & 63)];
+            if (ps) __stcg(ps + o, v);
           }
           consumer_sync<C::CT>();
           ++su;
-          (void)t_first;
         }
       } else {
         // ---------------------------------------------- attention stage --
-        // Each consumer warp owns 64 / CW keys of every 64-key entry and keeps
-        // its own online-softmax state (m, l, o) over all entries of a
-        // (batch, head) pair; lanes own D / 32 dimensions.  Warps merge once
-        // per pair, then CTAs merge through the partial slots.
         AttnSched s;
         attn_sched(p, s);
         const int Ctot = s.pre[8];
         int c0, c1;
         share(Ctot, G, g, c0, c1);
-        const int D = p.D;
-        const int EPL = D >> 5;               // 4 (D = 128) or 2 (D = 64)
-        constexpr int KPW = 64 / C::CW;       // keys per warp per entry
-        float* wm = scr;                      // [CW]      warp m
-        float* wl = scr + 32;                 // [CW]      warp l
-        float* wo = scr + 64;                 // [CW][128] warp o
+        const int D = p.D, hd = D >> 1, tph = D >> 6;
+        int pf = 0, np = 0;
+        if (c0 < c1) {
+          int b0, h0, k0, b1, h1, k1;
+          attn_entry(s, c0, b0, h0, k0);
+          attn_entry(s, c1 - 1, b1, h1, k1);
+          pf = b0 * p.H + h0;
+          np = b1 * p.H + h1 - pf + 1;
+        }
+        if (np > DF_MAX_PAIRS) {
+          if (tid == 0) atomicExch(p.status, DEV_STATUS_SCHEDULE);
+          np = DF_MAX_PAIRS;
+        }
+        // q, k, v of this CTA's (batch, head) pairs from the stage-1 partials:
+        // RoPE on q and k at the row's position, bf16 rounding as the cache
+        // stores them.  The owner of a pair's last key chunk appends k, v.
+        float* qkv = abuf;  // [np][3][D]
+        {
+          const DfPhase& q1 = s_ph[ph_i - 1];
+          const int nunits = np * 3 * tph;  // one per stage-1 tile: (pair, q/k/v, tile of the head)
+          for (int ui = tid; ui < nunits; ui += C::CT) {
+            const int j = ui % tph, r2 = ui / tph, prob = r2 % 3, pair = pf + r2 / 3;
+            const int h = pair % p.H;
+            if (!tile_slots(q1, q1.tile_start[prob] + h * tph + j, G, utab + ui * 16))
+              atomicExch(p.status, DEV_STATUS_SCHEDULE);
+          }
+          if (tid == 0) grid_wait(p.bar + ph_i - 1, G, abort_flag, p.status);
+          consumer_sync<C::CT>();
+          for (int e = tid; e < np * 3 * (hd >> 2); e += C::CT) {
+            const int i = (e % (hd >> 2)) * 4;
+            const int r2 = e / (hd >> 2);
+            const int prob = r2 % 3, pr = r2 / 3;
+            const int pair = pf + pr, b = pair / p.H, h = pair - b * p.H;
+            const int pos = s.L[b] - 1;
+            const short* u = utab + (r2 * tph + (i >> 5)) * 16;
+            float4 lo, hi;
+            gather4x2(part_prev, u, b * 64 + (i & 31), nullptr, u, b * 64 + (i & 31) + 32, nullptr, true, lo, hi);
+            if (prob < 2) {
+              const float4 cs = *reinterpret_cast<const float4*>(p.rope_cos + (long long)pos * hd + i);
+              const float4 sn = *reinterpret_cast<const float4*>(p.rope_sin + (long long)pos * hd + i);
+              const float4 l2 = make_float4(lo.x * cs.x - hi.x * sn.x, lo.y * cs.y - hi.y * sn.y,
+                                            lo.z * cs.z - hi.z * sn.z, lo.w * cs.w - hi.w * sn.w);
+              hi = make_float4(hi.x * cs.x + lo.x * sn.x, hi.y * cs.y + lo.y * sn.y, hi.z * cs.z + lo.z * sn.z,
+                               hi.w * cs.w + lo.w * sn.w);
+              lo = l2;
+            }
+            lo = round4(lo);
+            hi = round4(hi);
+            *reinterpret_cast<float4*>(qkv + (pr * 3 + prob) * D + i) = lo;
+            *reinterpret_cast<float4*>(qkv + (pr * 3 + prob) * D + i + hd) = hi;
+            if (prob > 0 && owner_of(s.pre[b] + h * s.nk[b] + s.nk[b] - 1, Ctot, G) == g) {
+              bf16* dst = (prob == 1 ? p.k_cache : p.v_cache) + ((long long)b * p.S_max + pos) * (p.H * D) +
+                          h * D;
+              uint2 o;
+              o.x = pack_bf2(lo.x, lo.y); o.y = pack_bf2(lo.z, lo.w);
+              *reinterpret_cast<uint2*>(dst + i) = o;
+              o.x = pack_bf2(hi.x, hi.y); o.y = pack_bf2(hi.z, hi.w);
+              *reinterpret_cast<uint2*>(dst + i + hd) = o;
+            }
+          }
+        }
+        consumer_sync<C::CT>();
+
+        // Each consumer warp owns 64 / CW keys of every 64-key entry and keeps
+        // its own online-softmax state (m, l, o) over all entries of a pair;
+        // lanes own D / 32 dimensions.  The key at the current position comes
+        // from qkv (its cache row may not be written yet).
+        const int EPL = D >> 5;
+        constexpr int KPW = 64 / C::CW;
+        float* wm = scr;       // [CW]
+        float* wl = scr + 32;  // [CW]
+        float* wo = scr + 64;  // [CW][128]
+        const int d0 = lane * EPL;
+        const int bx = d0 >> 6, ch = (d0 & 63) >> 3, sub = (d0 & 7) * 2;
         float qv[4] = {0.f, 0.f, 0.f, 0.f};
         float m_w = -INFINITY, l_w = 0.f;
         float ov[4] = {0.f, 0.f, 0.f, 0.f};
@@ -645,48 +844,53 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
         for (int c = c0; c < c1; ++c, ++seq) {
           int b, h, kc;
           attn_entry(s, c, b, h, kc);
-          const int pair_first = s.pre[b] + h * s.nk[b];
-          const int pair_last = pair_first + s.nk[b] - 1;
+          int pr = b * p.H + h - pf;
+          pr = pr < np ? pr : np - 1;  // only past the schedule limit (flagged above)
+          const int pair_last = s.pre[b] + h * s.nk[b] + s.nk[b] - 1;
           const int slot = seq % C::NSLOT;
           const uint32_t par = (uint32_t)(seq / C::NSLOT) & 1u;
           tc::mbar_wait(full + slot, par, abort_flag, p.status);  // on abort: run on, results discarded
+          const float* qn = qkv + pr * 3 * D + d0;
           if (c == c0 || kc == 0) {
-            m_w = -INFINITY; l_w = 0.f;
+            m_w = -INFINITY;
+            l_w = 0.f;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) ov[e] = 0.f;
-            const bf16* qp = p.q + ((long long)b * p.H + h) * D + lane * EPL;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) qv[e] = e < EPL ? bf2f(__ldcg(qp + e)) * p.scale_log2 : 0.f;
+            for (int e = 0; e < 4; ++e) {
+              ov[e] = 0.f;
+              qv[e] = e < EPL ? qn[e] * p.scale_log2 : 0.f;
+            }
           }
+          const int L = s.L[b], pos = L - 1;
           const uint8_t* kb = slots + slot * C::SLOT;
           const uint8_t* vb = kb + 16384;
-          // this lane's dims: d0 = lane * EPL .. + EPL (one 8- or 4-byte piece)
-          const int d0 = lane * EPL;
-          const int bx = d0 >> 6, ch = (d0 & 63) >> 3, sub = (d0 & 7) * 2;
-          float sc4[KPW];
+          float sc[KPW];
 #pragma unroll
           for (int i = 0; i < KPW; ++i) {
             const int j = warp * KPW + i;
-            const uint8_t* kp = kb + bx * 8192 + j * 128 + ((ch ^ (j & 7)) << 4) + sub;
             float dot = 0.f;
-            if (EPL == 4) {
-              const uint2 u = *reinterpret_cast<const uint2*>(kp);
-              dot = qv[0] * bf_lo(u.x) + qv[1] * bf_hi(u.x) + qv[2] * bf_lo(u.y) + qv[3] * bf_hi(u.y);
+            if (kc * 64 + j == pos) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                if (e < EPL) dot = fmaf(qv[e], qn[D + e], dot);
             } else {
-              const uint32_t u = *reinterpret_cast<const uint32_t*>(kp);
-              dot = qv[0] * bf_lo(u) + qv[1] * bf_hi(u);
+              const uint8_t* kp = kb + bx * 8192 + j * 128 + ((ch ^ (j & 7)) << 4) + sub;
+              if (EPL == 4) {
+                const uint2 u = *reinterpret_cast<const uint2*>(kp);
+                dot = qv[0] * bf_lo(u.x) + qv[1] * bf_hi(u.x) + qv[2] * bf_lo(u.y) + qv[3] * bf_hi(u.y);
+              } else {
+                const uint32_t u = *reinterpret_cast<const uint32_t*>(kp);
+                dot = qv[0] * bf_lo(u) + qv[1] * bf_hi(u);
+              }
             }
-            sc4[i] = dot;
+            sc[i] = dot;
           }
+          float mb = -INFINITY;
 #pragma unroll
           for (int i = 0; i < KPW; ++i) {
-            sc4[i] = warp_sum(sc4[i]);
-            const int key = kc * 64 + warp * KPW + i;
-            if (key >= s.L[b]) sc4[i] = -INFINITY;
+            sc[i] = warp_sum(sc[i]);
+            if (kc * 64 + warp * KPW + i >= L) sc[i] = -INFINITY;
+            mb = fmaxf(mb, sc[i]);
           }
-          float mb = sc4[0];
-#pragma unroll
-          for (int i = 1; i < KPW; ++i) mb = fmaxf(mb, sc4[i]);
           const float mn = fmaxf(m_w, mb);
           if (mn != -INFINITY) {
             const float corr = (m_w == -INFINITY) ? 0.f : exp2f(m_w - mn);
@@ -695,17 +899,23 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
             for (int e = 0; e < 4; ++e) ov[e] *= corr;
 #pragma unroll
             for (int i = 0; i < KPW; ++i) {
-              const float pj = (sc4[i] == -INFINITY) ? 0.f : exp2f(sc4[i] - mn);
+              const float pj = (sc[i] == -INFINITY) ? 0.f : exp2f(sc[i] - mn);
               l_w += pj;
               const int j = warp * KPW + i;
-              const uint8_t* vp = vb + bx * 8192 + j * 128 + ((ch ^ (j & 7)) << 4) + sub;
-              if (EPL == 4) {
-                const uint2 u = *reinterpret_cast<const uint2*>(vp);
-                ov[0] = fmaf(pj, bf_lo(u.x), ov[0]); ov[1] = fmaf(pj, bf_hi(u.x), ov[1]);
-                ov[2] = fmaf(pj, bf_lo(u.y), ov[2]); ov[3] = fmaf(pj, bf_hi(u.y), ov[3]);
+              if (kc * 64 + j == pos) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  if (e < EPL) ov[e] = fmaf(pj, qn[2 * D + e], ov[e]);
               } else {
-                const uint32_t u = *reinterpret_cast<const uint32_t*>(vp);
-                ov[0] = fmaf(pj, bf_lo(u), ov[0]); ov[1] = fmaf(pj, bf_hi(u), ov[1]);
+                const uint8_t* vp = vb + bx * 8192 + j * 128 + ((ch ^ (j & 7)) << 4) + sub;
+                if (EPL == 4) {
+                  const uint2 u = *reinterpret_cast<const uint2*>(vp);
+                  ov[0] = fmaf(pj, bf_lo(u.x), ov[0]); ov[1] = fmaf(pj, bf_hi(u.x), ov[1]);
+                  ov[2] = fmaf(pj, bf_lo(u.y), ov[2]); ov[3] = fmaf(pj, bf_hi(u.y), ov[3]);
+                } else {
+                  const uint32_t u = *reinterpret_cast<const uint32_t*>(vp);
+                  ov[0] = fmaf(pj, bf_lo(u), ov[0]); ov[1] = fmaf(pj, bf_hi(u), ov[1]);
+                }
               }
             }
             m_w = mn;
@@ -713,13 +923,12 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(empty + slot);
 
-          const bool pair_end = (c == c1 - 1) || (c == pair_last);
-          if (!pair_end) continue;
-          // ---- merge the warps of this CTA for pair (b, h) ----
+          if (c != c1 - 1 && c != pair_last) continue;
+          // ---- merge the warps; write this CTA's (m, l, o) partial of the pair ----
           if (lane == 0) { wm[warp] = m_w; wl[warp] = l_w; }
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            if (e < EPL) wo[warp * 128 + lane * EPL + e] = ov[e];
+            if (e < EPL) wo[warp * 128 + d0 + e] = ov[e];
           consumer_sync<C::CT>();
           float Mc = -INFINITY;
 #pragma unroll
@@ -731,87 +940,48 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
             Lc += wgt * wl[w2];
             if (tid < D) oc += wgt * wo[w2 * 128 + tid];
           }
-          const int pair = b * p.H + h;
-          const int gf = owner_of(pair_first, Ctot, G), gl = owner_of(pair_last, Ctot, G);
-          float* mypart = p.part + ((long long)g * DF_MAX_SU + (su < DF_MAX_SU ? su : DF_MAX_SU - 1)) *
-                                       DF_PART_STRIDE;
-          if (gf == gl) {
-            if (tid < D) p.att[((long long)b * p.H + h) * D + tid] = f2bf(oc / Lc);
-          } else {
-            if (tid < D) __stcg(mypart + 2 + tid, oc);
-            if (tid == 0) { __stcg(mypart, Mc); __stcg(mypart + 1, Lc); }
-            __threadfence();
-            consumer_sync<C::CT>();
-            if (tid == 0)
-              *s_flag = (atomicAdd(p.tilecnt + pair, 1) == count_owners(pair_first, pair_last, Ctot, G) - 1);
-            consumer_sync<C::CT>();
-            if (*s_flag) {
-              __threadfence();
-              float* cm = scr + 64 + C::CW * 128;   // [32] contributor m
-              float* cl = cm + 32;                   // [32] contributor l
-              int* cs = reinterpret_cast<int*>(cl + 32);  // [33] slot index, count
-              if (tid == 0) {
-                int n = 0;
-                for (int gg = gf; gg <= gl && n < 32; ++gg) {
-                  if (Ctot < G && !share_nonempty(Ctot, G, gg)) continue;
-                  const int c0g = gg * Ctot / G;
-                  int b2, h2, k2;
-                  attn_entry(s, c0g, b2, h2, k2);
-                  int sug = pair - (b2 * p.H + h2);
-                  sug = sug < DF_MAX_SU ? sug : DF_MAX_SU - 1;
-                  cs[n++] = gg * DF_MAX_SU + sug;
-                }
-                cs[32] = n;
-              }
-              consumer_sync<C::CT>();
-              const int ncon = cs[32];
-              if (tid < ncon) {
-                const float* pp = p.part + (long long)cs[tid] * DF_PART_STRIDE;
-                cm[tid] = __ldcg(pp);
-                cl[tid] = __ldcg(pp + 1);
-              }
-              consumer_sync<C::CT>();
-              float Mg = -INFINITY;
-              for (int k2 = 0; k2 < ncon; ++k2) Mg = fmaxf(Mg, cm[k2]);
-              float Lg = 0.f;
-              for (int k2 = 0; k2 < ncon; ++k2)
-                Lg += (cm[k2] == -INFINITY) ? 0.f : exp2f(cm[k2] - Mg) * cl[k2];
-              float* oh = scr + 64;  // reuse the warp-o area: [CT / D][D]
-              {
-                const int KG2 = C::CT / D;
-                const int dd = tid % D, kg = tid / D;
-                float oo = 0.f;
-                for (int k2 = kg; k2 < ncon; k2 += KG2) {
-                  const float wgt = (cm[k2] == -INFINITY) ? 0.f : exp2f(cm[k2] - Mg);
-                  oo += wgt * __ldcg(p.part + (long long)cs[k2] * DF_PART_STRIDE + 2 + dd);
-                }
-                oh[kg * D + dd] = oo;
-              }
-              consumer_sync<C::CT>();
-              if (tid < D) {
-                float o = 0.f;
-                for (int k2 = 0; k2 < C::CT / D; ++k2) o += oh[k2 * D + tid];
-                p.att[((long long)b * p.H + h) * D + tid] = f2bf(o / Lg);
-              }
-              if (tid == 0) p.tilecnt[pair] = 0;
-            }
+          float* ps = su < DF_MAX_SU ? part_cur + ((long long)g * DF_MAX_SU + su) * DF_PART_STRIDE : nullptr;
+          if (ps) {
+            if (tid < D) __stcg(ps + 4 + tid, oc);
+            if (tid == 0) { __stcg(ps, Mc); __stcg(ps + 1, Lc); }
+          } else if (tid == 0) {
+            atomicExch(p.status, DEV_STATUS_SCHEDULE);
           }
           consumer_sync<C::CT>();
           ++su;
         }
       }
       // ---- this CTA is done with stage ph_i ----
-      // Stores of this stage must be visible to the next stage's TMA / bulk
-      // copies (async proxy) issued by other CTAs.
-      asm volatile("fence.proxy.async.global;" ::: "memory");
       consumer_sync<C::CT>();
-      if (tid == 0) {
-        __threadfence();
-        red_release_add(p.bar + ph_i, 1);
+      // (the CTA barrier above orders every consumer's writes before this
+      // thread's release, which is cumulative over them)
+      if (tid == 0) red_release_add(p.bar + ph_i, 1);
+    }
+    // ---- final pass: x = x' + z V_dn for this CTA's 64-column tiles ----
+    if (tid == 0) grid_wait(p.bar + DF_NPHASE - 1, G, abort_flag, p.status);
+    consumer_sync<C::CT>();
+    {
+      const float* part8 = p.part + ((DF_NPHASE - 1) & 1) * half;
+      // record DF_NPHASE: tiles g, g + G, ... of the last stage
+      const int4* src = reinterpret_cast<const int4*>(p.sched + (long long)DF_NPHASE * G + g);
+      for (int w = tid; w < (int)(sizeof(SchedRec) / 16); w += C::CT) reinterpret_cast<int4*>(srec)[w] = __ldg(src + w);
+      consumer_sync<C::CT>();
+      const int nt = srec->nunits;
+      for (int e = tid; e < min(nt, DF_MAX_UNITS) * p.B * 16; e += C::CT) {
+        const int c4 = (e & 15) * 4, m = (e >> 4) % p.B, ui = (e >> 4) / p.B;
+        const long long o = (long long)m * p.d + (g + ui * G) * 64 + c4;
+        const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(p.xm + o));
+        float4 v = make_float4(bf_lo(raw.x), bf_hi(raw.x), bf_lo(raw.y), bf_hi(raw.y));
+        float4 sp, unused;
+        gather4x2(part8, utab + ui * 16, m * 64 + c4, nullptr, utab, 0, nullptr, false, sp, unused);
+        add4(v, sp);
+        uint2 w;
+        w.x = pack_bf2(v.x, v.y);
+        w.y = pack_bf2(v.z, v.w);
+        *reinterpret_cast<uint2*>(p.x + o) = w;
       }
     }
   }
-
   __syncthreads();
   if (tid == 0) {
     // The last CTA to finish resets the stage counters for the next launch.
@@ -823,6 +993,11 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
     }
   }
 }
+
+}  // namespace
+
+
+namespace {
 
 // ------------------------------------------------------------ the pack --
 // Entry (t, kc) of a stage -- rows [256 kc, 256 kc + kn) of column tile t --
@@ -886,25 +1061,18 @@ __global__ void __launch_bounds__(256) decode_pack_kernel(const __grid_constant_
   }
 }
 
-}  // namespace
 
 // ------------------------------------------------------------------ host --
 
-int decode_fused_supported(int B, int d, int D, int r, int r_f) {
-  return B >= 1 && B <= 8 && (D == 64 || D == 128) && d % 64 == 0 && r % 8 == 0 && r_f % 8 == 0;
-}
-
-// Stage table of one fused decode layer.  Activation pointers may be null
-// (when only the pack layout is wanted); Q, if given, receives each stage's
+// Stage table of one fused decode layer; Q, if given, receives each stage's
 // factor sources for the pack kernel.  Returns the pack size in bytes.
-long long build_stages(const DecodeLayerDesc& L, bf16* x, bf16* qbuf, const bf16* att, bf16* hbuf,
-                       float* z, DfPhase* P, PackStage* Q) {
+long long build_stages(const DecodeLayerDesc& L, DfPhase* P, PackStage* Q) {
   const int d = L.d, r = L.r, rf = L.r_f, f = L.f;
   memset(P, 0, sizeof(DfPhase) * DF_NPHASE);
   long long off = 0;
-  auto gemv = [&](int i, int pro, int epi, int map, int K, const bf16* const* src, const long long* ld) {
+  auto gemv = [&](int i, int map, int src, int K, const bf16* const* srcm, const long long* ld) {
     DfPhase& ph = P[i];
-    ph.type = DF_GEMV; ph.pro = pro; ph.epi = epi; ph.map = map; ph.K = K;
+    ph.type = DF_GEMV; ph.map = map; ph.src = src; ph.K = K;
     ph.nk = ceil_div(K, DF_KC);
     int T = 0;
     for (int j = 0; j < ph.nprob; ++j) {
@@ -916,56 +1084,163 @@ long long build_stages(const DecodeLayerDesc& L, bf16* x, bf16* qbuf, const bf16
     ph.pack_off = off;
     if (Q) {
       PackStage& q = Q[i];
-      q.off = off; q.K = K; q.T = T; q.map = map; q.nprob = ph.nprob; q.w_row2 = ph.w_row2;
+      q.off = off; q.K = K; q.T = T; q.map = map; q.nprob = ph.nprob;
+      q.w_row2 = map == MAP_SWIGLU ? rf : 0;
       for (int j = 0; j < 4; ++j) q.tile_start[j] = ph.tile_start[j];
-      for (int j = 0; j < ph.nprob; ++j) { q.N[j] = ph.N[j]; q.src[j] = src[j]; q.ld[j] = ld[j]; }
+      for (int j = 0; j < ph.nprob; ++j) { q.N[j] = ph.N[j]; q.src[j] = srcm[j]; q.ld[j] = ld[j]; }
     }
     off += (long long)T * K * 128;
   };
   // 0: z_qkv = rmsnorm(x) . [U_q | U_k | U_v]
-  P[0].nprob = 3;
-  for (int i = 0; i < 3; ++i) { P[0].N[i] = r; P[0].out_col[i] = i * r; }
-  P[0].a = x; P[0].a_f32 = 0; P[0].lda = d; P[0].norm_g = L.g1;
-  P[0].out32 = z; P[0].ldo32 = 3 * r;
-  { const long long ld[3] = {r, r, r}; gemv(0, PRO_RMSNORM, EPI_F32, MAP_PLAIN, d, L.U, ld); }
-  // 1: q, k, v = z . V  (+ RoPE; k, v appended at cache_seqlens)
+  P[0].nprob = 3; P[0].norm = 1; P[0].norm_g = L.g1;
+  for (int i = 0; i < 3; ++i) P[0].N[i] = r;
+  { const long long ld[3] = {r, r, r}; gemv(0, MAP_PLAIN, SRC_X, d, L.U, ld); }
+  // 1: q, k, v = z . V  (RoPE applied by the readers)
   P[1].nprob = 3;
-  for (int i = 0; i < 3; ++i) { P[1].N[i] = d; P[1].a_col[i] = i * r; P[1].kind[i] = i; }
-  P[1].a = z; P[1].a_f32 = 1; P[1].lda = 3 * r;
-  P[1].out16 = qbuf; P[1].ldo16 = d;
-  { const long long ld[3] = {d, d, d}; gemv(1, PRO_F32, EPI_QKV, MAP_ROPE, r, L.V, ld); }
+  for (int i = 0; i < 3; ++i) P[1].N[i] = d;
+  { const long long ld[3] = {d, d, d}; gemv(1, MAP_ROPE, SRC_PART, r, L.V, ld); }
   // 2: attention
   P[2].type = DF_ATTN;
+  P[2].pack_off = off;
   // 3: z = att . U_o
   P[3].nprob = 1; P[3].N[0] = r;
-  P[3].a = att; P[3].a_f32 = 0; P[3].lda = d; P[3].out32 = z; P[3].ldo32 = r;
-  { const long long ld[1] = {r}; gemv(3, PRO_BF16, EPI_F32, MAP_PLAIN, d, &L.U_o, ld); }
-  // 4: x += z . V_o
+  { const long long ld[1] = {r}; gemv(3, MAP_PLAIN, SRC_ATT, d, &L.U_o, ld); }
+  // 4: x' = x + z . V_o  (residual added by the readers)
   P[4].nprob = 1; P[4].N[0] = d;
-  P[4].a = z; P[4].a_f32 = 1; P[4].lda = r; P[4].out16 = x; P[4].ldo16 = d; P[4].resid = x; P[4].ldr = d;
-  { const long long ld[1] = {d}; gemv(4, PRO_F32, EPI_BF16, MAP_PLAIN, r, &L.V_o, ld); }
-  // 5: z = rmsnorm(x) . U_gu
-  P[5].nprob = 1; P[5].N[0] = 2 * rf;
-  P[5].a = x; P[5].a_f32 = 0; P[5].lda = d; P[5].norm_g = L.g2; P[5].out32 = z; P[5].ldo32 = 2 * rf;
-  { const long long ld[1] = {2 * rf}; gemv(5, PRO_RMSNORM, EPI_F32, MAP_PLAIN, d, &L.U_gu, ld); }
-  // 6: h = SiLU(z_g V_g) * (z_u V_u)
-  P[6].nprob = 1; P[6].N[0] = f; P[6].a_col[0] = 0; P[6].a_col2 = rf; P[6].w_row2 = rf;
-  P[6].a = z; P[6].a_f32 = 1; P[6].lda = 2 * rf; P[6].out16 = hbuf; P[6].ldo16 = f;
-  { const long long ld[1] = {f}; gemv(6, PRO_F32, EPI_SWIGLU, MAP_SWIGLU, rf, &L.V_gu, ld); }
-  // 7: z = h . U_dn
+  { const long long ld[1] = {d}; gemv(4, MAP_PLAIN, SRC_PART, r, &L.V_o, ld); }
+  // 5: z = rmsnorm(x') . U_gu
+  P[5].nprob = 1; P[5].N[0] = 2 * rf; P[5].norm = 1; P[5].norm_g = L.g2;
+  { const long long ld[1] = {2 * rf}; gemv(5, MAP_PLAIN, SRC_XMID, d, &L.U_gu, ld); }
+  // 6: gate and up halves: z_g V_g and z_u V_u, 32 + 32 columns per tile
+  P[6].nprob = 1; P[6].N[0] = f; P[6].a_col2 = rf;
+  { const long long ld[1] = {f}; gemv(6, MAP_SWIGLU, SRC_PART, rf, &L.V_gu, ld); }
+  // 7: z = h . U_dn, h = SiLU(gate) * up
   P[7].nprob = 1; P[7].N[0] = rf;
-  P[7].a = hbuf; P[7].a_f32 = 0; P[7].lda = f; P[7].out32 = z; P[7].ldo32 = rf;
-  { const long long ld[1] = {rf}; gemv(7, PRO_BF16, EPI_F32, MAP_PLAIN, f, &L.U_dn, ld); }
-  // 8: x += z . V_dn
+  { const long long ld[1] = {rf}; gemv(7, MAP_PLAIN, SRC_SWIGLU, f, &L.U_dn, ld); }
+  // 8: x'' = x' + z . V_dn  (added in the final pass)
   P[8].nprob = 1; P[8].N[0] = d;
-  P[8].a = z; P[8].a_f32 = 1; P[8].lda = rf; P[8].out16 = x; P[8].ldo16 = d; P[8].resid = x; P[8].ldr = d;
-  { const long long ld[1] = {d}; gemv(8, PRO_F32, EPI_BF16, MAP_PLAIN, rf, &L.V_dn, ld); }
+  { const long long ld[1] = {d}; gemv(8, MAP_PLAIN, SRC_PART, rf, &L.V_dn, ld); }
   return off;
 }
 
-long long decode_pack_bytes(const DecodeLayerDesc& L) {
+// Schedule records of every (stage, CTA) -- see SchedRec.  Returns false if
+// a CTA's share exceeds a record's fixed capacity.
+bool build_sched(const DfPhase* P, int G, int d, SchedRec* R) {
+  memset(R, 0, sizeof(SchedRec) * DF_NREC * G);
+  for (int i = 0; i < DF_NPHASE; ++i) {
+    const DfPhase& ph = P[i];
+    if (ph.type != DF_GEMV) continue;
+    const int Ctot = ph.T * ph.nk;
+    const int nseg = ph.map == MAP_SWIGLU ? 2 : 1;
+    const bool xin = ph.src == SRC_X || ph.src == SRC_XMID;
+    for (int g = 0; g < G; ++g) {
+      SchedRec& r = R[i * G + g];
+      const int c0 = g * Ctot / G, c1 = (g + 1) * Ctot / G;
+      if (c1 - c0 > DF_MAX_E) return false;
+      if (!xin) {
+        for (int c = c0; c < c1; ++c) {
+          const int t = c / ph.nk, kc = c - t * ph.nk;
+          int pi = 0;
+          for (int j = 1; j < ph.nprob; ++j)
+            if (t >= ph.tile_start[j]) pi = j;
+          const int key = pi << 8 | kc;
+          int ci = 0;
+          while (ci < r.n && r.clist[ci] != key) ++ci;
+          if (ci == r.n) {
+            if (r.n == 16 || (r.n + 1) * 256 * nseg > DF_ABUF_COLS) return false;
+            r.clist[r.n++] = key;
+          }
+          r.chunk_of[c - c0] = (uint8_t)ci;
+        }
+      }
+      const DfPhase& q = P[i > 0 ? i - 1 : 0];
+      if (ph.src == SRC_XMID) {
+        r.nunits = d >> 6;
+        for (int t = 0; t < r.nunits; ++t)
+          if (!tile_slots(P[4], t, G, r.utab[t])) return false;
+      } else if (ph.src == SRC_PART) {
+        r.nunits = r.n * nseg * 5;
+        for (int ui = 0; ui < r.nunits; ++ui) {
+          const int j = ui % 5, cs = ui / 5, seg = cs % nseg, ci = cs / nseg;
+          const int pi = r.clist[ci] >> 8, kc = r.clist[ci] & 255;
+          const int col0 = seg * ph.a_col2 + kc * DF_KC;
+          const int kn = std::min(DF_KC, ph.K - kc * DF_KC);
+          if ((col0 >> 6) + j <= (col0 + kn - 1) >> 6 &&
+              !tile_slots(q, q.tile_start[pi] + (col0 >> 6) + j, G, r.utab[ui]))
+            return false;
+        }
+      } else if (ph.src == SRC_SWIGLU) {
+        r.nunits = r.n * 8;
+        for (int ui = 0; ui < r.nunits; ++ui) {
+          const int t = ((r.clist[ui >> 3] & 255) * DF_KC >> 5) + (ui & 7);
+          if (t < q.T && !tile_slots(q, t, G, r.utab[ui])) return false;
+        }
+      }
+      if (r.nunits > DF_MAX_UNITS) return false;
+    }
+  }
+  // final pass: tiles g, g + G, ... of the last stage
+  for (int g = 0; g < G; ++g) {
+    SchedRec& r = R[DF_NPHASE * G + g];
+    for (int t = g; t < (d >> 6); t += G) {
+      if (r.nunits == DF_MAX_UNITS || !tile_slots(P[DF_NPHASE - 1], t, G, r.utab[r.nunits])) return false;
+      ++r.nunits;
+    }
+  }
+  return true;
+}
+
+// Byte offset of the schedule records in a pack of `factor_bytes`.
+long long sched_offset(long long factor_bytes) { return (factor_bytes + 127) / 128 * 128; }
+
+// Whether every CTA's share of every GEMV stage stays within the kernel's
+// fixed per-CTA limits (tiles touched, input chunks, contributor table).
+bool stages_fit(const DfPhase* P, int G, int MT, int D) {
+  const int CW = MT <= 2 ? 16 : 8;
+  const int red_bytes = std::max(CW * MT * 64 * 4, 2048);
+  for (int i = 0; i < DF_NPHASE; ++i) {
+    const DfPhase& ph = P[i];
+    if (ph.type != DF_GEMV) continue;
+    if (ph.nk > DF_MAX_NK) return false;
+    const int Ctot = ph.T * ph.nk;
+    if ((long long)Ctot * G >= (1LL << 31)) return false;
+    const int nseg = ph.map == MAP_SWIGLU ? 2 : 1;
+    for (int g = 0; g < G; ++g) {
+      const int c0 = g * Ctot / G, c1 = (g + 1) * Ctot / G;
+      if (c0 >= c1) continue;
+      if ((c1 - 1) / ph.nk - c0 / ph.nk + 1 > DF_MAX_SU) return false;
+      if (ph.src == SRC_X || ph.src == SRC_XMID) continue;
+      bool seen[3][DF_MAX_NK] = {};
+      int n = 0;
+      for (int c = c0; c < c1; ++c) {
+        const int t = c / ph.nk, kc = c - t * ph.nk;
+        int pi = 0;
+        for (int j = 1; j < ph.nprob; ++j)
+          if (t >= ph.tile_start[j]) pi = j;
+        if (!seen[pi][kc]) { seen[pi][kc] = true; ++n; }
+      }
+      if (n * 256 * nseg > DF_ABUF_COLS) return false;
+      int units = 0;
+      if (ph.src == SRC_PART) units = n * nseg * 5;
+      else if (ph.src == SRC_SWIGLU) units = n * 8;
+      else if (ph.src == SRC_ATT) units = n * MT * (DF_KC / D);
+      if (units > DF_MAX_UNITS) return false;
+      if (ph.src == SRC_ATT && units * DF_CMAX * 4 > red_bytes) return false;
+    }
+  }
+  return true;
+}
+
+}  // namespace
+
+int decode_fused_supported(int B, int d, int D, int r, int r_f) {
+  return B >= 1 && B <= 4 && (D == 64 || D == 128) && d % 64 == 0 && d <= DF_ABUF_COLS && r % 8 == 0 &&
+         r_f % 8 == 0;
+}
+
+long long decode_pack_bytes(const DecodeLayerDesc& L, int sm_count) {
   DfPhase P[DF_NPHASE];
-  return build_stages(L, nullptr, nullptr, nullptr, nullptr, nullptr, P, nullptr);
+  return sched_offset(build_stages(L, P, nullptr)) + (long long)sizeof(SchedRec) * DF_NREC * sm_count;
 }
 
 int decode_pack_launch(const DecodeLayerDesc& L, void* dst, long long bytes, int sm_count,
@@ -973,8 +1248,15 @@ int decode_pack_launch(const DecodeLayerDesc& L, void* dst, long long bytes, int
   DfPhase P[DF_NPHASE];
   PackParams pp;
   memset(&pp, 0, sizeof(pp));
-  const long long need = build_stages(L, nullptr, nullptr, nullptr, nullptr, nullptr, P, pp.st);
-  if (bytes < need) return FLASHSVD_ERR_INVALID_ARG;
+  const long long need = build_stages(L, P, pp.st);
+  const int G = sm_count;
+  const long long soff = sched_offset(need);
+  if (bytes < soff + (long long)sizeof(SchedRec) * DF_NREC * G) return FLASHSVD_ERR_INVALID_ARG;
+  std::vector<SchedRec> rec((size_t)DF_NREC * G);
+  if (!build_sched(P, G, L.d, rec.data())) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  // (pageable source: the copy is staged before this call returns)
+  FSVD_CUDA(cudaMemcpyAsync(static_cast<uint8_t*>(dst) + soff, rec.data(), sizeof(SchedRec) * rec.size(),
+                            cudaMemcpyHostToDevice, stream));
   // Stage 2 (attention) holds no factors: an empty range at stage 3's
   // offset lets the pack kernel's stage search pass over it.
   pp.st[2] = pp.st[3];
@@ -990,38 +1272,31 @@ int decode_pack_launch(const DecodeLayerDesc& L, void* dst, long long bytes, int
 }
 
 int decode_fused_launch(const DecodeLayerDesc& L, bf16* x, bf16* kc, bf16* vc, const int* seqlens,
-                        int B, int S_max, bf16* qbuf, bf16* att, bf16* hbuf, float* z, float* part,
-                        int* tilecnt, int* bar, int* done, int* status, int sm_count,
-                        cudaStream_t stream) {
+                        int B, int S_max, bf16* xm, float* part, long long part_floats, int* bar,
+                        int* done, int* status, int sm_count, cudaStream_t stream) {
   if (!L.pack) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  if (!decode_fused_supported(B, L.d, L.D, L.r, L.r_f) || L.f % 8) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  const int G = sm_count;
+  if (2LL * G * DF_MAX_SU * DF_PART_STRIDE > part_floats) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  // Attention: with equal lengths a CTA's share spans at most this many pairs.
+  if ((B * L.H + G - 1) / G + 1 > DF_MAX_PAIRS) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   DfParams p;
   memset(&p, 0, sizeof(p));
-  DfPhase* P = p.ph;
-  const long long pack_bytes = build_stages(L, x, qbuf, att, hbuf, z, P, nullptr);
+  const long long pack_bytes = build_stages(L, p.ph, nullptr);
+  if (!stages_fit(p.ph, G, B <= 1 ? 1 : (B <= 2 ? 2 : 4), L.D)) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   p.pack = static_cast<const uint8_t*>(L.pack);
+  // the pack holds the schedule records for this device's SM count
+  p.sched = reinterpret_cast<const SchedRec*>(p.pack + sched_offset(pack_bytes));
   const long long HD = (long long)L.H * L.D;
   FSVD_TRY(encode_map(&p.maps[0], kc, (long long)B * S_max, HD, HD, 64, 64, true));
   FSVD_TRY(encode_map(&p.maps[1], vc, (long long)B * S_max, HD, HD, 64, 64, true));
-  p.nphase = 9;
-
-  // Every CTA's share of a stage may touch at most DF_MAX_SU tiles.
-  const int G = sm_count;
-  for (int i = 0; i < 9; ++i) {
-    if (P[i].type != DF_GEMV) continue;
-    const int Ctot = P[i].T * P[i].nk;
-    const int per = ceil_div(Ctot, G);
-    if (ceil_div(per, P[i].nk) + 1 > DF_MAX_SU || P[i].T > 4096) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
-  }
-  // attention: a CTA's share spans at most (B*H)/G + 2 (batch, head) pairs
-  if ((B * L.H) / G + 3 > DF_MAX_SU || B * L.H > 4096) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
-
-  p.B = B; p.H = L.H; p.D = L.D; p.S_max = S_max;
+  p.B = B; p.H = L.H; p.D = L.D; p.S_max = S_max; p.d = L.d;
   p.eps = L.eps;
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)L.D);
-  p.seqlens = seqlens; p.k_cache = kc; p.v_cache = vc;
+  p.seqlens = seqlens;
+  p.x = x; p.xm = xm; p.k_cache = kc; p.v_cache = vc;
   p.rope_cos = L.rope_cos; p.rope_sin = L.rope_sin;
-  p.q = qbuf; p.att = att;
-  p.part = part; p.tilecnt = tilecnt; p.bar = bar; p.done = done; p.status = status;
+  p.part = part; p.bar = bar; p.done = done; p.status = status;
 
   const double bytes = (double)pack_bytes + 2.0 * 2.0 * B * (double)S_max * HD;
   const LaunchTag tag{"decode_layer_fused", bytes, 0.0};
@@ -1034,12 +1309,11 @@ int decode_fused_launch(const DecodeLayerDesc& L, bf16* x, bf16* kc, bf16* vc, c
       FSVD_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, DfCfg<MT_>::SMEM)); \
       configured = true;                                                                             \
     }                                                                                                \
-    return launch_pdl(tag, kern, dim3(G), dim3(DfCfg<MT_>::THREADS), (size_t)DfCfg<MT_>::SMEM, stream, p);   \
+    return launch_pdl(tag, kern, dim3(G), dim3(DfCfg<MT_>::THREADS), (size_t)DfCfg<MT_>::SMEM, stream, p); \
   }
   if (B <= 1) FSVD_DF_LAUNCH(1)
   if (B <= 2) FSVD_DF_LAUNCH(2)
-  if (B <= 4) FSVD_DF_LAUNCH(4)
-  FSVD_DF_LAUNCH(8)
+  FSVD_DF_LAUNCH(4)
 #undef FSVD_DF_LAUNCH
 }
 

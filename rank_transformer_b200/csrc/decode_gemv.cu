@@ -22,7 +22,6 @@ namespace fsvd {
 namespace {
 
 constexpr int GV_THREADS = 256;
-constexpr int GV_BATCH = 8;  // 16-byte weight vectors in flight per thread
 
 __device__ __forceinline__ void unpack8(const uint4& v, float* w) {
   w[0] = bf_lo(v.x); w[1] = bf_hi(v.x); w[2] = bf_lo(v.y); w[3] = bf_hi(v.y);

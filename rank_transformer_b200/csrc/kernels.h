@@ -111,16 +111,18 @@ struct DecodeLayerDesc {
   const void* pack;  // the layer's decode pack (decode_pack_launch), or null
 };
 int decode_fused_supported(int B, int d, int D, int r, int r_f);
-long long decode_pack_bytes(const DecodeLayerDesc& L);
+long long decode_pack_bytes(const DecodeLayerDesc& L, int sm_count);
 int decode_pack_launch(const DecodeLayerDesc& L, void* dst, long long bytes, int sm_count,
                        cudaStream_t stream);
+// Fused decode layer; x is updated in place.  xm: [B x d] bf16 scratch;
+// part: fp32 partial slots (>= 2 * sm_count * 16 * 640 floats); bar: 9 stage
+// counters and done: 1 counter, all zero between launches.
 int decode_fused_launch(const DecodeLayerDesc& L, bf16* x, bf16* kc, bf16* vc, const int* seqlens,
-                        int B, int S_max, bf16* qbuf, bf16* att, bf16* hbuf, float* z, float* part,
-                        int* tilecnt, int* bar, int* done, int* status, int sm_count,
-                        cudaStream_t stream);
+                        int B, int S_max, bf16* xm, float* part, long long part_floats, int* bar,
+                        int* done, int* status, int sm_count, cudaStream_t stream);
 int encode_map(CUtensorMap* map, const void* base, long long rows, long long cols, long long ld,
                int box_cols, int box_rows, bool swizzle128);
-constexpr int kFusedPartFloats = 148 * 16 * 640;  // per SM: 16 partial slots of 640 floats
+constexpr int kFusedPartFloats = 2 * 148 * 16 * 640;  // two halves; per SM 16 slots of 640 floats
 
 // ------------------------------------------------ prefill attention -------
 struct AttnPfParams {

@@ -55,7 +55,7 @@ def _bf16_normal(shape, std, gen, device):
 
 class DecoderModel:
     def __init__(self, cfg: DecoderConfig, B: int, S_max: int, seed: int = 0,
-                 device: str = "cuda", weights=None, decode_pack: bool = False):
+                 device: str = "cuda", weights=None, decode_pack: bool = True):
         self.cfg, self.B, self.S_max, self.device = cfg, B, S_max, device
         gen = torch.Generator(device=device)
         gen.manual_seed(seed)

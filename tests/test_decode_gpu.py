@@ -230,8 +230,9 @@ def test_decode_pack_layout(fs, shape):
     torch.cuda.synchronize()
     got = dev["pack"].cpu().numpy().view(np.uint16)
     exp = _expected_pack(w, d, H, D, f, r, r_f)
-    assert got.shape == exp.shape
-    assert np.array_equal(got, exp)
+    # the factor blocks come first; the kernel's schedule records follow them
+    assert got.size >= exp.size
+    assert np.array_equal(got[:exp.size], exp)
 
 
 @pytest.mark.parametrize("fused", [True, False])
