@@ -381,7 +381,8 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
   int* clist = srec->clist;
   short* utab = &srec->utab[0][0];
   float* s_rstd = reinterpret_cast<float*>(misc + sizeof(SchedRec));  // [8]
-  static_assert(sizeof(SchedRec) + 32 <= C::MISC_BYTES, "schedule record exceeds its shared copy");
+  AttnSched* s_as = reinterpret_cast<AttnSched*>(misc + sizeof(SchedRec) + 64);  // attention schedule
+  static_assert(sizeof(SchedRec) + 64 + sizeof(AttnSched) <= C::MISC_BYTES, "misc shared area");
   uint64_t* full = reinterpret_cast<uint64_t*>(misc + C::MISC_BYTES);
   uint64_t* empty = full + C::NSLOT;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + C::NSLOT);
@@ -505,6 +506,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
   } else {
     // ================================================= consumers ==========
     pdl_wait();
+    if (tid == 0) attn_sched(p, *s_as);  // lengths are fixed for the launch
     // lane bits: [1:0] 16-byte chunk, [2] row parity, [3] box, [..4] row lane;
     // a quarter warp then reads two consecutive 64-byte rows of one box.
     const int chunk = tid & 3, rsub = (tid >> 2) & 1, box = (tid >> 3) & 1, rowlane = tid >> 4;
@@ -543,14 +545,26 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
             if (tid == 0) atomicExch(p.status, DEV_STATUS_SCHEDULE);
             nunits = 0;
           }
-          AttnSched s;
-          attn_sched(p, s);
+          const AttnSched& s = *s_as;
           for (int ui = tid; ui < nunits; ui += C::CT) {
             short* u = utab + ui * 16;
             u[0] = 0;
             const int j = ui % hpc, r2 = ui / hpc, m = r2 % MT, ci = r2 / MT;
             const int hh = (clist[ci] & 255) * DF_KC / p.D + j;
             if (m < p.B && hh < p.H && !pair_slots(s, p.H, G, m, hh, u)) atomicExch(p.status, DEV_STATUS_SCHEDULE);
+          }
+        }
+        if (xin) {
+          // x (the layer input: fixed during the launch) into the input rows
+          const int d4 = p.d >> 2;
+          for (int e = tid; e < MT * d4; e += C::CT) {
+            const int m = e / d4, j = (e - m * d4) * 4;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (m < p.B) {
+              const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(p.x + (long long)m * p.d + j));
+              v = make_float4(bf_lo(raw.x), bf_hi(raw.x), bf_lo(raw.y), bf_hi(raw.y));
+            }
+            *reinterpret_cast<float4*>(abuf + m * DF_ABUF_COLS + j) = v;
           }
         }
         if (ph.norm) {
@@ -563,46 +577,32 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
         consumer_sync<C::CT>();
         // (2) the input itself, 4 consecutive values per group, two groups
         // per thread and step (their loads in flight together)
-        if (xin) {
-          // x (stage 0) or x' = x + (z V_o) (stage 5), whole rows, for RMSNorm
-          const int d4 = p.d >> 2, tot = MT * d4;
+        if (ph.src == SRC_XMID && nunits) {
+          // x' = x + (z V_o), rounded as the residual stream is stored
+          const int d4 = p.d >> 2, tot = p.B * d4;
           for (int e0 = tid; e0 < tot; e0 += 2 * C::CT) {
-            int ee[2] = {e0, e0 + C::CT};
-            float4 v[2], sp[2];
+            const int e1 = e0 + C::CT;
+            const bool h1 = e1 < tot;
+            const int m0 = e0 / d4, j0 = (e0 - m0 * d4) * 4;
+            const int m1 = h1 ? e1 / d4 : 0, j1 = h1 ? (e1 - m1 * d4) * 4 : 0;
+            float4 sp[2];
+            gather4x2(part_prev, utab + (j0 >> 6) * 16, m0 * 64 + (j0 & 63), nullptr, utab + (j1 >> 6) * 16,
+                      m1 * 64 + (j1 & 63), nullptr, h1, sp[0], sp[1]);
 #pragma unroll
             for (int k2 = 0; k2 < 2; ++k2) {
-              v[k2] = make_float4(0.f, 0.f, 0.f, 0.f);
-              const int m = ee[k2] / d4, j = (ee[k2] - m * d4) * 4;
-              if (ee[k2] < tot && m < p.B) {
-                const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(p.x + (long long)m * p.d + j));
-                v[k2] = make_float4(bf_lo(raw.x), bf_hi(raw.x), bf_lo(raw.y), bf_hi(raw.y));
+              if (k2 == 1 && !h1) continue;
+              const int m = k2 ? m1 : m0, j = k2 ? j1 : j0;
+              float4* a4 = reinterpret_cast<float4*>(abuf + m * DF_ABUF_COLS + j);
+              float4 v = *a4;
+              add4(v, sp[k2]);
+              v = round4(v);
+              *a4 = v;
+              if ((j >> 6) % G == g) {
+                uint2 o;
+                o.x = pack_bf2(v.x, v.y);
+                o.y = pack_bf2(v.z, v.w);
+                *reinterpret_cast<uint2*>(p.xm + (long long)m * p.d + j) = o;
               }
-            }
-            if (ph.src == SRC_XMID && nunits) {
-              const int m0 = ee[0] / d4, j0 = (ee[0] - m0 * d4) * 4;
-              const int m1 = ee[1] / d4, j1 = (ee[1] - m1 * d4) * 4;
-              const bool h0 = m0 < p.B, h1 = ee[1] < tot && m1 < p.B;
-              gather4x2(part_prev, utab + (h0 ? (j0 >> 6) : 0) * 16, m0 * 64 + (j0 & 63), nullptr,
-                        utab + (h1 ? (j1 >> 6) : 0) * 16, m1 * 64 + (j1 & 63), nullptr, h1, sp[0], sp[1]);
-  #pragma unroll
-            for (int k2 = 0; k2 < 2; ++k2) {
-                const int m = ee[k2] / d4, j = (ee[k2] - m * d4) * 4;
-                if (ee[k2] >= tot || m >= p.B) continue;
-                add4(v[k2], sp[k2]);
-                v[k2] = round4(v[k2]);
-                if ((j >> 6) % G == g) {
-                  uint2 o;
-                  o.x = pack_bf2(v[k2].x, v[k2].y);
-                  o.y = pack_bf2(v[k2].z, v[k2].w);
-                  *reinterpret_cast<uint2*>(p.xm + (long long)m * p.d + j) = o;
-                }
-              }
-            }
-#pragma unroll
-            for (int k2 = 0; k2 < 2; ++k2) {
-              if (ee[k2] >= tot) continue;
-              const int m = ee[k2] / d4, j = (ee[k2] - m * d4) * 4;
-              *reinterpret_cast<float4*>(abuf + m * DF_ABUF_COLS + j) = v[k2];
             }
           }
         } else if (ph.src == SRC_SWIGLU) {
@@ -633,8 +633,8 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
               v = round4(attn_gather4(part_prev, utab + ((ci * MT + m) * hpc + i / p.D) * 16, k % p.D));
             *reinterpret_cast<float4*>(abuf + m * DF_ABUF_COLS + ci * 256 + i) = v;
           }
-        } else {
-          // SRC_PART: fp32 rank activations z (plain column tiles of 64)
+        } else if (ph.src == SRC_PART) {
+          // fp32 rank activations z (plain column tiles of 64)
           const int tot = n * nseg * MT * 64;
           for (int e0 = tid; e0 < tot; e0 += 2 * C::CT) {
             const short* uu[2];
@@ -758,8 +758,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
         }
       } else {
         // ---------------------------------------------- attention stage --
-        AttnSched s;
-        attn_sched(p, s);
+        const AttnSched& s = *s_as;
         const int Ctot = s.pre[8];
         int c0, c1;
         share(Ctot, G, g, c0, c1);
@@ -826,20 +825,25 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
         }
         consumer_sync<C::CT>();
 
-        // Each consumer warp owns 64 / CW keys of every 64-key entry and keeps
-        // its own online-softmax state (m, l, o) over all entries of a pair;
-        // lanes own D / 32 dimensions.  The key at the current position comes
-        // from qkv (its cache row may not be written yet).
-        const int EPL = D >> 5;
+        // Each consumer warp owns KPW = 64 / CW keys of every 64-key entry;
+        // LPK = 32 / KPW lanes share a key, each holding cpl 16-byte chunks
+        // (8 dims each) of q, k, v and o.  A warp keeps its online-softmax
+        // state (m, and l, o per lane group) over all entries of a pair.
+        // The key at the current position comes from qkv (its cache row may
+        // not be written yet).
         constexpr int KPW = 64 / C::CW;
+        constexpr int LPK = 32 / KPW;
+        constexpr int CPL_MAX = 128 / (LPK * 8);
+        const int cpl = D / (LPK * 8);
+        const int grp = lane / LPK, sl = lane % LPK;
+        const int key_l = warp * KPW + grp;
         float* wm = scr;       // [CW]
         float* wl = scr + 32;  // [CW]
         float* wo = scr + 64;  // [CW][128]
-        const int d0 = lane * EPL;
-        const int bx = d0 >> 6, ch = (d0 & 63) >> 3, sub = (d0 & 7) * 2;
-        float qv[4] = {0.f, 0.f, 0.f, 0.f};
-        float m_w = -INFINITY, l_w = 0.f;
-        float ov[4] = {0.f, 0.f, 0.f, 0.f};
+        float qv[CPL_MAX * 8], ov[CPL_MAX * 8];
+#pragma unroll
+        for (int e = 0; e < CPL_MAX * 8; ++e) { qv[e] = 0.f; ov[e] = 0.f; }
+        float m_w = -INFINITY, l_g = 0.f;
         int su = 0;
         for (int c = c0; c < c1; ++c, ++seq) {
           int b, h, kc;
@@ -850,72 +854,75 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
           const int slot = seq % C::NSLOT;
           const uint32_t par = (uint32_t)(seq / C::NSLOT) & 1u;
           tc::mbar_wait(full + slot, par, abort_flag, p.status);  // on abort: run on, results discarded
-          const float* qn = qkv + pr * 3 * D + d0;
+          const float* qn = qkv + pr * 3 * D;
           if (c == c0 || kc == 0) {
             m_w = -INFINITY;
-            l_w = 0.f;
+            l_g = 0.f;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              ov[e] = 0.f;
-              qv[e] = e < EPL ? qn[e] * p.scale_log2 : 0.f;
-            }
+            for (int cc = 0; cc < CPL_MAX; ++cc)
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                ov[cc * 8 + e] = 0.f;
+                qv[cc * 8 + e] = cc < cpl ? qn[(sl * cpl + cc) * 8 + e] * p.scale_log2 : 0.f;
+              }
           }
           const int L = s.L[b], pos = L - 1;
+          const int key = kc * 64 + key_l;
           const uint8_t* kb = slots + slot * C::SLOT;
           const uint8_t* vb = kb + 16384;
-          float sc[KPW];
+          float dot = 0.f;
+          if (key == pos) {
 #pragma unroll
-          for (int i = 0; i < KPW; ++i) {
-            const int j = warp * KPW + i;
-            float dot = 0.f;
-            if (kc * 64 + j == pos) {
+            for (int cc = 0; cc < CPL_MAX; ++cc)
+              if (cc < cpl)
 #pragma unroll
-              for (int e = 0; e < 4; ++e)
-                if (e < EPL) dot = fmaf(qv[e], qn[D + e], dot);
-            } else {
-              const uint8_t* kp = kb + bx * 8192 + j * 128 + ((ch ^ (j & 7)) << 4) + sub;
-              if (EPL == 4) {
-                const uint2 u = *reinterpret_cast<const uint2*>(kp);
-                dot = qv[0] * bf_lo(u.x) + qv[1] * bf_hi(u.x) + qv[2] * bf_lo(u.y) + qv[3] * bf_hi(u.y);
-              } else {
-                const uint32_t u = *reinterpret_cast<const uint32_t*>(kp);
-                dot = qv[0] * bf_lo(u) + qv[1] * bf_hi(u);
+                for (int e = 0; e < 8; ++e) dot = fmaf(qv[cc * 8 + e], qn[D + (sl * cpl + cc) * 8 + e], dot);
+          } else {
+#pragma unroll
+            for (int cc = 0; cc < CPL_MAX; ++cc)
+              if (cc < cpl) {
+                const int gc = sl * cpl + cc;
+                const uint4 u = *reinterpret_cast<const uint4*>(kb + (gc >> 3) * 8192 + key_l * 128 +
+                                                                (((gc & 7) ^ (key_l & 7)) << 4));
+                const float kv[8] = {bf_lo(u.x), bf_hi(u.x), bf_lo(u.y), bf_hi(u.y),
+                                     bf_lo(u.z), bf_hi(u.z), bf_lo(u.w), bf_hi(u.w)};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) dot = fmaf(qv[cc * 8 + e], kv[e], dot);
               }
-            }
-            sc[i] = dot;
           }
-          float mb = -INFINITY;
 #pragma unroll
-          for (int i = 0; i < KPW; ++i) {
-            sc[i] = warp_sum(sc[i]);
-            if (kc * 64 + warp * KPW + i >= L) sc[i] = -INFINITY;
-            mb = fmaxf(mb, sc[i]);
-          }
+          for (int o = LPK / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+          const float sc = key < L ? dot : -INFINITY;
+          float mb = sc;
+#pragma unroll
+          for (int o = LPK; o < 32; o <<= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
           const float mn = fmaxf(m_w, mb);
-          if (mn != -INFINITY) {
-            const float corr = (m_w == -INFINITY) ? 0.f : exp2f(m_w - mn);
-            l_w *= corr;
+          if (mn != -INFINITY) {  // warp-uniform
+            const float corr = m_w == -INFINITY ? 0.f : exp2f(m_w - mn);
+            const float pj = sc == -INFINITY ? 0.f : exp2f(sc - mn);
+            l_g = l_g * corr + pj;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) ov[e] *= corr;
+            for (int e = 0; e < CPL_MAX * 8; ++e) ov[e] *= corr;
+            if (sc != -INFINITY) {
+              if (key == pos) {
 #pragma unroll
-            for (int i = 0; i < KPW; ++i) {
-              const float pj = (sc[i] == -INFINITY) ? 0.f : exp2f(sc[i] - mn);
-              l_w += pj;
-              const int j = warp * KPW + i;
-              if (kc * 64 + j == pos) {
+                for (int cc = 0; cc < CPL_MAX; ++cc)
+                  if (cc < cpl)
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                  if (e < EPL) ov[e] = fmaf(pj, qn[2 * D + e], ov[e]);
+                    for (int e = 0; e < 8; ++e)
+                      ov[cc * 8 + e] = fmaf(pj, qn[2 * D + (sl * cpl + cc) * 8 + e], ov[cc * 8 + e]);
               } else {
-                const uint8_t* vp = vb + bx * 8192 + j * 128 + ((ch ^ (j & 7)) << 4) + sub;
-                if (EPL == 4) {
-                  const uint2 u = *reinterpret_cast<const uint2*>(vp);
-                  ov[0] = fmaf(pj, bf_lo(u.x), ov[0]); ov[1] = fmaf(pj, bf_hi(u.x), ov[1]);
-                  ov[2] = fmaf(pj, bf_lo(u.y), ov[2]); ov[3] = fmaf(pj, bf_hi(u.y), ov[3]);
-                } else {
-                  const uint32_t u = *reinterpret_cast<const uint32_t*>(vp);
-                  ov[0] = fmaf(pj, bf_lo(u), ov[0]); ov[1] = fmaf(pj, bf_hi(u), ov[1]);
-                }
+#pragma unroll
+                for (int cc = 0; cc < CPL_MAX; ++cc)
+                  if (cc < cpl) {
+                    const int gc = sl * cpl + cc;
+                    const uint4 u = *reinterpret_cast<const uint4*>(vb + (gc >> 3) * 8192 + key_l * 128 +
+                                                                    (((gc & 7) ^ (key_l & 7)) << 4));
+                    const float vv[8] = {bf_lo(u.x), bf_hi(u.x), bf_lo(u.y), bf_hi(u.y),
+                                         bf_lo(u.z), bf_hi(u.z), bf_lo(u.w), bf_hi(u.w)};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ov[cc * 8 + e] = fmaf(pj, vv[e], ov[cc * 8 + e]);
+                  }
               }
             }
             m_w = mn;
@@ -924,11 +931,21 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
           if (lane == 0) tc::mbar_arrive(empty + slot);
 
           if (c != c1 - 1 && c != pair_last) continue;
-          // ---- merge the warps; write this CTA's (m, l, o) partial of the pair ----
-          if (lane == 0) { wm[warp] = m_w; wl[warp] = l_w; }
+          // ---- merge the lane groups, then the warps; write this CTA's
+          // (m, l, o) partial of the pair ----
+          float lw = l_g;
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if (e < EPL) wo[warp * 128 + d0 + e] = ov[e];
+          for (int o = LPK; o < 32; o <<= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+#pragma unroll
+          for (int cc = 0; cc < CPL_MAX; ++cc)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              float v = ov[cc * 8 + e];
+#pragma unroll
+              for (int o = LPK; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+              if (grp == 0 && cc < cpl) wo[warp * 128 + (sl * cpl + cc) * 8 + e] = v;
+            }
+          if (lane == 0) { wm[warp] = m_w; wl[warp] = lw; }
           consumer_sync<C::CT>();
           float Mc = -INFINITY;
 #pragma unroll
