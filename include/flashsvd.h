@@ -316,6 +316,40 @@ FLASHSVD_API int flashsvd_decode_pack_bytes(const flashsvd_layer* L, size_t* byt
 FLASHSVD_API int flashsvd_decode_pack(const flashsvd_layer* L, void* dst, size_t bytes,
                                       flashsvd_stream stream);
 
+/* ---------------------------------------------------------- decode plan ---
+ * FlashSVD v1.5 Technical Summary, Methodology 4, makes each layer's decode
+ * body one replay unit.  A decode plan goes one step further: the decode
+ * step of n consecutive decoder layers runs as ONE launch of the fused
+ * decode kernel, which streams the next layer's factors while the current
+ * layer finishes and hands each layer's output to the next on chip-wide
+ * partial sums, with no launch boundary in between.
+ *
+ * flashsvd_decode_plan_create: layers[0..n) (each with a decode pack, equal
+ *   d, H, D, f, norm_eps and RoPE tables; ranks may differ per layer), layer
+ *   i's caches k_caches[i], v_caches[i] ([B, S_max, H, D] bf16, device
+ *   pointers; host arrays of n pointers).  B <= 4.  Builds the kernel's
+ *   per-layer descriptors in device memory it owns (synchronous; not during
+ *   stream capture).  The layers' factors, packs and caches must outlive the
+ *   plan.
+ * flashsvd_decode_plan_forward: one decode step of all n layers in place on
+ *   x_inout [B x d]; positions are cache_seqlens[b] (device int32[B]); every
+ *   layer appends its new key and value there; cache_seqlens is not
+ *   incremented.  Same result as n DECODE-mode flashsvd_layer_forward calls.
+ *   Asynchronous, capturable, uses the context's scratch (one plan runs at a
+ *   time per context).
+ * Errors: INVALID_ARG, NOT_INITIALIZED, CAPTURE_UNSAFE (create during
+ *   capture), UNSUPPORTED_SHAPE (a layer without a pack, B > 4, shapes the
+ *   fused kernel does not cover), NO_MEMORY. */
+typedef struct flashsvd_decode_plan flashsvd_decode_plan;
+FLASHSVD_API int flashsvd_decode_plan_create(const flashsvd_layer* layers, int n_layers,
+                                             flashsvd_bf16* const* k_caches,
+                                             flashsvd_bf16* const* v_caches, int B, int S_max,
+                                             flashsvd_decode_plan** plan);
+FLASHSVD_API int flashsvd_decode_plan_forward(const flashsvd_decode_plan* plan,
+                                              flashsvd_bf16* x_inout,
+                                              const int32_t* cache_seqlens, flashsvd_stream stream);
+FLASHSVD_API int flashsvd_decode_plan_destroy(flashsvd_decode_plan* plan);
+
 /* Run one layer in place on x_inout ([B*S x d] bf16, token-major).
  * PREFILL_CAUSAL: positions 0..S-1; rotated keys and values are written to
  *   cache rows [0, S) of every batch entry; cache_seqlens is not read.

@@ -472,6 +472,61 @@ int flashsvd_decode_pack(const flashsvd_layer* L, void* dst, size_t bytes, flash
   return decode_pack_launch(decode_desc(L), dst, (long long)bytes, sms, (cudaStream_t)stream);
 }
 
+struct flashsvd_decode_plan {
+  DecodePlan* impl = nullptr;
+  int device = -1, B = 0, d = 0;
+};
+
+int flashsvd_decode_plan_create(const flashsvd_layer* layers, int n_layers, flashsvd_bf16* const* k_caches,
+                                flashsvd_bf16* const* v_caches, int B, int S_max,
+                                flashsvd_decode_plan** plan) {
+  FSVD_TRY(need_init());
+  if (!layers || n_layers <= 0 || !k_caches || !v_caches || !plan || B <= 0 || S_max <= 0)
+    return FLASHSVD_ERR_INVALID_ARG;
+  if (capturing(nullptr)) return FLASHSVD_ERR_CAPTURE_UNSAFE;
+  if (!g_fused_decode || g_ctx.sm_count > 148) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  std::vector<DecodeLayerDesc> descs((size_t)n_layers);
+  std::vector<bf16*> kc((size_t)n_layers), vc((size_t)n_layers);
+  for (int i = 0; i < n_layers; ++i) {
+    const flashsvd_layer* L = layers + i;
+    if (L->kind != FLASHSVD_DECODER) return FLASHSVD_ERR_INVALID_ARG;
+    if (!L->decode_pack || !pack_shapes_ok(L)) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+    if (!k_caches[i] || !v_caches[i]) return FLASHSVD_ERR_INVALID_ARG;
+    if (!aligned16(k_caches[i]) || !aligned16(v_caches[i])) return FLASHSVD_ERR_MISALIGNED;
+    descs[i] = decode_desc(L);
+    kc[i] = reinterpret_cast<bf16*>(k_caches[i]);
+    vc[i] = reinterpret_cast<bf16*>(v_caches[i]);
+  }
+  DecodePlan* impl = nullptr;
+  FSVD_TRY(decode_plan_create(descs.data(), n_layers, kc.data(), vc.data(), B, S_max, g_ctx.sm_count, &impl));
+  flashsvd_decode_plan* out = new flashsvd_decode_plan();
+  out->impl = impl;
+  out->device = g_ctx.device;
+  out->B = B;
+  out->d = layers[0].d;
+  *plan = out;
+  return FLASHSVD_OK;
+}
+
+int flashsvd_decode_plan_forward(const flashsvd_decode_plan* plan, flashsvd_bf16* x_inout,
+                                 const int32_t* cache_seqlens, flashsvd_stream stream) {
+  FSVD_TRY(need_init());
+  if (!plan || !x_inout || !cache_seqlens) return FLASHSVD_ERR_INVALID_ARG;
+  if (plan->device != g_ctx.device) return FLASHSVD_ERR_INVALID_ARG;
+  if (!aligned16(x_inout)) return FLASHSVD_ERR_MISALIGNED;
+  if (plan->d > g_ctx.max_hidden) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  return decode_plan_launch(plan->impl, reinterpret_cast<bf16*>(x_inout), cache_seqlens, g_ctx.xn, g_ctx.df_part,
+                            kFusedPartFloats, g_ctx.df_cnt, g_ctx.df_cnt + 32, g_ctx.status,
+                            (cudaStream_t)stream);
+}
+
+int flashsvd_decode_plan_destroy(flashsvd_decode_plan* plan) {
+  if (!plan) return FLASHSVD_OK;
+  decode_plan_destroy(plan->impl);
+  delete plan;
+  return FLASHSVD_OK;
+}
+
 int flashsvd_init(int device, int max_tokens, int max_rank, int max_hidden,
                   int max_ffn) {
   std::lock_guard<std::mutex> lock(g_mu);

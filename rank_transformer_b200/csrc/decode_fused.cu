@@ -59,7 +59,6 @@ constexpr int DF_KC = 256;            // rows per ring entry
 constexpr int DF_MAX_SU = 16;         // tiles (or attention pairs) per CTA and stage
 constexpr int DF_PART_STRIDE = 640;   // floats per partial slot (>= 4 x 64, >= 4 + 128)
 constexpr int DF_NPHASE = 9;
-constexpr int DF_NMAPS = 2;
 constexpr int DF_ABUF_COLS = 4096;    // floats per row of the stage-input buffer
 constexpr int DF_MAX_PAIRS = 8;       // attention (batch, head) pairs per CTA
 constexpr int DF_MAX_NK = 64;         // 256-row chunks per factor (K <= 16384)
@@ -68,7 +67,9 @@ constexpr int DF_MAX_UNITS = 96;      // tiles (or pairs) read per stage and CTA
 
 enum { DF_GEMV = 0, DF_ATTN = 1 };
 // How a stage's input is built from what the previous stage left.
-enum { SRC_X = 0, SRC_PART = 1, SRC_ATT = 2, SRC_XMID = 3, SRC_SWIGLU = 4 };
+// SRC_XOUT (stage 0 of every layer after the first): the previous layer's
+// output x'' = x' + z V_dn, summed from its last stage's partials.
+enum { SRC_X = 0, SRC_PART = 1, SRC_ATT = 2, SRC_XMID = 3, SRC_SWIGLU = 4, SRC_XOUT = 5 };
 
 struct DfPhase {
   int type, map, src, norm;
@@ -86,8 +87,9 @@ struct DfPhase {
 // first-use order, the chunk of each entry, and the contributor table of the
 // previous-stage tiles those chunks draw on.  Records 0..8 follow the
 // stages (attention-dependent tables are filled on the device); record 9
-// serves the final pass.
-constexpr int DF_NREC = DF_NPHASE + 1;
+// serves the final pass (tiles g, g + G, ... of the last stage) and record 10
+// the next layer's first stage (every tile of the last stage).
+constexpr int DF_NREC = DF_NPHASE + 2;
 constexpr int DF_MAX_E = 48;  // entries per CTA and stage
 struct SchedRec {
   int n, nunits, pad0, pad1;
@@ -97,31 +99,38 @@ struct SchedRec {
 };
 static_assert(sizeof(SchedRec) % 128 == 0, "schedule records stay 128-byte aligned");
 
-struct DfParams {
-  CUtensorMap maps[DF_NMAPS];  // the K and V cache views [B * S_max x H * D]
+// One decoder layer as the kernel sees it.
+struct alignas(64) DfLayer {
+  CUtensorMap kmap, vmap;      // the K and V cache views [B * S_max x H * D]
   const uint8_t* pack;
   const SchedRec* sched;       // [DF_NREC][G], inside the pack
+  bf16* k_cache;
+  bf16* v_cache;
   DfPhase ph[DF_NPHASE];
+};
+
+struct DfParams {
+  DfLayer inl;              // the layer, when layers is null
+  const DfLayer* layers;    // [nlayer] in device memory (several layers per launch)
+  int nlayer;
   int B, H, D, S_max, d;
   float eps, scale_log2;
   const int* seqlens;
-  bf16* x;        // layer input and output [B x d]
-  bf16* xm;       // x' (after the attention block) [B x d]
-  bf16* k_cache;
-  bf16* v_cache;
+  bf16* x;        // input of the first layer; output of the last
+  bf16* xm;       // x' (after a layer's attention block) [B x d]
   const float* rope_cos;
   const float* rope_sin;
-  float* part;    // [2][G][DF_MAX_SU][DF_PART_STRIDE]: stage s writes half s & 1
-  int* bar;       // [DF_NPHASE] arrivals per stage
+  float* part;    // [2][G][DF_MAX_SU][DF_PART_STRIDE]: global stage gs writes half gs & 1
+  int* bar;       // [DF_NPHASE] arrivals per stage, accumulated over the layers
   int* done;
   int* status;
 };
 
 template <int MT>
 struct DfCfg {
-  static constexpr int CW = MT <= 2 ? 16 : 8;        // consumer warps
+  static constexpr int CW = 16;                      // consumer warps
   static constexpr int CT = CW * 32;                 // consumer threads
-  static constexpr int THREADS = CT + 64;            // + producer and prefetch warps
+  static constexpr int THREADS = CT + 32;            // + the producer warp
   static constexpr int SLOT = 32768;
   static constexpr int NSLOT = MT == 1 ? 6 : (MT == 2 ? 5 : 4);
   static constexpr int ABUF_BYTES = MT * DF_ABUF_COLS * 4;
@@ -157,10 +166,10 @@ __device__ __forceinline__ void red_release_add(int* p, int v) {
 }
 __device__ __forceinline__ float bf_round(float v) { return bf2f(f2bf(v)); }
 
-// Bounded wait until every CTA has arrived at stage counter *bar.
-__device__ __forceinline__ void grid_wait(const int* bar, int G, volatile int* abort_flag, int* status) {
+// Bounded wait until stage counter *bar reaches target.
+__device__ __forceinline__ void grid_wait(const int* bar, int target, volatile int* abort_flag, int* status) {
   const long long t0 = clock64();
-  while (ld_acquire(bar) < G) {
+  while (ld_acquire(bar) < target) {
     if (*abort_flag) return;
     if (clock64() - t0 > tc::kWaitCycles) {
       *abort_flag = 1;
@@ -393,12 +402,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
   const int G = gridDim.x, g = blockIdx.x;
   const long long half = (long long)G * DF_MAX_SU * DF_PART_STRIDE;
 
-  {
-    // Stage descriptors are read in every inner loop: keep a shared copy.
-    const int* src = reinterpret_cast<const int*>(p.ph);
-    int* dst = reinterpret_cast<int*>(s_ph);
-    for (int i = tid; i < (int)(sizeof(DfPhase) * DF_NPHASE / 4); i += C::THREADS) dst[i] = src[i];
-  }
+  auto layer_of = [&](int l) -> const DfLayer* { return p.layers ? p.layers + l : &p.inl; };
   if (tid == 0) {
     for (int s = 0; s < C::NSLOT; ++s) {
       tc::mbar_init(full + s, 1);
@@ -412,95 +416,101 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
 
   if (warp == C::CW) {
     // =================================================== producer ==========
+    // Fills every ring entry in order, layer after layer: pack entries of the
+    // GEMV stages (the next layer's while the current one finishes), 64-key
+    // cache chunks of the attention stages.
     if (lane == 0) {
-      // L2 prefetch cursor over this CTA's pack entries, PF entries ahead of
-      // the copies into the ring.
+      // L2 prefetch cursor (layer, stage, entry), PF pack entries ahead
       constexpr int PF = 2;
-      int pf_ph = -1, pf_c = 0, pf_c1 = 0;
+      int pf_l = 0, pf_s = -1, pf_c = 0, pf_c1 = 0;
       auto pf_step = [&]() {
         while (pf_c >= pf_c1) {
-          if (pf_ph >= DF_NPHASE) return;
-          if (++pf_ph >= DF_NPHASE) return;
-          const DfPhase& q = s_ph[pf_ph];
+          if (pf_l >= p.nlayer) return;
+          if (++pf_s >= DF_NPHASE) {
+            pf_s = 0;
+            if (++pf_l >= p.nlayer) return;
+          }
+          const DfPhase& q = layer_of(pf_l)->ph[pf_s];
           if (q.type != DF_GEMV) { pf_c = pf_c1 = 0; continue; }
           share(q.T * q.nk, G, g, pf_c, pf_c1);
         }
-        const DfPhase& q = s_ph[pf_ph];
+        const DfLayer* Lq = layer_of(pf_l);
+        const DfPhase& q = Lq->ph[pf_s];
         const int t = pf_c / q.nk, kc = pf_c - t * q.nk;
         const int kn = min(DF_KC, q.K - kc * DF_KC);
-        prefetch_l2_bulk(p.pack + q.pack_off + (long long)t * q.K * 128 + (long long)kc * 32768,
+        prefetch_l2_bulk(Lq->pack + q.pack_off + (long long)t * q.K * 128 + (long long)kc * 32768,
                          (uint32_t)kn * 128u);
         ++pf_c;
       };
       for (int i = 0; i < PF; ++i) pf_step();
       int seq = 0;
       bool waited = false, ok = true;
-      for (int ph_i = 0; ph_i < DF_NPHASE && ok && !*abort_flag; ++ph_i) {
-        const DfPhase& ph = s_ph[ph_i];
-        int c0, c1;
-        if (ph.type == DF_ATTN) {
-          // K/V chunks of the dense cache (rows before the current position
-          // are fixed for this step; the current row is taken from q/k/v)
-          if (!waited) { pdl_wait(); waited = true; }
-          AttnSched s;
-          attn_sched(p, s);
-          share(s.pre[8], G, g, c0, c1);
-          const int NB = p.D >> 6;
+      AttnSched s;
+      int a0 = 0, a1 = 0;
+      const int NB = p.D >> 6;
+      for (int l = 0; l < p.nlayer && ok && !*abort_flag; ++l) {
+        const DfLayer* Ly = layer_of(l);
+        for (int ph_i = 0; ph_i < DF_NPHASE && ok && !*abort_flag; ++ph_i) {
+          const DfPhase& ph = Ly->ph[ph_i];
+          if (ph_i == 1) {
+            // History rows are fixed for this step: pull this layer's cache
+            // chunks of this CTA into L2 ahead of its attention stage.
+            if (!waited) {
+              pdl_wait();
+              waited = true;
+              attn_sched(p, s);
+              share(s.pre[8], G, g, a0, a1);
+            }
+            tc::tma_prefetch_desc(&Ly->kmap);
+            tc::tma_prefetch_desc(&Ly->vmap);
+            for (int c = a0; c < a1; ++c) {
+              int b, h, kc;
+              attn_entry(s, c, b, h, kc);
+              for (int bx = 0; bx < NB; ++bx) {
+                prefetch_l2_2d(&Ly->kmap, h * p.D + 64 * bx, b * p.S_max + kc * 64);
+                prefetch_l2_2d(&Ly->vmap, h * p.D + 64 * bx, b * p.S_max + kc * 64);
+              }
+            }
+          }
+          if (ph.type == DF_ATTN) {
+            // K/V chunks of the dense cache (rows before the current position
+            // are fixed for this step; the current row is taken from q/k/v)
+            for (int c = a0; c < a1; ++c, ++seq) {
+              const int slot = seq % C::NSLOT;
+              const uint32_t par = (uint32_t)(seq / C::NSLOT) & 1u;
+              if (!tc::mbar_wait_sleep(empty + slot, par ^ 1u, abort_flag, p.status)) { ok = false; break; }
+              uint8_t* base = slots + slot * C::SLOT;
+              int b, h, kc;
+              attn_entry(s, c, b, h, kc);
+              tc::mbar_expect_tx(full + slot, (uint32_t)(2 * NB * 8192));
+              const int row = b * p.S_max + kc * 64;
+              for (int bx = 0; bx < NB; ++bx) {
+                tc::tma_load_2d(base + bx * 8192, &Ly->kmap, full + slot, h * p.D + 64 * bx, row);
+                tc::tma_load_2d(base + 16384 + bx * 8192, &Ly->vmap, full + slot, h * p.D + 64 * bx, row);
+              }
+            }
+            continue;
+          }
+          int c0, c1;
+          share(ph.T * ph.nk, G, g, c0, c1);
           for (int c = c0; c < c1; ++c, ++seq) {
             const int slot = seq % C::NSLOT;
             const uint32_t par = (uint32_t)(seq / C::NSLOT) & 1u;
             if (!tc::mbar_wait_sleep(empty + slot, par ^ 1u, abort_flag, p.status)) { ok = false; break; }
-            uint8_t* base = slots + slot * C::SLOT;
-            int b, h, kc;
-            attn_entry(s, c, b, h, kc);
-            tc::mbar_expect_tx(full + slot, (uint32_t)(2 * NB * 8192));
-            const int row = b * p.S_max + kc * 64;
-            for (int bx = 0; bx < NB; ++bx) {
-              tc::tma_load_2d(base + bx * 8192, &p.maps[0], full + slot, h * p.D + 64 * bx, row);
-              tc::tma_load_2d(base + 16384 + bx * 8192, &p.maps[1], full + slot, h * p.D + 64 * bx, row);
-            }
+            const int t = c / ph.nk, kc = c - t * ph.nk;
+            const uint32_t box = (uint32_t)min(DF_KC, ph.K - kc * DF_KC) * 64u;
+            const uint8_t* e = Ly->pack + ph.pack_off + (long long)t * ph.K * 128 + (long long)kc * 32768;
+            uint8_t* w = slots + slot * C::SLOT;
+            tc::mbar_expect_tx(full + slot, 2u * box);
+            bulk_g2s(w, e, box, full + slot);
+            bulk_g2s(w + 16384, e + box, box, full + slot);
+            pf_step();
           }
-          continue;
-        }
-        share(ph.T * ph.nk, G, g, c0, c1);
-        for (int c = c0; c < c1; ++c, ++seq) {
-          const int slot = seq % C::NSLOT;
-          const uint32_t par = (uint32_t)(seq / C::NSLOT) & 1u;
-          if (!tc::mbar_wait_sleep(empty + slot, par ^ 1u, abort_flag, p.status)) { ok = false; break; }
-          const int t = c / ph.nk, kc = c - t * ph.nk;
-          const uint32_t box = (uint32_t)min(DF_KC, ph.K - kc * DF_KC) * 64u;
-          const uint8_t* e = p.pack + ph.pack_off + (long long)t * ph.K * 128 + (long long)kc * 32768;
-          uint8_t* w = slots + slot * C::SLOT;
-          tc::mbar_expect_tx(full + slot, 2u * box);
-          bulk_g2s(w, e, box, full + slot);
-          bulk_g2s(w + 16384, e + box, box, full + slot);
-          pf_step();
         }
       }
       if (*abort_flag) {
         const long long t0 = clock64();  // let copies in flight land
         while (clock64() - t0 < 2000000) {}
-      }
-    }
-  } else if (warp == C::CW + 1) {
-    // ================================================ K/V prefetch ==========
-    // History rows are fixed for this step: pull this CTA's chunks of the
-    // cache into L2 while the first stages stream their factors.
-    if (lane == 0) {
-      for (int i = 0; i < DF_NMAPS; ++i) tc::tma_prefetch_desc(&p.maps[i]);
-      pdl_wait();
-      AttnSched s;
-      attn_sched(p, s);
-      const int NB = p.D >> 6;
-      int a0, a1;
-      share(s.pre[8], G, g, a0, a1);
-      for (int c = a0; c < a1; ++c) {
-        int b, h, kc;
-        attn_entry(s, c, b, h, kc);
-        for (int bx = 0; bx < NB; ++bx) {
-          prefetch_l2_2d(&p.maps[0], h * p.D + 64 * bx, b * p.S_max + kc * 64);
-          prefetch_l2_2d(&p.maps[1], h * p.D + 64 * bx, b * p.S_max + kc * 64);
-        }
       }
     }
   } else {
@@ -514,21 +524,40 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
     const int row0 = 2 * rowlane + rsub;
     constexpr int RSTEP = C::CT / 8;
     int seq = 0;
+    for (int l = 0; l < p.nlayer; ++l) {
+    const DfLayer* Ly = layer_of(l);
+    {
+      // this layer's stage table, read in every inner loop
+      consumer_sync<C::CT>();
+      const int* src = reinterpret_cast<const int*>(Ly->ph);
+      int* dst = reinterpret_cast<int*>(s_ph);
+      for (int i = tid; i < (int)(sizeof(DfPhase) * DF_NPHASE / 4); i += C::CT) dst[i] = src[i];
+      consumer_sync<C::CT>();
+    }
     for (int ph_i = 0; ph_i < DF_NPHASE; ++ph_i) {
       const DfPhase& ph = s_ph[ph_i];
-      float* part_cur = p.part + (ph_i & 1) * half;
-      const float* part_prev = p.part + ((ph_i + 1) & 1) * half;
+      const int gs = l * DF_NPHASE + ph_i;  // global stage index
+      float* part_cur = p.part + (gs & 1) * half;
+      const float* part_prev = p.part + ((gs + 1) & 1) * half;
+      // the previous stage is complete on every CTA once its counter
+      // (accumulated over the layers) reaches prev_target
+      const int prev_ctr = ph_i > 0 ? ph_i - 1 : DF_NPHASE - 1;
+      const int prev_target = G * (ph_i > 0 ? l + 1 : l);
       if (ph.type == DF_GEMV) {
+        const int src = (ph_i == 0 && l > 0) ? SRC_XOUT : ph.src;
         const int Ctot = ph.T * ph.nk;
         int c0, c1;
         share(Ctot, G, g, c0, c1);
         const int nseg = ph.map == MAP_SWIGLU ? 2 : 1;
-        const bool xin = ph.src == SRC_X || ph.src == SRC_XMID;
+        const bool xin = src == SRC_X || src == SRC_XMID || src == SRC_XOUT;
         // this CTA's schedule record of the stage (static: from the pack)
         {
-          const int4* src = reinterpret_cast<const int4*>(p.sched + (long long)ph_i * G + g);
+          // (stage 0 after the first layer: the previous layer's record 10)
+          const SchedRec* r = src == SRC_XOUT ? layer_of(l - 1)->sched + (long long)(DF_NPHASE + 1) * G
+                                              : Ly->sched + (long long)ph_i * G;
+          const int4* rs = reinterpret_cast<const int4*>(r + g);
           int4* dst = reinterpret_cast<int4*>(srec);
-          for (int w = tid; w < (int)(sizeof(SchedRec) / 16); w += C::CT) dst[w] = __ldg(src + w);
+          for (int w = tid; w < (int)(sizeof(SchedRec) / 16); w += C::CT) dst[w] = __ldg(rs + w);
         }
         consumer_sync<C::CT>();
 
@@ -539,7 +568,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
         const int n = srec->n;
         const int hpc = DF_KC / p.D;  // heads per 256-column chunk
         int nunits = srec->nunits;
-        if (ph.src == SRC_ATT) {
+        if (src == SRC_ATT) {
           nunits = n * MT * hpc;
           if (nunits > DF_MAX_UNITS) {
             if (tid == 0) atomicExch(p.status, DEV_STATUS_SCHEDULE);
@@ -555,12 +584,13 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
           }
         }
         if (xin) {
-          // x (the layer input: fixed during the launch) into the input rows
+          // x (the layer input, complete before this stage) into the input
+          // rows; zero rows past B (SRC_XOUT: x is built after the barrier)
           const int d4 = p.d >> 2;
           for (int e = tid; e < MT * d4; e += C::CT) {
             const int m = e / d4, j = (e - m * d4) * 4;
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (m < p.B) {
+            if (m < p.B && src != SRC_XOUT) {
               const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(p.x + (long long)m * p.d + j));
               v = make_float4(bf_lo(raw.x), bf_hi(raw.x), bf_lo(raw.y), bf_hi(raw.y));
             }
@@ -573,12 +603,14 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
             asm volatile("prefetch.global.L1 [%0];" ::"l"(ph.norm_g + o));
         }
         // ---- wait for the previous stage on every CTA ----
-        if (ph_i > 0 && tid == 0) grid_wait(p.bar + ph_i - 1, G, abort_flag, p.status);
+        if ((ph_i > 0 || l > 0) && tid == 0) grid_wait(p.bar + prev_ctr, prev_target, abort_flag, p.status);
         consumer_sync<C::CT>();
         // (2) the input itself, 4 consecutive values per group, two groups
         // per thread and step (their loads in flight together)
-        if (ph.src == SRC_XMID && nunits) {
-          // x' = x + (z V_o), rounded as the residual stream is stored
+        if ((src == SRC_XMID || src == SRC_XOUT) && nunits) {
+          // x' = x + (z V_o) (SRC_XMID), or the previous layer's output
+          // x = x' + (z V_dn) (SRC_XOUT), rounded as the residual stream is
+          // stored; the owners of its 64-column tiles also store it
           const int d4 = p.d >> 2, tot = p.B * d4;
           for (int e0 = tid; e0 < tot; e0 += 2 * C::CT) {
             const int e1 = e0 + C::CT;
@@ -593,7 +625,13 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
               if (k2 == 1 && !h1) continue;
               const int m = k2 ? m1 : m0, j = k2 ? j1 : j0;
               float4* a4 = reinterpret_cast<float4*>(abuf + m * DF_ABUF_COLS + j);
-              float4 v = *a4;
+              float4 v;
+              if (src == SRC_XMID) {
+                v = *a4;
+              } else {
+                const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(p.xm + (long long)m * p.d + j));
+                v = make_float4(bf_lo(raw.x), bf_hi(raw.x), bf_lo(raw.y), bf_hi(raw.y));
+              }
               add4(v, sp[k2]);
               v = round4(v);
               *a4 = v;
@@ -601,11 +639,11 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
                 uint2 o;
                 o.x = pack_bf2(v.x, v.y);
                 o.y = pack_bf2(v.z, v.w);
-                *reinterpret_cast<uint2*>(p.xm + (long long)m * p.d + j) = o;
+                *reinterpret_cast<uint2*>((src == SRC_XMID ? p.xm : p.x) + (long long)m * p.d + j) = o;
               }
             }
           }
-        } else if (ph.src == SRC_SWIGLU) {
+        } else if (src == SRC_SWIGLU) {
           // h = SiLU(gate) * up; a SwiGLU tile holds 32 gate then 32 up columns
           const int tot = n * MT * 64;
           for (int e = tid; e < tot; e += C::CT) {
@@ -622,7 +660,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
             }
             *reinterpret_cast<float4*>(abuf + m * DF_ABUF_COLS + ci * 256 + i) = v;
           }
-        } else if (ph.src == SRC_ATT) {
+        } else if (src == SRC_ATT) {
           // attention output: dims k % D .. + 3 of head k / D of row m
           const int tot = n * MT * 64;
           for (int e = tid; e < tot; e += C::CT) {
@@ -633,7 +671,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
               v = round4(attn_gather4(part_prev, utab + ((ci * MT + m) * hpc + i / p.D) * 16, k % p.D));
             *reinterpret_cast<float4*>(abuf + m * DF_ABUF_COLS + ci * 256 + i) = v;
           }
-        } else if (ph.src == SRC_PART) {
+        } else if (src == SRC_PART) {
           // fp32 rank activations z (plain column tiles of 64)
           const int tot = n * nseg * MT * 64;
           for (int e0 = tid; e0 < tot; e0 += 2 * C::CT) {
@@ -788,7 +826,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
             if (!tile_slots(q1, q1.tile_start[prob] + h * tph + j, G, utab + ui * 16))
               atomicExch(p.status, DEV_STATUS_SCHEDULE);
           }
-          if (tid == 0) grid_wait(p.bar + ph_i - 1, G, abort_flag, p.status);
+          if (tid == 0) grid_wait(p.bar + prev_ctr, prev_target, abort_flag, p.status);
           consumer_sync<C::CT>();
           for (int e = tid; e < np * 3 * (hd >> 2); e += C::CT) {
             const int i = (e % (hd >> 2)) * 4;
@@ -813,7 +851,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
             *reinterpret_cast<float4*>(qkv + (pr * 3 + prob) * D + i) = lo;
             *reinterpret_cast<float4*>(qkv + (pr * 3 + prob) * D + i + hd) = hi;
             if (prob > 0 && owner_of(s.pre[b] + h * s.nk[b] + s.nk[b] - 1, Ctot, G) == g) {
-              bf16* dst = (prob == 1 ? p.k_cache : p.v_cache) + ((long long)b * p.S_max + pos) * (p.H * D) +
+              bf16* dst = (prob == 1 ? Ly->k_cache : Ly->v_cache) + ((long long)b * p.S_max + pos) * (p.H * D) +
                           h * D;
               uint2 o;
               o.x = pack_bf2(lo.x, lo.y); o.y = pack_bf2(lo.z, lo.w);
@@ -974,13 +1012,15 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
       // thread's release, which is cumulative over them)
       if (tid == 0) red_release_add(p.bar + ph_i, 1);
     }
-    // ---- final pass: x = x' + z V_dn for this CTA's 64-column tiles ----
-    if (tid == 0) grid_wait(p.bar + DF_NPHASE - 1, G, abort_flag, p.status);
+    }  // layers
+    // ---- final pass: x = x' + z V_dn of the last layer, this CTA's tiles ----
+    if (tid == 0) grid_wait(p.bar + DF_NPHASE - 1, G * p.nlayer, abort_flag, p.status);
     consumer_sync<C::CT>();
     {
-      const float* part8 = p.part + ((DF_NPHASE - 1) & 1) * half;
-      // record DF_NPHASE: tiles g, g + G, ... of the last stage
-      const int4* src = reinterpret_cast<const int4*>(p.sched + (long long)DF_NPHASE * G + g);
+      const float* part8 = p.part + ((p.nlayer * DF_NPHASE - 1) & 1) * half;
+      // record DF_NPHASE of the last layer: tiles g, g + G, ... of its last stage
+      const int4* src =
+          reinterpret_cast<const int4*>(layer_of(p.nlayer - 1)->sched + (long long)DF_NPHASE * G + g);
       for (int w = tid; w < (int)(sizeof(SchedRec) / 16); w += C::CT) reinterpret_cast<int4*>(srec)[w] = __ldg(src + w);
       consumer_sync<C::CT>();
       const int nt = srec->nunits;
@@ -1196,7 +1236,15 @@ bool build_sched(const DfPhase* P, int G, int d, SchedRec* R) {
       if (r.nunits > DF_MAX_UNITS) return false;
     }
   }
-  // final pass: tiles g, g + G, ... of the last stage
+  // record 10: every tile of the last stage (the next layer's input)
+  for (int g = 0; g < G; ++g) {
+    SchedRec& r = R[(DF_NPHASE + 1) * G + g];
+    r.nunits = d >> 6;
+    if (r.nunits > DF_MAX_UNITS) return false;
+    for (int t = 0; t < r.nunits; ++t)
+      if (!tile_slots(P[DF_NPHASE - 1], t, G, r.utab[t])) return false;
+  }
+  // record 9, the final pass: tiles g, g + G, ... of the last stage
   for (int g = 0; g < G; ++g) {
     SchedRec& r = R[DF_NPHASE * G + g];
     for (int t = g; t < (d >> 6); t += G) {
@@ -1213,7 +1261,7 @@ long long sched_offset(long long factor_bytes) { return (factor_bytes + 127) / 1
 // Whether every CTA's share of every GEMV stage stays within the kernel's
 // fixed per-CTA limits (tiles touched, input chunks, contributor table).
 bool stages_fit(const DfPhase* P, int G, int MT, int D) {
-  const int CW = MT <= 2 ? 16 : 8;
+  const int CW = 16;
   const int red_bytes = std::max(CW * MT * 64 * 4, 2048);
   for (int i = 0; i < DF_NPHASE; ++i) {
     const DfPhase& ph = P[i];
@@ -1288,36 +1336,45 @@ int decode_pack_launch(const DecodeLayerDesc& L, void* dst, long long bytes, int
   return cuda_status(cudaGetLastError());
 }
 
-int decode_fused_launch(const DecodeLayerDesc& L, bf16* x, bf16* kc, bf16* vc, const int* seqlens,
-                        int B, int S_max, bf16* xm, float* part, long long part_floats, int* bar,
-                        int* done, int* status, int sm_count, cudaStream_t stream) {
-  if (!L.pack) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+namespace {
+
+// The kernel's view of one layer (caches, pack, schedule, stage table).
+int fill_layer(const DecodeLayerDesc& L, bf16* kc, bf16* vc, int B, int S_max, int G, DfLayer* out,
+               long long* algo_bytes) {
+  if (!L.pack || !kc || !vc) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   if (!decode_fused_supported(B, L.d, L.D, L.r, L.r_f) || L.f % 8) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
-  const int G = sm_count;
-  if (2LL * G * DF_MAX_SU * DF_PART_STRIDE > part_floats) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   // Attention: with equal lengths a CTA's share spans at most this many pairs.
   if ((B * L.H + G - 1) / G + 1 > DF_MAX_PAIRS) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
-  DfParams p;
-  memset(&p, 0, sizeof(p));
-  const long long pack_bytes = build_stages(L, p.ph, nullptr);
-  if (!stages_fit(p.ph, G, B <= 1 ? 1 : (B <= 2 ? 2 : 4), L.D)) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
-  p.pack = static_cast<const uint8_t*>(L.pack);
+  memset(out, 0, sizeof(DfLayer));
+  const long long pack_bytes = build_stages(L, out->ph, nullptr);
+  if (!stages_fit(out->ph, G, B <= 1 ? 1 : (B <= 2 ? 2 : 4), L.D)) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  out->pack = static_cast<const uint8_t*>(L.pack);
   // the pack holds the schedule records for this device's SM count
-  p.sched = reinterpret_cast<const SchedRec*>(p.pack + sched_offset(pack_bytes));
+  out->sched = reinterpret_cast<const SchedRec*>(out->pack + sched_offset(pack_bytes));
   const long long HD = (long long)L.H * L.D;
-  FSVD_TRY(encode_map(&p.maps[0], kc, (long long)B * S_max, HD, HD, 64, 64, true));
-  FSVD_TRY(encode_map(&p.maps[1], vc, (long long)B * S_max, HD, HD, 64, 64, true));
+  FSVD_TRY(encode_map(&out->kmap, kc, (long long)B * S_max, HD, HD, 64, 64, true));
+  FSVD_TRY(encode_map(&out->vmap, vc, (long long)B * S_max, HD, HD, 64, 64, true));
+  out->k_cache = kc;
+  out->v_cache = vc;
+  // factor bytes of the layer, and the cache bytes at the longest context
+  const long long d = L.d, r = L.r, rf = L.r_f, f = L.f;
+  *algo_bytes = 2 * (4 * 2 * d * r + d * 2 * rf + 2 * rf * f + f * rf + rf * d) + 2LL * 2 * B * S_max * HD;
+  return FLASHSVD_OK;
+}
+
+void fill_common(DfParams& p, const DecodeLayerDesc& L, int B, int S_max, const int* seqlens, bf16* x,
+                 bf16* xm, float* part, int* bar, int* done, int* status) {
   p.B = B; p.H = L.H; p.D = L.D; p.S_max = S_max; p.d = L.d;
   p.eps = L.eps;
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)L.D);
   p.seqlens = seqlens;
-  p.x = x; p.xm = xm; p.k_cache = kc; p.v_cache = vc;
+  p.x = x; p.xm = xm;
   p.rope_cos = L.rope_cos; p.rope_sin = L.rope_sin;
   p.part = part; p.bar = bar; p.done = done; p.status = status;
+}
 
-  const double bytes = (double)pack_bytes + 2.0 * 2.0 * B * (double)S_max * HD;
-  const LaunchTag tag{"decode_layer_fused", bytes, 0.0};
-
+int launch_df(const DfParams& p, int G, double bytes, cudaStream_t stream) {
+  const LaunchTag tag{p.nlayer > 1 ? "decode_layers_fused" : "decode_layer_fused", bytes, 0.0};
 #define FSVD_DF_LAUNCH(MT_)                                                                          \
   {                                                                                                  \
     auto kern = decode_layer_kernel<MT_>;                                                            \
@@ -1328,10 +1385,88 @@ int decode_fused_launch(const DecodeLayerDesc& L, bf16* x, bf16* kc, bf16* vc, c
     }                                                                                                \
     return launch_pdl(tag, kern, dim3(G), dim3(DfCfg<MT_>::THREADS), (size_t)DfCfg<MT_>::SMEM, stream, p); \
   }
-  if (B <= 1) FSVD_DF_LAUNCH(1)
-  if (B <= 2) FSVD_DF_LAUNCH(2)
+  if (p.B <= 1) FSVD_DF_LAUNCH(1)
+  if (p.B <= 2) FSVD_DF_LAUNCH(2)
   FSVD_DF_LAUNCH(4)
 #undef FSVD_DF_LAUNCH
+}
+
+}  // namespace
+
+int decode_fused_launch(const DecodeLayerDesc& L, bf16* x, bf16* kc, bf16* vc, const int* seqlens,
+                        int B, int S_max, bf16* xm, float* part, long long part_floats, int* bar,
+                        int* done, int* status, int sm_count, cudaStream_t stream) {
+  const int G = sm_count;
+  if (2LL * G * DF_MAX_SU * DF_PART_STRIDE > part_floats) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  DfParams p;
+  memset(&p, 0, sizeof(p));
+  long long bytes = 0;
+  FSVD_TRY(fill_layer(L, kc, vc, B, S_max, G, &p.inl, &bytes));
+  p.layers = nullptr;
+  p.nlayer = 1;
+  fill_common(p, L, B, S_max, seqlens, x, xm, part, bar, done, status);
+  return launch_df(p, G, (double)bytes, stream);
+}
+
+struct DecodePlan {
+  DfParams p;           // layers points at dev; per-launch fields set at launch
+  DfLayer* dev = nullptr;
+  DecodeLayerDesc first;
+  int G = 0;
+  double bytes = 0.0;
+};
+
+int decode_plan_create(const DecodeLayerDesc* layers, int n, bf16* const* k_caches, bf16* const* v_caches,
+                       int B, int S_max, int sm_count, DecodePlan** out) {
+  if (!layers || n <= 0 || !k_caches || !v_caches || !out) return FLASHSVD_ERR_INVALID_ARG;
+  const int G = sm_count;
+  std::vector<DfLayer> host((size_t)n);
+  double bytes = 0.0;
+  for (int i = 0; i < n; ++i) {
+    const DecodeLayerDesc& L = layers[i];
+    // model-level shapes and tables must agree across the layers
+    if (L.d != layers[0].d || L.H != layers[0].H || L.D != layers[0].D || L.f != layers[0].f ||
+        L.eps != layers[0].eps || L.rope_cos != layers[0].rope_cos || L.rope_sin != layers[0].rope_sin)
+      return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+    long long b = 0;
+    FSVD_TRY(fill_layer(L, k_caches[i], v_caches[i], B, S_max, G, &host[i], &b));
+    bytes += (double)b;
+  }
+  DecodePlan* plan = new DecodePlan();
+  if (cudaMalloc(&plan->dev, sizeof(DfLayer) * n) != cudaSuccess) {
+    delete plan;
+    return FLASHSVD_ERR_NO_MEMORY;
+  }
+  const cudaError_t e = cudaMemcpy(plan->dev, host.data(), sizeof(DfLayer) * n, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    cudaFree(plan->dev);
+    delete plan;
+    return cuda_status(e);
+  }
+  memset(&plan->p, 0, sizeof(plan->p));
+  plan->p.layers = plan->dev;
+  plan->p.nlayer = n;
+  plan->first = layers[0];
+  plan->G = G;
+  plan->bytes = bytes;
+  plan->p.B = B;
+  plan->p.S_max = S_max;
+  *out = plan;
+  return FLASHSVD_OK;
+}
+
+int decode_plan_launch(const DecodePlan* plan, bf16* x, const int* seqlens, bf16* xm, float* part,
+                       long long part_floats, int* bar, int* done, int* status, cudaStream_t stream) {
+  if (2LL * plan->G * DF_MAX_SU * DF_PART_STRIDE > part_floats) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  DfParams p = plan->p;
+  fill_common(p, plan->first, plan->p.B, plan->p.S_max, seqlens, x, xm, part, bar, done, status);
+  return launch_df(p, plan->G, plan->bytes, stream);
+}
+
+void decode_plan_destroy(DecodePlan* plan) {
+  if (!plan) return;
+  cudaFree(plan->dev);
+  delete plan;
 }
 
 }  // namespace fsvd

@@ -120,6 +120,14 @@ int decode_pack_launch(const DecodeLayerDesc& L, void* dst, long long bytes, int
 int decode_fused_launch(const DecodeLayerDesc& L, bf16* x, bf16* kc, bf16* vc, const int* seqlens,
                         int B, int S_max, bf16* xm, float* part, long long part_floats, int* bar,
                         int* done, int* status, int sm_count, cudaStream_t stream);
+// Several layers in one launch (layer i on caches k_caches[i], v_caches[i]);
+// the plan owns a device copy of the layers' descriptors.
+struct DecodePlan;
+int decode_plan_create(const DecodeLayerDesc* layers, int n, bf16* const* k_caches, bf16* const* v_caches,
+                       int B, int S_max, int sm_count, DecodePlan** out);
+int decode_plan_launch(const DecodePlan* plan, bf16* x, const int* seqlens, bf16* xm, float* part,
+                       long long part_floats, int* bar, int* done, int* status, cudaStream_t stream);
+void decode_plan_destroy(DecodePlan* plan);
 int encode_map(CUtensorMap* map, const void* base, long long rows, long long cols, long long ld,
                int box_cols, int box_rows, bool swizzle128);
 constexpr int kFusedPartFloats = 2 * 148 * 16 * 640;  // two halves; per SM 16 slots of 640 floats

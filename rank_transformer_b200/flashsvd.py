@@ -72,6 +72,9 @@ _SIGS = {
     "flashsvd_set_decode_path": ([_i], _i),
     "flashsvd_decode_pack_bytes": ([_p, C.POINTER(C.c_size_t)], _i),
     "flashsvd_decode_pack": ([_p, _p, C.c_size_t, _p], _i),
+    "flashsvd_decode_plan_create": ([_p, _i, _p, _p, _i, _i, _p], _i),
+    "flashsvd_decode_plan_forward": ([_p, _p, _p, _p], _i),
+    "flashsvd_decode_plan_destroy": ([_p], _i),
     "flashsvd_profile_enable": ([_i], _i),
     "flashsvd_profile_report": ([C.c_char_p, _i, _i], _i),
     "flashsvd_lowrank_linear": ([_p, _p, _p, _p, _p, _i, _i, _i, _i, _p], _i),
@@ -275,6 +278,36 @@ class Graph:
     def destroy(self) -> None:
         if self.handle:
             _call("flashsvd_graph_destroy", self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+
+class DecodePlan:
+    """Owner of a flashsvd_decode_plan: the decode step of several decoder
+    layers (each with a decode pack) as one launch."""
+
+    def __init__(self, layers, k_caches, v_caches, B: int, S_max: int):
+        n = len(layers)
+        arr = (Layer * n)(*layers)
+        kc = (C.c_void_p * n)(*[ptr(t) for t in k_caches])
+        vc = (C.c_void_p * n)(*[ptr(t) for t in v_caches])
+        h = _p()
+        _call("flashsvd_decode_plan_create", arr, n, kc, vc, B, S_max, C.byref(h))
+        self.handle = h.value
+        self._keep = (arr, kc, vc)
+
+    def forward(self, x, cache_seqlens, stream=None) -> None:
+        _call("flashsvd_decode_plan_forward", self.handle, ptr(x), ptr(cache_seqlens),
+              stream_handle(stream))
+
+    def destroy(self) -> None:
+        if self.handle:
+            _call("flashsvd_decode_plan_destroy", self.handle)
             self.handle = None
 
     def __del__(self):

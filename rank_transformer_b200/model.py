@@ -109,6 +109,14 @@ class DecoderModel:
                 buf = torch.empty(n, dtype=torch.uint8, device=device)
                 fs.decode_pack(L, buf)
                 self.packs.append(buf)
+        # With a pack on every layer, the decode step of all layers runs as
+        # one launch of the fused kernel (a decode plan).
+        self.plan = None
+        if decode_pack and all(pk is not None for pk in self.packs):
+            try:
+                self.plan = fs.DecodePlan(self.structs, self.k_cache, self.v_cache, B, S_max)
+            except fs.FlashSVDError:
+                self.plan = None
         self.graphs = None
         self.step_graph = None
 
@@ -162,18 +170,35 @@ class DecoderModel:
         fs.greedy(self.logits, self.tokens, self.B, cfg.vocab, stream)
         fs.advance_seqlens(self.seqlens, self.B, stream)
 
+    def _layers_decode(self, stream):
+        if self.plan is not None:
+            self.plan.forward(self.x, self.seqlens, stream)
+            return
+        for i in range(self.cfg.layers):
+            fs.layer_forward(self.structs[i], self.x, self.k_cache[i], self.v_cache[i],
+                             self.seqlens, self.B, 1, self.S_max, fs.DECODE, stream)
+
     def decode_step_eager(self, stream=None):
         cfg = self.cfg
         fs.embed(self.tokens, self.emb, self.x, self.B, cfg.d, cfg.vocab, stream)
-        for i in range(cfg.layers):
-            fs.layer_forward(self.structs[i], self.x, self.k_cache[i], self.v_cache[i],
-                             self.seqlens, self.B, 1, self.S_max, fs.DECODE, stream)
+        self._layers_decode(stream)
         self._head(stream)
 
     def capture(self, stream, compose: bool = True):
         """Capture one graph per layer (plus the embedding and the head) and,
         with ``compose``, one graph for the whole step built from them."""
         cfg = self.cfg
+        if self.plan is not None:
+            # all layers are one launch: the step is one graph
+            with torch.cuda.stream(stream):
+                fs.capture_begin(stream)
+                fs.embed(self.tokens, self.emb, self.x, self.B, cfg.d, cfg.vocab, stream)
+                self.plan.forward(self.x, self.seqlens, stream)
+                self._head(stream)
+                g = fs.capture_end(stream)
+            self.graphs = [g]
+            self.step_graph = g
+            return
         with torch.cuda.stream(stream):
             fs.capture_begin(stream)
             fs.embed(self.tokens, self.emb, self.x, self.B, cfg.d, cfg.vocab, stream)

@@ -346,3 +346,70 @@ def test_decode_graph_replay_bitwise(fs):
         assert np.array_equal(a, b)
         assert np.array_equal(a, c)
     assert np.array_equal(kc_e, kc_g)
+
+
+def _torch_layer(fs, d, H, D, f, r, r_f, cos_t, sin_t, gen):
+    """Random bf16 layer on the device (no oracle involved) with its pack."""
+    def mat(rows, cols):
+        return (torch.randn(rows, cols, device="cuda", generator=gen) * rows ** -0.5).to(torch.bfloat16)
+    w = {}
+    for n in ("q", "k", "v", "o"):
+        w["U_" + n], w["V_" + n] = mat(d, r), mat(r, d)
+    w["U_gu"], w["V_gu"] = mat(d, 2 * r_f), mat(2 * r_f, f)
+    w["U_dn"], w["V_dn"] = mat(f, r_f), mat(r_f, d)
+    w["g1"] = (1 + 0.1 * torch.randn(d, device="cuda", generator=gen)).to(torch.bfloat16)
+    w["g2"] = (1 + 0.1 * torch.randn(d, device="cuda", generator=gen)).to(torch.bfloat16)
+    L = fs.Layer()
+    L.kind = fs.DECODER
+    L.d, L.H, L.D, L.f = d, H, D, f
+    L.norm_eps = 1e-5
+    L.norm1_g, L.norm2_g = w["g1"].data_ptr(), w["g2"].data_ptr()
+    for n in ("q", "k", "v", "o"):
+        F = getattr(L, n)
+        F.U, F.V, F.bias, F.r = w["U_" + n].data_ptr(), w["V_" + n].data_ptr(), None, r
+    L.U_gu, L.V_gu, L.r_f = w["U_gu"].data_ptr(), w["V_gu"].data_ptr(), r_f
+    L.down.U, L.down.V, L.down.bias, L.down.r = w["U_dn"].data_ptr(), w["V_dn"].data_ptr(), None, r_f
+    L.rope_cos, L.rope_sin = cos_t.data_ptr(), sin_t.data_ptr()
+    w["pack"] = torch.empty(fs.decode_pack_bytes(L), dtype=torch.uint8, device="cuda")
+    fs.decode_pack(L, w["pack"])
+    return L, w
+
+
+@pytest.mark.parametrize("shape", ["tiny-mixed-ranks", "7b-2-layers"])
+@pytest.mark.parametrize("B", [1, 4])
+def test_decode_plan_matches_layer_calls(fs, shape, B):
+    """A decode plan (all layers in one launch) gives bit-identical x and
+    caches to one fused DECODE layer_forward call per layer: each layer's
+    input is summed from the previous layer's partials in the same order
+    the per-layer final pass uses."""
+    if shape == "tiny-mixed-ranks":
+        d, H, D, f, P = 256, 4, 64, 688, 100
+        ranks = [(64, 64), (128, 96), (64, 128)]
+    else:
+        d, H, D, f, P = 4096, 32, 128, 11008, 2048
+        ranks = [(1216, 1792), (832, 1216)]
+    S_max = P + 4
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(7)
+    cos_t = torch.empty((S_max, D // 2), dtype=torch.float32, device="cuda")
+    sin_t = torch.empty_like(cos_t)
+    fs.rope_table(cos_t, sin_t, S_max, D, 10000.0)
+    layers = [_torch_layer(fs, d, H, D, f, r, rf, cos_t, sin_t, gen) for r, rf in ranks]
+    kc0 = [torch.randn(B, S_max, H, D, device="cuda", generator=gen).to(torch.bfloat16) for _ in layers]
+    vc0 = [torch.randn(B, S_max, H, D, device="cuda", generator=gen).to(torch.bfloat16) for _ in layers]
+    x0 = torch.randn(B, d, device="cuda", generator=gen).to(torch.bfloat16)
+    seq = torch.full((B,), P, dtype=torch.int32, device="cuda")
+
+    x_a, kc_a, vc_a = x0.clone(), [k.clone() for k in kc0], [v.clone() for v in vc0]
+    for (L, _), kc, vc in zip(layers, kc_a, vc_a):
+        fs.layer_forward(L, x_a, kc, vc, seq, B, 1, S_max, fs.DECODE)
+    x_b, kc_b, vc_b = x0.clone(), [k.clone() for k in kc0], [v.clone() for v in vc0]
+    plan = fs.DecodePlan([L for L, _ in layers], kc_b, vc_b, B, S_max)
+    plan.forward(x_b, seq)
+    torch.cuda.synchronize()
+    fs.check_device_status()
+    plan.destroy()
+    assert torch.equal(x_a.view(torch.int16), x_b.view(torch.int16))
+    for a, b in zip(kc_a + vc_a, kc_b + vc_b):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert torch.isfinite(x_b.float()).all()
