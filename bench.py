@@ -41,6 +41,8 @@ def parse():
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=32,
+                    help="decoder layers (default 32; fewer only for small profiling cases)")
     ap.add_argument("--profile-step", action="store_true",
                     help="after warm-up, run one prefill and two decode steps inside an NVTX "
                          "range 'profile_step' (for an ncu launch list) and exit")
@@ -48,6 +50,29 @@ def parse():
 
 
 # ------------------------------------------------------------ peaks ------
+
+def ncu_traffic(kernel: str, layers: int):
+    """DRAM bytes per launch of the fused decode kernel from the committed
+    ncu capture (profiles/decode_layers_fused_*.md: per-layer traffic of a
+    2-layer launch, scaled to `layers`); None when the kernel source has
+    changed since that capture or for other kernels."""
+    import hashlib
+    import re as _re
+    if kernel != "decode_layers_fused":
+        return None
+    prof = os.path.join(ROOT, "profiles", "decode_layers_fused_llama7b_2layers_b1_ctx2048.md")
+    src = os.path.join(ROOT, "rank_transformer_b200", "csrc", "decode_fused.cu")
+    try:
+        text = open(prof).read()
+        sha = hashlib.sha1(open(src, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    m = _re.search(r"sha1 \(rank_transformer_b200/csrc/decode_fused.cu\): ([0-9a-f]{40})", text)
+    t = _re.search(r"= ([0-9.]+) MB per layer", text)
+    if not m or not t or m.group(1) != sha:
+        return None
+    return float(t.group(1)) * 1e6 * layers
+
 
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -207,7 +232,8 @@ def run_ours(args):
     from rank_transformer_b200.model import LLAMA7B, DecoderModel
 
     B = args.batch
-    cfg = LLAMA7B
+    import dataclasses
+    cfg = dataclasses.replace(LLAMA7B, layers=args.layers)
     S_max = PROMPT + DECODE_STEPS
     fs.init(local, max_tokens=B * PROMPT, max_rank=2368, max_hidden=cfg.d, max_ffn=cfg.f)
     model = DecoderModel(cfg, B, S_max, seed=1234 + rank)
@@ -291,16 +317,25 @@ def run_ours(args):
 
     # Dominant decode kernel: per-launch CUDA-event timings of one eager
     # decode step (the profiler brackets each library launch on the stream).
+    # Steps at contexts PROMPT .. PROMPT + 2 (the timed region covers
+    # PROMPT .. PROMPT + 127).
+    model.seqlens.fill_(PROMPT)
     fs.profile_enable(True)
     with torch.cuda.stream(stream):
-        model.decode_step_eager(stream)
-        model.decode_step_eager(stream)
+        for _ in range(3):
+            model.decode_step_eager(stream)
     prof = fs.profile_report(reset=True)
     fs.profile_enable(False)
     prof = {k: v for k, v in prof.items() if v["launches"] > 0}
     top = max(prof, key=lambda k: prof[k]["ms"])
     tp = prof[top]
-    achieved = (tp["bytes"] / tp["launches"]) / (tp["ms"] / tp["launches"] / 1e3) / 1e9
+    if top == "decode_layers_fused":
+        # one launch = every decoder layer of a step: its algorithmic bytes
+        # at the mean profiled context
+        alg_per_launch = model.layers_decode_bytes(PROMPT + 1)
+    else:
+        alg_per_launch = tp["bytes"] / tp["launches"]
+    achieved = alg_per_launch / (tp["ms"] / tp["launches"] / 1e3) / 1e9
 
     # End to end through the public call: pinned host prompt in, generated
     # tokens out, on the same stream, timed with events around everything.
@@ -330,7 +365,9 @@ def run_ours(args):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": f"llama2-7b-shaped low-rank decoder (rho=0.6, r=1216/1792), "
                                    f"B={B}, prefill {PROMPT} + {DECODE_STEPS} greedy decode steps, "
-                                   f"per-layer CUDA graphs",
+                                   + ("decode step = embedding + one fused launch of all 32 layers "
+                                      "+ head, replayed as one CUDA graph" if model.plan is not None
+                                      else "per-layer CUDA graphs"),
                        "batch": B, "prompt": PROMPT, "decode_steps": DECODE_STEPS,
                        "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (7.75 GB of factors streamed per step)"},
@@ -339,8 +376,13 @@ def run_ours(args):
                            "frac": dec_gbs / peaks["hbm_gbs"],
                            "bytes_per_step": step_bytes / DECODE_STEPS},
             "roofline": {"bound": "hbm", "kernel": top, "achieved": achieved,
+                         "algorithmic_bytes_per_launch": alg_per_launch,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                         "frac": achieved / peaks["hbm_gbs"],
+                         "traffic": ncu_traffic(top, cfg.layers),
+                         "traffic_source": "ncu dram__bytes_read+write of a 2-layer launch, "
+                                           "scaled per layer (profiles/decode_layers_fused_"
+                                           "llama7b_2layers_b1_ctx2048.md)",
                          "launches_timed": tp["launches"],
                          "peak_source": peaks["source"] + " (burst copy)"},
             "kernel_times_ms": {k: round(v["ms"], 4) for k, v in sorted(prof.items())},

@@ -5,9 +5,13 @@ the forward pass is a libflashsvd call.
 
 ``DecoderModel``: Llama-shaped pre-norm decoder whose seven per-layer
 projections are rank-r factor pairs (q, k, v, o, packed gate|up, down), a
-dense LM head and a contiguous bf16 KV cache per layer.  Decode runs one
-replayable CUDA graph per layer (FlashSVD v1.5 explainer, Technical Summary,
-Methodology 4), with positions held in device memory.
+dense LM head and a contiguous bf16 KV cache per layer.  Each layer's
+factors are also kept as a decode pack, and the decoder layers of a decode
+step run as one fused launch (a decode plan); the step (embedding, layers,
+head) is captured and replayed as a CUDA graph (FlashSVD v1.5 explainer,
+Technical Summary, Methodology 4), with positions held in device memory.
+Without packs, decode replays one graph per layer over the per-stage
+kernels.
 
 ``EncoderModel``: BERT-shaped post-LN encoder with every linear factorized.
 """
@@ -240,6 +244,17 @@ class DecoderModel:
         kv = 2 * cfg.layers * (context + 1) * cfg.d * 2 * self.B
         act = self.B * cfg.d * 2 * 2 * cfg.layers
         return self.weight_bytes() + kv + act
+
+    def layers_decode_bytes(self, context: int) -> int:
+        """Algorithmic HBM bytes of the decoder layers of one decode step
+        (the work of one decode-plan launch): every layer's factors and norm
+        gains once, its K/V history at cache length ``context`` plus the new
+        rows, and the activations in and out."""
+        cfg = self.cfg
+        n = sum(t.numel() for w in self.layers for k, t in w.items())
+        kv = 2 * cfg.layers * (context + 1) * cfg.d * 2 * self.B
+        act = self.B * cfg.d * 2 * 2 * cfg.layers
+        return 2 * n + kv + act
 
     # --------------------------------------------------------- generate --
     def generate(self, prompt_host, steps: int, stream=None):
