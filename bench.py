@@ -51,6 +51,22 @@ def parse():
 
 # ------------------------------------------------------------ peaks ------
 
+def max_over_ranks(values, world: int, device):
+    """Element-wise max of per-rank timings over all ranks (every rank gets
+    the result); a no-op for one rank."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms: float) -> float:
+    """Units of all ranks per second, over the slowest rank's time."""
+    return world * units_per_rank / (ms / 1e3)
+
+
 def ncu_traffic(kernel: str, layers: int):
     """DRAM bytes per launch of the fused decode kernel from the committed
     ncu capture (profiles/decode_layers_fused_*.md: per-layer traffic of a
@@ -299,15 +315,9 @@ def run_ours(args):
     pre_ms = sum(e[0].elapsed_time(e[1]) for e in events)
     dec_ms = sum(e[1].elapsed_time(e[2]) for e in events)
     tot_ms = sum(e[0].elapsed_time(e[2]) for e in events)
-    t = torch.tensor([pre_ms, dec_ms, tot_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    pre_ms, dec_ms, tot_ms = t.tolist()
-
-    dec_tokens = world * B * DECODE_STEPS * args.steps
-    pre_tokens = world * B * PROMPT * args.steps
-    value = dec_tokens / (dec_ms / 1e3)
-    prefill_tok_s = pre_tokens / (pre_ms / 1e3)
+    pre_ms, dec_ms, tot_ms = max_over_ranks([pre_ms, dec_ms, tot_ms], world, "cuda")
+    value = whole_job_rate(B * DECODE_STEPS * args.steps, world, dec_ms)
+    prefill_tok_s = whole_job_rate(B * PROMPT * args.steps, world, pre_ms)
     peaks = measured_peaks()
 
     # Decode-step roofline: algorithmic bytes of the 128 steps / decode time.
@@ -347,8 +357,8 @@ def run_ours(args):
         out = model.generate(prompt_host, DECODE_STEPS, stream)
         e1.record(stream)
     stream.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    e2e_value = world * B * DECODE_STEPS / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1)], world, "cuda")[0]
+    e2e_value = whole_job_rate(B * DECODE_STEPS, world, e2e_ms)
     assert out.shape == (B, DECODE_STEPS)
 
     cpu = None
