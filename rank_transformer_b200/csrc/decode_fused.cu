@@ -332,13 +332,25 @@ __device__ __forceinline__ float4 round4(float4 v) {
   return make_float4(bf_round(v.x), bf_round(v.y), bf_round(v.z), bf_round(v.w));
 }
 
+// (a0, a1) += x * (y0, y1): one packed fp32x2 FMA (sm_100).
+__device__ __forceinline__ void ffma2(float& a0, float& a1, float x, float y0, float y1) {
+  asm("{\n\t.reg .b64 acc, xx, yy;\n\t"
+      "mov.b64 acc, {%0, %1};\n\t"
+      "mov.b64 xx, {%2, %2};\n\t"
+      "mov.b64 yy, {%3, %4};\n\t"
+      "fma.rn.f32x2 acc, xx, yy, acc;\n\t"
+      "mov.b64 {%0, %1}, acc;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(x), "f"(y0), "f"(y1));
+}
+
 // acc[m][0..7] += A[m][kk] * W[kk][8 columns] over this thread's rows of a
 // 256-row entry.  a points at the entry's input chunk (row m at
-// m * DF_ABUF_COLS); NORM scales it by rstd[m] * g[kk].  Rows at or beyond kn
+// m * DF_ABUF_COLS).  FULL: all 256 rows are valid; else rows at or beyond kn
 // are masked (their shared memory holds stale data).
-template <int MT, int NORM, int RSTEP>
+template <int MT, int RSTEP, bool FULL>
 __device__ __forceinline__ void entry_mac(float (&acc)[MT][8], const uint8_t* w, const float* a, int kn,
-                                          int row0, const bf16* g, const float* rstd) {
+                                          int row0) {
   constexpr int IT = DF_KC / RSTEP;
   uint4 u[IT];
   float av[IT][MT];
@@ -349,23 +361,18 @@ __device__ __forceinline__ void entry_mac(float (&acc)[MT][8], const uint8_t* w,
 #pragma unroll
     for (int m = 0; m < MT; ++m) av[i][m] = a[m * DF_ABUF_COLS + kk];
   }
-  float gk[IT];
 #pragma unroll
   for (int i = 0; i < IT; ++i) {
-    const int kk = row0 + RSTEP * i;
-    gk[i] = NORM ? bf2f(g[kk < kn ? kk : 0]) : 1.f;
-  }
-#pragma unroll
-  for (int i = 0; i < IT; ++i) {
-    const bool valid = row0 + RSTEP * i < kn;
-    const float wv[8] = {bf_lo(u[i].x), bf_hi(u[i].x), bf_lo(u[i].y), bf_hi(u[i].y),
-                         bf_lo(u[i].z), bf_hi(u[i].z), bf_lo(u[i].w), bf_hi(u[i].w)};
+    const bool valid = FULL || row0 + RSTEP * i < kn;
+    uint4 q = u[i];
+    if (!FULL && !valid) q = make_uint4(0u, 0u, 0u, 0u);
+    const float wv[8] = {bf_lo(q.x), bf_hi(q.x), bf_lo(q.y), bf_hi(q.y),
+                         bf_lo(q.z), bf_hi(q.z), bf_lo(q.w), bf_hi(q.w)};
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
-      float x = NORM ? av[i][m] * (rstd[m] * gk[i]) : av[i][m];
-      x = valid ? x : 0.f;
+      const float x = (FULL || valid) ? av[i][m] : 0.f;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) acc[m][j] = fmaf(x, valid ? wv[j] : 0.f, acc[m][j]);
+      for (int j = 0; j < 8; j += 2) ffma2(acc[m][j], acc[m][j + 1], x, wv[j], wv[j + 1]);
     }
   }
 }
@@ -760,18 +767,20 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
           const int k0 = kc * DF_KC;
           const int kn = min(DF_KC, ph.K - k0);
           const uint8_t* w = slots + slot * C::SLOT + box * 16384 + chunk * 16;
-          if (ph.norm) {
-            entry_mac<MT, 0, RSTEP>(acc, w, abuf + k0, kn, row0, nullptr, s_rstd);
-          } else {
-            const int off = srec->chunk_of[c - c0] * 256 * nseg + (nseg == 2 ? box * 256 : 0);
-            entry_mac<MT, 0, RSTEP>(acc, w, abuf + off, kn, row0, nullptr, s_rstd);
-          }
+          const float* ain = ph.norm ? abuf + k0
+                                     : abuf + srec->chunk_of[c - c0] * 256 * nseg + (nseg == 2 ? box * 256 : 0);
+          if (kn == DF_KC) entry_mac<MT, RSTEP, true>(acc, w, ain, kn, row0);
+          else entry_mac<MT, RSTEP, false>(acc, w, ain, kn, row0);
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(empty + slot);
 
           const bool tile_end = (c == c1 - 1) || (kc == ph.nk - 1);
           if (!tile_end) continue;
           // ---- this CTA's partial of tile t ----
+          // (tile ends alternate between two scratch areas when both fit, so
+          // one CTA barrier per tile end suffices)
+          constexpr bool kDual = C::SCR_BYTES >= C::RED_BYTES;
+          float* rb = (kDual && (su & 1)) ? scr : red;
 #pragma unroll
           for (int m = 0; m < MT; ++m)
 #pragma unroll
@@ -780,7 +789,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
               v += __shfl_xor_sync(0xffffffffu, v, 4);
               v += __shfl_xor_sync(0xffffffffu, v, 16);
               acc[m][j] = 0.f;
-              if ((lane & 20) == 0) red[(warp * MT + m) * 64 + cg * 8 + j] = v;
+              if ((lane & 20) == 0) rb[(warp * MT + m) * 64 + cg * 8 + j] = v;
             }
           consumer_sync<C::CT>();
           float* ps = su < DF_MAX_SU ? part_cur + ((long long)g * DF_MAX_SU + su) * DF_PART_STRIDE : nullptr;
@@ -788,10 +797,10 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
           for (int o = tid; o < MT * 64; o += C::CT) {
             float v = 0.f;
 #pragma unroll
-            for (int w8 = 0; w8 < C::CW; ++w8) v += red[(w8 * MT + (o >> 6)) * 64 + (o & 63)];
+            for (int w8 = 0; w8 < C::CW; ++w8) v += rb[(w8 * MT + (o >> 6)) * 64 + (o & 63)];
             if (ps) __stcg(ps + o, v);
           }
-          consumer_sync<C::CT>();
+          if (!kDual) consumer_sync<C::CT>();
           ++su;
         }
       } else {
