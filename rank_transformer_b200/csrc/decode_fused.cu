@@ -328,6 +328,31 @@ __device__ __forceinline__ float4 attn_gather4(const float* buf, const short* u,
   return make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
 }
 
+// Sum of 4 consecutive floats at idx over one unit's partial slots, in CTA
+// order; up to eight slots' loads in flight together.
+__device__ __forceinline__ float4 gather4_one(const float* buf, const short* u, int idx) {
+  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int n = u[0];
+  for (int c0 = 0; c0 < n; c0 += 8) {
+    float4 a[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      a[c] = c0 + c < n ? __ldcg(reinterpret_cast<const float4*>(buf + (long long)u[1 + c0 + c] * DF_PART_STRIDE + idx))
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      if (c0 + c < n) add4(s, a[c]);
+  }
+  return s;
+}
+
+template <int MT>
+__device__ __forceinline__ void add_sq(float (&ssq)[MT], int m, const float4& v) {
+#pragma unroll
+  for (int mm = 0; mm < MT; ++mm)
+    if (mm == m) ssq[mm] += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+}
+
 __device__ __forceinline__ float4 round4(float4 v) {
   return make_float4(bf_round(v.x), bf_round(v.y), bf_round(v.z), bf_round(v.w));
 }
@@ -590,6 +615,9 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
             if (m < p.B && hh < p.H && !pair_slots(s, p.H, G, m, hh, u)) atomicExch(p.status, DEV_STATUS_SCHEDULE);
           }
         }
+        float ssq[MT];  // RMSNorm: sum of squares of this thread's input values
+#pragma unroll
+        for (int m = 0; m < MT; ++m) ssq[m] = 0.f;
         if (xin) {
           // x (the layer input, complete before this stage) into the input
           // rows; zero rows past B (SRC_XOUT: x is built after the barrier)
@@ -600,6 +628,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
             if (m < p.B && src != SRC_XOUT) {
               const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(p.x + (long long)m * p.d + j));
               v = make_float4(bf_lo(raw.x), bf_hi(raw.x), bf_lo(raw.y), bf_hi(raw.y));
+              if (src == SRC_X) add_sq<MT>(ssq, m, v);
             }
             *reinterpret_cast<float4*>(abuf + m * DF_ABUF_COLS + j) = v;
           }
@@ -641,6 +670,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
               }
               add4(v, sp[k2]);
               v = round4(v);
+              add_sq<MT>(ssq, m, v);
               *a4 = v;
               if ((j >> 6) % G == g) {
                 uint2 o;
@@ -681,6 +711,26 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
         } else if (src == SRC_PART) {
           // fp32 rank activations z (plain column tiles of 64)
           const int tot = n * nseg * MT * 64;
+          if (tot <= C::CT) {
+            // at most one group per thread: all its slots' loads at once
+            const int e = tid;
+            if (e < tot) {
+              const int i = (e & 63) * 4;
+              int rest = e >> 6;
+              const int m = rest % MT;
+              rest /= MT;
+              const int seg = rest % nseg, ci = rest / nseg;
+              const int kc = clist[ci] & 255;
+              const int k = kc * DF_KC + i;
+              float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+              if (m < p.B && k < ph.K && nunits) {
+                const int col = seg * ph.a_col2 + k, col0 = seg * ph.a_col2 + kc * DF_KC;
+                v = gather4_one(part_prev, utab + ((ci * nseg + seg) * 5 + (col >> 6) - (col0 >> 6)) * 16,
+                                m * 64 + (col & 63));
+              }
+              *reinterpret_cast<float4*>(abuf + m * DF_ABUF_COLS + ci * 256 * nseg + seg * 256 + i) = v;
+            }
+          } else
           for (int e0 = tid; e0 < tot; e0 += 2 * C::CT) {
             const short* uu[2];
             const float* ww[2];
@@ -721,14 +771,10 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
         }
         consumer_sync<C::CT>();
         if (ph.norm) {
-          // rstd of each row of the stage input
+          // rstd of each row of the stage input (squares summed while building it)
+#pragma unroll
           for (int m = 0; m < MT; ++m) {
-            float ss = 0.f;
-            for (int j = tid; j < p.d; j += C::CT) {
-              const float v = abuf[m * DF_ABUF_COLS + j];
-              ss = fmaf(v, v, ss);
-            }
-            ss = warp_sum(ss);
+            const float ss = warp_sum(ssq[m]);
             if (lane == 0) red[warp * MT + m] = ss;
           }
           consumer_sync<C::CT>();
@@ -758,7 +804,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
         for (int m = 0; m < MT; ++m)
 #pragma unroll
           for (int j = 0; j < 8; ++j) acc[m][j] = 0.f;
-        int su = 0;
+        int su = 0, npend = 0;
         for (int c = c0; c < c1; ++c, ++seq) {
           const int slot = seq % C::NSLOT;
           const uint32_t par = (uint32_t)(seq / C::NSLOT) & 1u;
@@ -776,11 +822,13 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
 
           const bool tile_end = (c == c1 - 1) || (kc == ph.nk - 1);
           if (!tile_end) continue;
-          // ---- this CTA's partial of tile t ----
-          // (tile ends alternate between two scratch areas when both fit, so
-          // one CTA barrier per tile end suffices)
-          constexpr bool kDual = C::SCR_BYTES >= C::RED_BYTES;
-          float* rb = (kDual && (su & 1)) ? scr : red;
+          // ---- tile t done: each warp parks its column sums in shared
+          // memory; the CTA sums pending tiles once the area is full or the
+          // stage's entries are done (one CTA barrier for several tiles) ----
+          constexpr int kTileFloats = C::CW * MT * 64;
+          constexpr int kCap = (C::RED_BYTES + C::SCR_BYTES) / (kTileFloats * 4);  // red and scr are adjacent
+          static_assert(kCap >= 1, "tile-sum area");
+          float* tb = red + npend * kTileFloats;
 #pragma unroll
           for (int m = 0; m < MT; ++m)
 #pragma unroll
@@ -789,19 +837,23 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
               v += __shfl_xor_sync(0xffffffffu, v, 4);
               v += __shfl_xor_sync(0xffffffffu, v, 16);
               acc[m][j] = 0.f;
-              if ((lane & 20) == 0) rb[(warp * MT + m) * 64 + cg * 8 + j] = v;
+              if ((lane & 20) == 0) tb[(warp * MT + m) * 64 + cg * 8 + j] = v;
             }
+          ++npend;
+          ++su;
+          if (npend < kCap && c != c1 - 1) continue;
           consumer_sync<C::CT>();
-          float* ps = su < DF_MAX_SU ? part_cur + ((long long)g * DF_MAX_SU + su) * DF_PART_STRIDE : nullptr;
-          if (!ps && tid == 0) atomicExch(p.status, DEV_STATUS_SCHEDULE);
-          for (int o = tid; o < MT * 64; o += C::CT) {
+          for (int o = tid; o < npend * MT * 64; o += C::CT) {
+            const int pt = o / (MT * 64), oo = o - pt * MT * 64;
+            const int sp = su - npend + pt;
             float v = 0.f;
 #pragma unroll
-            for (int w8 = 0; w8 < C::CW; ++w8) v += rb[(w8 * MT + (o >> 6)) * 64 + (o & 63)];
-            if (ps) __stcg(ps + o, v);
+            for (int w8 = 0; w8 < C::CW; ++w8) v += red[pt * kTileFloats + (w8 * MT + (oo >> 6)) * 64 + (oo & 63)];
+            if (sp < DF_MAX_SU) __stcg(part_cur + ((long long)g * DF_MAX_SU + sp) * DF_PART_STRIDE + oo, v);
+            else if (oo == 0) atomicExch(p.status, DEV_STATUS_SCHEDULE);
           }
-          if (!kDual) consumer_sync<C::CT>();
-          ++su;
+          if (c != c1 - 1) consumer_sync<C::CT>();  // the area is reused by later tiles
+          npend = 0;
         }
       } else {
         // ---------------------------------------------- attention stage --
