@@ -34,6 +34,7 @@ struct Ctx {
   bf16* zb = nullptr;          // [rows x 2*max_rank] prefill rank activations
   float* df_part = nullptr;    // fused decode: per-CTA partial slots
   int* df_cnt = nullptr;       // fused decode: tile counters, stage barriers, done counter
+  int* zcnt = nullptr;         // prefill: per 128-row block counters of the z discard
   int rows = 0;                // rows of the scratch above
 };
 
@@ -42,7 +43,7 @@ std::mutex g_mu;
 
 void free_ctx(Ctx& c) {
   void* ptrs[] = {c.z, c.part, c.counters, c.apart, c.acounters, c.status,
-                  c.xn, c.q, c.att, c.h, c.zb, c.df_part, c.df_cnt};
+                  c.xn, c.q, c.att, c.h, c.zb, c.df_part, c.df_cnt, c.zcnt};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   c = Ctx();
@@ -207,6 +208,7 @@ PfLinear pf_base(const bf16* x, long long ldx, const flashsvd_factor& F, int M,
   p.y = y; p.ldy = ldy; p.M = M; p.d = d; p.r = F.r; p.n = n;
   p.epi = PF_EPI_BF16;
   p.z = g_ctx.zb;
+  p.zcnt = g_ctx.zcnt;
   p.status = g_ctx.status;
   return p;
 }
@@ -567,11 +569,13 @@ int flashsvd_init(int device, int max_tokens, int max_rank, int max_hidden,
   FSVD_ALLOC(c.zb, (size_t)c.rows * 2 * max_rank * sizeof(bf16));
   FSVD_ALLOC(c.df_part, (size_t)kFusedPartFloats * sizeof(float));
   FSVD_ALLOC(c.df_cnt, (size_t)(4096 + 64) * sizeof(int));
+  FSVD_ALLOC(c.zcnt, (size_t)(c.rows / 128 + 1) * sizeof(int));
 #undef FSVD_ALLOC
   if (e == cudaSuccess) e = cudaMemset(c.counters, 0, kCountersN * sizeof(int));
   if (e == cudaSuccess) e = cudaMemset(c.acounters, 0, kCountersN * sizeof(int));
   if (e == cudaSuccess) e = cudaMemset(c.status, 0, 64 * sizeof(int));
   if (e == cudaSuccess) e = cudaMemset(c.df_cnt, 0, (4096 + 64) * sizeof(int));
+  if (e == cudaSuccess) e = cudaMemset(c.zcnt, 0, (c.rows / 128 + 1) * sizeof(int));
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
     free_ctx(c);
@@ -602,6 +606,7 @@ int flashsvd_check_device_status(flashsvd_stream stream) {
     FSVD_CUDA(cudaMemset(g_ctx.df_cnt, 0, (4096 + 64) * sizeof(int)));
     FSVD_CUDA(cudaMemset(g_ctx.counters, 0, kCountersN * sizeof(int)));
     FSVD_CUDA(cudaMemset(g_ctx.acounters, 0, kCountersN * sizeof(int)));
+    FSVD_CUDA(cudaMemset(g_ctx.zcnt, 0, (g_ctx.rows / 128 + 1) * sizeof(int)));
     return word == DEV_STATUS_SCHEDULE ? FLASHSVD_ERR_UNSUPPORTED_SHAPE : FLASHSVD_ERR_TIMEOUT;
   }
   return FLASHSVD_OK;

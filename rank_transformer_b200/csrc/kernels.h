@@ -96,6 +96,7 @@ struct PfLinear {
   int kind; bf16* cache; int S, S_max, HD, D;
   const float* rope_cos; const float* rope_sin;
   bf16* z;                           // [M x r] bf16 scratch for the rank activations
+  int* zcnt;                         // [ceil(M / 128)] zero counters: z blocks discarded from L2 after use, or null
   int* status;
 };
 int prefill_linear_launch(const PfLinear& p, cudaStream_t stream);

@@ -78,6 +78,12 @@ struct TcArgs {
   int kind; bf16* cache; int S, S_max, HD, D;
   const float* rope_cos; const float* rope_sin;
   int* status;
+  // Stage 2 of a factorized linear: the rank activation z (A operand, rows of
+  // zld elements) is dead once every column tile of a 128-row block has
+  // consumed it; the last CTA to finish a block (counter zcnt[block], zero
+  // between launches) discards the block's L2 lines, so z is never written
+  // back to HBM.
+  const bf16* zdrop; long long zld; int* zcnt;
 };
 
 __device__ __forceinline__ void store8(bf16* p, const float* v) {
@@ -350,6 +356,28 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(tempty + buf);
+      if (a.zdrop && q == 0) {
+        // This tile's MMAs are complete: every TMA read of its z rows is
+        // done.  One warp counts the block's finished column tiles; the last
+        // CTA's warp discards the block's z lines (whole 128-byte lines
+        // inside rows [m0, m0 + 128) only).
+        const int mb = t % a.tiles_m;
+        const unsigned act = __activemask();
+        int last = 0;
+        if (lane == 0) {
+          last = atomicAdd(a.zcnt + mb, 1) == a.tiles_n - 1;
+          if (last) a.zcnt[mb] = 0;
+        }
+        last = __shfl_sync(act, last, __ffs(act) - 1);
+        if (last) {
+          const long long b0 = (long long)m0 * a.zld * 2;
+          const long long b1 = (long long)min(m0 + BM, a.M) * a.zld * 2;
+          const uintptr_t base = reinterpret_cast<uintptr_t>(a.zdrop);
+          const uintptr_t l0 = (base + b0 + 127) & ~(uintptr_t)127, l1 = (base + b1) & ~(uintptr_t)127;
+          for (uintptr_t ln = l0 + (uintptr_t)lane * 128; ln < l1; ln += 32 * 128)
+            asm volatile("discard.global.L2 [%0], 128;" ::"l"(ln) : "memory");
+        }
+      }
     }
   }
 
@@ -446,6 +474,7 @@ int prefill_linear_launch(const PfLinear& p, cudaStream_t stream) {
   a2.kind = p.kind; a2.cache = p.cache; a2.S = p.S; a2.S_max = p.S_max; a2.HD = p.HD; a2.D = p.D;
   a2.rope_cos = p.rope_cos; a2.rope_sin = p.rope_sin;
   a2.status = p.status;
+  if (p.zcnt) { a2.zdrop = p.z; a2.zld = p.r; a2.zcnt = p.zcnt; }
   return gemm(p.z, p.r, p.r, p.V, p.n, p.r, a2, p.epi, dual, dual ? "tc_stage2_swiglu" : "tc_stage2_zv",
               stream);
 }
