@@ -41,6 +41,11 @@ def parse():
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["decode7b", "linear-sweep", "bert", "mixed-rank"],
+                    default="decode7b",
+                    help="decode7b (default): the headline line; the others print one JSON "
+                         "line per measured case of the isolated-linear sweep, the BERT-shaped "
+                         "encoder and the mixed-rank model (1 GPU)")
     ap.add_argument("--layers", type=int, default=32,
                     help="decoder layers (default 32; fewer only for small profiling cases)")
     ap.add_argument("--profile-step", action="store_true",
@@ -409,10 +414,186 @@ def run_ours(args):
     return 0
 
 
+# ------------------------------------------------------- other workloads --
+
+def _event_ms(fn, reps, stream):
+    import torch
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(reps):
+        fn(i)
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def run_linear_sweep(args):
+    """Isolated factorized linears, Llama-7B shapes: square 4096x4096 and the
+    packed gate|up 4096 -> 2x11008 (+SwiGLU), r in {512, 1024, 2048}, M in
+    {1, 8, 32} (HBM-bound GEMV path) and {512, 2048} (tcgen05 path).  Random
+    factors of the SVD shapes; the calls rotate over enough factor copies
+    that the factors come from HBM (2x L2 worth)."""
+    import torch
+    sys.path.insert(0, ROOT)
+    from rank_transformer_b200 import flashsvd as fs
+    torch.cuda.set_device(0)
+    fs.init(0, max_tokens=2048, max_rank=4096, max_hidden=4096, max_ffn=11008)
+    peaks = measured_peaks()
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    stream = torch.cuda.Stream()
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(5)
+    d, f = 4096, 11008
+
+    def mat(r_, c_):
+        return (torch.randn(r_, c_, device="cuda", generator=gen) * r_ ** -0.5).to(torch.bfloat16)
+
+    for shape in ("square", "gateup"):
+        for r in (512, 1024, 2048):
+            if shape == "square":
+                fp_bytes = 2 * (d * r + r * d)
+            else:
+                fp_bytes = 2 * (d * 2 * r + 2 * r * f)
+            copies = max(1, min(64, math.ceil(2 * l2 / fp_bytes)))
+            facs = [(mat(d, r), mat(r, d)) if shape == "square" else (mat(d, 2 * r), mat(2 * r, f))
+                    for _ in range(copies)]
+            for M in (1, 8, 32, 512, 2048):
+                x = torch.randn(M, d, device="cuda", generator=gen).to(torch.bfloat16)
+                n = d if shape == "square" else f
+                y = torch.empty(M, n, device="cuda", dtype=torch.bfloat16)
+                if shape == "square":
+                    call = lambda i: fs.lowrank_linear(x, facs[i % copies][0], facs[i % copies][1], None,
+                                                       y, M, d, r, d, stream)
+                    flops = 2 * M * r * (d + d)
+                    bytes_ = 2 * (d * r + r * d + M * d + M * d)
+                else:
+                    call = lambda i: fs.gateup_swiglu(x, facs[i % copies][0], facs[i % copies][1], y, M, d,
+                                                      r, f, stream)
+                    flops = 2 * M * (d * 2 * r + 2 * r * f)
+                    bytes_ = 2 * (d * 2 * r + 2 * r * f + M * d + M * f)
+                with torch.cuda.stream(stream):
+                    for i in range(10):
+                        call(i)
+                    ms = _event_ms(call, 50, stream)
+                fs.check_device_status(stream)
+                gbs, tfs = bytes_ / (ms / 1e3) / 1e9, flops / (ms / 1e3) / 1e12
+                hbm_bound = M <= 32
+                print(json.dumps({
+                    "workload": "linear-sweep", "shape": "4096x4096" if shape == "square" else
+                    "gate|up 4096->2x11008 +SwiGLU", "r": r, "M": M, "us": round(ms * 1e3, 2),
+                    "path": "split-K GEMV" if M <= 32 else "tcgen05 GEMM",
+                    "bound": "hbm" if hbm_bound else "tensor",
+                    "achieved": round(gbs if hbm_bound else tfs, 1),
+                    "unit": "GB/s" if hbm_bound else "TFLOP/s",
+                    "frac": round(gbs / peaks["hbm_gbs"] if hbm_bound else tfs / peaks["bf16_tflops"], 3),
+                    "algorithmic_bytes": bytes_, "flops": flops, "factor_copies": copies}), flush=True)
+            del facs
+            torch.cuda.empty_cache()
+    return 0
+
+
+def run_bert(args):
+    """BERT-Base-shaped low-rank encoder: 12 layers, hidden 768, 12 heads,
+    FFN 3072 (GELU), every linear at rank 192 with bias, batch 32 x 512,
+    bf16, N(0,1) inputs (GLUE is not here; same shapes)."""
+    import torch
+    sys.path.insert(0, ROOT)
+    from rank_transformer_b200 import flashsvd as fs
+    from rank_transformer_b200.model import EncoderModel
+    torch.cuda.set_device(0)
+    B, S = 32, 512
+    fs.init(0, max_tokens=B * S, max_rank=192, max_hidden=768, max_ffn=3072)
+    peaks = measured_peaks()
+    m = EncoderModel(B=B, S=S, seed=3)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(4)
+    x0 = torch.randn(B * S, 768, device="cuda", generator=gen).to(torch.bfloat16)
+    x = x0.clone()
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            x.copy_(x0)
+            m.forward(x, stream)
+        ms = _event_ms(lambda i: m.forward(x, stream), 10, stream)
+    fs.check_device_status(stream)
+    tf = m.flops() / (ms / 1e3) / 1e12
+    M, d, f, r = B * S, 768, 3072, 192
+    # activations the forward keeps in device memory: hidden x, K/V buffers,
+    # and the library's per-layer temporaries for this shape (q / attention
+    # output / FFN intermediate / bf16 rank activations z)
+    act = 2 * (M * d + 2 * M * d + 2 * M * d + M * f + M * r)
+    print(json.dumps({
+        "workload": "bert", "config": {"layers": 12, "hidden": d, "heads": 12, "ffn": f, "rank": r,
+                                       "batch": B, "seq": S},
+        "ms_per_forward": round(ms, 3), "sequences_per_s": round(B / (ms / 1e3), 1),
+        "tokens_per_s": round(M / (ms / 1e3)), "tflops": round(tf, 1),
+        "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 3),
+        "activation_bytes": act, "unfused_z_bytes_avoided_per_linear": 2 * M * r,
+        "note": "the rank activation z of each linear stays in L2 (discarded after use)"}), flush=True)
+    return 0
+
+
+def run_mixed(args):
+    """Same 7B-shaped model with one retention ratio per layer drawn from
+    {0.4, 0.6, 0.8}: prefill B=4 x 2048 (tcgen05 path), then 256 greedy
+    decode steps (B=4, decode plan)."""
+    import dataclasses
+    import torch
+    sys.path.insert(0, ROOT)
+    from rank_transformer_b200 import flashsvd as fs
+    from rank_transformer_b200 import synth
+    from rank_transformer_b200.model import LLAMA7B, DecoderModel
+    torch.cuda.set_device(0)
+    B, S, steps = 4, PROMPT, 256
+    cfg = dataclasses.replace(LLAMA7B, rho=synth.mixed_rho(11, LLAMA7B.layers))
+    fs.init(0, max_tokens=B * S, max_rank=2368, max_hidden=cfg.d, max_ffn=cfg.f)
+    peaks = measured_peaks()
+    model = DecoderModel(cfg, B, S + steps, seed=21)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(22)
+    prompt = torch.randint(0, cfg.vocab, (B, S), generator=gen, device="cuda", dtype=torch.int32)
+    stream = torch.cuda.Stream()
+    model.capture(stream)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    with torch.cuda.stream(stream):
+        for rep_ in range(2):
+            ev[0].record(stream)
+            model.prefill(prompt, stream)
+            ev[1].record(stream)
+            for _ in range(steps):
+                model.decode_step(stream)
+            ev[2].record(stream)
+    stream.synchronize()
+    fs.check_device_status(stream)
+    pre_ms, dec_ms = ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2])
+    lin = 2 * B * S * sum(cfg.layer_params(i) for i in range(cfg.layers))
+    head = 2 * B * cfg.d * cfg.vocab
+    attn = cfg.layers * 4 * B * S * S * cfg.d / 2
+    pf_flops = lin + head + attn
+    model.release_graphs()
+    print(json.dumps({
+        "workload": "mixed-rank", "rho_per_layer": list(cfg.rho),
+        "ranks_per_layer": [list(cfg.ranks(i)) for i in range(cfg.layers)],
+        "batch": B, "prompt": S, "decode_steps": steps,
+        "prefill_tok_s": round(B * S / (pre_ms / 1e3)), "prefill_ms": round(pre_ms, 2),
+        "prefill_tflops": round(pf_flops / (pre_ms / 1e3) / 1e12, 1),
+        "prefill_frac_of_bf16_peak": round(pf_flops / (pre_ms / 1e3) / 1e12 / peaks["bf16_tflops"], 3),
+        "decode_tok_s": round(B * steps / (dec_ms / 1e3), 1), "decode_ms": round(dec_ms, 2),
+        "e2e_latency_ms": round(pre_ms + dec_ms, 2),
+        "decode_path": "decode plan" if model.plan is not None else "per-stage"}), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "linear-sweep":
+        return run_linear_sweep(args)
+    if args.workload == "bert":
+        return run_bert(args)
+    if args.workload == "mixed-rank":
+        return run_mixed(args)
     return run_ours(args)
 
 

@@ -106,12 +106,11 @@ class DecoderModel:
         if decode_pack:
             for L in self.structs:
                 try:
-                    n = fs.decode_pack_bytes(L)
+                    buf = torch.empty(fs.decode_pack_bytes(L), dtype=torch.uint8, device=device)
+                    fs.decode_pack(L, buf)
                 except fs.FlashSVDError:
-                    self.packs.append(None)
-                    continue
-                buf = torch.empty(n, dtype=torch.uint8, device=device)
-                fs.decode_pack(L, buf)
+                    L.decode_pack = None  # shapes the fused kernel does not cover
+                    buf = None
                 self.packs.append(buf)
         # With a pack on every layer, the decode step of all layers runs as
         # one launch of the fused kernel (a decode plan).

@@ -64,6 +64,13 @@ def rank_for_ratio(rho: float, d_in: int, d_out: int, multiple: int = 64) -> int
     return int(multiple * round(exact / multiple))
 
 
+def mixed_rho(seed: int, layers: int, choices=(0.4, 0.6, 0.8)) -> tuple:
+    """One retention ratio per layer, drawn uniformly from ``choices`` in
+    layer order with a seeded PCG64 generator (mixed-rank model)."""
+    rng = rng_for(seed)
+    return tuple(float(choices[i]) for i in rng.integers(0, len(choices), size=layers))
+
+
 def _haar_columns(rng: np.random.Generator, n: int, k: int) -> np.ndarray:
     """n x k matrix with orthonormal columns, Haar distributed (QR of a
     Gaussian with the signs of R's diagonal folded into Q)."""
