@@ -312,6 +312,7 @@ int layer_prefill(const flashsvd_layer* L, bf16* x, bf16* kc, bf16* vc,
   a.q = g_ctx.q; a.k = kc; a.v = vc; a.out = g_ctx.att;
   a.B = B; a.S = S; a.H = L->H; a.D = L->D; a.S_max = S_max; a.causal = 1;
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)L->D);
+  a.status = g_ctx.status;
   FSVD_TRY(attn_prefill_launch(a, s));
   {
     PfLinear p = pf_base(g_ctx.att, d, L->o, M, d, d, x, d);
@@ -347,6 +348,7 @@ int layer_encoder(const flashsvd_layer* L, bf16* x, bf16* kc, bf16* vc,
   a.q = g_ctx.q; a.k = kc; a.v = vc; a.out = g_ctx.att;
   a.B = B; a.S = S; a.H = L->H; a.D = L->D; a.S_max = S_max; a.causal = 0;
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)L->D);
+  a.status = g_ctx.status;
   FSVD_TRY(attn_prefill_launch(a, s));
   {
     PfLinear p = pf_base(g_ctx.att, d, L->o, M, d, d, g_ctx.xn, d);
@@ -741,6 +743,7 @@ int flashsvd_prefill_attn(const flashsvd_bf16* q, const flashsvd_bf16* k_cache,
   a.q = (const bf16*)q; a.k = (const bf16*)k_cache; a.v = (const bf16*)v_cache; a.out = (bf16*)out;
   a.B = B; a.S = S; a.H = H; a.D = D; a.S_max = S_max; a.causal = causal ? 1 : 0;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.status = g_ctx.status;
   return attn_prefill_launch(a, stream);
 }
 

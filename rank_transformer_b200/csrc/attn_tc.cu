@@ -1,0 +1,354 @@
+// Prefill attention on the 5th-generation tensor cores.
+//
+// FlashSVD v1.5 (gist.science explainer), Technical Summary, Methodology 2:
+// prefill keeps its own attention kernel (the dense-KV path is the decode
+// one); here it reads the same dense [B, S_max, H, D] cache the prefill's
+// q/k/v epilogue wrote.  Causal (decoder) or bidirectional (encoder).
+//
+// One CTA per (128-query tile, batch row, head), 6 warps:
+//   warp 0  TMA: Q once, then 128-key K and V tiles into a 2-stage ring;
+//   warp 1  TMEM owner and MMA issuer: S = Q K^T into one of two 128-column
+//           TMEM buffers, then O += P V into a D-column TMEM accumulator;
+//   warps 2-9  two threads per query row (each half of the keys and of O):
+//           load S from TMEM, mask, online softmax (exp2 domain, the row max
+//           exchanged through shared memory), rescale O in TMEM when the
+//           row's reference max moves, write P (bf16) into 128-byte-swizzled
+//           shared memory as the next MMA's A operand; at the end O / l.
+// All operand tiles are 128-byte swizzled; S of tile j+1 is computed while
+// the softmax of tile j runs.  Every wait is bounded.
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace fsvd {
+namespace {
+
+constexpr int AT_BM = 128;   // queries per CTA
+constexpr int AT_BN = 128;   // keys per tile
+constexpr int AT_THREADS = 320;  // TMA warp, MMA warp, 8 softmax warps
+
+template <int D>
+struct AtLayout {
+  static constexpr int KB = D / 64;              // 64-column blocks of a head
+  static constexpr int TILE = AT_BN * 128;       // one [128 x 64] bf16 block, 16 KB
+  static constexpr int Q_OFF = 0;
+  static constexpr int K_OFF = Q_OFF + KB * TILE;
+  static constexpr int V_OFF = K_OFF + 2 * KB * TILE;
+  static constexpr int P_OFF = V_OFF + 2 * KB * TILE;
+  static constexpr int BAR_OFF = P_OFF + 2 * TILE;
+  static constexpr int X_OFF = BAR_OFF + 256;     // [2 tiles][2 halves][128] row partials
+  static constexpr int SMEM = 1024 + X_OFF + 2 * 2 * 128 * 4;
+  static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+struct AtParams {
+  int B, S, H, S_max;
+  float scale_log2;
+  bf16* out;      // [B*S x H*D]
+  int* status;
+};
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(AT_THREADS, 1)
+attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AtParams p) {
+  using L = AtLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+  uint64_t* kv_full = q_full + 1;    // [2]
+  uint64_t* kv_empty = kv_full + 2;  // [2]
+  uint64_t* s_full = kv_empty + 2;   // [2]
+  uint64_t* s_empty = s_full + 2;    // [2]
+  uint64_t* p_full = s_empty + 2;
+  uint64_t* o_done = p_full + 1;
+  uint64_t* drain = o_done + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // heaviest (longest causal) query tiles first
+  const int qt = gridDim.x - 1 - blockIdx.x;
+  const int bh = blockIdx.y, b = bh / p.H, h = bh - b * p.H;
+  const int m0 = qt * AT_BM;
+  const int nt_all = (p.S + AT_BN - 1) / AT_BN;
+  const int nt = CAUSAL ? min(nt_all, (m0 + AT_BM + AT_BN - 1) / AT_BN) : nt_all;
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(kv_full + i, 1);
+      tc::mbar_init(kv_empty + i, 1);
+      tc::mbar_init(s_full + i, 1);
+      tc::mbar_init(s_empty + i, 8);
+    }
+    tc::mbar_init(p_full, 8);
+    tc::mbar_init(o_done, 1);
+    tc::mbar_init(drain, 1);
+    *abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tc::tma_prefetch_desc(&tmQ);
+    tc::tma_prefetch_desc(&tmK);
+    tc::tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_holder, 512);  // S0 [0,128), S1 [128,256), O [256, 256 + D)
+    tc::tmem_relinquish();
+    tc::fence_before_sync();
+  }
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_holder;
+
+  pdl_launch_dependents();
+  pdl_wait();
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA --
+    if (lane == 0) {
+      const int hx = h * D;
+      tc::mbar_expect_tx(q_full, (uint32_t)(L::KB * L::TILE));
+      for (int kb = 0; kb < L::KB; ++kb)
+        tc::tma_load_2d(smem + L::Q_OFF + kb * L::TILE, &tmQ, q_full, hx + 64 * kb, b * p.S + m0);
+      for (int j = 0; j < nt; ++j) {
+        const int st = j & 1;
+        if (!tc::mbar_wait(kv_empty + st, ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag, p.status)) break;
+        tc::mbar_expect_tx(kv_full + st, (uint32_t)(2 * L::KB * L::TILE));
+        const int row = b * p.S_max + j * AT_BN;
+        for (int kb = 0; kb < L::KB; ++kb) {
+          tc::tma_load_2d(smem + L::K_OFF + (st * L::KB + kb) * L::TILE, &tmK, kv_full + st, hx + 64 * kb, row);
+          tc::tma_load_2d(smem + L::V_OFF + (st * L::KB + kb) * L::TILE, &tmV, kv_full + st, hx + 64 * kb, row);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = tc::idesc_bf16(AT_BN, false);  // B = K rows, K-major
+      constexpr uint32_t IDESC_O = tc::idesc_bf16(D, true);       // B = V rows, MN-major
+      const uint32_t sq = tc::smem_u32(smem + L::Q_OFF);
+      const uint32_t sp = tc::smem_u32(smem + L::P_OFF);
+      bool ok = tc::mbar_wait(q_full, 0, abort_flag, p.status);
+      auto issue_pv = [&](int j) {
+        // O (+)= P_j V_j once the softmax has written P_j (and rescaled O)
+        if (!tc::mbar_wait(p_full, (uint32_t)j & 1u, abort_flag, p.status)) return false;
+        tc::fence_after_sync();
+        const uint32_t sv = tc::smem_u32(smem + L::V_OFF + (j & 1) * L::KB * L::TILE);
+#pragma unroll
+        for (int k = 0; k < AT_BN / 16; ++k) {
+          const uint64_t ad = tc::sdesc_sw128(sp + (k >> 2) * L::TILE + (k & 3) * 32, 16, 1024);
+          const uint64_t bd = tc::sdesc_sw128(sv + k * 2048, L::TILE, 1024);
+          tc::mma_bf16(tmem + 256, ad, bd, IDESC_O, (j > 0 || k > 0) ? 1u : 0u);
+        }
+        tc::mma_commit(o_done);
+        tc::mma_commit(kv_empty + (j & 1));
+        return true;
+      };
+      for (int j = 0; j < nt && ok; ++j) {
+        const int st = j & 1;
+        if (!(ok = tc::mbar_wait(kv_full + st, (uint32_t)(j >> 1) & 1u, abort_flag, p.status))) break;
+        if (!(ok = tc::mbar_wait(s_empty + st, ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag, p.status))) break;
+        tc::fence_after_sync();
+        const uint32_t sk = tc::smem_u32(smem + L::K_OFF + st * L::KB * L::TILE);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint64_t ad = tc::sdesc_sw128(sq + (k >> 2) * L::TILE + (k & 3) * 32, 16, 1024);
+          const uint64_t bd = tc::sdesc_sw128(sk + (k >> 2) * L::TILE + (k & 3) * 32, 16, 1024);
+          tc::mma_bf16(tmem + st * AT_BN, ad, bd, IDESC_S, k > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(s_full + st);
+        if (j > 0) ok = issue_pv(j - 1);
+      }
+      if (ok && nt > 0) issue_pv(nt - 1);
+      // every MMA this thread issued has completed once `drain` fires
+      tc::mma_commit(drain);
+      const long long t0 = clock64();
+      while (!tc::mbar_try_wait(drain, 0) && clock64() - t0 < tc::kWaitCycles) {}
+    }
+  } else {
+    // ------------------------------------------------- softmax, epilogue --
+    // Warp w (2..9) reads TMEM lanes 32 (w % 4) .. + 31; warps 2-5 take keys
+    // [0, 64) of a tile and O columns [0, D/2), warps 6-9 the other halves.
+    const int quad = warp & 3;
+    const int hf = (warp - 2) >> 2;
+    const int r = quad * 32 + lane;       // query row within the tile
+    const int q = m0 + r;                 // query position
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    float* xr = reinterpret_cast<float*>(smem + L::X_OFF);  // [2][2][128]
+    const float sc = p.scale_log2;
+    float m = -INFINITY, l = 0.f;         // m: reference max, scaled units
+    uint8_t* sP = smem + L::P_OFF;
+    constexpr int HC = AT_BN / 2;         // keys per thread
+    constexpr int OC = D / 2;             // O columns per thread
+    // tcgen05.ld / st are warp-collective: wait results are made
+    // warp-uniform.  The 8 softmax warps meet at a named barrier every tile,
+    // so the loop never exits early: after a failed wait it runs on without
+    // touching tensor memory.
+    auto wwait = [&](uint64_t* bar, uint32_t par) {
+      return __all_sync(0xffffffffu, tc::mbar_wait(bar, par, abort_flag, p.status)) != 0;
+    };
+    auto sm_sync = [] { asm volatile("bar.sync 1, 256;" ::: "memory"); };
+    bool ok = true;
+    for (int j = 0; j < nt; ++j) {
+      const int st = j & 1;
+      ok = ok && wwait(s_full + st, (uint32_t)(j >> 1) & 1u);
+      float s[HC];
+      if (ok) {
+        tc::fence_after_sync();
+#pragma unroll
+        for (int c = 0; c < HC / 32; ++c)
+          tc::tmem_ld32(tmem + lane_base + st * AT_BN + hf * HC + c * 32, reinterpret_cast<uint32_t*>(s + c * 32));
+        tc::tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int c = 0; c < HC; ++c) s[c] = -INFINITY;
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(s_empty + st);
+      // mask (raw scores: the scale is positive) and partial row max
+      const int n0 = j * AT_BN + hf * HC;
+      const bool need_mask = n0 + HC > p.S || (CAUSAL && n0 + HC - 1 > m0);
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int c = 0; c < HC; ++c) {
+        if (need_mask) {
+          const int key = n0 + c;
+          if (key >= p.S || (CAUSAL && key > q)) s[c] = -INFINITY;
+        }
+        mx4[c & 3] = fmaxf(mx4[c & 3], s[c]);
+      }
+      float* xt = xr + st * 256;
+      xt[hf * 128 + r] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      sm_sync();
+      const float rawmax = fmaxf(xt[r], xt[128 + r]);
+      const float mx = rawmax == -INFINITY ? -INFINITY : rawmax * sc;
+      // PV of tile j-1 must be complete before O is rescaled or P rewritten
+      if (j > 0) ok = ok && wwait(o_done, (uint32_t)(j - 1) & 1u);
+      tc::fence_after_sync();
+      // The row's reference m (P = 2^(s sc - m)) moves up only when the tile
+      // max exceeds it by more than 8: P stays <= 2^8 (exact enough in bf16
+      // and in the fp32 sums), O and l keep the same reference, and O is
+      // rescaled rarely.
+      const bool raise = m == -INFINITY || mx > m + 8.f;
+      const float m_new = raise ? fmaxf(mx, m) : m;
+      const bool grow = j > 0 && raise && m != -INFINITY;
+      if (ok && __any_sync(0xffffffffu, grow)) {
+        const float corr = grow ? exp2f(m - m_new) : 1.f;
+        l *= corr;
+#pragma unroll
+        for (int c = 0; c < OC / 32; ++c) {
+          uint32_t o[32];
+          tc::tmem_ld32(tmem + lane_base + 256 + hf * OC + c * 32, o);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
+          tc::tmem_st32(tmem + lane_base + 256 + hf * OC + c * 32, o);
+        }
+        tc::tmem_st_wait();
+      }
+      m = m_new;
+      // P = 2^(s sc - m), bf16, this half of row r of the swizzled A operand
+      const float mneg = m == -INFINITY ? 0.f : -m;
+      float l4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ch = 0; ch < HC / 8; ++ch) {
+        float pv[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float x = s[ch * 8 + e];
+          pv[e] = (x == -INFINITY) ? 0.f : exp2f(fmaf(x, sc, mneg));
+          l4[e & 3] += pv[e];
+        }
+        uint4 u;
+        u.x = pack_bf2(pv[0], pv[1]); u.y = pack_bf2(pv[2], pv[3]);
+        u.z = pack_bf2(pv[4], pv[5]); u.w = pack_bf2(pv[6], pv[7]);
+        *reinterpret_cast<uint4*>(sP + hf * L::TILE + r * 128 + ((ch ^ (r & 7)) << 4)) = u;
+      }
+      l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+      tc::fence_proxy_async_smem();   // P is read by the tensor cores
+      tc::fence_before_sync();        // O rows rewritten in TMEM above
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(p_full);
+    }
+    // ---- O / l -> bf16 ----
+    const bool fin = ok && nt > 0 && wwait(o_done, (uint32_t)(nt - 1) & 1u);
+    sm_sync();  // every partner has read the last tile's row maxima
+    xr[hf * 128 + r] = l;
+    sm_sync();
+    const float lt = xr[r] + xr[128 + r];
+    if (fin) {
+      tc::fence_after_sync();
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      const long long HD = (long long)p.H * D;
+      bf16* og = p.out + ((long long)b * p.S + q) * HD + (long long)h * D + hf * OC;
+#pragma unroll
+      for (int c = 0; c < OC / 32; ++c) {
+        uint32_t o[32];
+        tc::tmem_ld32(tmem + lane_base + 256 + hf * OC + c * 32, o);
+        tc::tmem_ld_wait();
+        if (q < p.S) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 u;
+            u.x = pack_bf2(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
+            u.y = pack_bf2(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+            u.z = pack_bf2(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
+            u.w = pack_bf2(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
+            *reinterpret_cast<uint4*>(og + c * 32 + e) = u;
+          }
+        }
+      }
+    }
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  if (*abort_flag && warp == 0 && lane == 0) {
+    // let copies still in flight land before shared memory is released
+    const long long t0 = clock64();
+    while (clock64() - t0 < 2000000) {}
+  }
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D, bool CAUSAL>
+int launch_at(const AttnPfParams& ap, cudaStream_t stream) {
+  using L = AtLayout<D>;
+  auto kern = attn_prefill_tc_kernel<D, CAUSAL>;
+  static bool configured = false;
+  if (!configured) {
+    FSVD_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM));
+    configured = true;
+  }
+  const long long HD = (long long)ap.H * D;
+  CUtensorMap mq, mk, mv;
+  FSVD_TRY(encode_map(&mq, ap.q, (long long)ap.B * ap.S, HD, HD, 64, AT_BM, true));
+  FSVD_TRY(encode_map(&mk, ap.k, (long long)ap.B * ap.S_max, HD, HD, 64, AT_BN, true));
+  FSVD_TRY(encode_map(&mv, ap.v, (long long)ap.B * ap.S_max, HD, HD, 64, AT_BN, true));
+  AtParams p;
+  p.B = ap.B; p.S = ap.S; p.H = ap.H; p.S_max = ap.S_max;
+  p.scale_log2 = ap.scale_log2;
+  p.out = ap.out;
+  p.status = ap.status;
+  const dim3 grid(ceil_div(ap.S, AT_BM), ap.B * ap.H);
+  const double S = ap.S;
+  const double flops = 4.0 * ap.B * ap.H * S * S * D * (CAUSAL ? 0.5 : 1.0);
+  const LaunchTag tag{CAUSAL ? "attn_prefill_causal" : "attn_prefill_bidir", 2.0 * 4.0 * ap.B * S * HD, flops};
+  return launch_pdl(tag, kern, grid, dim3(AT_THREADS), (size_t)L::SMEM, stream, mq, mk, mv, p);
+}
+
+}  // namespace
+
+int attn_prefill_tc_launch(const AttnPfParams& p, cudaStream_t stream) {
+  if (!p.status) return FLASHSVD_ERR_NOT_INITIALIZED;
+  if (p.D == 128) return p.causal ? launch_at<128, true>(p, stream) : launch_at<128, false>(p, stream);
+  if (p.D == 64) return p.causal ? launch_at<64, true>(p, stream) : launch_at<64, false>(p, stream);
+  return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+}
+
+}  // namespace fsvd

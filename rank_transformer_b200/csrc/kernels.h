@@ -138,7 +138,9 @@ struct AttnPfParams {
   const bf16* q; const bf16* k; const bf16* v; bf16* out;
   int B, S, H, D, S_max, causal;
   float scale_log2;
+  int* status;       // device status word (bounded waits)
 };
 int attn_prefill_launch(const AttnPfParams& p, cudaStream_t stream);
+int attn_prefill_tc_launch(const AttnPfParams& p, cudaStream_t stream);
 
 }  // namespace fsvd

@@ -238,6 +238,10 @@ int launch_attn(const AttnPfParams& p, cudaStream_t stream) {
 }  // namespace
 
 int attn_prefill_launch(const AttnPfParams& p, cudaStream_t stream) {
+  // tcgen05 kernel (attn_tc.cu) for every shape it covers; this mma.sync
+  // kernel remains for the rest
+  const int st = attn_prefill_tc_launch(p, stream);
+  if (st != FLASHSVD_ERR_UNSUPPORTED_SHAPE && st != FLASHSVD_ERR_NOT_INITIALIZED) return st;
   if (p.D == 128) return p.causal ? launch_attn<128, true>(p, stream) : launch_attn<128, false>(p, stream);
   if (p.D == 64) return p.causal ? launch_attn<64, true>(p, stream) : launch_attn<64, false>(p, stream);
   return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
