@@ -171,12 +171,82 @@ __global__ void advance_kernel(int* seqlens, int B) {
   for (int b = threadIdx.x; b < B; b += blockDim.x) seqlens[b] += 1;
 }
 
+// Rows of up to 2048 elements: one warp per row (VPL 16-byte vectors per
+// lane), eight rows per CTA, no CTA barriers.
+constexpr int WR_ROWS = 8;
+
+template <int VPL, bool LN>
+__global__ void __launch_bounds__(WR_ROWS * 32)
+norm_warp_kernel(const bf16* x, const bf16* g, const bf16* b, bf16* y, int M, int d, float eps) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * WR_ROWS + (threadIdx.x >> 5);
+  if (row >= M) return;
+  float v[VPL][8];
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int c = (lane + i * 32) * 8;
+    if (c < d) {
+      ld8(x + row * d + c, v[i]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) s = LN ? s + v[i][j] : fmaf(v[i][j], v[i][j], s);
+    }
+  }
+  s = warp_sum(s);
+  float mean = 0.f, rs;
+  if (LN) {
+    mean = s / (float)d;
+    float q = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i)
+      if ((lane + i * 32) * 8 < d)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float t = v[i][j] - mean;
+          q = fmaf(t, t, q);
+        }
+    rs = rsqrtf(warp_sum(q) / (float)d + eps);
+  } else {
+    rs = rsqrtf(s / (float)d + eps);
+  }
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int c = (lane + i * 32) * 8;
+    if (c < d) {
+      float gg[8], bb[8], o[8];
+      ld8(g + c, gg);
+      if (LN) ld8(b + c, bb);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) o[j] = LN ? (v[i][j] - mean) * rs * gg[j] + bb[j] : v[i][j] * rs * gg[j];
+      st8(y + row * d + c, o);
+    }
+  }
+}
+
+template <bool LN>
+int norm_warp_launch(const bf16* x, const bf16* g, const bf16* b, bf16* y, int M, int d, float eps,
+                     cudaStream_t s) {
+  const LaunchTag tag{LN ? "layernorm" : "rmsnorm", 4.0 * M * d, 0.0};
+  const dim3 grid(ceil_div(M, WR_ROWS)), block(WR_ROWS * 32);
+  switch (ceil_div(d, 256)) {
+    case 1: return launch_pdl(tag, norm_warp_kernel<1, LN>, grid, block, 0, s, x, g, b, y, M, d, eps);
+    case 2: return launch_pdl(tag, norm_warp_kernel<2, LN>, grid, block, 0, s, x, g, b, y, M, d, eps);
+    case 3: return launch_pdl(tag, norm_warp_kernel<3, LN>, grid, block, 0, s, x, g, b, y, M, d, eps);
+    case 4: return launch_pdl(tag, norm_warp_kernel<4, LN>, grid, block, 0, s, x, g, b, y, M, d, eps);
+    case 5: case 6: return launch_pdl(tag, norm_warp_kernel<6, LN>, grid, block, 0, s, x, g, b, y, M, d, eps);
+    default: return launch_pdl(tag, norm_warp_kernel<8, LN>, grid, block, 0, s, x, g, b, y, M, d, eps);
+  }
+}
+
 }  // namespace
 
 int rmsnorm_launch(const bf16* x, const bf16* g, bf16* y, int M, int d,
                    float eps, cudaStream_t s) {
   if (d > NT * ROW_VEC * 8) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return FLASHSVD_OK;
+  if (d <= 2048) return norm_warp_launch<false>(x, g, nullptr, y, M, d, eps, s);
   return launch_pdl(LaunchTag{"rmsnorm", 4.0 * M * d, 0.0}, rmsnorm_kernel, dim3(M), dim3(NT), 0, s, x, g, y, d, eps);
 }
 
@@ -184,6 +254,7 @@ int layernorm_launch(const bf16* x, const bf16* g, const bf16* b, bf16* y,
                      int M, int d, float eps, cudaStream_t s) {
   if (d > NT * ROW_VEC * 8) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return FLASHSVD_OK;
+  if (d <= 2048) return norm_warp_launch<true>(x, g, b, y, M, d, eps, s);
   return launch_pdl(LaunchTag{"layernorm", 4.0 * M * d, 0.0}, layernorm_kernel, dim3(M), dim3(NT), 0, s, x, g, b, y, d, eps);
 }
 
