@@ -65,7 +65,7 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int TC_THREADS = 192;
+constexpr int TC_THREADS = 320;  // TMA warp, MMA warp, 8 epilogue warps
 
 struct TcArgs {
   int M, N, K;          // per half for the dual (SwiGLU) form
@@ -138,7 +138,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(tfull + b, 1);
-      tc::mbar_init(tempty + b, 4);
+      tc::mbar_init(tempty + b, 8);
     }
     tc::mbar_init(drain, 1);
     *abort_flag = 0;
@@ -237,7 +237,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
   } else {
     // --------------------------------------------------------- epilogue --
+    // Warp w reads TMEM lanes 32 (w % 4) .. + 31 (its 32 rows); the two
+    // warps of a lane quadrant take alternate 32-column chunks of the tile.
     const int q = warp & 3;
+    const int part = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     int it = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
@@ -256,13 +259,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const int half = a.D >> 1;
         const int hc = half >> 5;  // chunks per half head
         const int bq = mok ? m / a.S : 0, tq = mok ? m - bq * a.S : 0;
+        int pair = 0;
         for (int c = 0; c < BN / 32; ++c) {
           if ((c % (2 * hc)) >= hc) continue;  // second-half chunks ride along
+          if ((pair++ & 1) != part) continue;
+          const int n = n0 + c * 32;
           uint32_t r0[32], r1[32];
           tc::tmem_ld32(tb + c * 32, r0);
           tc::tmem_ld32(tb + (c + hc) * 32, r1);
           tc::tmem_ld_wait();
-          const int n = n0 + c * 32;
           if (!mok || n >= a.N) continue;
           float lo[32], hi[32];
 #pragma unroll
@@ -304,13 +309,32 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           }
         }
       } else {
+        // A warp owns pairs of chunks (64 columns: whole 128-byte lines of
+        // a row), so no output line is shared between the two warps of a
+        // quadrant.  Residual and bias are read before the accumulator
+        // wait: the residual may be the output buffer itself (in-place
+        // update), and reading it up front keeps the loads off the stores.
         for (int c = 0; c < BN / 32; ++c) {
+          if (((c >> 1) & 1) != part) continue;
+          const int n = n0 + c * 32;
+          constexpr bool PLAIN = !DUAL && EPI != PF_EPI_F32;
+          uint4 rr[PLAIN ? 4 : 1], bb[PLAIN ? 4 : 1];
+          if (PLAIN) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              const int ng = n + 8 * g;
+              const bool in = mok && ng < a.N;
+              rr[g] = (in && a.resid) ? *reinterpret_cast<const uint4*>(a.resid + (long long)m * a.ldr + ng)
+                                      : make_uint4(0u, 0u, 0u, 0u);
+              bb[g] = (in && a.bias) ? *reinterpret_cast<const uint4*>(a.bias + ng) : make_uint4(0u, 0u, 0u, 0u);
+            }
+          }
+          __syncwarp();
           uint32_t r0[32];
           uint32_t r1[DUAL ? 32 : 1];
           tc::tmem_ld32(tb + c * 32, r0);
           if (DUAL) tc::tmem_ld32(tb + BN + c * 32, r1);
           tc::tmem_ld_wait();
-          const int n = n0 + c * 32;
           if (!mok) continue;
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
@@ -332,21 +356,20 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 v[j] = v[j] / (1.f + expf(-v[j])) * u;
               }
             } else {
+              const int gi = PLAIN ? g : 0;
+              const uint32_t bw[4] = {bb[gi].x, bb[gi].y, bb[gi].z, bb[gi].w};
+              const uint32_t rw[4] = {rr[gi].x, rr[gi].y, rr[gi].z, rr[gi].w};
               if (a.bias) {
-                float b[8];
-                load8(a.bias + ng, b);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] += b[j];
+                for (int j = 0; j < 4; ++j) { v[2 * j] += bf_lo(bw[j]); v[2 * j + 1] += bf_hi(bw[j]); }
               }
               if (EPI == PF_EPI_GELU) {
 #pragma unroll
                 for (int j = 0; j < 8; ++j) v[j] = 0.5f * v[j] * (1.f + erff(v[j] * 0.70710678118654752f));
               }
               if (a.resid) {
-                float rr[8];
-                load8(a.resid + (long long)m * a.ldr + ng, rr);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] += rr[j];
+                for (int j = 0; j < 4; ++j) { v[2 * j] += bf_lo(rw[j]); v[2 * j + 1] += bf_hi(rw[j]); }
               }
             }
             store8(a.y + (long long)m * a.ldy + ng, v);
@@ -356,7 +379,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(tempty + buf);
-      if (a.zdrop && q == 0) {
+      if (a.zdrop && q == 0 && part == 0) {
         // This tile's MMAs are complete: every TMA read of its z rows is
         // done.  One warp counts the block's finished column tiles; the last
         // CTA's warp discards the block's z lines (whole 128-byte lines
@@ -475,8 +498,11 @@ int prefill_linear_launch(const PfLinear& p, cudaStream_t stream) {
   a2.rope_cos = p.rope_cos; a2.rope_sin = p.rope_sin;
   a2.status = p.status;
   if (p.zcnt) { a2.zdrop = p.z; a2.zld = p.r; a2.zcnt = p.zcnt; }
-  return gemm(p.z, p.r, p.r, p.V, p.n, p.r, a2, p.epi, dual, dual ? "tc_stage2_swiglu" : "tc_stage2_zv",
-              stream);
+  const char* name = dual                  ? "tc_stage2_swiglu"
+                     : p.epi == PF_EPI_QKV ? "tc_stage2_qkv_rope"
+                     : p.resid             ? "tc_stage2_zv_resid"
+                                           : "tc_stage2_zv";
+  return gemm(p.z, p.r, p.r, p.V, p.n, p.r, a2, p.epi, dual, name, stream);
 }
 
 int prefill_dense_launch(const PfLinear& p, cudaStream_t stream) {
