@@ -134,11 +134,11 @@ struct DfCfg {
   static constexpr int SLOT = 32768;
   static constexpr int NSLOT = MT == 1 ? 6 : (MT == 2 ? 5 : 4);
   static constexpr int ABUF_BYTES = MT * DF_ABUF_COLS * 4;
-  static constexpr int RED_BYTES = CW * MT * 64 * 4 > 2048 ? CW * MT * 64 * 4 : 2048;
+  static constexpr int RED_BYTES = 512;              // per-warp sums of squares (RMSNorm)
   static constexpr int SCR_BYTES = (64 + CW * 128) * 4;
-  static constexpr int MISC_BYTES = 4608;  // chunk map and list, rstd, contributor table
+  static constexpr int MISC_BYTES = 6656;  // two schedule records, rstd, attention schedule
   static constexpr int BAR_BYTES = 512;
-  static constexpr int PH_BYTES = 768;     // copy of the stage table
+  static constexpr int PH_BYTES = 2 * 768;  // two copies of a layer's record tail (stage table)
   static constexpr int SMEM = 1024 + NSLOT * SLOT + ABUF_BYTES + RED_BYTES + SCR_BYTES + MISC_BYTES +
                               BAR_BYTES + PH_BYTES;
   static_assert(SMEM <= 232448, "shared memory budget");
@@ -369,43 +369,86 @@ __device__ __forceinline__ void ffma2(float& a0, float& a1, float x, float y0, f
       : "f"(x), "f"(y0), "f"(y1));
 }
 
-// acc[m][0..7] += A[m][kk] * W[kk][8 columns] over this thread's rows of a
-// 256-row entry.  a points at the entry's input chunk (row m at
-// m * DF_ABUF_COLS).  FULL: all 256 rows are valid; else rows at or beyond kn
-// are masked (their shared memory holds stale data).
-template <int MT, int RSTEP, bool FULL>
-__device__ __forceinline__ void entry_mac(float (&acc)[MT][8], const uint8_t* w, const float* a, int kn,
-                                          int row0) {
-  constexpr int IT = DF_KC / RSTEP;
-  uint4 u[IT];
-  float av[IT][MT];
+// acc[m][0..3] += A[m][kk] * W[kk][4 columns] over this lane's rows of a
+// ring entry.  w points at the warp's region of the entry: 16-byte pieces
+// (rows 2p and 2p + 1 of the warp's 4 columns), piece p = 32 i + lane, so
+// every load of the warp reads 512 consecutive bytes.  a points at the
+// entry's input chunk (row m at m * DF_ABUF_COLS).  FULL: all 256 rows are
+// valid; else pieces at or beyond kn / 2 are skipped (kn is even).
+template <int MT, bool FULL>
+__device__ __forceinline__ void entry_mac(float (&acc)[MT][4], const uint8_t* w, const float* a, int kn,
+                                          int lane) {
+  uint4 u[4];
+  float2 av[4][MT];
 #pragma unroll
-  for (int i = 0; i < IT; ++i) {
-    const int kk = row0 + RSTEP * i;
-    u[i] = *reinterpret_cast<const uint4*>(w + kk * 64);
+  for (int i = 0; i < 4; ++i) {
+    const int pc = 32 * i + lane;
+    const bool valid = FULL || 2 * pc < kn;
+    u[i] = valid ? *reinterpret_cast<const uint4*>(w + pc * 16) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-    for (int m = 0; m < MT; ++m) av[i][m] = a[m * DF_ABUF_COLS + kk];
+    for (int m = 0; m < MT; ++m)
+      av[i][m] = valid ? *reinterpret_cast<const float2*>(a + m * DF_ABUF_COLS + 2 * pc) : make_float2(0.f, 0.f);
   }
 #pragma unroll
-  for (int i = 0; i < IT; ++i) {
-    const bool valid = FULL || row0 + RSTEP * i < kn;
-    uint4 q = u[i];
-    if (!FULL && !valid) q = make_uint4(0u, 0u, 0u, 0u);
-    const float wv[8] = {bf_lo(q.x), bf_hi(q.x), bf_lo(q.y), bf_hi(q.y),
-                         bf_lo(q.z), bf_hi(q.z), bf_lo(q.w), bf_hi(q.w)};
+  for (int i = 0; i < 4; ++i) {
+    const float w0[4] = {bf_lo(u[i].x), bf_hi(u[i].x), bf_lo(u[i].y), bf_hi(u[i].y)};
+    const float w1[4] = {bf_lo(u[i].z), bf_hi(u[i].z), bf_lo(u[i].w), bf_hi(u[i].w)};
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
-      const float x = (FULL || valid) ? av[i][m] : 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; j += 2) ffma2(acc[m][j], acc[m][j + 1], x, wv[j], wv[j + 1]);
+      ffma2(acc[m][0], acc[m][1], av[i][m].x, w0[0], w0[1]);
+      ffma2(acc[m][2], acc[m][3], av[i][m].x, w0[2], w0[3]);
+      ffma2(acc[m][0], acc[m][1], av[i][m].y, w1[0], w1[1]);
+      ffma2(acc[m][2], acc[m][3], av[i][m].y, w1[2], w1[3]);
     }
   }
+}
+
+// Sum each of V values over the 32 lanes of a warp (V a power of 2, 4..16)
+// as a reduce-scatter: rounds with lane masks 16, 8, ... halve the values a
+// lane keeps, the rest are plain butterflies.  Returns the sum of value
+// scatter_index(lane), identical on the lanes that share it.
+template <int V>
+__device__ __forceinline__ float warp_reduce_scatter(float (&v)[V], int lane) {
+#pragma unroll
+  for (int n = V, s = 16; n > 1; n >>= 1, s >>= 1) {
+    const bool hi = (lane & s) != 0;
+#pragma unroll
+    for (int j = 0; j < n / 2; ++j) {
+      const float send = hi ? v[j] : v[j + n / 2];
+      const float keep = hi ? v[j + n / 2] : v[j];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+    }
+  }
+  float r = v[0];
+#pragma unroll
+  for (int s = 16 / V; s >= 1; s >>= 1) r += __shfl_xor_sync(0xffffffffu, r, s);
+  return r;
+}
+template <int V>
+__device__ __forceinline__ int scatter_index(int lane) {
+  int idx = 0;
+#pragma unroll
+  for (int n = V, s = 16; n > 1; n >>= 1, s >>= 1)
+    if (lane & s) idx += n / 2;
+  return idx;
 }
 
 __device__ __forceinline__ void prefetch_l2_2d(const CUtensorMap* tm, int c0, int c1) {
   asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(tm), "r"(c0), "r"(c1)
                : "memory");
 }
+
+template <int A, int B>
+struct RED_OK {
+  static constexpr bool value = A >= B;
+};
+
+// Asynchronous 16-byte global -> shared copy (completion: cp_async_wait).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 template <int MT>
 __global__ void __launch_bounds__(DfCfg<MT>::THREADS, 1)
@@ -418,17 +461,29 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
   float* red = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(abuf) + C::ABUF_BYTES);
   float* scr = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(red) + C::RED_BYTES);
   uint8_t* misc = reinterpret_cast<uint8_t*>(scr) + C::SCR_BYTES;
-  SchedRec* srec = reinterpret_cast<SchedRec*>(misc);    // this CTA's record of the current stage
+  // Two schedule-record buffers: GEMV stage k reads buffer k & 1 while the
+  // record of stage k + 1 lands in the other one (asynchronous copy).
+  SchedRec* const srec_buf = reinterpret_cast<SchedRec*>(misc);
+  SchedRec* srec = srec_buf;  // this CTA's record of the current stage
   int* clist = srec->clist;
   short* utab = &srec->utab[0][0];
-  float* s_rstd = reinterpret_cast<float*>(misc + sizeof(SchedRec));  // [8]
-  AttnSched* s_as = reinterpret_cast<AttnSched*>(misc + sizeof(SchedRec) + 64);  // attention schedule
-  static_assert(sizeof(SchedRec) + 64 + sizeof(AttnSched) <= C::MISC_BYTES, "misc shared area");
+  float* s_rstd = reinterpret_cast<float*>(misc + 2 * sizeof(SchedRec));  // [8]
+  AttnSched* s_as = reinterpret_cast<AttnSched*>(misc + 2 * sizeof(SchedRec) + 64);  // attention schedule
+  static_assert(RED_OK<C::RED_BYTES, C::CW * MT * 4>::value, "norm sums area");
+  static_assert(2 * sizeof(SchedRec) + 64 + sizeof(AttnSched) <= C::MISC_BYTES, "misc shared area");
   uint64_t* full = reinterpret_cast<uint64_t*>(misc + C::MISC_BYTES);
   uint64_t* empty = full + C::NSLOT;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + C::NSLOT);
-  DfPhase* s_ph = reinterpret_cast<DfPhase*>(reinterpret_cast<uint8_t*>(full) + C::BAR_BYTES);
-  static_assert(sizeof(DfPhase) * DF_NPHASE <= C::PH_BYTES, "stage table exceeds its shared copy");
+  // consumers' copy of the current layer's record tail: pack, sched,
+  // k_cache, v_cache, then the stage table
+  // (layer l reads copy l & 1; the next layer's lands in the other one)
+  uint8_t* const s_lyb_buf = reinterpret_cast<uint8_t*>(full) + C::BAR_BYTES;
+  uint8_t* s_lyb = s_lyb_buf;
+  DfPhase* s_ph = reinterpret_cast<DfPhase*>(s_lyb + (offsetof(DfLayer, ph) - offsetof(DfLayer, pack)));
+  constexpr int LYQ = (int)(offsetof(DfLayer, ph) + sizeof(DfPhase) * DF_NPHASE - offsetof(DfLayer, pack)) / 16;
+  static_assert(LYQ * 16 <= C::PH_BYTES / 2 && offsetof(DfLayer, pack) % 16 == 0 &&
+                    (offsetof(DfLayer, ph) + sizeof(DfPhase) * DF_NPHASE - offsetof(DfLayer, pack)) % 16 == 0,
+                "layer record tail exceeds its shared copy");
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, g = blockIdx.x;
@@ -530,12 +585,10 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
             const uint32_t par = (uint32_t)(seq / C::NSLOT) & 1u;
             if (!tc::mbar_wait_sleep(empty + slot, par ^ 1u, abort_flag, p.status)) { ok = false; break; }
             const int t = c / ph.nk, kc = c - t * ph.nk;
-            const uint32_t box = (uint32_t)min(DF_KC, ph.K - kc * DF_KC) * 64u;
+            const uint32_t bytes = (uint32_t)min(DF_KC, ph.K - kc * DF_KC) * 128u;
             const uint8_t* e = Ly->pack + ph.pack_off + (long long)t * ph.K * 128 + (long long)kc * 32768;
-            uint8_t* w = slots + slot * C::SLOT;
-            tc::mbar_expect_tx(full + slot, 2u * box);
-            bulk_g2s(w, e, box, full + slot);
-            bulk_g2s(w + 16384, e + box, box, full + slot);
+            tc::mbar_expect_tx(full + slot, bytes);
+            bulk_g2s(slots + slot * C::SLOT, e, bytes, full + slot);
             pf_step();
           }
         }
@@ -549,22 +602,60 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
     // ================================================= consumers ==========
     pdl_wait();
     if (tid == 0) attn_sched(p, *s_as);  // lengths are fixed for the launch
-    // lane bits: [1:0] 16-byte chunk, [2] row parity, [3] box, [..4] row lane;
-    // a quarter warp then reads two consecutive 64-byte rows of one box.
-    const int chunk = tid & 3, rsub = (tid >> 2) & 1, box = (tid >> 3) & 1, rowlane = tid >> 4;
-    const int cg = box * 4 + chunk;
-    const int row0 = 2 * rowlane + rsub;
-    constexpr int RSTEP = C::CT / 8;
+    // Consumer warp w owns columns 4 w .. 4 w + 3 of every ring entry (box
+    // w / 8) over all of the entry's rows: a tile's column sums need no
+    // exchange between warps.
+    const int box = warp >> 3;
     int seq = 0;
+    // Schedule record of the next GEMV stage, one 16-byte piece per thread
+    // (stage 0 after the first layer uses the previous layer's record 10).
+    // All of it comes from the current layer's records (sched_cur); the
+    // next layer's record tail is loaded into registers during the last stage.
+    bool rec_ready = false, ly_ready = false;
+    int gidx = 0;  // GEMV stages done in this launch: the current one reads srec_buf[gidx & 1]
+    const SchedRec* sched_cur = nullptr;
+    auto rec_fetch = [&](int rl, int rph, int buf) {
+      static_assert(sizeof(SchedRec) / 16 <= C::CT, "one 16-byte piece of the record per thread");
+      const SchedRec* r = sched_cur + (long long)((rph == 0 && rl > 0) ? DF_NPHASE + 1 : rph) * G;
+      SchedRec* dst = srec_buf + buf;
+      if (tid < (int)(sizeof(SchedRec) / 16))
+        cp_async16(reinterpret_cast<uint4*>(dst) + tid, reinterpret_cast<const uint4*>(r + g) + tid);
+      cp_async_commit();
+      rec_ready = true;
+    };
+    // layers after the first come from the device array p.layers
+    auto ly_fetch = [&](int rl) {
+      if (tid < LYQ)
+        cp_async16(s_lyb_buf + (rl & 1) * (C::PH_BYTES / 2) + tid * 16,
+                   reinterpret_cast<const uint4*>(&p.layers[rl].pack) + tid);
+      cp_async_commit();
+      ly_ready = true;
+    };
+    // record of the GEMV stage after (rl, rph) into buffer buf
+    auto next_gemv_stage = [&](int rl, int rph, int buf) {
+      ++rph;
+      if (rph < DF_NPHASE && s_ph[rph].type != DF_GEMV) ++rph;
+      if (rph >= DF_NPHASE) { rph = 0; ++rl; }
+      if (rl < p.nlayer) {
+        rec_fetch(rl, rph, buf);
+        if (rph == 0) ly_fetch(rl);
+      }
+    };
     for (int l = 0; l < p.nlayer; ++l) {
-    const DfLayer* Ly = layer_of(l);
     {
-      // this layer's stage table, read in every inner loop
+      // this layer's pointers and stage table, read in every inner loop
       consumer_sync<C::CT>();
-      const int* src = reinterpret_cast<const int*>(Ly->ph);
-      int* dst = reinterpret_cast<int*>(s_ph);
-      for (int i = tid; i < (int)(sizeof(DfPhase) * DF_NPHASE / 4); i += C::CT) dst[i] = src[i];
+      s_lyb = s_lyb_buf + (l & 1) * (C::PH_BYTES / 2);
+      s_ph = reinterpret_cast<DfPhase*>(s_lyb + (offsetof(DfLayer, ph) - offsetof(DfLayer, pack)));
+      if (l == 0) {
+        if (tid < LYQ) reinterpret_cast<uint4*>(s_lyb)[tid] = reinterpret_cast<const uint4*>(&layer_of(0)->pack)[tid];
+      } else {
+        if (!ly_ready) ly_fetch(l);
+        cp_async_wait();
+      }
+      ly_ready = false;
       consumer_sync<C::CT>();
+      sched_cur = *reinterpret_cast<const SchedRec* const*>(s_lyb + (offsetof(DfLayer, sched) - offsetof(DfLayer, pack)));
     }
     for (int ph_i = 0; ph_i < DF_NPHASE; ++ph_i) {
       const DfPhase& ph = s_ph[ph_i];
@@ -582,15 +673,14 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
         share(Ctot, G, g, c0, c1);
         const int nseg = ph.map == MAP_SWIGLU ? 2 : 1;
         const bool xin = src == SRC_X || src == SRC_XMID || src == SRC_XOUT;
-        // this CTA's schedule record of the stage (static: from the pack)
-        {
-          // (stage 0 after the first layer: the previous layer's record 10)
-          const SchedRec* r = src == SRC_XOUT ? layer_of(l - 1)->sched + (long long)(DF_NPHASE + 1) * G
-                                              : Ly->sched + (long long)ph_i * G;
-          const int4* rs = reinterpret_cast<const int4*>(r + g);
-          int4* dst = reinterpret_cast<int4*>(srec);
-          for (int w = tid; w < (int)(sizeof(SchedRec) / 16); w += C::CT) dst[w] = __ldg(rs + w);
-        }
+        // this CTA's schedule record of the stage (static: from the pack),
+        // copied while the previous stage ran
+        srec = srec_buf + (gidx & 1);
+        clist = srec->clist;
+        utab = &srec->utab[0][0];
+        if (!rec_ready) rec_fetch(l, ph_i, gidx & 1);
+        cp_async_wait();
+        rec_ready = false;
         consumer_sync<C::CT>();
 
         // ---- the stage input, built from what the previous stage left ----
@@ -798,13 +888,14 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
           consumer_sync<C::CT>();
         }
 
+        next_gemv_stage(l, ph_i, (gidx + 1) & 1);  // its record loads under this stage's entries
         // ---- entries ----
-        float acc[MT][8];
+        float acc[MT][4];
 #pragma unroll
         for (int m = 0; m < MT; ++m)
 #pragma unroll
-          for (int j = 0; j < 8; ++j) acc[m][j] = 0.f;
-        int su = 0, npend = 0;
+          for (int j = 0; j < 4; ++j) acc[m][j] = 0.f;
+        int su = 0;
         for (int c = c0; c < c1; ++c, ++seq) {
           const int slot = seq % C::NSLOT;
           const uint32_t par = (uint32_t)(seq / C::NSLOT) & 1u;
@@ -812,51 +903,45 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
           const int t = c / ph.nk, kc = c - t * ph.nk;
           const int k0 = kc * DF_KC;
           const int kn = min(DF_KC, ph.K - k0);
-          const uint8_t* w = slots + slot * C::SLOT + box * 16384 + chunk * 16;
+          const uint8_t* w = slots + slot * C::SLOT + warp * 8 * kn;
           const float* ain = ph.norm ? abuf + k0
                                      : abuf + srec->chunk_of[c - c0] * 256 * nseg + (nseg == 2 ? box * 256 : 0);
-          if (kn == DF_KC) entry_mac<MT, RSTEP, true>(acc, w, ain, kn, row0);
-          else entry_mac<MT, RSTEP, false>(acc, w, ain, kn, row0);
+          if (kn == DF_KC) entry_mac<MT, true>(acc, w, ain, kn, lane);
+          else entry_mac<MT, false>(acc, w, ain, kn, lane);
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(empty + slot);
 
           const bool tile_end = (c == c1 - 1) || (kc == ph.nk - 1);
           if (!tile_end) continue;
-          // ---- tile t done: each warp parks its column sums in shared
-          // memory; the CTA sums pending tiles once the area is full or the
-          // stage's entries are done (one CTA barrier for several tiles) ----
-          constexpr int kTileFloats = C::CW * MT * 64;
-          constexpr int kCap = (C::RED_BYTES + C::SCR_BYTES) / (kTileFloats * 4);  // red and scr are adjacent
-          static_assert(kCap >= 1, "tile-sum area");
-          float* tb = red + npend * kTileFloats;
+          // ---- tile t done: the warp's 4 x MT column sums, reduced over
+          // its lanes, go straight to this CTA's partial slot ----
+          constexpr int V = 4 * MT;
+          float v[V];
 #pragma unroll
           for (int m = 0; m < MT; ++m)
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              float v = acc[m][j];
-              v += __shfl_xor_sync(0xffffffffu, v, 4);
-              v += __shfl_xor_sync(0xffffffffu, v, 16);
-              acc[m][j] = 0.f;
-              if ((lane & 20) == 0) tb[(warp * MT + m) * 64 + cg * 8 + j] = v;
+            for (int j = 0; j < 4; ++j) { v[m * 4 + j] = acc[m][j]; acc[m][j] = 0.f; }
+          const float sum = warp_reduce_scatter<V>(v, lane);
+          if (su < DF_MAX_SU) {
+            if ((lane & (32 / V - 1)) == 0) {
+              const int idx = scatter_index<V>(lane);
+              __stcg(part_cur + ((long long)g * DF_MAX_SU + su) * DF_PART_STRIDE + (idx >> 2) * 64 + warp * 4 +
+                         (idx & 3),
+                     sum);
             }
-          ++npend;
-          ++su;
-          if (npend < kCap && c != c1 - 1) continue;
-          consumer_sync<C::CT>();
-          for (int o = tid; o < npend * MT * 64; o += C::CT) {
-            const int pt = o / (MT * 64), oo = o - pt * MT * 64;
-            const int sp = su - npend + pt;
-            float v = 0.f;
-#pragma unroll
-            for (int w8 = 0; w8 < C::CW; ++w8) v += red[pt * kTileFloats + (w8 * MT + (oo >> 6)) * 64 + (oo & 63)];
-            if (sp < DF_MAX_SU) __stcg(part_cur + ((long long)g * DF_MAX_SU + sp) * DF_PART_STRIDE + oo, v);
-            else if (oo == 0) atomicExch(p.status, DEV_STATUS_SCHEDULE);
+          } else if (lane == 0) {
+            atomicExch(p.status, DEV_STATUS_SCHEDULE);
           }
-          if (c != c1 - 1) consumer_sync<C::CT>();  // the area is reused by later tiles
-          npend = 0;
+          ++su;
         }
       } else {
         // ---------------------------------------------- attention stage --
+        // (contributor tables in the previous GEMV stage's record buffer;
+        // the next one's record lands in the other)
+        srec = srec_buf + ((gidx + 1) & 1);
+        clist = srec->clist;
+        utab = &srec->utab[0][0];
+        next_gemv_stage(l, ph_i, gidx & 1);
         const AttnSched& s = *s_as;
         const int Ctot = s.pre[8];
         int c0, c1;
@@ -912,7 +997,9 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
             *reinterpret_cast<float4*>(qkv + (pr * 3 + prob) * D + i) = lo;
             *reinterpret_cast<float4*>(qkv + (pr * 3 + prob) * D + i + hd) = hi;
             if (prob > 0 && owner_of(s.pre[b] + h * s.nk[b] + s.nk[b] - 1, Ctot, G) == g) {
-              bf16* dst = (prob == 1 ? Ly->k_cache : Ly->v_cache) + ((long long)b * p.S_max + pos) * (p.H * D) +
+              bf16* dst = *reinterpret_cast<bf16* const*>(
+                              s_lyb + (prob == 1 ? offsetof(DfLayer, k_cache) : offsetof(DfLayer, v_cache)) -
+                              offsetof(DfLayer, pack)) + ((long long)b * p.S_max + pos) * (p.H * D) +
                           h * D;
               uint2 o;
               o.x = pack_bf2(lo.x, lo.y); o.y = pack_bf2(lo.z, lo.w);
@@ -1068,6 +1155,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
         }
       }
       // ---- this CTA is done with stage ph_i ----
+      if (ph.type == DF_GEMV) ++gidx;
       consumer_sync<C::CT>();
       // (the CTA barrier above orders every consumer's writes before this
       // thread's release, which is cumulative over them)
@@ -1118,11 +1206,14 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
 namespace {
 
 // ------------------------------------------------------------ the pack --
-// Entry (t, kc) of a stage -- rows [256 kc, 256 kc + kn) of column tile t --
-// is stored as box 0 then box 1, each [kn x 32] bf16 row-major (64-byte
-// rows), at byte offset  stage_off + t * K * 128 + kc * 32768.  A box's 32
-// source columns (and, for the SwiGLU map, source rows) follow the stage's
-// output map; columns at or beyond the factor's width are zero.
+// Entry (t, kc) of a stage -- rows [256 kc, 256 kc + kn) of column tile t,
+// 128 kn bytes at byte offset  stage_off + t * K * 128 + kc * 32768 -- holds
+// 16 warp regions of 8 kn bytes.  Region w covers the entry's columns
+// 4 w .. 4 w + 3 (box w / 8: entry columns 0..31 are box 0, 32..63 box 1) as
+// kn / 2 pieces of 16 bytes; piece p holds rows 2p and 2p + 1 of those 4
+// columns, row-major.  A box's 32 source columns (and, for the SwiGLU map,
+// source rows) follow the stage's output map; columns at or beyond the
+// factor's width are zero.
 struct PackStage {
   long long off;
   int K, T, map, nprob, w_row2;
@@ -1154,14 +1245,14 @@ __global__ void __launch_bounds__(256) decode_pack_kernel(const __grid_constant_
     rem -= (long long)kc << 15;
     const int k0 = kc * DF_KC;
     const int kn = min(DF_KC, st.K - k0);
-    const int box = rem >= (long long)kn * 64 ? 1 : 0;
-    rem -= (long long)box * kn * 64;
-    const int row = (int)(rem >> 6), chunk = (int)((rem >> 4) & 3);
+    const int wr = (int)(rem / (8LL * kn));  // consumer warp region
+    const int pc = (int)((rem - (long long)wr * 8 * kn) >> 4);
+    const int box = wr >> 3;
     int pi = 0;
     for (int j = 1; j < 3; ++j)
       if (j < st.nprob && t >= st.tile_start[j]) pi = j;
     const int tl = t - st.tile_start[pi];
-    long long srow = k0 + row;
+    long long srow = k0 + 2 * pc;
     int col;
     if (st.map == MAP_PLAIN) {
       col = 64 * tl + 32 * box;
@@ -1172,9 +1263,14 @@ __global__ void __launch_bounds__(256) decode_pack_kernel(const __grid_constant_
       col = 32 * tl;
       srow += box * st.w_row2;
     }
-    col += 8 * chunk;
+    col += 4 * (wr & 7);
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (col < st.N[pi]) v = __ldg(reinterpret_cast<const uint4*>(st.src[pi] + srow * st.ld[pi] + col));
+    if (col < st.N[pi]) {
+      const bf16* r0 = st.src[pi] + srow * st.ld[pi] + col;
+      const uint2 a0 = __ldg(reinterpret_cast<const uint2*>(r0));
+      const uint2 a1 = __ldg(reinterpret_cast<const uint2*>(r0 + st.ld[pi]));
+      v = make_uint4(a0.x, a0.y, a1.x, a1.y);
+    }
     *reinterpret_cast<uint4*>(p.dst + byte) = v;
   }
 }

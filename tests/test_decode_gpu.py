@@ -184,21 +184,27 @@ def _layer_struct(fs, w, d, H, D, f, r, r_f, cos_t, sin_t, pack=True):
 
 def _expected_pack(w, d, H, D, f, r, r_f):
     """The decode pack written out from its definition in the header: per
-    stage, per column tile, per 256-row chunk, box 0 then box 1, each
-    [rows x 32] bf16 row-major; zero beyond a factor's width."""
+    stage, per column tile, per 256-row chunk (kn rows), 16 regions of 4
+    columns (region w: box w // 8, columns 4 (w % 8) .. + 3 of the box), each
+    kn / 2 pieces of rows (2p, 2p + 1) x those 4 columns, row-major; zero
+    beyond a factor's width."""
     def tiles(mats, K, cols_of_tile, ntiles, rows_of_box=None):
         out = []
         for M, T in zip(mats, ntiles):
             for t in range(T):
                 for k0 in range(0, K, 256):
                     kn = min(256, K - k0)
+                    boxes = []
                     for b in range(2):
                         c0 = cols_of_tile(t, b)
                         rs = rows_of_box(b) if rows_of_box else 0
                         blk = np.zeros((kn, 32), dtype=np.uint16)
                         src = M[rs + k0: rs + k0 + kn, c0: c0 + 32]
                         blk[:, :src.shape[1]] = src
-                        out.append(blk.ravel())
+                        boxes.append(blk)
+                    for wr in range(16):
+                        cols = boxes[wr // 8][:, 4 * (wr % 8): 4 * (wr % 8) + 4]  # [kn x 4]
+                        out.append(cols.reshape(kn // 2, 2, 4).ravel())
         return out
     plain = lambda t, b: 64 * t + 32 * b
     def rope(t, b):
