@@ -353,6 +353,11 @@ __device__ __forceinline__ void add_sq(float (&ssq)[MT], int m, const float4& v)
     if (mm == m) ssq[mm] += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
 }
 
+// v * g[j .. j + 3] (bf16 gains)
+__device__ __forceinline__ float4 gain4(float4 v, const bf16* g, int j) {
+  const uint2 gr = __ldg(reinterpret_cast<const uint2*>(g + j));
+  return make_float4(v.x * bf_lo(gr.x), v.y * bf_hi(gr.x), v.z * bf_lo(gr.y), v.w * bf_hi(gr.y));
+}
 __device__ __forceinline__ float4 round4(float4 v) {
   return make_float4(bf_round(v.x), bf_round(v.y), bf_round(v.z), bf_round(v.w));
 }
@@ -467,7 +472,6 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
   SchedRec* srec = srec_buf;  // this CTA's record of the current stage
   int* clist = srec->clist;
   short* utab = &srec->utab[0][0];
-  float* s_rstd = reinterpret_cast<float*>(misc + 2 * sizeof(SchedRec));  // [8]
   AttnSched* s_as = reinterpret_cast<AttnSched*>(misc + 2 * sizeof(SchedRec) + 64);  // attention schedule
   static_assert(RED_OK<C::RED_BYTES, C::CW * MT * 4>::value, "norm sums area");
   static_assert(2 * sizeof(SchedRec) + 64 + sizeof(AttnSched) <= C::MISC_BYTES, "misc shared area");
@@ -718,7 +722,10 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
             if (m < p.B && src != SRC_XOUT) {
               const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(p.x + (long long)m * p.d + j));
               v = make_float4(bf_lo(raw.x), bf_hi(raw.x), bf_lo(raw.y), bf_hi(raw.y));
-              if (src == SRC_X) add_sq<MT>(ssq, m, v);
+              if (src == SRC_X) {
+                add_sq<MT>(ssq, m, v);
+                if (ph.norm) v = gain4(v, ph.norm_g, j);
+              }
             }
             *reinterpret_cast<float4*>(abuf + m * DF_ABUF_COLS + j) = v;
           }
@@ -761,7 +768,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
               add4(v, sp[k2]);
               v = round4(v);
               add_sq<MT>(ssq, m, v);
-              *a4 = v;
+              *a4 = ph.norm ? gain4(v, ph.norm_g, j) : v;
               if ((j >> 6) % G == g) {
                 uint2 o;
                 o.x = pack_bf2(v.x, v.y);
@@ -859,33 +866,26 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
             }
           }
         }
-        consumer_sync<C::CT>();
+        // RMSNorm: the input holds x * g; rstd(x) scales the column sums at
+        // each tile's end.  Per-warp sums of squares go out with this barrier.
         if (ph.norm) {
-          // rstd of each row of the stage input (squares summed while building it)
 #pragma unroll
           for (int m = 0; m < MT; ++m) {
             const float ss = warp_sum(ssq[m]);
             if (lane == 0) red[warp * MT + m] = ss;
           }
-          consumer_sync<C::CT>();
-          if (tid < MT) {
+        }
+        consumer_sync<C::CT>();
+        float rstd[MT];
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          rstd[m] = 1.f;
+          if (ph.norm) {
             float ss = 0.f;
 #pragma unroll
-            for (int w = 0; w < C::CW; ++w) ss += red[w * MT + tid];
-            s_rstd[tid] = rsqrtf(ss / (float)p.d + p.eps);
+            for (int w = 0; w < C::CW; ++w) ss += red[w * MT + m];
+            rstd[m] = rsqrtf(ss / (float)p.d + p.eps);
           }
-          consumer_sync<C::CT>();
-          // the normalized input x * (rstd * g), once for all entries
-          for (int e = tid; e < MT * (p.d >> 2); e += C::CT) {
-            const int m = e / (p.d >> 2), j = (e - m * (p.d >> 2)) * 4;
-            const uint2 gr = __ldg(reinterpret_cast<const uint2*>(ph.norm_g + j));
-            const float r = s_rstd[m];
-            float4* a4 = reinterpret_cast<float4*>(abuf + m * DF_ABUF_COLS + j);
-            float4 v = *a4;
-            v.x *= r * bf_lo(gr.x); v.y *= r * bf_hi(gr.x); v.z *= r * bf_lo(gr.y); v.w *= r * bf_hi(gr.y);
-            *a4 = v;
-          }
-          consumer_sync<C::CT>();
         }
 
         next_gemv_stage(l, ph_i, (gidx + 1) & 1);  // its record loads under this stage's entries
@@ -925,9 +925,13 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
           if (su < DF_MAX_SU) {
             if ((lane & (32 / V - 1)) == 0) {
               const int idx = scatter_index<V>(lane);
+              float r = rstd[0];
+#pragma unroll
+              for (int m = 1; m < MT; ++m)
+                if ((idx >> 2) == m) r = rstd[m];
               __stcg(part_cur + ((long long)g * DF_MAX_SU + su) * DF_PART_STRIDE + (idx >> 2) * 64 + warp * 4 +
                          (idx & 3),
-                     sum);
+                     sum * r);
             }
           } else if (lane == 0) {
             atomicExch(p.status, DEV_STATUS_SCHEDULE);
