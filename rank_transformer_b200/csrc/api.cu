@@ -87,6 +87,8 @@ GvParams gv_base() {
   memset(&p, 0, sizeof(p));
   p.part = g_ctx.part;
   p.counters = g_ctx.counters;
+  p.part_cap = (long long)g_ctx.part_elems;
+  p.counters_cap = kCountersN;
   return p;
 }
 

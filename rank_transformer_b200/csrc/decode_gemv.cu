@@ -60,6 +60,10 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int cg = tid & 7, rr = tid >> 3;
   const int tile = blockIdx.x, split = blockIdx.y;
+  // row group blockIdx.z: rows m0 .. m0 + Mg - 1 of the launch's p.M rows
+  const int m0 = p.m0 + blockIdx.z * MT;
+  const int Mg = min(MT, p.M - blockIdx.z * MT);
+  const long long slot = (long long)blockIdx.z * gridDim.x + tile;  // partials / counter of this tile
 
   int pi = 0;
 #pragma unroll
@@ -97,8 +101,8 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
     float* ssq = red;  // [8 warps][MT] scratch, reused below
     for (int m = 0; m < MT; ++m) {
       float ss = 0.f;
-      if (m < p.M) {
-        const bf16* xr = p.x + (long long)(p.m0 + m) * p.ldx;
+      if (m < Mg) {
+        const bf16* xr = p.x + (long long)(m0 + m) * p.ldx;
         for (int c = tid * 8; c < p.K; c += GV_THREADS * 8) {
           float w[8];
           unpack8(*reinterpret_cast<const uint4*>(xr + c), w);
@@ -127,9 +131,9 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
       const int m = rem / kc8;
       const int kk = (rem - m * kc8) * 8;
       float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      if (m < p.M && kk < kn) {
+      if (m < Mg && kk < kn) {
         const int acol = (seg ? P.a_col2 : P.a_col) + k0 + kk;
-        const long long row = p.m0 + m;
+        const long long row = m0 + m;
         if (PRO == PRO_F32) {
           const float4* src = reinterpret_cast<const float4*>(p.a32 + row * p.lda + acol);
           const float4 u0 = src[0], u1 = src[1];
@@ -212,7 +216,7 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
   }
 
   if (p.splits > 1) {
-    float* mypart = p.part + ((long long)tile * p.splits + split) * NOUT;
+    float* mypart = p.part + (slot * p.splits + split) * NOUT;
 #pragma unroll
     for (int q = 0; q < PER; ++q) {
       const int o = tid + q * GV_THREADS;
@@ -220,13 +224,13 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
     }
     __threadfence();
     __syncthreads();
-    if (tid == 0) s_last = (atomicAdd(p.counters + tile, 1) == p.splits - 1);
+    if (tid == 0) s_last = (atomicAdd(p.counters + slot, 1) == p.splits - 1);
     __syncthreads();
     if (!s_last) return;
     __threadfence();
     // Sum the split partials: LPO threads per output, each a fixed stride
     // of splits, combined by a fixed shuffle tree (deterministic order).
-    const float* tp = p.part + (long long)tile * p.splits * NOUT;
+    const float* tp = p.part + slot * p.splits * NOUT;
     constexpr int LPO = NOUT >= GV_THREADS ? 1 : GV_THREADS / NOUT;
 #pragma unroll
     for (int q = 0; q < PER; ++q) {
@@ -248,7 +252,7 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
       for (int w = 1; w < LPO; w <<= 1) s += __shfl_xor_sync(0xffffffffu, s, w);
       val[q] = s;
     }
-    if (tid == 0) p.counters[tile] = 0;  // ready for the next launch
+    if (tid == 0) p.counters[slot] = 0;  // ready for the next launch
   }
 
   // ---- epilogue on the finished [MT x 64] tile ----
@@ -270,8 +274,8 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
     for (int o = tid; o < NOUT; o += GV_THREADS) {
       const int m = o >> 6, c = o & 63;
       const int gc = tile_col<MAP>(t, c, p.D);
-      if (m >= p.M || gc >= P.N) continue;
-      const long long row = p.m0 + m;
+      if (m >= Mg || gc >= P.N) continue;
+      const long long row = m0 + m;
       float v = fin[o];
       if (EPI == EPI_F32) {
         p.out32[row * p.ldo32 + P.out_col + gc] = v;
@@ -285,8 +289,8 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
     const int half = p.D >> 1;
     for (int o = tid; o < MT * 32; o += GV_THREADS) {
       const int m = o >> 5, c = o & 31;
-      if (m >= p.M) continue;
-      const int b = p.m0 + m;
+      if (m >= Mg) continue;
+      const int b = m0 + m;
       int pos = p.seqlens[b];
       pos = pos < 0 ? 0 : (pos >= p.S_max ? p.S_max - 1 : pos);
       const int glo = tile_col<MAP>(t, c, p.D);
@@ -309,10 +313,10 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
     for (int o = tid; o < MT * 32; o += GV_THREADS) {
       const int m = o >> 5, c = o & 31;
       const int fc = t * 32 + c;
-      if (m >= p.M || fc >= P.N) continue;
+      if (m >= Mg || fc >= P.N) continue;
       const float g = fin[m * 64 + c], u = fin[m * 64 + c + 32];
       const float h = g / (1.f + expf(-g)) * u;
-      p.out16[(long long)(p.m0 + m) * p.ldo16 + fc] = f2bf(h);
+      p.out16[(long long)(m0 + m) * p.ldo16 + fc] = f2bf(h);
     }
   }
 }
@@ -356,7 +360,7 @@ int launch_one(const GvParams& p, int total_tiles, cudaStream_t stream) {
   for (int i = 0; i < p.nprob; ++i)
     flops += 2.0 * p.M * (double)p.K * p.prob[i].N * (EPI == EPI_SWIGLU ? 2.0 : 1.0);
   const LaunchTag tag{gv_name(PRO, EPI), gv_bytes(p, PRO, EPI), flops};
-  return launch_pdl(tag, kern, dim3(total_tiles, p.splits), dim3(GV_THREADS), smem, stream, p);
+  return launch_pdl(tag, kern, dim3(total_tiles, p.splits, ceil_div(p.M, MT)), dim3(GV_THREADS), smem, stream, p);
 }
 
 template <int PRO, int EPI, int MAP>
@@ -383,19 +387,26 @@ int gemv_launch(GvParams p, int pro, int epi, int map, int total_rows,
     tiles += gemv_tiles_for(map, p.prob[i].N, p.D);
   }
   for (int i = p.nprob; i < 4; ++i) p.tile_start[i] = tiles;
-  // Split K so that about `target_ctas` CTAs (one resident wave) cover the
-  // launch, with at most 512 factor rows (64 KB) per CTA.
-  int splits = target_ctas / (tiles > 0 ? tiles : 1);
+  // One launch for all rows: groups of up to 8 rows are the third grid
+  // dimension (each CTA of a group re-reads its factor block, from L2 after
+  // the first).  Split K so that about `target_ctas` CTAs (one resident
+  // wave) cover the launch, with at most 512 factor rows (64 KB) per CTA.
+  const int groups = ceil_div(total_rows, 8);
+  const int slots = tiles * groups;
+  int splits = target_ctas / (slots > 0 ? slots : 1);
   splits = splits < 1 ? 1 : splits;
   const int max_splits = ceil_div(p.K, 32);
   splits = splits > max_splits ? max_splits : splits;
   p.KC = round_up(ceil_div(p.K, splits), 32);
   p.KC = p.KC > 512 ? 512 : p.KC;
   p.splits = ceil_div(p.K, p.KC);
-
-  for (int m0 = 0; m0 < total_rows; m0 += 8) {
-    p.m0 = m0;
-    p.M = total_rows - m0 < 8 ? total_rows - m0 : 8;
+  const int mt = total_rows <= 1 ? 1 : (total_rows <= 2 ? 2 : (total_rows <= 4 ? 4 : 8));
+  if ((long long)slots > p.counters_cap ||
+      (p.splits > 1 && (long long)slots * p.splits * mt * 64 > p.part_cap))
+    return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  {
+    p.m0 = 0;
+    p.M = total_rows;
     int st = FLASHSVD_ERR_INVALID_ARG;
 #define FSVD_GV(PRO_, EPI_, MAP_) \
     if (pro == PRO_ && epi == EPI_ && map == MAP_) st = launch_mt<PRO_, EPI_, MAP_>(p, tiles, stream);

@@ -46,12 +46,13 @@ struct GvParams {
   const float* rope_cos; const float* rope_sin;     // [S_max x D/2]
   // workspace
   float* part; int* counters;
+  long long part_cap; int counters_cap;             // their sizes (floats, ints)
 };
 
 enum GvMap { MAP_PLAIN = 0, MAP_ROPE = 1, MAP_SWIGLU = 2 };
 
 // Host launcher: fills tile_start/splits/KC, picks the row-tile variant and
-// launches once per group of 8 rows.
+// launches once (row groups of up to 8 as the grid's third dimension).
 int gemv_launch(GvParams p, int pro, int epi, int map, int total_rows,
                 int target_ctas, cudaStream_t stream);
 int gemv_tiles_for(int map, int N, int D);

@@ -111,6 +111,7 @@ extern "C" int flashsvd_lowrank_linear_noalloc(const flashsvd_bf16* x, const fla
   p1.x = reinterpret_cast<const bf16*>(x); p1.ldx = d;
   p1.out32 = s->z; p1.ldo32 = r;
   p1.part = s->part; p1.counters = s->counters;
+  p1.part_cap = kNaPartFloats; p1.counters_cap = kNaCounters;
   FSVD_TRY(gemv_launch(p1, PRO_BF16, EPI_F32, MAP_PLAIN, M, target, stream));
 
   GvParams p2;
@@ -121,5 +122,6 @@ extern "C" int flashsvd_lowrank_linear_noalloc(const flashsvd_bf16* x, const fla
   p2.out16 = reinterpret_cast<bf16*>(y); p2.ldo16 = n;
   p2.bias = reinterpret_cast<const bf16*>(bias);
   p2.part = s->part; p2.counters = s->counters;
+  p2.part_cap = kNaPartFloats; p2.counters_cap = kNaCounters;
   return gemv_launch(p2, PRO_F32, EPI_BF16, MAP_PLAIN, M, target, stream);
 }

@@ -64,6 +64,7 @@ def test_lowrank_linear_svd_factors(fs):
 
 
 @pytest.mark.parametrize("M,d,r_f,f,r_dn", [(1, 256, 64, 688, 64), (5, 256, 64, 688, 64),
+                                           (20, 256, 64, 688, 64),
                                            (1, 4096, 1792, 11008, 1792),
                                            (8, 4096, 512, 11008, 1024)])
 def test_packed_mlp_decode(fs, M, d, r_f, f, r_dn):
