@@ -28,6 +28,23 @@ __device__ __forceinline__ void unpack8(const uint4& v, float* w) {
   w[4] = bf_lo(v.z); w[5] = bf_hi(v.z); w[6] = bf_lo(v.w); w[7] = bf_hi(v.w);
 }
 
+// (a0, a1) += x * (y0, y1): one packed fp32x2 FMA (sm_100).
+__device__ __forceinline__ void gv_ffma2(float& a0, float& a1, float x, float y0, float y1) {
+  asm("{\n\t.reg .b64 acc, xx, yy;\n\t"
+      "mov.b64 acc, {%0, %1};\n\t"
+      "mov.b64 xx, {%2, %2};\n\t"
+      "mov.b64 yy, {%3, %4};\n\t"
+      "fma.rn.f32x2 acc, xx, yy, acc;\n\t"
+      "mov.b64 {%0, %1}, acc;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(x), "f"(y0), "f"(y1));
+}
+
+// Split partial stride: the MT x 64 tile plus 8 floats (RMSNORM: the
+// split's sums of squares of its rows).
+template <int MT>
+__host__ __device__ constexpr int gv_part_stride() { return MT * 64 + 8; }
+
 // Global output column of tile column c (0..63) for the column map.
 template <int MAP>
 __device__ __forceinline__ int tile_col(int t, int c, int D) {
@@ -54,7 +71,7 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
   float* As = sm;                                   // [NSEG][MT][KC] fp32
   float* red = As + NSEG * MT * p.KC;               // [8][MT][64] fp32
   bf16* Ws = reinterpret_cast<bf16*>(red + 8 * MT * 64);  // [KC][64] bf16
-  __shared__ float s_rstd[MT];
+  __shared__ float s_ssq[MT];  // RMSNORM: sums of squares of this CTA's row slices, then of whole rows
   __shared__ int s_last;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -96,32 +113,12 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
 
   pdl_wait();
   // ---- stage the activation slice A[m0+m, acol + k0 .. + KC) in fp32 ----
-  if (PRO == PRO_RMSNORM) {
-    // Sum of squares of each row: all 256 threads read the row at once.
-    float* ssq = red;  // [8 warps][MT] scratch, reused below
-    for (int m = 0; m < MT; ++m) {
-      float ss = 0.f;
-      if (m < Mg) {
-        const bf16* xr = p.x + (long long)(m0 + m) * p.ldx;
-        for (int c = tid * 8; c < p.K; c += GV_THREADS * 8) {
-          float w[8];
-          unpack8(*reinterpret_cast<const uint4*>(xr + c), w);
+  // RMSNorm: the staged slice holds x * g; the squares of x are summed
+  // over this CTA's slice here and over the splits by the reducer, which
+  // scales the finished tile by rstd (no pass over the whole row per CTA).
+  float ss_t[MT];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) ss = fmaf(w[j], w[j], ss);
-        }
-      }
-      ss = warp_sum(ss);
-      if (lane == 0) ssq[warp * MT + m] = ss;
-    }
-    __syncthreads();
-    if (tid < MT) {
-      float ss = 0.f;
-#pragma unroll
-      for (int w = 0; w < GV_THREADS / 32; ++w) ss += ssq[w * MT + tid];
-      s_rstd[tid] = rsqrtf(ss / (float)p.K + p.eps);
-    }
-    __syncthreads();
-  }
+  for (int m = 0; m < MT; ++m) ss_t[m] = 0.f;
   {
     const int kc8 = p.KC >> 3;
     const int items = NSEG * MT * kc8;
@@ -142,11 +139,16 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
         } else {
           unpack8(*reinterpret_cast<const uint4*>(p.x + row * p.ldx + acol), a);
           if (PRO == PRO_RMSNORM) {
-            float g[8];
+            float g[8], ss = 0.f;
             unpack8(*reinterpret_cast<const uint4*>(p.norm_g + acol), g);
-            const float rs = s_rstd[m];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) a[j] = a[j] * rs * g[j];
+            for (int j = 0; j < 8; ++j) {
+              ss = fmaf(a[j], a[j], ss);
+              a[j] *= g[j];
+            }
+#pragma unroll
+            for (int mm = 0; mm < MT; ++mm)
+              if (mm == m) ss_t[mm] += ss;
           }
         }
       }
@@ -155,7 +157,20 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
       dst[1] = make_float4(a[4], a[5], a[6], a[7]);
     }
   }
+  if (PRO == PRO_RMSNORM) {
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      const float ss = warp_sum(ss_t[m]);
+      if (lane == 0) red[warp * MT + m] = ss;
+    }
+  }
   __syncthreads();
+  if (PRO == PRO_RMSNORM && tid < MT) {
+    float ss = 0.f;
+#pragma unroll
+    for (int w = 0; w < GV_THREADS / 32; ++w) ss += red[w * MT + tid];
+    s_ssq[tid] = ss;  // (red is next written after the barrier below)
+  }
 
   // ---- multiply-accumulate from shared memory ----
   cp_async_wait_all();
@@ -177,7 +192,7 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
       for (int m = 0; m < MT; ++m) {
         const float a = Aseg[m * p.KC + kk];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[m][j] = fmaf(a, w[j], acc[m][j]);
+        for (int j = 0; j < 8; j += 2) gv_ffma2(acc[m][j], acc[m][j + 1], a, w[j], w[j + 1]);
       }
     }
   }
@@ -216,12 +231,14 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
   }
 
   if (p.splits > 1) {
-    float* mypart = p.part + (slot * p.splits + split) * NOUT;
+    constexpr int NP = gv_part_stride<MT>();
+    float* mypart = p.part + (slot * p.splits + split) * NP;
 #pragma unroll
     for (int q = 0; q < PER; ++q) {
       const int o = tid + q * GV_THREADS;
       if (o < NOUT) __stcg(mypart + o, val[q]);
     }
+    if (PRO == PRO_RMSNORM && tid < MT) __stcg(mypart + NOUT + tid, s_ssq[tid]);
     __threadfence();
     __syncthreads();
     if (tid == 0) s_last = (atomicAdd(p.counters + slot, 1) == p.splits - 1);
@@ -230,7 +247,7 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
     __threadfence();
     // Sum the split partials: LPO threads per output, each a fixed stride
     // of splits, combined by a fixed shuffle tree (deterministic order).
-    const float* tp = p.part + slot * p.splits * NOUT;
+    const float* tp = p.part + slot * p.splits * NP;
     constexpr int LPO = NOUT >= GV_THREADS ? 1 : GV_THREADS / NOUT;
 #pragma unroll
     for (int q = 0; q < PER; ++q) {
@@ -240,17 +257,22 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
       if (o < NOUT) {
         int sp = sub;
         for (; sp + 3 * LPO < p.splits; sp += 4 * LPO) {
-          const float v0 = __ldcg(tp + (long long)sp * NOUT + o);
-          const float v1 = __ldcg(tp + (long long)(sp + LPO) * NOUT + o);
-          const float v2 = __ldcg(tp + (long long)(sp + 2 * LPO) * NOUT + o);
-          const float v3 = __ldcg(tp + (long long)(sp + 3 * LPO) * NOUT + o);
+          const float v0 = __ldcg(tp + (long long)sp * NP + o);
+          const float v1 = __ldcg(tp + (long long)(sp + LPO) * NP + o);
+          const float v2 = __ldcg(tp + (long long)(sp + 2 * LPO) * NP + o);
+          const float v3 = __ldcg(tp + (long long)(sp + 3 * LPO) * NP + o);
           s += ((v0 + v1) + (v2 + v3));
         }
-        for (; sp < p.splits; sp += LPO) s += __ldcg(tp + (long long)sp * NOUT + o);
+        for (; sp < p.splits; sp += LPO) s += __ldcg(tp + (long long)sp * NP + o);
       }
 #pragma unroll
       for (int w = 1; w < LPO; w <<= 1) s += __shfl_xor_sync(0xffffffffu, s, w);
       val[q] = s;
+    }
+    if (PRO == PRO_RMSNORM && tid < MT) {
+      float ss = 0.f;  // sums of squares of the whole rows, in split order
+      for (int sp = 0; sp < p.splits; ++sp) ss += __ldcg(tp + (long long)sp * NP + NOUT + tid);
+      s_ssq[tid] = ss;
     }
     if (tid == 0) p.counters[slot] = 0;  // ready for the next launch
   }
@@ -277,6 +299,7 @@ gemv_splitk_kernel(const __grid_constant__ GvParams p) {
       if (m >= Mg || gc >= P.N) continue;
       const long long row = m0 + m;
       float v = fin[o];
+      if (PRO == PRO_RMSNORM) v *= rsqrtf(s_ssq[m] / (float)p.K + p.eps);
       if (EPI == EPI_F32) {
         p.out32[row * p.ldo32 + P.out_col + gc] = v;
       } else {
@@ -402,7 +425,7 @@ int gemv_launch(GvParams p, int pro, int epi, int map, int total_rows,
   p.splits = ceil_div(p.K, p.KC);
   const int mt = total_rows <= 1 ? 1 : (total_rows <= 2 ? 2 : (total_rows <= 4 ? 4 : 8));
   if ((long long)slots > p.counters_cap ||
-      (p.splits > 1 && (long long)slots * p.splits * mt * 64 > p.part_cap))
+      (p.splits > 1 && (long long)slots * p.splits * (mt * 64 + 8) > p.part_cap))
     return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   {
     p.m0 = 0;

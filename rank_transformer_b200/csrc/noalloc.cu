@@ -65,7 +65,7 @@ long long partials_needed(int K, int tiles, int rows, int target) {
   KC = KC > 512 ? 512 : KC;
   splits = ceil_div(K, KC);
   const int mt = rows <= 1 ? 1 : rows <= 2 ? 2 : rows <= 4 ? 4 : 8;
-  return (long long)tiles * splits * mt * 64;
+  return (long long)tiles * splits * (mt * 64 + 8);  // split partial stride of the GEMV
 }
 
 }  // namespace
