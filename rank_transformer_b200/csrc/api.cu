@@ -215,6 +215,27 @@ PfLinear pf_base(const bf16* x, long long ldx, const flashsvd_factor& F, int M,
   return p;
 }
 
+// Stage 1 of the q, k, v projections of x in one grouped tcgen05 launch,
+// into three regions of the rank-activation scratch; false (nothing
+// launched) when they do not fit it together.
+bool qkv_stage1_grouped(const bf16* x, int d, int M, const flashsvd_factor* const* F, bf16** z,
+                        cudaStream_t s, int* st) {
+  const long long need = (long long)M * (F[0]->r + F[1]->r + F[2]->r);
+  if (need > (long long)g_ctx.rows * 2 * g_ctx.max_rank) return false;
+  const bf16* U[3];
+  int r[3];
+  long long off = 0;
+  for (int i = 0; i < 3; ++i) {
+    U[i] = cb(F[i]->U);
+    r[i] = F[i]->r;
+    z[i] = g_ctx.zb + off;
+    off += (long long)M * r[i];
+    if (!aligned16(z[i]) || r[i] % 8) return false;
+  }
+  *st = prefill_stage1_grouped(x, d, d, M, 3, U, r, z, g_ctx.status, s);
+  return true;
+}
+
 bool g_fused_decode = true;
 
 // Whether the fused decode layer (and hence a decode pack) covers L's shapes.
@@ -302,8 +323,13 @@ int layer_prefill(const flashsvd_layer* L, bf16* x, bf16* kc, bf16* vc,
   FSVD_TRY(rmsnorm_launch(x, cb(L->norm1_g), g_ctx.xn, M, d, L->norm_eps, s));
   const flashsvd_factor* F[3] = {&L->q, &L->k, &L->v};
   bf16* dst[3] = {g_ctx.q, kc, vc};
+  bf16* zg[3];
+  int gst = FLASHSVD_OK;
+  const bool grouped = qkv_stage1_grouped(g_ctx.xn, d, M, F, zg, s, &gst);
+  FSVD_TRY(gst);
   for (int i = 0; i < 3; ++i) {
     PfLinear p = pf_base(g_ctx.xn, d, *F[i], M, d, d, g_ctx.q, d);
+    if (grouped) { p.z = zg[i]; p.z_ready = 1; }
     p.epi = PF_EPI_QKV; p.kind = i; p.cache = dst[i]; p.S = S; p.S_max = S_max;
     p.HD = d; p.D = L->D;
     if (i < 2) { p.rope_cos = L->rope_cos; p.rope_sin = L->rope_sin; }
@@ -339,8 +365,13 @@ int layer_encoder(const flashsvd_layer* L, bf16* x, bf16* kc, bf16* vc,
   const int d = L->d, M = B * S;
   const flashsvd_factor* F[3] = {&L->q, &L->k, &L->v};
   bf16* dst[3] = {g_ctx.q, kc, vc};
+  bf16* zg[3];
+  int gst = FLASHSVD_OK;
+  const bool grouped = qkv_stage1_grouped(x, d, M, F, zg, s, &gst);
+  FSVD_TRY(gst);
   for (int i = 0; i < 3; ++i) {
     PfLinear p = pf_base(x, d, *F[i], M, d, d, g_ctx.q, d);
+    if (grouped) { p.z = zg[i]; p.z_ready = 1; }
     p.epi = PF_EPI_QKV; p.kind = i; p.cache = dst[i]; p.S = S; p.S_max = S_max;
     p.HD = d; p.D = L->D;
     FSVD_TRY(prefill_linear_launch(p, s));

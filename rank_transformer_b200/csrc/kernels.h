@@ -99,8 +99,13 @@ struct PfLinear {
   bf16* z;                           // [M x r] bf16 scratch for the rank activations
   int* zcnt;                         // [ceil(M / 128)] zero counters: z blocks discarded from L2 after use, or null
   int* status;
+  int z_ready;                       // z already holds x . U (stage 1 skipped)
 };
 int prefill_linear_launch(const PfLinear& p, cudaStream_t stream);
+// Stage 1 of n <= 3 factorized linears sharing x, in one tcgen05 launch:
+// z[i] [M x r[i]] = x . U[i] (bf16, row stride r[i]).
+int prefill_stage1_grouped(const bf16* x, long long ldx, int d, int M, int n, const bf16* const* U,
+                           const int* r, bf16* const* z, int* status, cudaStream_t stream);
 int prefill_dense_launch(const PfLinear& p, cudaStream_t stream);
 
 // --------------------------------------------- fused decode layer ---------

@@ -84,7 +84,18 @@ struct TcArgs {
   // between launches) discards the block's L2 lines, so z is never written
   // back to HBM.
   const bf16* zdrop; long long zld; int* zcnt;
+  // Grouped form (plain bf16 epilogue only): nprob problems share A; the
+  // global column-tile index runs over problem 0's tiles, then 1's, then
+  // 2's (first tile pt[i]); problem i has B map i, output gy[i] (row
+  // stride gldy[i]) and width gN[i].  nprob <= 1: a.y, a.ldy, a.N.
+  int nprob; int pt[3];
+  bf16* gy[3]; long long gldy[3]; int gN[3];
 };
+
+// Problem of global column tile gn of a grouped launch, and its first tile.
+__device__ __forceinline__ int group_of(const TcArgs& a, int gn) {
+  return a.nprob <= 1 ? 0 : (gn >= a.pt[1]) + (a.nprob > 2 && gn >= a.pt[2]);
+}
 
 __device__ __forceinline__ void store8(bf16* p, const float* v) {
   uint4 u;
@@ -113,6 +124,7 @@ struct Layout {
 template <int BN, int STAGES, bool DUAL, int EPI>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
                const __grid_constant__ TcArgs a) {
   using L = Layout<BN, STAGES, DUAL>;
   extern __shared__ uint8_t smem_raw[];
@@ -147,6 +159,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   if (warp == 0 && lane == 0) {
     tc::tma_prefetch_desc(&tmA);
     tc::tma_prefetch_desc(&tmB);
+    if (a.nprob > 1) tc::tma_prefetch_desc(&tmB1);
+    if (a.nprob > 2) tc::tma_prefetch_desc(&tmB2);
   }
   if (warp == 1) {
     tc::tmem_alloc(tmem_holder, L::TMEM_COLS);
@@ -168,7 +182,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       int issued = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-        const int m0 = (t % a.tiles_m) * BM, n0 = (t / a.tiles_m) * BN;
+        const int gn = t / a.tiles_m, gp = group_of(a, gn);
+        const int m0 = (t % a.tiles_m) * BM, n0 = (gn - (gp ? a.pt[gp] : 0)) * BN;
+        const CUtensorMap* mB = gp == 0 ? &tmB : (gp == 1 ? &tmB1 : &tmB2);
         for (int kb = 0; kb < kb_total; ++kb) {
           if (!tc::mbar_wait(empty + stage, phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
           tc::mbar_expect_tx(full + stage, L::STAGE_BYTES);
@@ -180,7 +196,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           uint8_t* sB = sA + L::A_BYTES;
           tc::tma_load_2d(sA, &tmA, full + stage, ka, m0);
 #pragma unroll
-          for (int j = 0; j < BN / 64; ++j) tc::tma_load_2d(sB + j * 8192, &tmB, full + stage, n0 + 64 * j, kr);
+          for (int j = 0; j < BN / 64; ++j) tc::tma_load_2d(sB + j * 8192, mB, full + stage, n0 + 64 * j, kr);
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -248,7 +264,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const uint32_t tph = (uint32_t)(it >> 1) & 1u;
       if (!tc::mbar_wait(tfull + buf, tph, abort_flag, a.status)) break;
       tc::fence_after_sync();
-      const int m0 = (t % a.tiles_m) * BM, n0 = (t / a.tiles_m) * BN;
+      const int gn = t / a.tiles_m, gp = group_of(a, gn);
+      const int m0 = (t % a.tiles_m) * BM, n0 = (gn - (gp ? a.pt[gp] : 0)) * BN;
+      // this tile's output (grouped launches: its problem's)
+      bf16* const ty = a.nprob > 1 ? a.gy[gp] : a.y;
+      const long long tldy = a.nprob > 1 ? a.gldy[gp] : a.ldy;
+      const int tN = a.nprob > 1 ? a.gN[gp] : a.N;
       const int m = m0 + row;
       const bool mok = m < a.M;
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * L::ACC_COLS);
@@ -323,7 +344,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
               const int ng = n + 8 * g;
-              const bool in = mok && ng < a.N;
+              const bool in = mok && ng < tN;
               rr[g] = (in && a.resid) ? *reinterpret_cast<const uint4*>(a.resid + (long long)m * a.ldr + ng)
                                       : make_uint4(0u, 0u, 0u, 0u);
               bb[g] = (in && a.bias) ? *reinterpret_cast<const uint4*>(a.bias + ng) : make_uint4(0u, 0u, 0u, 0u);
@@ -339,7 +360,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
             const int ng = n + 8 * g;
-            if (ng >= a.N) break;
+            if (ng >= tN) break;
             float v[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) v[j] = __uint_as_float(r0[8 * g + j]);
@@ -372,7 +393,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 for (int j = 0; j < 4; ++j) { v[2 * j] += bf_lo(rw[j]); v[2 * j + 1] += bf_hi(rw[j]); }
               }
             }
-            store8(a.y + (long long)m * a.ldy + ng, v);
+            store8(ty + (long long)m * tldy + ng, v);
           }
         }
       }
@@ -436,8 +457,8 @@ double gemm_bytes(const TcArgs& a, bool dual) {
 }
 
 template <int BN, int STAGES, bool DUAL, int EPI>
-int launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, TcArgs a, const char* name,
-              cudaStream_t stream) {
+int launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb1, const CUtensorMap& mb2,
+              TcArgs a, const char* name, cudaStream_t stream) {
   using L = Layout<BN, STAGES, DUAL>;
   auto kern = tc_gemm_kernel<BN, STAGES, DUAL, EPI>;
   static bool configured = false;
@@ -446,12 +467,24 @@ int launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, TcArgs a, const char
     configured = true;
   }
   a.tiles_m = ceil_div(a.M, BM);
-  a.tiles_n = ceil_div(a.N, BN);
+  if (a.nprob > 1) {
+    // grouped: problem i's column tiles start at pt[i]; a.N = total width
+    int nt = 0;
+    a.N = 0;
+    for (int i = 0; i < a.nprob; ++i) {
+      a.pt[i] = nt;
+      nt += ceil_div(a.gN[i], BN);
+      a.N += a.gN[i];
+    }
+    a.tiles_n = nt;
+  } else {
+    a.tiles_n = ceil_div(a.N, BN);
+  }
   const int tiles = a.tiles_m * a.tiles_n;
   const int grid = tiles < sm_count() ? tiles : sm_count();
   const double flops = 2.0 * a.M * (double)a.N * a.K * (DUAL ? 2.0 : 1.0);
   const LaunchTag tag{name, gemm_bytes(a, DUAL), flops};
-  return launch_pdl(tag, kern, dim3(grid), dim3(TC_THREADS), (size_t)L::SMEM, stream, ma, mb, a);
+  return launch_pdl(tag, kern, dim3(grid), dim3(TC_THREADS), (size_t)L::SMEM, stream, ma, mb, mb1, mb2, a);
 }
 
 // One tensor-core GEMM C = A . B with the given epilogue.
@@ -461,19 +494,38 @@ int gemm(const bf16* A, long long lda, long long a_cols, const bf16* B, long lon
   FSVD_TRY(make_map(&ma, A, a.M, a_cols, lda, BM));
   if (dual) {
     FSVD_TRY(make_map(&mb, B, b_rows, a.N, ldb, BK));
-    return launch_tc<128, 6, true, PF_EPI_SWIGLU>(ma, mb, a, name, stream);
+    return launch_tc<128, 6, true, PF_EPI_SWIGLU>(ma, mb, mb, mb, a, name, stream);
   }
   FSVD_TRY(make_map(&mb, B, b_rows, a.N, ldb, BK));
   switch (epi) {
-    case PF_EPI_BF16: return launch_tc<256, 4, false, PF_EPI_BF16>(ma, mb, a, name, stream);
-    case PF_EPI_GELU: return launch_tc<256, 4, false, PF_EPI_GELU>(ma, mb, a, name, stream);
-    case PF_EPI_QKV: return launch_tc<256, 4, false, PF_EPI_QKV>(ma, mb, a, name, stream);
-    case PF_EPI_F32: return launch_tc<256, 4, false, PF_EPI_F32>(ma, mb, a, name, stream);
+    case PF_EPI_BF16: return launch_tc<256, 4, false, PF_EPI_BF16>(ma, mb, mb, mb, a, name, stream);
+    case PF_EPI_GELU: return launch_tc<256, 4, false, PF_EPI_GELU>(ma, mb, mb, mb, a, name, stream);
+    case PF_EPI_QKV: return launch_tc<256, 4, false, PF_EPI_QKV>(ma, mb, mb, mb, a, name, stream);
+    case PF_EPI_F32: return launch_tc<256, 4, false, PF_EPI_F32>(ma, mb, mb, mb, a, name, stream);
     default: return FLASHSVD_ERR_INVALID_ARG;
   }
 }
 
 }  // namespace
+
+int prefill_stage1_grouped(const bf16* x, long long ldx, int d, int M, int n, const bf16* const* U,
+                           const int* r, bf16* const* z, int* status, cudaStream_t stream) {
+  if (n < 1 || n > 3) return FLASHSVD_ERR_INVALID_ARG;
+  TcArgs a;
+  memset(&a, 0, sizeof(a));
+  a.M = M; a.K = d;
+  a.status = status;
+  a.nprob = n;
+  CUtensorMap ma, mb[3];
+  FSVD_TRY(make_map(&ma, x, M, d, ldx, BM));
+  for (int i = 0; i < n; ++i) {
+    FSVD_TRY(make_map(&mb[i], U[i], d, r[i], r[i], BK));
+    a.gy[i] = z[i]; a.gldy[i] = r[i]; a.gN[i] = r[i];
+  }
+  a.y = z[0]; a.ldy = r[0];
+  return launch_tc<256, 4, false, PF_EPI_BF16>(ma, mb[0], mb[n > 1 ? 1 : 0], mb[n > 2 ? 2 : 0], a,
+                                               "tc_stage1_xu_grouped", stream);
+}
 
 int prefill_linear_launch(const PfLinear& p, cudaStream_t stream) {
   if (!p.z) return FLASHSVD_ERR_NOT_INITIALIZED;
@@ -486,7 +538,7 @@ int prefill_linear_launch(const PfLinear& p, cudaStream_t stream) {
   a1.M = p.M; a1.N = p.r; a1.K = p.d;
   a1.y = p.z; a1.ldy = p.r;
   a1.status = p.status;
-  FSVD_TRY(gemm(p.x, p.ldx, p.d, p.U, p.r, p.d, a1, PF_EPI_BF16, false, "tc_stage1_xu", stream));
+  if (!p.z_ready) FSVD_TRY(gemm(p.x, p.ldx, p.d, p.U, p.r, p.d, a1, PF_EPI_BF16, false, "tc_stage1_xu", stream));
   // Stage 2: y = epilogue(z . V).
   TcArgs a2;
   memset(&a2, 0, sizeof(a2));
