@@ -165,6 +165,12 @@ __device__ __forceinline__ void red_release_add(int* p, int v) {
   asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 __device__ __forceinline__ float bf_round(float v) { return bf2f(f2bf(v)); }
+// 2^x with the hardware approximation (relative error ~2^-22; 2^-inf = +0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 // Bounded wait until stage counter *bar reaches target.
 __device__ __forceinline__ void grid_wait(const int* bar, int target, volatile int* abort_flag, int* status) {
@@ -318,7 +324,7 @@ __device__ __forceinline__ float4 attn_gather4(const float* buf, const short* u,
     for (int c = 0; c < 4; ++c) {
       if (mc[c] == -INFINITY) continue;
       const float Mn = fmaxf(M, mc[c]);
-      const float a = M == -INFINITY ? 0.f : exp2f(M - Mn), b = exp2f(mc[c] - Mn);
+      const float a = M == -INFINITY ? 0.f : ex2_approx(M - Mn), b = ex2_approx(mc[c] - Mn);
       Ls = Ls * a + lc[c] * b;
       O = make_float4(O.x * a + oc[c].x * b, O.y * a + oc[c].y * b, O.z * a + oc[c].z * b, O.w * a + oc[c].w * b);
       M = Mn;
@@ -1088,8 +1094,8 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
           for (int o = LPK; o < 32; o <<= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
           const float mn = fmaxf(m_w, mb);
           if (mn != -INFINITY) {  // warp-uniform
-            const float corr = m_w == -INFINITY ? 0.f : exp2f(m_w - mn);
-            const float pj = sc == -INFINITY ? 0.f : exp2f(sc - mn);
+            const float corr = m_w == -INFINITY ? 0.f : ex2_approx(m_w - mn);
+            const float pj = sc == -INFINITY ? 0.f : ex2_approx(sc - mn);
             l_g = l_g * corr + pj;
 #pragma unroll
             for (int e = 0; e < CPL_MAX * 8; ++e) ov[e] *= corr;
@@ -1143,7 +1149,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
           float Lc = 0.f, oc = 0.f;
 #pragma unroll
           for (int w2 = 0; w2 < C::CW; ++w2) {
-            const float wgt = (wm[w2] == -INFINITY) ? 0.f : exp2f(wm[w2] - Mc);
+            const float wgt = (wm[w2] == -INFINITY) ? 0.f : ex2_approx(wm[w2] - Mc);
             Lc += wgt * wl[w2];
             if (tid < D) oc += wgt * wo[w2 * 128 + tid];
           }
