@@ -1066,7 +1066,8 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
           const int key = kc * 64 + key_l;
           const uint8_t* kb = slots + slot * C::SLOT;
           const uint8_t* vb = kb + 16384;
-          float dot = 0.f;
+          // two partial dots (even / odd dims) keep the FMA chains short
+          float dot = 0.f, dot1 = 0.f;
           if (key == pos) {
 #pragma unroll
             for (int cc = 0; cc < CPL_MAX; ++cc)
@@ -1083,9 +1084,13 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
                 const float kv[8] = {bf_lo(u.x), bf_hi(u.x), bf_lo(u.y), bf_hi(u.y),
                                      bf_lo(u.z), bf_hi(u.z), bf_lo(u.w), bf_hi(u.w)};
 #pragma unroll
-                for (int e = 0; e < 8; ++e) dot = fmaf(qv[cc * 8 + e], kv[e], dot);
+                for (int e = 0; e < 8; e += 2) {
+                  dot = fmaf(qv[cc * 8 + e], kv[e], dot);
+                  dot1 = fmaf(qv[cc * 8 + e + 1], kv[e + 1], dot1);
+                }
               }
           }
+          dot += dot1;
 #pragma unroll
           for (int o = LPK / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
           const float sc = key < L ? dot : -INFINITY;
