@@ -32,6 +32,16 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// (a0, a1) += (b0, b1) as one packed fp32x2 add.
+__device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 aa, bb;\n\t"
+      "mov.b64 aa, {%0, %1};\n\t"
+      "mov.b64 bb, {%2, %3};\n\t"
+      "add.rn.f32x2 aa, aa, bb;\n\t"
+      "mov.b64 {%0, %1}, aa;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(b0), "f"(b1));
+}
 // (x0, x1) * s + (c, c) as one packed fp32x2 FMA.
 __device__ __forceinline__ void fma2_sc(float& x0, float& x1, float sc, float c) {
   asm("{\n\t.reg .b64 xx, ss, cc;\n\t"
@@ -279,8 +289,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           fma2_sc(x0, x1, sc, mneg);  // masked keys: -inf, and 2^-inf = 0
           pv[e] = ex2_approx(x0);
           pv[e + 1] = ex2_approx(x1);
-          l4[e & 3] += pv[e];
-          l4[(e + 1) & 3] += pv[e + 1];
+          add2(l4[e & 3], l4[(e + 1) & 3], pv[e], pv[e + 1]);
         }
         uint4 u;
         u.x = pack_bf2(pv[0], pv[1]); u.y = pack_bf2(pv[2], pv[3]);
