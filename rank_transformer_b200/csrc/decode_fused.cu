@@ -17,14 +17,17 @@
 //
 // Factors.  They are read from the layer's decode pack: every factor matrix
 // re-tiled once, at load time, so that each ring entry (256 rows x 64 output
-// columns, as two [rows x 32] boxes) is one contiguous block of HBM, stored
-// in consumption order.  Whole blocks stream near the HBM copy rate; 64- or
-// 128-byte row pieces spaced at the matrix pitch do not.
+// columns, laid out as 16 per-warp regions of 4 columns) is one contiguous
+// block of HBM, stored in consumption order.  Whole blocks stream near the
+// HBM copy rate; 64- or 128-byte row pieces spaced at the matrix pitch do
+// not.
 //
 // Reduction ("reduce on read").  A CTA's share of a stage is a contiguous
 // range of (tile, 256-row chunk) entries, so a column tile's K range is
-// split over a few CTAs.  A CTA writes one fp32 partial per tile it touched
-// and nothing else: no atomics, no last-arriver combine.  After the grid
+// split over a few CTAs.  Consumer warp w owns columns 4w..4w+3 of every
+// entry, so a tile's column sums are complete inside each warp; the CTA
+// writes one fp32 partial per tile it touched and nothing else: no atomics,
+// no last-arriver combine.  After the grid
 // barrier, each CTA builds the stage input it needs by summing those
 // partials (in CTA order, so every reader gets the same bits) and applying
 // the previous stage's epilogue as it reads: RoPE and bf16 rounding of q/k/v,
@@ -34,15 +37,17 @@
 // Hence the K/V chunks themselves depend on no stage and are loaded as soon
 // as ring slots free up.
 //
-// Roles per CTA (CW consumer warps + 2 producer warps):
-//   warp CW   producer: fills every ring entry in order -- bulk copies of
-//             pack entries for the GEMV stages (prefetched ahead into L2),
-//             TMA loads of 64-key cache chunks for attention; it never waits
-//             for activations.
-//   warp CW+1 prefetches this CTA's cache chunks into L2 at kernel start.
+// Roles per CTA (CW consumer warps + 1 producer warp):
+//   warp CW   producer: fills every ring entry in order -- one bulk copy
+//             per pack entry for the GEMV stages (prefetched two entries
+//             ahead into L2), TMA loads of 64-key cache chunks for attention
+//             (a layer's chunks of this CTA are prefetched into L2 at its
+//             stage 1); it never waits for activations.
 //   consumers multiply-accumulate ring entries against the stage input
 //             built in shared memory, and run attention with per-warp
-//             online-softmax state.
+//             online-softmax state.  The next GEMV stage's schedule record
+//             and the next layer's stage table are copied (cp.async) into
+//             second shared-memory buffers while the current stage runs.
 // All waits are bounded; a timeout sets the device status word.
 #include <algorithm>
 #include <cstring>

@@ -14,8 +14,11 @@
 //               (M=128, N=BN, K=16) into one of two accumulator buffers and
 //               frees ring slots / publishes finished tiles with
 //               tcgen05.commit;
-//   warps 2..5  read the accumulator with tcgen05.ld (one TMEM lane
-//               quadrant each), apply the fused epilogue and store.
+//   warps 2..9  read the accumulator with tcgen05.ld (two warps per TMEM
+//               lane quadrant, alternate 64-column pairs), apply the fused
+//               epilogue and store.
+// A grouped launch runs up to three GEMMs that share A (q, k, v stage 1):
+// their column tiles follow one another, each with its own B and output.
 // Every wait is bounded: on expiry the CTA raises the device status word
 // and winds down (waits for its own copies, frees tensor memory).
 #include <cstring>
