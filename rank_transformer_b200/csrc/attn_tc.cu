@@ -5,7 +5,8 @@
 // one); here it reads the same dense [B, S_max, H, D] cache the prefill's
 // q/k/v epilogue wrote.  Causal (decoder) or bidirectional (encoder).
 //
-// One CTA per (128-query tile, batch row, head), 6 warps:
+// Persistent CTAs (one per SM) walk the (128-query tile, batch row, head)
+// items, heaviest first; 10 warps:
 //   warp 0  TMA: Q once, then 128-key K and V tiles into a 2-stage ring;
 //   warp 1  TMEM owner and MMA issuer: S = Q K^T into one of two 128-column
 //           TMEM buffers, then O += P V into a D-column TMEM accumulator;
@@ -90,16 +91,30 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   uint64_t* p_full = s_empty + 2;
   uint64_t* o_done = p_full + 1;
   uint64_t* drain = o_done + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* q_empty = drain + 1;     // the item's S MMAs are done: Q may be reloaded
+  uint64_t* o_free = q_empty + 1;    // the epilogue has read O (count 8)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(o_free + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // heaviest (longest causal) query tiles first
-  const int qt = gridDim.x - 1 - blockIdx.x;
-  const int bh = blockIdx.y, b = bh / p.H, h = bh - b * p.H;
-  const int m0 = qt * AT_BM;
+  // Persistent: work item k = (query tile, batch row, head), heaviest
+  // (longest causal) query tiles first; CTA c takes items c, c + G, ...
+  // Barrier phases run on across items: T counts this CTA's key tiles, I
+  // its items.
+  const int qtiles = (p.S + AT_BM - 1) / AT_BM;
+  const int BH = p.B * p.H;
+  const int NW = qtiles * BH;
   const int nt_all = (p.S + AT_BN - 1) / AT_BN;
-  const int nt = CAUSAL ? min(nt_all, (m0 + AT_BM + AT_BN - 1) / AT_BN) : nt_all;
+  struct Item { int b, h, m0, nt; };
+  auto item_of = [&](int k) {
+    Item it;
+    const int qt = qtiles - 1 - k / BH, bh = k - (k / BH) * BH;
+    it.b = bh / p.H;
+    it.h = bh - it.b * p.H;
+    it.m0 = qt * AT_BM;
+    it.nt = CAUSAL ? min(nt_all, (it.m0 + AT_BM + AT_BN - 1) / AT_BN) : nt_all;
+    return it;
+  };
 
   if (threadIdx.x == 0) {
     tc::mbar_init(q_full, 1);
@@ -112,6 +127,8 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     tc::mbar_init(p_full, 8);
     tc::mbar_init(o_done, 1);
     tc::mbar_init(drain, 1);
+    tc::mbar_init(q_empty, 1);
+    tc::mbar_init(o_free, 8);
     *abort_flag = 0;
     tc::fence_barrier_init();
   }
@@ -135,19 +152,26 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA --
     if (lane == 0) {
-      const int hx = h * D;
-      tc::mbar_expect_tx(q_full, (uint32_t)(L::KB * L::TILE));
-      for (int kb = 0; kb < L::KB; ++kb)
-        tc::tma_load_2d(smem + L::Q_OFF + kb * L::TILE, &tmQ, q_full, hx + 64 * kb, b * p.S + m0);
-      for (int j = 0; j < nt; ++j) {
-        const int st = j & 1;
-        if (!tc::mbar_wait(kv_empty + st, ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag, p.status)) break;
-        tc::mbar_expect_tx(kv_full + st, (uint32_t)(2 * L::KB * L::TILE));
-        const int row = b * p.S_max + j * AT_BN;
-        for (int kb = 0; kb < L::KB; ++kb) {
-          tc::tma_load_2d(smem + L::K_OFF + (st * L::KB + kb) * L::TILE, &tmK, kv_full + st, hx + 64 * kb, row);
-          tc::tma_load_2d(smem + L::V_OFF + (st * L::KB + kb) * L::TILE, &tmV, kv_full + st, hx + 64 * kb, row);
+      int T = 0;
+      bool ok = true;
+      for (int k = blockIdx.x, I = 0; k < NW && ok; k += gridDim.x, ++I) {
+        const Item it = item_of(k);
+        const int hx = it.h * D;
+        if (!(ok = tc::mbar_wait(q_empty, ((uint32_t)I & 1u) ^ 1u, abort_flag, p.status))) break;
+        tc::mbar_expect_tx(q_full, (uint32_t)(L::KB * L::TILE));
+        for (int kb = 0; kb < L::KB; ++kb)
+          tc::tma_load_2d(smem + L::Q_OFF + kb * L::TILE, &tmQ, q_full, hx + 64 * kb, it.b * p.S + it.m0);
+        for (int j = 0; j < it.nt; ++j) {
+          const int t = T + j, st = t & 1;
+          if (!(ok = tc::mbar_wait(kv_empty + st, ((uint32_t)(t >> 1) & 1u) ^ 1u, abort_flag, p.status))) break;
+          tc::mbar_expect_tx(kv_full + st, (uint32_t)(2 * L::KB * L::TILE));
+          const int row = it.b * p.S_max + j * AT_BN;
+          for (int kb = 0; kb < L::KB; ++kb) {
+            tc::tma_load_2d(smem + L::K_OFF + (st * L::KB + kb) * L::TILE, &tmK, kv_full + st, hx + 64 * kb, row);
+            tc::tma_load_2d(smem + L::V_OFF + (st * L::KB + kb) * L::TILE, &tmV, kv_full + st, hx + 64 * kb, row);
+          }
         }
+        T += it.nt;
       }
     }
   } else if (warp == 1) {
@@ -157,38 +181,49 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       constexpr uint32_t IDESC_O = tc::idesc_bf16(D, true);       // B = V rows, MN-major
       const uint32_t sq = tc::smem_u32(smem + L::Q_OFF);
       const uint32_t sp = tc::smem_u32(smem + L::P_OFF);
-      bool ok = tc::mbar_wait(q_full, 0, abort_flag, p.status);
-      auto issue_pv = [&](int j) {
-        // O (+)= P_j V_j once the softmax has written P_j (and rescaled O)
-        if (!tc::mbar_wait(p_full, (uint32_t)j & 1u, abort_flag, p.status)) return false;
-        tc::fence_after_sync();
-        const uint32_t sv = tc::smem_u32(smem + L::V_OFF + (j & 1) * L::KB * L::TILE);
+      bool ok = true;
+      int T = 0;
+      for (int k = blockIdx.x, I = 0; k < NW && ok; k += gridDim.x, ++I) {
+        const Item it = item_of(k);
+        // O (+)= P_t V_t once the softmax has written P_t (and rescaled O);
+        // an item's first P V overwrites O, so the previous item's epilogue
+        // must have read it
+        auto issue_pv = [&](int t, bool first) {
+          if (!tc::mbar_wait(p_full, (uint32_t)t & 1u, abort_flag, p.status)) return false;
+          if (first && !tc::mbar_wait(o_free, ((uint32_t)I & 1u) ^ 1u, abort_flag, p.status)) return false;
+          tc::fence_after_sync();
+          const uint32_t sv = tc::smem_u32(smem + L::V_OFF + (t & 1) * L::KB * L::TILE);
 #pragma unroll
-        for (int k = 0; k < AT_BN / 16; ++k) {
-          const uint64_t ad = tc::sdesc_sw128(sp + (k >> 2) * L::TILE + (k & 3) * 32, 16, 1024);
-          const uint64_t bd = tc::sdesc_sw128(sv + k * 2048, L::TILE, 1024);
-          tc::mma_bf16(tmem + 256, ad, bd, IDESC_O, (j > 0 || k > 0) ? 1u : 0u);
-        }
-        tc::mma_commit(o_done);
-        tc::mma_commit(kv_empty + (j & 1));
-        return true;
-      };
-      for (int j = 0; j < nt && ok; ++j) {
-        const int st = j & 1;
-        if (!(ok = tc::mbar_wait(kv_full + st, (uint32_t)(j >> 1) & 1u, abort_flag, p.status))) break;
-        if (!(ok = tc::mbar_wait(s_empty + st, ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag, p.status))) break;
-        tc::fence_after_sync();
-        const uint32_t sk = tc::smem_u32(smem + L::K_OFF + st * L::KB * L::TILE);
+          for (int kk = 0; kk < AT_BN / 16; ++kk) {
+            const uint64_t ad = tc::sdesc_sw128(sp + (kk >> 2) * L::TILE + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = tc::sdesc_sw128(sv + kk * 2048, L::TILE, 1024);
+            tc::mma_bf16(tmem + 256, ad, bd, IDESC_O, (!first || kk > 0) ? 1u : 0u);
+          }
+          tc::mma_commit(o_done);
+          tc::mma_commit(kv_empty + (t & 1));
+          return true;
+        };
+        if (!(ok = tc::mbar_wait(q_full, (uint32_t)I & 1u, abort_flag, p.status))) break;
+        for (int j = 0; j < it.nt && ok; ++j) {
+          const int t = T + j, st = t & 1;
+          if (!(ok = tc::mbar_wait(kv_full + st, (uint32_t)(t >> 1) & 1u, abort_flag, p.status))) break;
+          if (!(ok = tc::mbar_wait(s_empty + st, ((uint32_t)(t >> 1) & 1u) ^ 1u, abort_flag, p.status))) break;
+          tc::fence_after_sync();
+          const uint32_t sk = tc::smem_u32(smem + L::K_OFF + st * L::KB * L::TILE);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint64_t ad = tc::sdesc_sw128(sq + (k >> 2) * L::TILE + (k & 3) * 32, 16, 1024);
-          const uint64_t bd = tc::sdesc_sw128(sk + (k >> 2) * L::TILE + (k & 3) * 32, 16, 1024);
-          tc::mma_bf16(tmem + st * AT_BN, ad, bd, IDESC_S, k > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ad = tc::sdesc_sw128(sq + (kk >> 2) * L::TILE + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = tc::sdesc_sw128(sk + (kk >> 2) * L::TILE + (kk & 3) * 32, 16, 1024);
+            tc::mma_bf16(tmem + st * AT_BN, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          tc::mma_commit(s_full + st);
+          if (j > 0) ok = issue_pv(t - 1, j == 1);
         }
-        tc::mma_commit(s_full + st);
-        if (j > 0) ok = issue_pv(j - 1);
+        if (!ok) break;
+        tc::mma_commit(q_empty);  // fires once this item's S MMAs are done
+        if (it.nt > 0) ok = issue_pv(T + it.nt - 1, it.nt == 1);
+        T += it.nt;
       }
-      if (ok && nt > 0) issue_pv(nt - 1);
       // every MMA this thread issued has completed once `drain` fires
       tc::mma_commit(drain);
       const long long t0 = clock64();
@@ -201,11 +236,10 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     const int quad = warp & 3;
     const int hf = (warp - 2) >> 2;
     const int r = quad * 32 + lane;       // query row within the tile
-    const int q = m0 + r;                 // query position
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     float* xr = reinterpret_cast<float*>(smem + L::X_OFF);  // [2][2][128]
     const float sc = p.scale_log2;
-    float m = -INFINITY, l = 0.f;         // m: reference max, scaled units
+    float m, l;                           // m: reference max, scaled units
     uint8_t* sP = smem + L::P_OFF;
     constexpr int HC = AT_BN / 2;         // keys per thread
     constexpr int OC = D / 2;             // O columns per thread
@@ -218,9 +252,18 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     };
     auto sm_sync = [] { asm volatile("bar.sync 1, 256;" ::: "memory"); };
     bool ok = true;
+    int T = 0;
+    // (every item and tile is visited even after a failed wait, so that the
+    // named barriers stay matched)
+    for (int k = blockIdx.x, I = 0; k < NW; k += gridDim.x, ++I) {
+    const Item it = item_of(k);
+    const int m0 = it.m0, nt = it.nt, b = it.b, h = it.h;
+    const int q = m0 + r;                 // query position
+    m = -INFINITY;
+    l = 0.f;
     for (int j = 0; j < nt; ++j) {
-      const int st = j & 1;
-      ok = ok && wwait(s_full + st, (uint32_t)(j >> 1) & 1u);
+      const int t = T + j, st = t & 1;
+      ok = ok && wwait(s_full + st, (uint32_t)(t >> 1) & 1u);
       float s[HC];
       if (ok) {
         tc::fence_after_sync();
@@ -253,7 +296,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       const float rawmax = fmaxf(xt[r], xt[128 + r]);
       const float mx = rawmax == -INFINITY ? -INFINITY : rawmax * sc;
       // PV of tile j-1 must be complete before O is rescaled or P rewritten
-      if (j > 0) ok = ok && wwait(o_done, (uint32_t)(j - 1) & 1u);
+      if (j > 0) ok = ok && wwait(o_done, (uint32_t)(t - 1) & 1u);
       tc::fence_after_sync();
       // The row's reference m (P = 2^(s sc - m)) moves up only when the tile
       // max exceeds it by more than 8: P stays <= 2^8 (exact enough in bf16
@@ -303,11 +346,12 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       if (lane == 0) tc::mbar_arrive(p_full);
     }
     // ---- O / l -> bf16 ----
-    const bool fin = ok && nt > 0 && wwait(o_done, (uint32_t)(nt - 1) & 1u);
+    const bool fin = ok && nt > 0 && wwait(o_done, (uint32_t)(T + nt - 1) & 1u);
     sm_sync();  // every partner has read the last tile's row maxima
     xr[hf * 128 + r] = l;
     sm_sync();
     const float lt = xr[r] + xr[128 + r];
+    sm_sync();  // both halves have read l before the next item's maxima reuse xr
     if (fin) {
       tc::fence_after_sync();
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
@@ -331,6 +375,12 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         }
       }
     }
+    // O is read: the next item's first P V may overwrite it
+    tc::fence_before_sync();
+    __syncwarp();
+    if (lane == 0) tc::mbar_arrive(o_free);
+    T += nt;
+    }  // items
   }
 
   tc::fence_before_sync();
@@ -365,7 +415,14 @@ int launch_at(const AttnPfParams& ap, cudaStream_t stream) {
   p.scale_log2 = ap.scale_log2;
   p.out = ap.out;
   p.status = ap.status;
-  const dim3 grid(ceil_div(ap.S, AT_BM), ap.B * ap.H);
+  const int items = ceil_div(ap.S, AT_BM) * ap.B * ap.H;
+  int sms = 148;
+  {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  const dim3 grid(items < sms ? items : sms);
   const double S = ap.S;
   const double flops = 4.0 * ap.B * ap.H * S * S * D * (CAUSAL ? 0.5 : 1.0);
   const LaunchTag tag{CAUSAL ? "attn_prefill_causal" : "attn_prefill_bidir", 2.0 * 4.0 * ap.B * S * HD, flops};
