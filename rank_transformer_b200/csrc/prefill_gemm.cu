@@ -100,6 +100,26 @@ __device__ __forceinline__ int group_of(const TcArgs& a, int gn) {
   return a.nprob <= 1 ? 0 : (gn >= a.pt[1]) + (a.nprob > 2 && gn >= a.pt[2]);
 }
 
+// GELU(v) = v * Phi(v) = 0.5 v (1 + erf(v / sqrt 2)), with erf from
+// Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26:
+// erf(x) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-x^2),
+// t = 1 / (1 + p x), x >= 0 (odd extension), |error| <= 1.5e-7 -- below the
+// bf16 rounding of the output, and branch-free (one reciprocal, one exp2).
+__device__ __forceinline__ float gelu_erf(float v) {
+  const float x = fabsf(v) * 0.70710678118654752f;
+  float t;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t) : "f"(fmaf(0.3275911f, x, 1.f)));
+  float poly = fmaf(1.061405429f, t, -1.453152027f);
+  poly = fmaf(poly, t, 1.421413741f);
+  poly = fmaf(poly, t, -0.284496736f);
+  poly = fmaf(poly, t, 0.254829592f);
+  poly *= t;
+  float e;  // exp(-x^2) = 2^(-x^2 log2 e)
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-x * x * 1.4426950408889634f));
+  const float erf_abs = fmaf(-poly, e, 1.f);
+  return 0.5f * v * (1.f + copysignf(erf_abs, v));
+}
+
 __device__ __forceinline__ void store8(bf16* p, const float* v) {
   uint4 u;
   u.x = pack_bf2(v[0], v[1]); u.y = pack_bf2(v[2], v[3]);
@@ -389,7 +409,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
               }
               if (EPI == PF_EPI_GELU) {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] = 0.5f * v[j] * (1.f + erff(v[j] * 0.70710678118654752f));
+                for (int j = 0; j < 8; ++j) v[j] = gelu_erf(v[j]);
               }
               if (a.resid) {
 #pragma unroll
