@@ -33,6 +33,12 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 // (a0, a1) += (b0, b1) as one packed fp32x2 add.
 __device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
   asm("{\n\t.reg .b64 aa, bb;\n\t"
@@ -281,15 +287,16 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       // mask (raw scores: the scale is positive) and partial row max
       const int n0 = j * AT_BN + hf * HC;
       const bool need_mask = n0 + HC > p.S || (CAUSAL && n0 + HC - 1 > m0);
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (need_mask) {
 #pragma unroll
-      for (int c = 0; c < HC; ++c) {
-        if (need_mask) {
+        for (int c = 0; c < HC; ++c) {
           const int key = n0 + c;
           if (key >= p.S || (CAUSAL && key > q)) s[c] = -INFINITY;
         }
-        mx4[c & 3] = fmaxf(mx4[c & 3], s[c]);
       }
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int c = 0; c < HC; c += 2) mx4[(c >> 1) & 3] = max3(mx4[(c >> 1) & 3], s[c], s[c + 1]);
       float* xt = xr + st * 256;
       xt[hf * 128 + r] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       sm_sync();
