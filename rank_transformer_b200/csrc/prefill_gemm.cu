@@ -104,20 +104,55 @@ __device__ __forceinline__ int group_of(const TcArgs& a, int gn) {
 // Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26:
 // erf(x) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-x^2),
 // t = 1 / (1 + p x), x >= 0 (odd extension), |error| <= 1.5e-7 -- below the
-// bf16 rounding of the output, and branch-free (one reciprocal, one exp2).
-__device__ __forceinline__ float gelu_erf(float v) {
-  const float x = fabsf(v) * 0.70710678118654752f;
-  float t;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t) : "f"(fmaf(0.3275911f, x, 1.f)));
-  float poly = fmaf(1.061405429f, t, -1.453152027f);
-  poly = fmaf(poly, t, 1.421413741f);
-  poly = fmaf(poly, t, -0.284496736f);
-  poly = fmaf(poly, t, 0.254829592f);
-  poly *= t;
-  float e;  // exp(-x^2) = 2^(-x^2 log2 e)
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-x * x * 1.4426950408889634f));
-  const float erf_abs = fmaf(-poly, e, 1.f);
-  return 0.5f * v * (1.f + copysignf(erf_abs, v));
+// bf16 rounding of the output, and branch-free (one reciprocal, one exp2);
+// gelu_erf2 below evaluates it on two values with packed fp32x2 arithmetic.
+
+// Packed fp32x2 helpers: (a0, a1) op (b0, b1) [op (c0, c1)] in one instruction.
+__device__ __forceinline__ void fma_x2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                       float c1) {
+  asm("{\n\t.reg .b64 aa, bb, cc;\n\t"
+      "mov.b64 aa, {%2, %3};\n\t"
+      "mov.b64 bb, {%4, %5};\n\t"
+      "mov.b64 cc, {%6, %7};\n\t"
+      "fma.rn.f32x2 aa, aa, bb, cc;\n\t"
+      "mov.b64 {%0, %1}, aa;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void mul_x2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 aa, bb;\n\t"
+      "mov.b64 aa, {%2, %3};\n\t"
+      "mov.b64 bb, {%4, %5};\n\t"
+      "mul.rn.f32x2 aa, aa, bb;\n\t"
+      "mov.b64 {%0, %1}, aa;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void gelu_erf2(float& v0, float& v1) {
+  float x0, x1;
+  mul_x2(x0, x1, fabsf(v0), fabsf(v1), 0.70710678118654752f, 0.70710678118654752f);
+  float d0, d1, t0, t1;
+  fma_x2(d0, d1, 0.3275911f, 0.3275911f, x0, x1, 1.f, 1.f);
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t0) : "f"(d0));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t1) : "f"(d1));
+  float p0, p1;
+  fma_x2(p0, p1, 1.061405429f, 1.061405429f, t0, t1, -1.453152027f, -1.453152027f);
+  fma_x2(p0, p1, p0, p1, t0, t1, 1.421413741f, 1.421413741f);
+  fma_x2(p0, p1, p0, p1, t0, t1, -0.284496736f, -0.284496736f);
+  fma_x2(p0, p1, p0, p1, t0, t1, 0.254829592f, 0.254829592f);
+  mul_x2(p0, p1, p0, p1, t0, t1);
+  float q0, q1, e0, e1;
+  mul_x2(q0, q1, x0, x1, x0, x1);
+  mul_x2(q0, q1, q0, q1, -1.4426950408889634f, -1.4426950408889634f);
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e0) : "f"(q0));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e1) : "f"(q1));
+  float a0, a1;  // erf(|x|)
+  fma_x2(a0, a1, -p0, -p1, e0, e1, 1.f, 1.f);
+  a0 = copysignf(a0, v0);
+  a1 = copysignf(a1, v1);
+  float h0, h1;  // 0.5 v
+  mul_x2(h0, h1, v0, v1, 0.5f, 0.5f);
+  fma_x2(v0, v1, h0, h1, a0, a1, h0, h1);  // 0.5 v (1 + erf) = 0.5 v + 0.5 v erf
 }
 
 __device__ __forceinline__ void store8(bf16* p, const float* v) {
@@ -409,7 +444,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
               }
               if (EPI == PF_EPI_GELU) {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] = gelu_erf(v[j]);
+                for (int j = 0; j < 8; j += 2) gelu_erf2(v[j], v[j + 1]);
               }
               if (a.resid) {
 #pragma unroll
