@@ -454,11 +454,6 @@ __device__ __forceinline__ void prefetch_l2_2d(const CUtensorMap* tm, int c0, in
                : "memory");
 }
 
-template <int A, int B>
-struct RED_OK {
-  static constexpr bool value = A >= B;
-};
-
 // Asynchronous 16-byte global -> shared copy (completion: cp_async_wait).
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(dst)), "l"(src) : "memory");
@@ -484,7 +479,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
   int* clist = srec->clist;
   short* utab = &srec->utab[0][0];
   AttnSched* s_as = reinterpret_cast<AttnSched*>(misc + 2 * sizeof(SchedRec) + 64);  // attention schedule
-  static_assert(RED_OK<C::RED_BYTES, C::CW * MT * 4>::value, "norm sums area");
+  static_assert(C::RED_BYTES >= C::CW * MT * 4, "norm sums area");
   static_assert(2 * sizeof(SchedRec) + 64 + sizeof(AttnSched) <= C::MISC_BYTES, "misc shared area");
   uint64_t* full = reinterpret_cast<uint64_t*>(misc + C::MISC_BYTES);
   uint64_t* empty = full + C::NSLOT;
@@ -1438,8 +1433,6 @@ long long sched_offset(long long factor_bytes) { return (factor_bytes + 127) / 1
 // Whether every CTA's share of every GEMV stage stays within the kernel's
 // fixed per-CTA limits (tiles touched, input chunks, contributor table).
 bool stages_fit(const DfPhase* P, int G, int MT, int D) {
-  const int CW = 16;
-  const int red_bytes = std::max(CW * MT * 64 * 4, 2048);
   for (int i = 0; i < DF_NPHASE; ++i) {
     const DfPhase& ph = P[i];
     if (ph.type != DF_GEMV) continue;
@@ -1467,7 +1460,6 @@ bool stages_fit(const DfPhase* P, int G, int MT, int D) {
       else if (ph.src == SRC_SWIGLU) units = n * 8;
       else if (ph.src == SRC_ATT) units = n * MT * (DF_KC / D);
       if (units > DF_MAX_UNITS) return false;
-      if (ph.src == SRC_ATT && units * DF_CMAX * 4 > red_bytes) return false;
     }
   }
   return true;
