@@ -122,11 +122,13 @@ FLASHSVD_API int flashsvd_profile_report(char* buf, int buflen, int reset);
  * rank-r intermediate is reduced on the fly, never materialised as a
  * full-size activation); [v1.5] Problem Statement (prefill and decode have
  * different bottlenecks, so each phase has its own kernel).
- *   M <= 32 (decode): split-K GEMV over U, then over V; the intermediate
- *     z = x.U [M x r] stays fp32 in a small L2-resident workspace.
- *   M > 32 (prefill): tcgen05 tensor-core kernel; each 128-row tile of z is
- *     computed into tensor memory, rounded to bf16 into shared memory and
- *     multiplied by V on chip; z never reaches global memory.
+ *   M <= 32 (decode): split-K GEMV over U, then over V (rows in groups of
+ *     8, one launch per stage); the intermediate z = x.U [M x r] stays fp32
+ *     in a small L2-resident workspace.
+ *   M > 32 (prefill): two tcgen05 tensor-core launches; z is rounded to
+ *     bf16 into a library scratch that stays in L2 between them, and the
+ *     second launch discards each 128-row block of z from L2 once every
+ *     column tile has read it, so z is never written back to HBM.
  * Sizes: 1 <= M <= max_tokens; d, r, n multiples of 8 (prefill: d, r
  * multiples of 64 as well); r <= max_rank.
  */
