@@ -202,15 +202,30 @@ __host__ __device__ __forceinline__ bool share_nonempty(int C, int G, int g) {
   return (g + 1) * C / G > g * C / G;
 }
 
-// Attention entry layout: for each batch row b, H heads x nk_b chunks of 64
-// keys (nk_b from the current length L_b = position + 1).
+// Attention entry layout: for each batch row b, H heads x ne_b entries of
+// 64 keys, ne_b = max(nk_b, m) with nk_b the chunks of the current length
+// L_b = position + 1; entries past nk_b are empty (nothing loaded or
+// computed).  The entries are split evenly over the first Ga CTAs.  Two
+// per-CTA limits follow from the choice of Ga and m, whatever the lengths:
+//  - a pair's entries (at most Ctot / H of them) span at most
+//    ceil(Ga / H) + 1 <= DF_CMAX CTAs, as Ga <= (DF_CMAX - 1) H;
+//  - a share of S <= ceil(Ctot / Ga) entries meets at most
+//    1 + ceil((S - 1) / m) pairs, as every pair has m entries or more; with
+//    Ctot <= raw + B H m and m >= raw / ((DF_MAX_PAIRS - 1) Ga - B H) that
+//    is at most DF_MAX_PAIRS (the host checks (DF_MAX_PAIRS - 1) Ga > B H).
+// With equal lengths m <= nk_b, so nothing is padded.
 struct AttnSched {
   int nk[8];
+  int ne[8];
   int pre[9];
   int L[8];
+  int Ga;
 };
-__device__ __forceinline__ void attn_sched(const DfParams& p, AttnSched& s) {
-  s.pre[0] = 0;
+__host__ __device__ __forceinline__ int attn_ctas(int G, int H) {
+  return G < (DF_CMAX - 1) * H ? G : (DF_CMAX - 1) * H;
+}
+__device__ __forceinline__ void attn_sched(const DfParams& p, int G, AttnSched& s) {
+  int raw = 0;
   for (int b = 0; b < 8; ++b) {
     if (b < p.B) {
       int pos = p.seqlens[b];
@@ -221,15 +236,32 @@ __device__ __forceinline__ void attn_sched(const DfParams& p, AttnSched& s) {
       s.L[b] = 0;
       s.nk[b] = 0;
     }
-    s.pre[b + 1] = s.pre[b] + p.H * s.nk[b];
+    raw += p.H * s.nk[b];
+  }
+  s.Ga = attn_ctas(G, p.H);
+  const int den = (DF_MAX_PAIRS - 1) * s.Ga - p.B * p.H;
+  const int m = den > 0 ? max(1, (raw + den - 1) / den) : 1;
+  s.pre[0] = 0;
+  for (int b = 0; b < 8; ++b) {
+    s.ne[b] = b < p.B ? max(s.nk[b], m) : 0;
+    s.pre[b + 1] = s.pre[b] + p.H * s.ne[b];
   }
 }
 __device__ __forceinline__ void attn_entry(const AttnSched& s, int c, int& b, int& h, int& kc) {
   b = 0;
   while (b < 7 && c >= s.pre[b + 1]) ++b;
   const int r = c - s.pre[b];
-  h = r / s.nk[b];
-  kc = r - h * s.nk[b];
+  h = r / s.ne[b];
+  kc = r - h * s.ne[b];
+}
+// This CTA's attention entries [c0, c1) (empty past the first Ga CTAs).
+__device__ __forceinline__ void attn_share(const AttnSched& s, int g, int& c0, int& c1) {
+  if (g < s.Ga) {
+    c0 = (int)((long long)g * s.pre[8] / s.Ga);
+    c1 = (int)((long long)(g + 1) * s.pre[8] / s.Ga);
+  } else {
+    c0 = c1 = 0;
+  }
 }
 
 // Contributors of a tile (or attention pair) are the CTAs whose shares hold
@@ -252,11 +284,12 @@ __host__ __device__ __forceinline__ bool tile_slots(const DfPhase& q, int t, int
   return ok;
 }
 
-// Attention pair (b, h).
-__device__ __forceinline__ bool pair_slots(const AttnSched& s, int H, int G, int b, int h, short* u) {
-  const int Ctot = s.pre[8];
-  const int e0 = s.pre[b] + h * s.nk[b];
-  const int gf = owner_of(e0, Ctot, G), gl = owner_of(e0 + s.nk[b] - 1, Ctot, G);
+// Attention pair (b, h): every CTA whose share meets the pair's entries
+// (empty ones included) writes one partial of it.
+__device__ __forceinline__ bool pair_slots(const AttnSched& s, int H, int b, int h, short* u) {
+  const int Ctot = s.pre[8], G = s.Ga;
+  const int e0 = s.pre[b] + h * s.ne[b];
+  const int gf = owner_of(e0, Ctot, G), gl = owner_of(e0 + s.ne[b] - 1, Ctot, G);
   int n = 0;
   bool ok = true;
   for (int gg = gf; gg <= gl; ++gg) {
@@ -555,14 +588,15 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
             if (!waited) {
               pdl_wait();
               waited = true;
-              attn_sched(p, s);
-              share(s.pre[8], G, g, a0, a1);
+              attn_sched(p, G, s);
+              attn_share(s, g, a0, a1);
             }
             tc::tma_prefetch_desc(&Ly->kmap);
             tc::tma_prefetch_desc(&Ly->vmap);
             for (int c = a0; c < a1; ++c) {
               int b, h, kc;
               attn_entry(s, c, b, h, kc);
+              if (kc >= s.nk[b]) continue;  // padding
               for (int bx = 0; bx < NB; ++bx) {
                 prefetch_l2_2d(&Ly->kmap, h * p.D + 64 * bx, b * p.S_max + kc * 64);
                 prefetch_l2_2d(&Ly->vmap, h * p.D + 64 * bx, b * p.S_max + kc * 64);
@@ -572,13 +606,15 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
           if (ph.type == DF_ATTN) {
             // K/V chunks of the dense cache (rows before the current position
             // are fixed for this step; the current row is taken from q/k/v)
-            for (int c = a0; c < a1; ++c, ++seq) {
-              const int slot = seq % C::NSLOT;
-              const uint32_t par = (uint32_t)(seq / C::NSLOT) & 1u;
-              if (!tc::mbar_wait_sleep(empty + slot, par ^ 1u, abort_flag, p.status)) { ok = false; break; }
-              uint8_t* base = slots + slot * C::SLOT;
+            for (int c = a0; c < a1; ++c) {
               int b, h, kc;
               attn_entry(s, c, b, h, kc);
+              if (kc >= s.nk[b]) continue;  // padding: no ring entry
+              const int slot = seq % C::NSLOT;
+              const uint32_t par = (uint32_t)(seq / C::NSLOT) & 1u;
+              ++seq;
+              if (!tc::mbar_wait_sleep(empty + slot, par ^ 1u, abort_flag, p.status)) { ok = false; break; }
+              uint8_t* base = slots + slot * C::SLOT;
               tc::mbar_expect_tx(full + slot, (uint32_t)(2 * NB * 8192));
               const int row = b * p.S_max + kc * 64;
               for (int bx = 0; bx < NB; ++bx) {
@@ -611,7 +647,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
   } else {
     // ================================================= consumers ==========
     pdl_wait();
-    if (tid == 0) attn_sched(p, *s_as);  // lengths are fixed for the launch
+    if (tid == 0) attn_sched(p, G, *s_as);  // lengths are fixed for the launch
     // Consumer warp w owns columns 4 w .. 4 w + 3 of every ring entry (box
     // w / 8) over all of the entry's rows: a tile's column sums need no
     // exchange between warps.
@@ -712,7 +748,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
             u[0] = 0;
             const int j = ui % hpc, r2 = ui / hpc, m = r2 % MT, ci = r2 / MT;
             const int hh = (clist[ci] & 255) * DF_KC / p.D + j;
-            if (m < p.B && hh < p.H && !pair_slots(s, p.H, G, m, hh, u)) atomicExch(p.status, DEV_STATUS_SCHEDULE);
+            if (m < p.B && hh < p.H && !pair_slots(s, p.H, m, hh, u)) atomicExch(p.status, DEV_STATUS_SCHEDULE);
           }
         }
         float ssq[MT];  // RMSNorm: sum of squares of this thread's input values
@@ -955,7 +991,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
         const AttnSched& s = *s_as;
         const int Ctot = s.pre[8];
         int c0, c1;
-        share(Ctot, G, g, c0, c1);
+        attn_share(s, g, c0, c1);
         const int D = p.D, hd = D >> 1, tph = D >> 6;
         int pf = 0, np = 0;
         if (c0 < c1) {
@@ -1006,7 +1042,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
             hi = round4(hi);
             *reinterpret_cast<float4*>(qkv + (pr * 3 + prob) * D + i) = lo;
             *reinterpret_cast<float4*>(qkv + (pr * 3 + prob) * D + i + hd) = hi;
-            if (prob > 0 && owner_of(s.pre[b] + h * s.nk[b] + s.nk[b] - 1, Ctot, G) == g) {
+            if (prob > 0 && owner_of(s.pre[b] + h * s.ne[b] + s.nk[b] - 1, Ctot, s.Ga) == g) {
               bf16* dst = *reinterpret_cast<bf16* const*>(
                               s_lyb + (prob == 1 ? offsetof(DfLayer, k_cache) : offsetof(DfLayer, v_cache)) -
                               offsetof(DfLayer, pack)) + ((long long)b * p.S_max + pos) * (p.H * D) +
@@ -1041,15 +1077,12 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
         for (int e = 0; e < CPL_MAX * 8; ++e) { qv[e] = 0.f; ov[e] = 0.f; }
         float m_w = -INFINITY, l_g = 0.f;
         int su = 0;
-        for (int c = c0; c < c1; ++c, ++seq) {
+        for (int c = c0; c < c1; ++c) {
           int b, h, kc;
           attn_entry(s, c, b, h, kc);
           int pr = b * p.H + h - pf;
           pr = pr < np ? pr : np - 1;  // only past the schedule limit (flagged above)
-          const int pair_last = s.pre[b] + h * s.nk[b] + s.nk[b] - 1;
-          const int slot = seq % C::NSLOT;
-          const uint32_t par = (uint32_t)(seq / C::NSLOT) & 1u;
-          tc::mbar_wait(full + slot, par, abort_flag, p.status);  // on abort: run on, results discarded
+          const int pair_last = s.pre[b] + h * s.ne[b] + s.ne[b] - 1;
           const float* qn = qkv + pr * 3 * D;
           if (c == c0 || kc == 0) {
             m_w = -INFINITY;
@@ -1062,74 +1095,80 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
                 qv[cc * 8 + e] = cc < cpl ? qn[(sl * cpl + cc) * 8 + e] * p.scale_log2 : 0.f;
               }
           }
-          const int L = s.L[b], pos = L - 1;
-          const int key = kc * 64 + key_l;
-          const uint8_t* kb = slots + slot * C::SLOT;
-          const uint8_t* vb = kb + 16384;
-          // two partial dots (even / odd dims) keep the FMA chains short
-          float dot = 0.f, dot1 = 0.f;
-          if (key == pos) {
+          if (kc < s.nk[b]) {  // padding entries hold no keys
+            const int slot = seq % C::NSLOT;
+            const uint32_t par = (uint32_t)(seq / C::NSLOT) & 1u;
+            ++seq;
+            tc::mbar_wait(full + slot, par, abort_flag, p.status);  // on abort: run on, results discarded
+            const int L = s.L[b], pos = L - 1;
+            const int key = kc * 64 + key_l;
+            const uint8_t* kb = slots + slot * C::SLOT;
+            const uint8_t* vb = kb + 16384;
+            // two partial dots (even / odd dims) keep the FMA chains short
+            float dot = 0.f, dot1 = 0.f;
+            if (key == pos) {
 #pragma unroll
-            for (int cc = 0; cc < CPL_MAX; ++cc)
-              if (cc < cpl)
+              for (int cc = 0; cc < CPL_MAX; ++cc)
+                if (cc < cpl)
 #pragma unroll
-                for (int e = 0; e < 8; ++e) dot = fmaf(qv[cc * 8 + e], qn[D + (sl * cpl + cc) * 8 + e], dot);
-          } else {
+                  for (int e = 0; e < 8; ++e) dot = fmaf(qv[cc * 8 + e], qn[D + (sl * cpl + cc) * 8 + e], dot);
+            } else {
 #pragma unroll
-            for (int cc = 0; cc < CPL_MAX; ++cc)
-              if (cc < cpl) {
-                const int gc = sl * cpl + cc;
-                const uint4 u = *reinterpret_cast<const uint4*>(kb + (gc >> 3) * 8192 + key_l * 128 +
-                                                                (((gc & 7) ^ (key_l & 7)) << 4));
-                const float kv[8] = {bf_lo(u.x), bf_hi(u.x), bf_lo(u.y), bf_hi(u.y),
-                                     bf_lo(u.z), bf_hi(u.z), bf_lo(u.w), bf_hi(u.w)};
+              for (int cc = 0; cc < CPL_MAX; ++cc)
+                if (cc < cpl) {
+                  const int gc = sl * cpl + cc;
+                  const uint4 u = *reinterpret_cast<const uint4*>(kb + (gc >> 3) * 8192 + key_l * 128 +
+                                                                  (((gc & 7) ^ (key_l & 7)) << 4));
+                  const float kv[8] = {bf_lo(u.x), bf_hi(u.x), bf_lo(u.y), bf_hi(u.y),
+                                       bf_lo(u.z), bf_hi(u.z), bf_lo(u.w), bf_hi(u.w)};
 #pragma unroll
-                for (int e = 0; e < 8; e += 2) {
-                  dot = fmaf(qv[cc * 8 + e], kv[e], dot);
-                  dot1 = fmaf(qv[cc * 8 + e + 1], kv[e + 1], dot1);
+                  for (int e = 0; e < 8; e += 2) {
+                    dot = fmaf(qv[cc * 8 + e], kv[e], dot);
+                    dot1 = fmaf(qv[cc * 8 + e + 1], kv[e + 1], dot1);
+                  }
+                }
+            }
+            dot += dot1;
+#pragma unroll
+            for (int o = LPK / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+            const float sc = key < L ? dot : -INFINITY;
+            float mb = sc;
+#pragma unroll
+            for (int o = LPK; o < 32; o <<= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+            const float mn = fmaxf(m_w, mb);
+            if (mn != -INFINITY) {  // warp-uniform
+              const float corr = m_w == -INFINITY ? 0.f : ex2_approx(m_w - mn);
+              const float pj = sc == -INFINITY ? 0.f : ex2_approx(sc - mn);
+              l_g = l_g * corr + pj;
+#pragma unroll
+              for (int e = 0; e < CPL_MAX * 8; ++e) ov[e] *= corr;
+              if (sc != -INFINITY) {
+                if (key == pos) {
+#pragma unroll
+                  for (int cc = 0; cc < CPL_MAX; ++cc)
+                    if (cc < cpl)
+#pragma unroll
+                      for (int e = 0; e < 8; ++e)
+                        ov[cc * 8 + e] = fmaf(pj, qn[2 * D + (sl * cpl + cc) * 8 + e], ov[cc * 8 + e]);
+                } else {
+#pragma unroll
+                  for (int cc = 0; cc < CPL_MAX; ++cc)
+                    if (cc < cpl) {
+                      const int gc = sl * cpl + cc;
+                      const uint4 u = *reinterpret_cast<const uint4*>(vb + (gc >> 3) * 8192 + key_l * 128 +
+                                                                      (((gc & 7) ^ (key_l & 7)) << 4));
+                      const float vv[8] = {bf_lo(u.x), bf_hi(u.x), bf_lo(u.y), bf_hi(u.y),
+                                           bf_lo(u.z), bf_hi(u.z), bf_lo(u.w), bf_hi(u.w)};
+#pragma unroll
+                      for (int e = 0; e < 8; ++e) ov[cc * 8 + e] = fmaf(pj, vv[e], ov[cc * 8 + e]);
+                    }
                 }
               }
-          }
-          dot += dot1;
-#pragma unroll
-          for (int o = LPK / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-          const float sc = key < L ? dot : -INFINITY;
-          float mb = sc;
-#pragma unroll
-          for (int o = LPK; o < 32; o <<= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
-          const float mn = fmaxf(m_w, mb);
-          if (mn != -INFINITY) {  // warp-uniform
-            const float corr = m_w == -INFINITY ? 0.f : ex2_approx(m_w - mn);
-            const float pj = sc == -INFINITY ? 0.f : ex2_approx(sc - mn);
-            l_g = l_g * corr + pj;
-#pragma unroll
-            for (int e = 0; e < CPL_MAX * 8; ++e) ov[e] *= corr;
-            if (sc != -INFINITY) {
-              if (key == pos) {
-#pragma unroll
-                for (int cc = 0; cc < CPL_MAX; ++cc)
-                  if (cc < cpl)
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                      ov[cc * 8 + e] = fmaf(pj, qn[2 * D + (sl * cpl + cc) * 8 + e], ov[cc * 8 + e]);
-              } else {
-#pragma unroll
-                for (int cc = 0; cc < CPL_MAX; ++cc)
-                  if (cc < cpl) {
-                    const int gc = sl * cpl + cc;
-                    const uint4 u = *reinterpret_cast<const uint4*>(vb + (gc >> 3) * 8192 + key_l * 128 +
-                                                                    (((gc & 7) ^ (key_l & 7)) << 4));
-                    const float vv[8] = {bf_lo(u.x), bf_hi(u.x), bf_lo(u.y), bf_hi(u.y),
-                                         bf_lo(u.z), bf_hi(u.z), bf_lo(u.w), bf_hi(u.w)};
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) ov[cc * 8 + e] = fmaf(pj, vv[e], ov[cc * 8 + e]);
-                  }
-              }
+              m_w = mn;
             }
-            m_w = mn;
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(empty + slot);
           }
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(empty + slot);
 
           if (c != c1 - 1 && c != pair_last) continue;
           // ---- merge the lane groups, then the warps; write this CTA's
@@ -1512,8 +1551,9 @@ int fill_layer(const DecodeLayerDesc& L, bf16* kc, bf16* vc, int B, int S_max, i
                long long* algo_bytes) {
   if (!L.pack || !kc || !vc) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   if (!decode_fused_supported(B, L.d, L.D, L.r, L.r_f) || L.f % 8) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
-  // Attention: with equal lengths a CTA's share spans at most this many pairs.
-  if ((B * L.H + G - 1) / G + 1 > DF_MAX_PAIRS) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  // Attention: the schedule keeps each CTA within DF_MAX_PAIRS pairs for
+  // any lengths when this holds (see AttnSched).
+  if ((DF_MAX_PAIRS - 1) * attn_ctas(G, L.H) <= B * L.H) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   memset(out, 0, sizeof(DfLayer));
   const long long pack_bytes = build_stages(L, out->ph, nullptr);
   if (!stages_fit(out->ph, G, B <= 1 ? 1 : (B <= 2 ? 2 : 4), L.D)) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;

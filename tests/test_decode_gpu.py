@@ -311,6 +311,52 @@ def test_decoder_layer_decode_7b_shape(fs, B):
     fs.set_decode_path(True)
 
 
+RAGGED_CASES = [
+    # (d, H, D, f, r, positions of the batch rows)
+    (256, 4, 64, 688, 64, [3999]),                 # few heads, long context
+    (256, 4, 64, 688, 64, [0, 3999, 76]),          # an empty history among long rows
+    (256, 4, 64, 688, 64, [7999, 0, 5, 0]),        # short rows beside a long one
+    (2048, 32, 64, 1376, 128, [2999, 0, 0, 0]),    # 32 heads, three one-key rows
+    (2048, 16, 128, 1376, 128, [16383]),           # the longest context, 16384 keys
+]
+
+
+@pytest.mark.parametrize("fused", [True, False])
+@pytest.mark.parametrize("case", RAGGED_CASES, ids=lambda c: f"H{c[1]}D{c[2]}pos{'-'.join(map(str, c[5]))}")
+def test_decoder_layer_decode_ragged_lengths(fs, case, fused):
+    """One decode step of a layer whose batch rows sit at very different
+    positions (long contexts, an empty history, few heads), fused and
+    per-stage paths, against the oracle: the layer output and the k, v rows
+    appended at each row's position."""
+    d, H, D, f, r, pos = case
+    B, S_max = len(pos), max(pos) + 1
+    rng = synth.rng_for(12 + B * 131 + S_max)
+    w = synth.decoder_layer_weights(rng, d, f, r, r, gain_jitter=0.1)
+    cos_t = torch.empty((S_max, D // 2), dtype=torch.float32, device="cuda")
+    sin_t = torch.empty_like(cos_t)
+    fs.rope_table(cos_t, sin_t, S_max, D, 10000.0)
+    L, dev = _layer_struct(fs, w, d, H, D, f, r, r, cos_t, sin_t)
+    kc0 = synth.normal_bf16(rng, (B, S_max, H, D))
+    vc0 = synth.normal_bf16(rng, (B, S_max, H, D))
+    xt = synth.normal_bf16(rng, (B, d))
+    y, kn, vn = oracle.decoder_layer_decode(oracle.from_bf16(xt), oracle.widen_layer(w), H,
+                                            oracle.from_bf16(kc0), oracle.from_bf16(vc0), pos)
+    fs.set_decode_path(fused)
+    try:
+        kc, vc = dev_bf16(kc0), dev_bf16(vc0)
+        seq = torch.tensor(pos, dtype=torch.int32, device="cuda")
+        x = dev_bf16(xt)
+        fs.layer_forward(L, x, kc, vc, seq, B, 1, S_max, fs.DECODE)
+        torch.cuda.synchronize()
+        fs.check_device_status()
+    finally:
+        fs.set_decode_path(True)
+    assert_parity(host_f64(x), y, f"ragged decode fused={fused}")
+    for b in range(B):
+        assert_parity(host_f64(kc[b, pos[b]]), kn[b], f"appended k row {b} fused={fused}")
+        assert_parity(host_f64(vc[b, pos[b]]), vn[b], f"appended v row {b} fused={fused}")
+
+
 def test_decode_graph_replay_bitwise(fs):
     d, H, D, f, r, P, B = 256, 4, 64, 688, 64, 100, 2
     S_max = P + 8
