@@ -41,11 +41,13 @@ def parse():
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["decode7b", "linear-sweep", "bert", "mixed-rank"],
+    ap.add_argument("--workload", choices=["decode7b", "linear-sweep", "bert", "mixed-rank",
+                                           "long-decode"],
                     default="decode7b",
                     help="decode7b (default): the headline line; the others print one JSON "
                          "line per measured case of the isolated-linear sweep, the BERT-shaped "
-                         "encoder and the mixed-rank model (1 GPU)")
+                         "encoder, the mixed-rank model and decode over long histories "
+                         "(1 GPU)")
     ap.add_argument("--layers", type=int, default=32,
                     help="decoder layers (default 32; fewer only for small profiling cases)")
     ap.add_argument("--profile-step", action="store_true",
@@ -584,6 +586,69 @@ def run_mixed(args):
     return 0
 
 
+def run_long_decode(args):
+    """Decode over long histories: the 7B-shaped model with every layer's
+    cache filled with a random history (N(0, 1) bf16) and the lengths set
+    directly, at contexts 2048 / 4096 / 8192 / 16320 for B = 1 and B = 4,
+    plus one B = 4 batch of very different lengths; each point times 64
+    graph-replayed steps (embedding, one decode-plan launch of all 32
+    layers, head) after 3 warm-up steps.  Algorithmic bytes per step: every
+    factor, norm gain and the head once, each row's K/V history of every
+    layer once, the new K/V rows and the activations.  The caches
+    (8.6 GB per row at 16384 positions) exceed L2."""
+    import torch
+    sys.path.insert(0, ROOT)
+    from rank_transformer_b200 import flashsvd as fs
+    from rank_transformer_b200.model import LLAMA7B, DecoderModel
+    torch.cuda.set_device(0)
+    cfg, S_max, steps, warm = LLAMA7B, 16384, 64, 3
+    contexts = (2048, 4096, 8192, S_max - steps)
+    fs.init(0, max_tokens=256, max_rank=2368, max_hidden=cfg.d, max_ffn=cfg.f)
+    peaks = measured_peaks()
+    stream = torch.cuda.Stream()
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(31)
+    for B in (1, 4):
+        model = DecoderModel(cfg, B, S_max, seed=41 + B)
+        with torch.cuda.stream(stream):
+            for kc, vc in zip(model.k_cache, model.v_cache):
+                kc.normal_(generator=gen)
+                vc.normal_(generator=gen)
+            model.tokens.copy_(torch.randint(0, cfg.vocab, (B,), generator=gen, device="cuda",
+                                             dtype=torch.int32))
+        model.capture(stream)
+        points = [[c] * B for c in contexts]
+        if B == 4:
+            points.append([S_max - steps, 4096, 1024, 64])
+        for lens in points:
+            start = torch.tensor(lens, dtype=torch.int32, device="cuda")
+            with torch.cuda.stream(stream):
+                model.seqlens.copy_(start)
+                for _ in range(warm):
+                    model.decode_step(stream)
+                model.seqlens.copy_(start)
+                ms = _event_ms(lambda i: model.decode_step(stream), steps, stream)
+            fs.check_device_status(stream)
+            # mean history per step: the lengths grow by one each step
+            hist = sum(c + (steps - 1) / 2 + 1 for c in lens)
+            kv = 2 * cfg.layers * hist * cfg.d * 2
+            act = B * cfg.d * 2 * 2 * cfg.layers
+            byts = model.weight_bytes() + kv + act
+            gbs = byts / (ms / 1e3) / 1e9
+            print(json.dumps({
+                "workload": "long-decode", "batch": B, "context": lens,
+                "decode_steps": steps, "tok_s": round(B / (ms / 1e3), 1),
+                "ms_per_step": round(ms, 3), "bytes_per_step": int(byts),
+                "achieved_gbs": round(gbs, 1), "peak_gbs": peaks["hbm_gbs"],
+                "frac": round(gbs / peaks["hbm_gbs"], 3),
+                "decode_path": "decode plan" if model.plan is not None else "per-stage",
+                "data": "synthetic (random weights and histories)"}), flush=True)
+        model.release_graphs()
+        del model
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -594,6 +659,8 @@ def main():
         return run_bert(args)
     if args.workload == "mixed-rank":
         return run_mixed(args)
+    if args.workload == "long-decode":
+        return run_long_decode(args)
     return run_ours(args)
 
 

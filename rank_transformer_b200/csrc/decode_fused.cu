@@ -212,7 +212,8 @@ __host__ __device__ __forceinline__ bool share_nonempty(int C, int G, int g) {
 //  - a share of S <= ceil(Ctot / Ga) entries meets at most
 //    1 + ceil((S - 1) / m) pairs, as every pair has m entries or more; with
 //    Ctot <= raw + B H m and m >= raw / ((DF_MAX_PAIRS - 1) Ga - B H) that
-//    is at most DF_MAX_PAIRS (the host checks (DF_MAX_PAIRS - 1) Ga > B H).
+//    is at most DF_MAX_PAIRS.  The host checks (DF_MAX_PAIRS - 1) Ga >= 2 B H,
+//    so m <= max nk_b and Ctot <= B H max nk_b, and keeps Ctot Ga < 2^31.
 // With equal lengths m <= nk_b, so nothing is padded.
 struct AttnSched {
   int nk[8];
@@ -254,11 +255,11 @@ __device__ __forceinline__ void attn_entry(const AttnSched& s, int c, int& b, in
   h = r / s.ne[b];
   kc = r - h * s.ne[b];
 }
-// This CTA's attention entries [c0, c1) (empty past the first Ga CTAs).
+// This CTA's attention entries [c0, c1) (empty past the first Ga CTAs;
+// 32-bit: the host keeps entries x Ga below 2^31).
 __device__ __forceinline__ void attn_share(const AttnSched& s, int g, int& c0, int& c1) {
   if (g < s.Ga) {
-    c0 = (int)((long long)g * s.pre[8] / s.Ga);
-    c1 = (int)((long long)(g + 1) * s.pre[8] / s.Ga);
+    share(s.pre[8], s.Ga, g, c0, c1);
   } else {
     c0 = c1 = 0;
   }
@@ -1552,8 +1553,10 @@ int fill_layer(const DecodeLayerDesc& L, bf16* kc, bf16* vc, int B, int S_max, i
   if (!L.pack || !kc || !vc) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   if (!decode_fused_supported(B, L.d, L.D, L.r, L.r_f) || L.f % 8) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   // Attention: the schedule keeps each CTA within DF_MAX_PAIRS pairs for
-  // any lengths when this holds (see AttnSched).
-  if ((DF_MAX_PAIRS - 1) * attn_ctas(G, L.H) <= B * L.H) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  // any lengths when these hold (see AttnSched).
+  const int Ga = attn_ctas(G, L.H);
+  if ((DF_MAX_PAIRS - 1) * Ga < 2 * B * L.H) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)B * L.H * ((S_max + 63) / 64) * Ga >= (1LL << 31)) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   memset(out, 0, sizeof(DfLayer));
   const long long pack_bytes = build_stages(L, out->ph, nullptr);
   if (!stages_fit(out->ph, G, B <= 1 ? 1 : (B <= 2 ? 2 : 4), L.D)) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
