@@ -337,11 +337,17 @@ FLASHSVD_API int flashsvd_decode_pack(const flashsvd_layer* L, void* dst, size_t
  *   x_inout [B x d]; positions are cache_seqlens[b] (device int32[B]); every
  *   layer appends its new key and value there; cache_seqlens is not
  *   incremented.  Same result as n DECODE-mode flashsvd_layer_forward calls.
+ *   The positions may differ freely across the rows (any mix of lengths up
+ *   to S_max): the attention work, 64-key chunks of every (row, head), is
+ *   split evenly over the CTAs whatever the lengths.
  *   Asynchronous, capturable, uses the context's scratch (one plan runs at a
  *   time per context).
  * Errors: INVALID_ARG, NOT_INITIALIZED, CAPTURE_UNSAFE (create during
  *   capture), UNSUPPORTED_SHAPE (a layer without a pack, B > 4, shapes the
- *   fused kernel does not cover), NO_MEMORY. */
+ *   fused kernel does not cover: among them 7 * min(SMs, 14 H) < 2 B H, or
+ *   B H ceil(S_max / 64) min(SMs, 14 H) >= 2^31), NO_MEMORY.  A DECODE-mode
+ *   flashsvd_layer_forward on a layer the fused kernel does not cover runs
+ *   the per-stage kernels instead. */
 typedef struct flashsvd_decode_plan flashsvd_decode_plan;
 FLASHSVD_API int flashsvd_decode_plan_create(const flashsvd_layer* layers, int n_layers,
                                              flashsvd_bf16* const* k_caches,
