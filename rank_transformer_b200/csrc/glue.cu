@@ -145,9 +145,21 @@ greedy_kernel(const float* logits, int* next, int vocab) {
   const float* row = logits + (long long)blockIdx.x * vocab;
   float bv = -INFINITY;
   int bi = 0x7fffffff;
-  for (int j = threadIdx.x; j < vocab; j += blockDim.x) {
-    const float v = row[j];
-    if (v > bv) { bv = v; bi = j; }  // j increases: ties keep the lower index
+  // GR_UNROLL independent loads in flight per thread (one at a time would
+  // leave the row's read bound by the load latency, ~30 in a row per thread
+  // at a 32000-entry vocabulary)
+  constexpr int GR_UNROLL = 16;
+  const int stride = blockDim.x;
+  for (int j0 = threadIdx.x; j0 < vocab; j0 += stride * GR_UNROLL) {
+    float v[GR_UNROLL];
+#pragma unroll
+    for (int u = 0; u < GR_UNROLL; ++u) {
+      const int j = j0 + u * stride;
+      v[u] = j < vocab ? __ldg(row + j) : -INFINITY;
+    }
+#pragma unroll
+    for (int u = 0; u < GR_UNROLL; ++u)
+      if (v[u] > bv) { bv = v[u]; bi = j0 + u * stride; }  // j increases: ties keep the lower index
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {

@@ -162,6 +162,26 @@ def test_glue_kernels(fs):
     assert list(sl.cpu().numpy()) == [6, 8]
 
 
+@pytest.mark.parametrize("vocab", [32000, 32003, 70001])
+def test_greedy_large_vocab(fs, vocab):
+    """Greedy pick over vocabularies that give every thread many entries:
+    the maximum in the last entry, a tie between entries far apart (lowest
+    index wins), a row of equal values, the maximum in the first entry, and
+    a plain random row; against the oracle's argmax."""
+    rng = synth.rng_for(4100 + vocab)
+    logits = rng.standard_normal((5, vocab)).astype(np.float32)
+    logits[0, vocab - 1] = 40.0
+    logits[1, 7] = logits[1, vocab // 2 + 3] = logits[1, vocab - 2] = 40.0
+    logits[2, :] = 1.5
+    logits[3, 0] = 40.0
+    nxt = torch.empty(5, dtype=torch.int32, device="cuda")
+    fs.greedy(torch.from_numpy(logits).cuda(), nxt, 5, vocab)
+    torch.cuda.synchronize()
+    got = list(nxt.cpu().numpy())
+    assert got == list(oracle.greedy(logits))
+    assert got[:4] == [vocab - 1, 7, 0, 0]
+
+
 def _layer_struct(fs, w, d, H, D, f, r, r_f, cos_t, sin_t, pack=True):
     """Layer descriptor over device copies of w; with pack, also the decode
     pack that the fused decode kernel streams (kept alive in dev)."""
