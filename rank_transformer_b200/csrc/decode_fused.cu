@@ -70,6 +70,33 @@ constexpr int DF_MAX_NK = 64;         // 256-row chunks per factor (K <= 16384)
 constexpr int DF_CMAX = 15;           // contributing CTAs per tile (or pair) read
 constexpr int DF_MAX_UNITS = 96;      // tiles (or pairs) read per stage and CTA
 
+#ifdef FLASHSVD_TRACE
+// Stage timeline (trace builds only; the product build compiles none of
+// it): per (layer, stage, CTA) of the last launch, four points -- stage
+// entry, previous stage complete on every CTA (grid barrier passed), stage
+// input built, stage done (before the release) -- each as %globaltimer ns
+// (comparable across SMs) and clock64 cycles (exact within a CTA).
+constexpr int DF_TRACE_LAYERS = 64;
+constexpr int DF_TRACE_CTAS = 148;
+__device__ unsigned long long g_df_trace[DF_TRACE_LAYERS][9][DF_TRACE_CTAS][2][4];
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+#define DF_TRACE(l, ph, k)                                                     \
+  do {                                                                         \
+    if (tid == 0 && (l) < DF_TRACE_LAYERS && g < DF_TRACE_CTAS) {              \
+      g_df_trace[l][ph][g][0][k] = global_ns();                                \
+      g_df_trace[l][ph][g][1][k] = (unsigned long long)clock64();              \
+    }                                                                          \
+  } while (0)
+#else
+#define DF_TRACE(l, ph, k) \
+  do {                     \
+  } while (0)
+#endif
+
 enum { DF_GEMV = 0, DF_ATTN = 1 };
 // How a stage's input is built from what the previous stage left.
 // SRC_XOUT (stage 0 of every layer after the first): the previous layer's
@@ -713,6 +740,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
       // (accumulated over the layers) reaches prev_target
       const int prev_ctr = ph_i > 0 ? ph_i - 1 : DF_NPHASE - 1;
       const int prev_target = G * (ph_i > 0 ? l + 1 : l);
+      DF_TRACE(l, ph_i, 0);
       if (ph.type == DF_GEMV) {
         const int src = (ph_i == 0 && l > 0) ? SRC_XOUT : ph.src;
         const int Ctot = ph.T * ph.nk;
@@ -780,6 +808,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
         }
         // ---- wait for the previous stage on every CTA ----
         if ((ph_i > 0 || l > 0) && tid == 0) grid_wait(p.bar + prev_ctr, prev_target, abort_flag, p.status);
+        DF_TRACE(l, ph_i, 1);
         consumer_sync<C::CT>();
         // (2) the input itself, 4 consecutive values per group, two groups
         // per thread and step (their loads in flight together)
@@ -931,6 +960,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
           }
         }
 
+        DF_TRACE(l, ph_i, 2);
         next_gemv_stage(l, ph_i, (gidx + 1) & 1);  // its record loads under this stage's entries
         // ---- entries ----
         float acc[MT][4];
@@ -1020,6 +1050,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
               atomicExch(p.status, DEV_STATUS_SCHEDULE);
           }
           if (tid == 0) grid_wait(p.bar + prev_ctr, prev_target, abort_flag, p.status);
+          DF_TRACE(l, ph_i, 1);
           consumer_sync<C::CT>();
           for (int e = tid; e < np * 3 * (hd >> 2); e += C::CT) {
             const int i = (e % (hd >> 2)) * 4;
@@ -1057,6 +1088,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
           }
         }
         consumer_sync<C::CT>();
+        DF_TRACE(l, ph_i, 2);
 
         // Each consumer warp owns KPW = 64 / CW keys of every 64-key entry;
         // LPK = 32 / KPW lanes share a key, each holding cpl 16-byte chunks
@@ -1212,6 +1244,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
       // ---- this CTA is done with stage ph_i ----
       if (ph.type == DF_GEMV) ++gidx;
       consumer_sync<C::CT>();
+      DF_TRACE(l, ph_i, 3);
       // (the CTA barrier above orders every consumer's writes before this
       // thread's release, which is cumulative over them)
       if (tid == 0) red_release_add(p.bar + ph_i, 1);
@@ -1682,3 +1715,19 @@ void decode_plan_destroy(DecodePlan* plan) {
 }
 
 }  // namespace fsvd
+
+#ifdef FLASHSVD_TRACE
+// Trace builds only (not part of the public ABI): the stage timeline of the
+// fused decode kernel's last launches, laid out as
+// u64 [64 layers][9 stages][148 CTAs][2: ns, cycles][4 points].
+extern "C" __attribute__((visibility("default"))) int flashsvd_trace_read(void* host, size_t bytes) {
+  if (!host) return FLASHSVD_ERR_INVALID_ARG;
+  const size_t n = bytes < sizeof(fsvd::g_df_trace) ? bytes : sizeof(fsvd::g_df_trace);
+  return cudaMemcpyFromSymbol(host, fsvd::g_df_trace, n) == cudaSuccess ? FLASHSVD_OK : FLASHSVD_ERR_CUDA;
+}
+extern "C" __attribute__((visibility("default"))) int flashsvd_trace_clear(void) {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, fsvd::g_df_trace) != cudaSuccess) return FLASHSVD_ERR_CUDA;
+  return cudaMemset(p, 0, sizeof(fsvd::g_df_trace)) == cudaSuccess ? FLASHSVD_OK : FLASHSVD_ERR_CUDA;
+}
+#endif

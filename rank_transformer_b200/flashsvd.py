@@ -12,7 +12,9 @@ import ctypes as C
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libflashsvd.so")
+# FLASHSVD_LIBRARY selects another build of the same library (the trace
+# build, libflashsvd_trace.so); by default the in-tree product library.
+LIB_PATH = os.environ.get("FLASHSVD_LIBRARY") or os.path.join(_HERE, "libflashsvd.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(

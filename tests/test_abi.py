@@ -41,6 +41,13 @@ def test_every_declared_symbol_is_exported(fs):
         assert name in fs.EXPORTED, f"{name} not bound in flashsvd.py"
 
 
+def test_product_library_has_no_trace_code(fs):
+    """The stage-timeline hooks exist only in the trace build
+    (libflashsvd_trace.so); the product library exports none of them."""
+    for name in ("flashsvd_trace_read", "flashsvd_trace_clear"):
+        assert not hasattr(fs.lib, name), name
+
+
 def test_status_strings(fs):
     assert fs.lib.flashsvd_status_string(0) == b"ok"
     for s in range(1, 9):
