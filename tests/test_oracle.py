@@ -276,6 +276,132 @@ def pin_head_and_greedy(o):
     _close(logits, o.rmsnorm(emb[toks], np.ones(8)))
 
 
+def _two_token_case(eps=0.0):
+    """Hand-worked two-token, two-head decoder example (d = 4, H = 2, D = 2,
+    every factor the identity, RMSNorm with g = 1, MLP off).
+
+    x0 = [1, 1, 1, 1] and x1 = [sqrt2, 0, 0, sqrt2] both have mean square 1,
+    so n1 = c x with c = 1 / sqrt(1 + eps), and q = k = v = n1.  Head 0 holds
+    dims (0, 1), head 1 dims (2, 3).  RoPE at position 0 is the identity; at
+    position 1 it turns each head's pair by 1 radian.  Token 0 sees only
+    itself: a0 = v0.  Token 1, head 0: q = c sqrt2 [cos 1, sin 1]; its
+    scores (scale 1/sqrt2) to k0 = c [1, 1] and to itself are
+    c^2 (cos 1 + sin 1) and c^2 sqrt2.  Head 1: q = c sqrt2 [-sin 1, cos 1],
+    scores c^2 (cos 1 - sin 1) and c^2 sqrt2.  The values are not rotated.
+    """
+    s2, c1, s1 = math.sqrt(2.0), math.cos(1.0), math.sin(1.0)
+    c = 1.0 / math.sqrt(1.0 + eps)
+    x = np.array([[1.0, 1.0, 1.0, 1.0], [s2, 0.0, 0.0, s2]])
+    I = np.eye(4)
+    w = {n: I for n in ("U_q", "V_q", "U_k", "V_k", "U_v", "V_v", "U_o", "V_o")}
+    w.update(U_gu=np.concatenate([I, I], 1), V_gu=np.concatenate([I, I], 0),
+             U_dn=I, V_dn=np.zeros((4, 4)), g1=np.ones(4), g2=np.ones(4))
+
+    def two_key(a, b):          # softmax weight of the first of two scores
+        return 1.0 / (1.0 + math.exp(b - a))
+    p_h0 = two_key(c * c * (c1 + s1), c * c * s2)
+    p_h1 = two_key(c * c * (c1 - s1), c * c * s2)
+    a1 = c * np.array([p_h0 * 1 + (1 - p_h0) * s2, p_h0 * 1 + (1 - p_h0) * 0,
+                       p_h1 * 1 + (1 - p_h1) * 0, p_h1 * 1 + (1 - p_h1) * s2])
+    y = np.stack([x[0] + c * x[0], x[1] + a1])
+    k_rot = c * np.array([[[1.0, 1.0], [1.0, 1.0]],
+                          [[s2 * c1, s2 * s1], [-s2 * s1, s2 * c1]]])
+    return x, w, y, k_rot
+
+
+def pin_decoder_layer_worked_example(o):
+    # Prefill over both tokens, and decode of token 1 against a cache that
+    # holds only token 0 (written out by hand), give the hand-worked rows.
+    x, w, y, k_rot = _two_token_case()
+    yp, kp, vp = o.decoder_layer_prefill(x, w, 2, eps=0.0)
+    _close(yp, y)
+    _close(kp, k_rot)
+    _close(vp, x.reshape(2, 2, 2))
+    k_hist = np.array([[[[1.0, 1.0], [1.0, 1.0]]]])
+    v_hist = k_hist.copy()
+    yd, kd, vd = o.decoder_layer_decode(x[1:], w, 2, k_hist, v_hist, [1], eps=0.0)
+    _close(yd[0], y[1])
+    _close(kd[0], k_rot[1])
+    _close(vd[0], x[1].reshape(2, 2))
+
+
+def pin_decoder_mlp_branch(o):
+    # Attention branch off (V_o = 0): h = x.  Closed-form MLP factors
+    # U_gu = [I | I], V_gu = [diag(a); I], U_dn = V_dn = I make the branch
+    # SiLU(a * n2) * n2 with n2 = rmsnorm(x) under the SECOND gain g2, which
+    # differs from g1 here; y = x + that.  Prefill and decode alike.
+    rng = _rng(13)
+    d, H = 8, 2
+    I = np.eye(d)
+    a = rng.standard_normal(d)
+    w = _tiny_layer(rng, d=d, H=H, f=d, r=d)
+    w.update(V_o=np.zeros((d, d)), U_gu=np.concatenate([I, I], 1),
+             V_gu=np.concatenate([np.diag(a), I], 0), U_dn=I, V_dn=I,
+             g2=1.0 + 0.5 * rng.standard_normal(d))
+    x = rng.standard_normal((3, d))
+    ms = np.mean(x * x, axis=1, keepdims=True)
+    n2 = x / np.sqrt(ms + o.RMS_EPS) * w["g2"]
+    expect = x + (a * n2) / (1.0 + np.exp(-a * n2)) * n2
+    _close(o.decoder_layer_prefill(x, w, H)[0], expect, 1e-11)
+    D = d // H
+    hist = rng.standard_normal((3, 4, H, D))
+    yd = o.decoder_layer_decode(x, w, H, hist, hist, [4, 2, 0])[0]
+    _close(yd, expect, 1e-11)
+
+
+def pin_bert_layer_closed_form(o):
+    # Query factor and bias zero: every score is 0, so each token averages
+    # the values of ALL tokens (bidirectional).  With U_v = V_v = U_o =
+    # V_o = I:  h = LN1(x + mean_t(x) + b_v + b_o).
+    # FFN with U_up = I, V_up = diag(a), U_dn = V_dn = I:
+    #   y = LN2(h + GELU(a * h + b_up) + b_dn),  GELU(t) = t * Phi(t).
+    rng = _rng(14)
+    S, d, H = 5, 8, 2
+    I = np.eye(d)
+    a = rng.standard_normal(d)
+    w = {"U_q": np.zeros((d, d)), "V_q": I, "b_q": np.zeros(d),
+         "U_k": rng.standard_normal((d, d)), "V_k": I, "b_k": rng.standard_normal(d),
+         "U_v": I, "V_v": I, "b_v": rng.standard_normal(d),
+         "U_o": I, "V_o": I, "b_o": rng.standard_normal(d),
+         "U_up": I, "V_up": np.diag(a), "b_up": rng.standard_normal(d),
+         "U_dn": I, "V_dn": I, "b_dn": rng.standard_normal(d)}
+    for n in ("ln1", "ln2"):
+        w[n + "_g"] = 1.0 + 0.3 * rng.standard_normal(d)
+        w[n + "_b"] = 0.3 * rng.standard_normal(d)
+    x = rng.standard_normal((S, d))
+
+    def ln(t, g, b):
+        mu = t.mean(axis=1, keepdims=True)
+        var = ((t - mu) ** 2).mean(axis=1, keepdims=True)
+        return (t - mu) / np.sqrt(var + o.LN_EPS) * g + b
+    h = ln(x + x.mean(axis=0, keepdims=True) + w["b_v"] + w["b_o"], w["ln1_g"], w["ln1_b"])
+    t = a * h + w["b_up"]
+    y = ln(h + t * norm.cdf(t) + w["b_dn"], w["ln2_g"], w["ln2_b"])
+    _close(o.bert_layer(x, w, H), y, 1e-10)
+
+
+def pin_model_and_head(o):
+    # Output head with a square, non-symmetric W (a transposed W changes the
+    # result): rows of mean square 1, g = 1, eps = 0 give logits = x W.
+    x = np.array([[1.0, -1.0, 1.0, -1.0], [2.0, 0.0, 0.0, 0.0]])
+    W = np.array([[1.0, 2.0, 0.0, 0.0], [0.0, 1.0, 0.0, 5.0],
+                  [3.0, 0.0, 1.0, 0.0], [0.0, 0.0, 7.0, 1.0]])
+    _close(o.lm_head(x, np.ones(4), W, eps=0.0), [[4.0, 1.0, -6.0, -6.0], [2.0, 4.0, 0.0, 0.0]])
+    # One-layer model over the worked two-token example: embedding rows
+    # chosen so emb[tokens] = x; logits = rmsnorm(y) W; the cache holds the
+    # rotated keys and the plain values.
+    eps = o.RMS_EPS
+    xs, w, y, k_rot = _two_token_case(eps)
+    emb = np.zeros((5, 4))
+    emb[3], emb[1] = xs[0], xs[1]
+    logits, cache = o.decoder_model_prefill(np.array([3, 1]), emb, [w], np.ones(4), W, H=2)
+    yn = y / np.sqrt(np.mean(y * y, axis=1, keepdims=True) + eps)
+    _close(logits, yn @ W)
+    assert len(cache) == 1
+    _close(cache[0][0], k_rot)
+    _close(cache[0][1], xs.reshape(2, 2, 2) / math.sqrt(1.0 + eps))
+
+
 def pin_from_bf16(o):
     bits = np.array([0x3F80, 0xBF80, 0x4049, 0x0000, 0x8000, 0x7F7F, 0x0001], np.uint16)
     want = [1.0, -1.0, 3.140625, 0.0, -0.0, 3.3895313892515355e38, 9.183549615799121e-41]
@@ -287,7 +413,8 @@ PINS = [pin_lowrank_worked_example, pin_lowrank_associativity,
         pin_packed_equals_unpacked, pin_packed_mlp_closed_form, pin_rmsnorm,
         pin_layernorm, pin_rope, pin_attention, pin_decode_matches_prefill,
         pin_decoder_layer_special_cases, pin_bert_layer, pin_head_and_greedy,
-        pin_from_bf16]
+        pin_from_bf16, pin_decoder_layer_worked_example, pin_decoder_mlp_branch,
+        pin_bert_layer_closed_form, pin_model_and_head]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -399,11 +526,48 @@ def _mut_bert_causal(m):
     m.attention = lambda q, k, v, causal=False, q_offset=0: orig(q, k, v, True, q_offset)
 
 
+
+def _source_mutant(old, new, name):
+    """A mistake planted by editing the oracle's source text: every
+    occurrence of ``old`` becomes ``new`` and the edited source is executed
+    in the fresh module's namespace."""
+    def mutate(m):
+        src = open(m.__file__).read()
+        assert old in src, f"mutation anchor missing: {old!r}"
+        exec(compile(src.replace(old, new), m.__file__, "exec"), m.__dict__)
+    mutate.__name__ = name
+    return mutate
+
+
+_mut_second_norm_uses_g1 = _source_mutant(
+    'rmsnorm(h_res, w["g2"], eps)', 'rmsnorm(h_res, w["g1"], eps)', "_mut_second_norm_uses_g1")
+_mut_bert_drops_b_up = _source_mutant(
+    'w["V_up"], w["b_up"]', 'w["V_up"], None', "_mut_bert_drops_b_up")
+_mut_rope_on_values = _source_mutant(
+    "    k = np.stack([rope(k[:, h], pos) for h in range(H)], axis=1)\n",
+    "    k = np.stack([rope(k[:, h], pos) for h in range(H)], axis=1)\n"
+    "    v = np.stack([rope(v[:, h], pos) for h in range(H)], axis=1)\n",
+    "_mut_rope_on_values")
+_mut_heads_interleaved = _source_mutant(
+    "return x.reshape(T, H, HD // H)", "return x.reshape(T, HD // H, H).transpose(0, 2, 1)",
+    "_mut_heads_interleaved")
+_mut_decode_position_shift = _source_mutant(
+    "np.full(H, p)", "np.full(H, p + 1)", "_mut_decode_position_shift")
+_mut_head_transposed = _source_mutant(
+    "y = np.asarray(x, np.float64) @ np.asarray(W, np.float64)",
+    "y = np.asarray(x, np.float64) @ np.asarray(W, np.float64).T", "_mut_head_transposed")
+_mut_model_skips_final_norm = _source_mutant(
+    "return dense_linear(rmsnorm(x, g_final, eps), W_lm)", "return dense_linear(x, W_lm)",
+    "_mut_model_skips_final_norm")
+
 MUTANTS = [_mut_rope_sign, _mut_rope_interleaved, _mut_attention_noscale,
            _mut_attention_causal_strict, _mut_swiglu_swapped,
            _mut_rmsnorm_nosquare, _mut_layernorm_unbiased,
            _mut_lowrank_drops_bias, _mut_decode_forgets_current,
-           _mut_gelu_tanh, _mut_silu_sigmoid_only, _mut_bert_causal]
+           _mut_gelu_tanh, _mut_silu_sigmoid_only, _mut_bert_causal,
+           _mut_second_norm_uses_g1, _mut_bert_drops_b_up, _mut_rope_on_values,
+           _mut_heads_interleaved, _mut_decode_position_shift, _mut_head_transposed,
+           _mut_model_skips_final_norm]
 
 
 @pytest.mark.parametrize("mutate", MUTANTS, ids=[f.__name__ for f in MUTANTS])
