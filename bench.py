@@ -354,6 +354,22 @@ def run_ours(args):
         alg_per_launch = tp["bytes"] / tp["launches"]
     achieved = alg_per_launch / (tp["ms"] / tp["launches"] / 1e3) / 1e9
 
+    # Prefill roofline (tensor-core bound): algorithmic FLOPs of the timed
+    # prefills / their time, and the dominant prefill kernel from one eager
+    # prefill with every launch bracketed by CUDA events on its stream.
+    pf_flops = model.prefill_flops(PROMPT)
+    pf_tfs = pf_flops * args.steps / (pre_ms / 1e3) / 1e12
+    fs.profile_enable(True)
+    with torch.cuda.stream(stream):
+        model.prefill(prompt, stream)
+    pprof = fs.profile_report(reset=True)
+    fs.profile_enable(False)
+    pprof = {k: v for k, v in pprof.items() if v["launches"] > 0}
+    ptop = max(pprof, key=lambda k: pprof[k]["ms"])
+    pk = pprof[ptop]
+    pk_tfs = pk["flops"] / (pk["ms"] / 1e3) / 1e12
+    pf_total_ms = sum(v["ms"] for v in pprof.values())
+
     # End to end through the public call: pinned host prompt in, generated
     # tokens out, on the same stream, timed with events around everything.
     prompt_host = torch.empty((B, PROMPT), dtype=torch.int32, pin_memory=True)
@@ -388,7 +404,17 @@ def run_ours(args):
                        "batch": B, "prompt": PROMPT, "decode_steps": DECODE_STEPS,
                        "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (7.75 GB of factors streamed per step)"},
-            "prefill": {"value": prefill_tok_s, "unit": "tok/s", "ms_per_step": pre_ms / args.steps},
+            "prefill": {
+                "value": prefill_tok_s, "unit": "tok/s", "ms_per_step": pre_ms / args.steps,
+                "roofline": {"bound": "tensor", "achieved": pf_tfs, "unit": "TFLOP/s",
+                             "peak": peaks["bf16_tflops"], "frac": pf_tfs / peaks["bf16_tflops"],
+                             "frac_of_sustained": pf_tfs / peaks["bf16_tflops_sustained"],
+                             "flops_per_step": pf_flops,
+                             "peak_source": peaks["source"] + " (dense bf16 GEMM, burst)"},
+                "top_kernel": {"kernel": ptop, "launches": pk["launches"],
+                               "share": pk["ms"] / pf_total_ms, "achieved": pk_tfs,
+                               "unit": "TFLOP/s", "frac": pk_tfs / peaks["bf16_tflops"]},
+                "kernel_times_ms": {k: round(v["ms"], 4) for k, v in sorted(pprof.items())}},
             "decode_hbm": {"achieved_gbs": dec_gbs, "peak_gbs": peaks["hbm_gbs"],
                            "frac": dec_gbs / peaks["hbm_gbs"],
                            "bytes_per_step": step_bytes / DECODE_STEPS},

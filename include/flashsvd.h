@@ -232,8 +232,13 @@ FLASHSVD_API int flashsvd_advance_seqlens(int32_t* cache_seqlens, int B,
  * scratch (rank activations, split partial sums, tile counters) is one fixed
  * array of about 2.2 MiB in device memory that every GPU which loads the
  * library holds until the process exits.
- * Limits: 1 <= M <= 8, r <= 4096, d and n <= 16384 (all multiples of 8) and
- * the split partial sums must fit the array; anything larger returns
+ * Limits: 1 <= M <= 8, r <= 4096, d and n <= 16384 (all multiples of 8),
+ * and the split partial sums of both products must fit the array.  The call
+ * accepts a shape exactly when, for (K, N) = (d, r) and (K, N) = (r, n),
+ *     ceil(K / 512) * ceil(N / 64) * (64 m + 8) <= 524288,
+ * with m = 1, 2, 4, 8 for M = 1, 2, 3..4, 5..8 (on GPUs of up to 336 SMs).
+ * Every shape with d, n <= 8192 and r <= 2048, or with d, n, r <= 4096,
+ * passes at any M <= 8.  Anything else returns
  * FLASHSVD_ERR_UNSUPPORTED_SHAPE and launches nothing.
  * The first call on each device looks up the array's device address with
  * that device current; make that first call before any stream capture.

@@ -407,11 +407,8 @@ template <int D, bool CAUSAL>
 int launch_at(const AttnPfParams& ap, cudaStream_t stream) {
   using L = AtLayout<D>;
   auto kern = attn_prefill_tc_kernel<D, CAUSAL>;
-  static bool configured = false;
-  if (!configured) {
-    FSVD_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM));
-    configured = true;
-  }
+  static SmemAttrOnce smem_once;
+  FSVD_TRY(set_smem_once(smem_once, kern, L::SMEM));
   const long long HD = (long long)ap.H * D;
   CUtensorMap mq, mk, mv;
   FSVD_TRY(encode_map(&mq, ap.q, (long long)ap.B * ap.S, HD, HD, 64, AT_BM, true));
@@ -438,7 +435,7 @@ int launch_at(const AttnPfParams& ap, cudaStream_t stream) {
 
 }  // namespace
 
-int attn_prefill_tc_launch(const AttnPfParams& p, cudaStream_t stream) {
+int attn_prefill_launch(const AttnPfParams& p, cudaStream_t stream) {
   if (!p.status) return FLASHSVD_ERR_NOT_INITIALIZED;
   if (p.D == 128) return p.causal ? launch_at<128, true>(p, stream) : launch_at<128, false>(p, stream);
   if (p.D == 64) return p.causal ? launch_at<64, true>(p, stream) : launch_at<64, false>(p, stream);

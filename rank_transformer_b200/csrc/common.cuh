@@ -77,6 +77,26 @@ inline int launch_pdl(const LaunchTag& tag, void (*kernel)(KArgs...), dim3 grid,
   return FLASHSVD_OK;
 }
 
+// Raise `kernel`'s dynamic shared-memory limit to `bytes` on the current
+// device.  cudaFuncSetAttribute applies to the device that is current when it
+// runs, so the flag is kept per device (a call site keeps one `SmemAttrOnce`
+// per kernel instantiation).  Two threads racing here both set the same
+// value, which is harmless.
+struct SmemAttrOnce {
+  std::atomic<bool> done[64];
+};
+
+template <typename Kern>
+inline int set_smem_once(SmemAttrOnce& once, Kern kernel, int bytes) {
+  int dev = 0;
+  FSVD_CUDA(cudaGetDevice(&dev));
+  const bool tracked = dev >= 0 && dev < 64;
+  if (tracked && once.done[dev].load(std::memory_order_acquire)) return FLASHSVD_OK;
+  FSVD_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  if (tracked) once.done[dev].store(true, std::memory_order_release);
+  return FLASHSVD_OK;
+}
+
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 inline int round_up(int a, int b) { return ceil_div(a, b) * b; }
 inline bool aligned16(const void* p) { return (((uintptr_t)p) & 15u) == 0; }

@@ -1623,11 +1623,8 @@ int launch_df(const DfParams& p, int G, double bytes, cudaStream_t stream) {
 #define FSVD_DF_LAUNCH(MT_)                                                                          \
   {                                                                                                  \
     auto kern = decode_layer_kernel<MT_>;                                                            \
-    static bool configured = false;                                                                  \
-    if (!configured) {                                                                               \
-      FSVD_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, DfCfg<MT_>::SMEM)); \
-      configured = true;                                                                             \
-    }                                                                                                \
+    static SmemAttrOnce smem_once;                                                                   \
+    FSVD_TRY(set_smem_once(smem_once, kern, DfCfg<MT_>::SMEM));                                      \
     return launch_pdl(tag, kern, dim3(G), dim3(DfCfg<MT_>::THREADS), (size_t)DfCfg<MT_>::SMEM, stream, p); \
   }
   if (p.B <= 1) FSVD_DF_LAUNCH(1)

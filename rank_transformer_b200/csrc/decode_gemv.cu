@@ -373,11 +373,8 @@ int launch_one(const GvParams& p, int total_tiles, cudaStream_t stream) {
   const size_t smem = (size_t)(NSEG * MT * p.KC + 8 * MT * 64) * sizeof(float) +
                       (size_t)p.KC * 64 * sizeof(bf16);
   auto kern = gemv_splitk_kernel<MT, PRO, EPI, MAP>;
-  static bool configured = false;  // once per instantiation
-  if (!configured) {
-    FSVD_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
-    configured = true;
-  }
+  static SmemAttrOnce smem_once;  // per instantiation, per device
+  FSVD_TRY(set_smem_once(smem_once, kern, 200 * 1024));
   if (smem > 200 * 1024) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   double flops = 0.0;
   for (int i = 0; i < p.nprob; ++i)

@@ -147,6 +147,5 @@ struct AttnPfParams {
   int* status;       // device status word (bounded waits)
 };
 int attn_prefill_launch(const AttnPfParams& p, cudaStream_t stream);
-int attn_prefill_tc_launch(const AttnPfParams& p, cudaStream_t stream);
 
 }  // namespace fsvd

@@ -519,11 +519,8 @@ int launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& m
               TcArgs a, const char* name, cudaStream_t stream) {
   using L = Layout<BN, STAGES, DUAL>;
   auto kern = tc_gemm_kernel<BN, STAGES, DUAL, EPI>;
-  static bool configured = false;
-  if (!configured) {
-    FSVD_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM));
-    configured = true;
-  }
+  static SmemAttrOnce smem_once;
+  FSVD_TRY(set_smem_once(smem_once, kern, L::SMEM));
   a.tiles_m = ceil_div(a.M, BM);
   if (a.nprob > 1) {
     // grouped: problem i's column tiles start at pt[i]; a.N = total width

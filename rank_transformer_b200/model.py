@@ -45,8 +45,11 @@ class DecoderConfig:
         return r_a, r_f
 
     def layer_params(self, layer: int) -> int:
+        """Factor parameters of one layer: q, k, v, o at rank r_a
+        (r_a * 2d each), the packed gate|up pair U_gu [d x 2 r_f] and V_gu
+        [2 r_f x f], and the down pair U_dn [f x r_f], V_dn [r_f x d]."""
         r_a, r_f = self.ranks(layer)
-        return 4 * r_a * 2 * self.d + r_f * (self.d + 2 * self.f) + r_f * (self.f + self.d)
+        return 4 * r_a * 2 * self.d + 2 * r_f * (self.d + self.f) + r_f * (self.f + self.d)
 
 
 LLAMA7B = DecoderConfig()
@@ -59,7 +62,12 @@ def _bf16_normal(shape, std, gen, device):
 
 class DecoderModel:
     def __init__(self, cfg: DecoderConfig, B: int, S_max: int, seed: int = 0,
-                 device: str = "cuda", weights=None, decode_pack: bool = True):
+                 device: str = "cuda", weights=None, head=None, decode_pack: bool = True):
+        """``weights``: optional list of per-layer dicts of device bf16
+        tensors (U_q, V_q, ..., U_gu, V_gu, U_dn, V_dn, g1, g2); ``head``:
+        optional dict with the device tensors emb [vocab x d], g_final [d]
+        and W_lm [d x vocab].  Whatever is not given is random-initialised
+        from ``seed``."""
         self.cfg, self.B, self.S_max, self.device = cfg, B, S_max, device
         gen = torch.Generator(device=device)
         gen.manual_seed(seed)
@@ -81,8 +89,8 @@ class DecoderModel:
                 w["g1"] = torch.ones(d, dtype=torch.bfloat16, device=device)
                 w["g2"] = torch.ones(d, dtype=torch.bfloat16, device=device)
             self.layers.append(w)
-        if weights is not None and "emb" in weights:
-            self.emb, self.g_final, self.W_lm = weights["emb"], weights["g_final"], weights["W_lm"]
+        if head is not None:
+            self.emb, self.g_final, self.W_lm = head["emb"], head["g_final"], head["W_lm"]
         else:
             self.emb = _bf16_normal((cfg.vocab, d), 1.0, gen, device)
             self.g_final = torch.ones(d, dtype=torch.bfloat16, device=device)
@@ -254,6 +262,18 @@ class DecoderModel:
         kv = 2 * cfg.layers * (context + 1) * cfg.d * 2 * self.B
         act = self.B * cfg.d * 2 * 2 * cfg.layers
         return 2 * n + kv + act
+
+    def prefill_flops(self, S: int) -> float:
+        """Algorithmic FLOPs of one prefill of B prompts of S tokens: every
+        factorized linear over B*S rows (2 flops per multiply-add of both
+        factors), causal attention (q.k and p.v over the S(S+1)/2 visible
+        pairs of every head), and the head on the last position of each
+        prompt."""
+        cfg = self.cfg
+        lin = 2.0 * self.B * S * sum(cfg.layer_params(i) for i in range(cfg.layers))
+        attn = cfg.layers * 4.0 * self.B * cfg.H * cfg.D * S * (S + 1) / 2
+        head = 2.0 * self.B * cfg.d * cfg.vocab
+        return lin + attn + head
 
     # --------------------------------------------------------- generate --
     def generate(self, prompt_host, steps: int, stream=None):

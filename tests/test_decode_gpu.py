@@ -298,7 +298,7 @@ def test_decoder_layer_decode_steps(fs, B, fused):
     fs.set_decode_path(True)
 
 
-@pytest.mark.parametrize("B", [1, 8])
+@pytest.mark.parametrize("B", [1, 4, 8])
 def test_decoder_layer_decode_7b_shape(fs, B):
     """One Llama-2-7B-shaped low-rank layer (hidden 4096, 32 heads of 128,
     SwiGLU 11008, ranks 1216 / 1792) decoding at context 2048 on a random
