@@ -520,22 +520,65 @@ def run_linear_sweep(args):
     return 0
 
 
+def _unfused_encoder_layer(x, w, B, S, H, eps):
+    """One post-LN encoder layer in plain PyTorch eager, the unfused
+    execution the streamed path is compared with: every factorized linear
+    as two torch.matmul calls (the rank activation z materialised), torch's
+    erf GELU, LayerNorm and scaled_dot_product_attention (no score matrix)."""
+    import torch.nn.functional as F
+    import torch
+    M, d = x.shape
+    D = d // H
+
+    def lin(t, n):
+        return torch.matmul(torch.matmul(t, w["U_" + n]), w["V_" + n]) + w["b_" + n]
+
+    def heads(t):
+        return t.view(B, S, H, D).transpose(1, 2)
+    a = F.scaled_dot_product_attention(heads(lin(x, "q")), heads(lin(x, "k")), heads(lin(x, "v")))
+    a = a.transpose(1, 2).reshape(M, d)
+    h = F.layer_norm(x + lin(a, "o"), (d,), w["ln1_g"], w["ln1_b"], eps)
+    u = F.gelu(lin(h, "up"))
+    return F.layer_norm(h + lin(u, "dn"), (d,), w["ln2_g"], w["ln2_b"], eps)
+
+
 def run_bert(args):
     """BERT-Base-shaped low-rank encoder: 12 layers, hidden 768, 12 heads,
     FFN 3072 (GELU), every linear at rank 192 with bias, batch 32 x 512,
-    bf16, N(0,1) inputs (GLUE is not here; same shapes)."""
+    bf16, N(0,1) inputs (GLUE is not here; same shapes).  Throughput, the
+    streamed FFN kernel's share, and memory against unfused execution:
+    peak activation = device memory the forward holds beyond weights and
+    input; transient = the largest intra-layer temporaries.  Unfused (torch
+    eager, two matmuls per linear): torch allocator peaks.  Ours: the
+    library workspace measured with cudaMemGetInfo around creating it (the
+    part that grows with the token count: a workspace for these tokens
+    minus one for 32 tokens) plus the caller's K/V buffers; no [M x f]
+    buffer is allocated (max_ffn = 8), since the FFN is streamed."""
     import torch
     sys.path.insert(0, ROOT)
     from rank_transformer_b200 import flashsvd as fs
     from rank_transformer_b200.model import EncoderModel
     torch.cuda.set_device(0)
-    B, S = 32, 512
-    fs.init(0, max_tokens=B * S, max_rank=192, max_hidden=768, max_ffn=3072)
+    B, S, d, H, f, r, nl = 32, 512, 768, 12, 3072, 192, 12
+    M = B * S
     peaks = measured_peaks()
-    m = EncoderModel(B=B, S=S, seed=3)
+
+    def ws_bytes(tokens):
+        torch.cuda.synchronize()
+        free0 = torch.cuda.mem_get_info()[0]
+        ctx = fs.Context(0, max_tokens=tokens, max_rank=r, max_hidden=d, max_ffn=8)
+        free1 = torch.cuda.mem_get_info()[0]
+        ctx.destroy()
+        return free0 - free1
+    ws_full, ws_small = ws_bytes(M), ws_bytes(32)
+    fs.init(0, max_tokens=M, max_rank=r, max_hidden=d, max_ffn=8)
+    before = torch.cuda.memory_allocated()
+    m = EncoderModel(layers=nl, B=B, S=S, seed=3)
+    model_bytes = torch.cuda.memory_allocated() - before   # weights + K/V buffers
+    kv_bytes = m.k_buf.numel() * 2 + m.v_buf.numel() * 2
     gen = torch.Generator(device="cuda")
     gen.manual_seed(4)
-    x0 = torch.randn(B * S, 768, device="cuda", generator=gen).to(torch.bfloat16)
+    x0 = torch.randn(M, d, device="cuda", generator=gen).to(torch.bfloat16)
     x = x0.clone()
     stream = torch.cuda.Stream()
     with torch.cuda.stream(stream):
@@ -544,20 +587,74 @@ def run_bert(args):
             m.forward(x, stream)
         ms = _event_ms(lambda i: m.forward(x, stream), 10, stream)
     fs.check_device_status(stream)
+    fs.profile_enable(True)
+    with torch.cuda.stream(stream):
+        m.forward(x, stream)
+    prof = fs.profile_report(reset=True)
+    fs.profile_enable(False)
     tf = m.flops() / (ms / 1e3) / 1e12
-    M, d, f, r = B * S, 768, 3072, 192
-    # activations the forward keeps in device memory: hidden x, K/V buffers,
-    # and the library's per-layer temporaries for this shape (q / attention
-    # output / FFN intermediate / bf16 rank activations z)
-    act = 2 * (M * d + 2 * M * d + 2 * M * d + M * f + M * r)
-    print(json.dumps({
-        "workload": "bert", "config": {"layers": 12, "hidden": d, "heads": 12, "ffn": f, "rank": r,
+    ours_act = (ws_full - ws_small) + kv_bytes
+
+    # unfused torch eager over the same weights and input
+    with torch.cuda.stream(stream):
+        torch.cuda.synchronize()
+        xu = x0.clone()
+        base = torch.cuda.memory_allocated()
+        torch.cuda.reset_peak_memory_stats()
+        t = xu
+        transient = 0
+        for w in m.layers:
+            live = torch.cuda.memory_allocated()
+            torch.cuda.reset_peak_memory_stats()
+            t = _unfused_encoder_layer(t, w, B, S, H, m.eps)
+            transient = max(transient, torch.cuda.max_memory_allocated() - live)
+        torch.cuda.synchronize()
+        del t
+        torch.cuda.reset_peak_memory_stats()
+        base = torch.cuda.memory_allocated()
+        t = xu
+        for w in m.layers:
+            t = _unfused_encoder_layer(t, w, B, S, H, m.eps)
+        torch.cuda.synchronize()
+        unfused_act = torch.cuda.max_memory_allocated() - base
+        del t
+
+        def unfused_fwd(i):
+            t = xu
+            for w in m.layers:
+                t = _unfused_encoder_layer(t, w, B, S, H, m.eps)
+        for _ in range(2):
+            unfused_fwd(0)
+        ms_unfused = _event_ms(unfused_fwd, 3, stream)
+    ffn = prof.get("ffn_stream")
+    line = {
+        "workload": "bert", "config": {"layers": nl, "hidden": d, "heads": H, "ffn": f, "rank": r,
                                        "batch": B, "seq": S},
         "ms_per_forward": round(ms, 3), "sequences_per_s": round(B / (ms / 1e3), 1),
         "tokens_per_s": round(M / (ms / 1e3)), "tflops": round(tf, 1),
         "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 3),
-        "activation_bytes": act, "unfused_z_bytes_avoided_per_linear": 2 * M * r,
-        "note": "the rank activation z of each linear stays in L2 (discarded after use)"}), flush=True)
+        "memory": {
+            "ours_peak_activation_bytes": ours_act,
+            "ours_workspace_bytes": ws_full, "ours_fixed_workspace_bytes": ws_small,
+            "kv_buffer_bytes": kv_bytes, "model_allocation_bytes": model_bytes,
+            "unfused_peak_activation_bytes": unfused_act,
+            "unfused_peak_transient_bytes": transient,
+            "ours_transient_bytes": ours_act,
+            "peak_activation_reduction": round(1 - ours_act / unfused_act, 3),
+            "transient_reduction": round(1 - ours_act / transient, 3),
+            "how": "unfused: torch allocator peak during the forward minus the memory live "
+                   "before it (transient: per layer, minus the live hidden state); ours: "
+                   "cudaMemGetInfo delta of a workspace for these tokens minus one for 32 tokens, "
+                   "plus the caller's K/V buffers (the forward allocates nothing)"},
+        "unfused_ms_per_forward": round(ms_unfused, 3),
+        "kernel_times_ms": {k: round(v["ms"], 4) for k, v in sorted(prof.items())},
+    }
+    if ffn:
+        ffn_tf = ffn["flops"] / (ffn["ms"] / 1e3) / 1e12
+        line["ffn_stream"] = {"launches": ffn["launches"], "ms": round(ffn["ms"], 4),
+                              "tflops": round(ffn_tf, 1),
+                              "frac_of_bf16_peak": round(ffn_tf / peaks["bf16_tflops"], 3)}
+    print(json.dumps(line), flush=True)
     return 0
 
 

@@ -25,8 +25,10 @@
  *     flashsvd_check_device_status().
  *   - Compute calls allocate nothing, never synchronise and copy nothing
  *     between host and device, so they may be captured in a CUDA graph.
- *     They use the library workspace made by flashsvd_init(): calls that
- *     share it must be ordered on one stream (overlapping calls race).
+ *     They use the workspace of the calling thread's context (see
+ *     flashsvd_ctx_create; by default the one made by flashsvd_init()):
+ *     calls that share a workspace must be ordered on one stream
+ *     (overlapping calls race).
  *   - Read-only factor pointers may alias each other (shared bases,
  *     [v1.5] Methodology 1, Basis Sharing).  Outputs must not alias inputs
  *     except where a call says "in place".
@@ -88,8 +90,36 @@ FLASHSVD_API int flashsvd_init(int device, int max_tokens, int max_rank, int max
                   int max_ffn);
 FLASHSVD_API int flashsvd_shutdown(void);
 
-/* Synchronise `stream`, then read and clear the device status word written
- * by kernels whose bounded waits expired.  Returns FLASHSVD_OK or
+/* ------------------------------------------------------------ contexts --
+ * A context is one workspace (the scratch listed under flashsvd_init) plus
+ * its device status word, on one device.  Every compute call uses the
+ * context bound to the calling host thread, or the default context of
+ * flashsvd_init when none is bound.  Calls that share a context must be
+ * ordered on one stream; work that should overlap (two streams, two host
+ * threads, two models on one GPU, or one model per GPU from one process)
+ * gives each its own context.
+ * flashsvd_ctx_create: allocate a context on `device` with the limits of
+ *   flashsvd_init (cudaMalloc; not during stream capture:
+ *   FLASHSVD_ERR_CAPTURE_UNSAFE; FLASHSVD_ERR_NO_MEMORY).  The calling
+ *   thread's current device is left as it was.
+ * flashsvd_ctx_bind: bind `ctx` to the calling host thread and make its
+ *   device current (NULL returns the thread to the default context).  A
+ *   context may be bound by several threads, but their calls then share
+ *   its workspace.  Decode plans and captured graphs hold the addresses of
+ *   the workspace that was current when they were made (plans: when they
+ *   run), so a context must outlive them.
+ * flashsvd_ctx_destroy: synchronise the context's device and free it; the
+ *   calling thread is unbound from it if it was bound.  It must not be
+ *   bound by another thread or used by a graph that still runs.
+ */
+typedef struct flashsvd_ctx flashsvd_ctx;
+FLASHSVD_API int flashsvd_ctx_create(int device, int max_tokens, int max_rank, int max_hidden,
+                                     int max_ffn, flashsvd_ctx** ctx);
+FLASHSVD_API int flashsvd_ctx_bind(flashsvd_ctx* ctx);
+FLASHSVD_API int flashsvd_ctx_destroy(flashsvd_ctx* ctx);
+
+/* Synchronise `stream`, then read and clear the current context's device
+ * status word, written by kernels whose bounded waits expired.  Returns FLASHSVD_OK or
  * FLASHSVD_ERR_TIMEOUT (or FLASHSVD_ERR_CUDA if the stream reports an
  * error). */
 FLASHSVD_API int flashsvd_check_device_status(flashsvd_stream stream);
@@ -162,6 +192,31 @@ FLASHSVD_API int flashsvd_packed_gateup_mlp(const flashsvd_bf16* x,
 FLASHSVD_API int flashsvd_gateup_swiglu(const flashsvd_bf16* x, const flashsvd_bf16* U_gu,
                            const flashsvd_bf16* V_gu, flashsvd_bf16* h, int M,
                            int d, int r_f, int f, flashsvd_stream stream);
+
+/* ------------------------------------------------- streamed low-rank FFN --
+ * [v1] abstract: the encoder FFN's intermediate activations are streamed
+ * through tiles instead of being materialised.
+ *   y[M x d] = GELU((x . U_up) . V_up + b_up) . U_dn . V_dn + b_dn + resid
+ * x [M x d], U_up [d x r_up], V_up [r_up x f], U_dn [f x r_dn],
+ * V_dn [r_dn x d]; b_up [f], b_dn [d] and resid [M x d] may be NULL; resid
+ * may equal y.  GELU is the erf form.  z1 = x . U_up is one tcgen05 launch
+ * into the library scratch (kept in L2 and discarded there after use); the
+ * rest is ONE kernel per 128-row tile that runs f in 128-column chunks:
+ * the chunk of GELU(z1 . V_up + b_up) goes from tensor memory through the
+ * GELU warps into shared memory and straight into the rank-r_dn
+ * accumulator of U_dn, so the [M x f] activation is never written to
+ * memory.  ENCODER-layer flashsvd_layer_forward uses it for the FFN.
+ * Sizes: d a multiple of 64; r_up, r_dn multiples of 64 in [64, 256]; f a
+ * multiple of 8; M <= max_tokens.  Other shapes return
+ * FLASHSVD_ERR_UNSUPPORTED_SHAPE (the encoder layer then runs the FFN as
+ * two factorized linears with the [M x f] activation in the workspace).
+ */
+FLASHSVD_API int flashsvd_lowrank_ffn(const flashsvd_bf16* x, const flashsvd_bf16* U_up,
+                                      const flashsvd_bf16* V_up, const flashsvd_bf16* b_up,
+                                      const flashsvd_bf16* U_dn, const flashsvd_bf16* V_dn,
+                                      const flashsvd_bf16* b_dn, const flashsvd_bf16* resid,
+                                      flashsvd_bf16* y, int M, int d, int r_up, int f, int r_dn,
+                                      flashsvd_stream stream);
 
 /* ------------------------------------------------ dense-KV decode attention --
  * [v1.5] Methodology 2 ("reconstruct the present, read the past

@@ -262,6 +262,18 @@ def decoder_layer_decode(x, w, H, k_hist, v_hist, pos, eps=RMS_EPS):
     return y, k_new, v
 
 
+# ------------------------------------------------------------ encoder FFN --
+
+def lowrank_gelu_ffn(x, U_up, V_up, b_up, U_dn, V_dn, b_dn):
+    """Low-rank GELU FFN of an encoder layer ([v1] abstract: the FFN of
+    BERT-class encoders with both projections factorized; its intermediate
+    activation is what the streamed kernel never materialises):
+
+        y = lowrank(GELU(lowrank(x, U_up, V_up, b_up)), U_dn, V_dn, b_dn)
+    """
+    return lowrank_linear(gelu(lowrank_linear(x, U_up, V_up, b_up)), U_dn, V_dn, b_dn)
+
+
 # --------------------------------------------------------- encoder layer --
 
 def bert_layer(x, w, H, eps=LN_EPS):
@@ -281,9 +293,8 @@ def bert_layer(x, w, H, eps=LN_EPS):
                  axis=1).reshape(S, d)
     h = layernorm(x + lowrank_linear(a, w["U_o"], w["V_o"], w["b_o"]),
                   w["ln1_g"], w["ln1_b"], eps)
-    u = gelu(lowrank_linear(h, w["U_up"], w["V_up"], w["b_up"]))
-    return layernorm(h + lowrank_linear(u, w["U_dn"], w["V_dn"], w["b_dn"]),
-                     w["ln2_g"], w["ln2_b"], eps)
+    f = lowrank_gelu_ffn(h, w["U_up"], w["V_up"], w["b_up"], w["U_dn"], w["V_dn"], w["b_dn"])
+    return layernorm(h + f, w["ln2_g"], w["ln2_b"], eps)
 
 
 # ------------------------------------------------------------ model head --

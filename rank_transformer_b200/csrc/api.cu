@@ -38,8 +38,13 @@ struct Ctx {
   int rows = 0;                // rows of the scratch above
 };
 
-Ctx g_ctx;
+// The default context (flashsvd_init / flashsvd_shutdown) and the context a
+// host thread has bound with flashsvd_ctx_bind (none: the default).
+Ctx g_default;
+thread_local Ctx* t_ctx = nullptr;
 std::mutex g_mu;
+
+inline Ctx& cur() { return t_ctx ? *t_ctx : g_default; }
 
 void free_ctx(Ctx& c) {
   void* ptrs[] = {c.z, c.part, c.counters, c.apart, c.acounters, c.status,
@@ -49,13 +54,58 @@ void free_ctx(Ctx& c) {
   c = Ctx();
 }
 
+// Allocate and clear a context's workspace on `device` (which must be
+// current).  On failure nothing stays allocated.
+int alloc_ctx(Ctx& c, int device, int max_tokens, int max_rank, int max_hidden, int max_ffn) {
+  c = Ctx();
+  c.device = device;
+  c.max_tokens = max_tokens; c.max_rank = max_rank;
+  c.max_hidden = max_hidden; c.max_ffn = max_ffn;
+  cudaDeviceGetAttribute(&c.sm_count, cudaDevAttrMultiProcessorCount, device);
+  c.rows = max_tokens > DECODE_MAX_ROWS ? max_tokens : DECODE_MAX_ROWS;
+  const int wide = max_ffn > max_hidden ? max_ffn : max_hidden;
+  c.z_elems = (size_t)DECODE_MAX_ROWS * 3 * (max_rank > wide / 2 ? max_rank : wide / 2) + 4096;
+  c.part_elems = (size_t)16 << 20;
+  c.apart_elems = (size_t)16 << 20;  // split-sequence partials of decode attention
+  cudaError_t e = cudaSuccess;
+#define FSVD_ALLOC(ptr, bytes) \
+  if (e == cudaSuccess) e = cudaMalloc((void**)&(ptr), (bytes));
+  FSVD_ALLOC(c.z, c.z_elems * sizeof(float));
+  FSVD_ALLOC(c.part, c.part_elems * sizeof(float));
+  FSVD_ALLOC(c.counters, kCountersN * sizeof(int));
+  FSVD_ALLOC(c.apart, c.apart_elems * sizeof(float));
+  FSVD_ALLOC(c.acounters, kCountersN * sizeof(int));
+  FSVD_ALLOC(c.status, 64 * sizeof(int));
+  FSVD_ALLOC(c.xn, (size_t)c.rows * max_hidden * sizeof(bf16));
+  FSVD_ALLOC(c.q, (size_t)c.rows * max_hidden * sizeof(bf16));
+  FSVD_ALLOC(c.att, (size_t)c.rows * max_hidden * sizeof(bf16));
+  FSVD_ALLOC(c.h, (size_t)c.rows * max_ffn * sizeof(bf16));
+  FSVD_ALLOC(c.zb, (size_t)c.rows * 2 * max_rank * sizeof(bf16));
+  FSVD_ALLOC(c.df_part, (size_t)kFusedPartFloats * sizeof(float));
+  FSVD_ALLOC(c.df_cnt, (size_t)(4096 + 64) * sizeof(int));
+  FSVD_ALLOC(c.zcnt, (size_t)(c.rows / 128 + 1) * sizeof(int));
+#undef FSVD_ALLOC
+  if (e == cudaSuccess) e = cudaMemset(c.counters, 0, kCountersN * sizeof(int));
+  if (e == cudaSuccess) e = cudaMemset(c.acounters, 0, kCountersN * sizeof(int));
+  if (e == cudaSuccess) e = cudaMemset(c.status, 0, 64 * sizeof(int));
+  if (e == cudaSuccess) e = cudaMemset(c.df_cnt, 0, (4096 + 64) * sizeof(int));
+  if (e == cudaSuccess) e = cudaMemset(c.zcnt, 0, (c.rows / 128 + 1) * sizeof(int));
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    free_ctx(c);
+    g_last_cuda_error = (int)e;
+    return e == cudaErrorMemoryAllocation ? FLASHSVD_ERR_NO_MEMORY : FLASHSVD_ERR_CUDA;
+  }
+  return FLASHSVD_OK;
+}
+
 bool capturing(cudaStream_t s) {
   cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
   if (cudaStreamIsCapturing(s, &st) != cudaSuccess) return false;
   return st != cudaStreamCaptureStatusNone;
 }
 
-int need_init() { return g_ctx.device < 0 ? FLASHSVD_ERR_NOT_INITIALIZED : FLASHSVD_OK; }
+int need_init() { return cur().device < 0 ? FLASHSVD_ERR_NOT_INITIALIZED : FLASHSVD_OK; }
 
 inline const bf16* cb(const flashsvd_bf16* p) { return reinterpret_cast<const bf16*>(p); }
 
@@ -70,14 +120,14 @@ int check_w8(int v) {
   return (v % 8) ? FLASHSVD_ERR_UNSUPPORTED_SHAPE : FLASHSVD_OK;
 }
 
-int target_ctas() { return g_ctx.sm_count * 3; }
+int target_ctas() { return cur().sm_count * 3; }
 
 // Capacity guard for decode attention: one partial of D + 2 floats per
 // (batch, head, 64-key chunk).
 int attn_fits(int B, int H, int D, int S_max) {
   const size_t chunks = (size_t)ceil_div(S_max, 64);
   if (chunks > 1024 || (size_t)B * H > (size_t)kCountersN ||
-      (size_t)B * H * chunks * (D + 2) > g_ctx.apart_elems)
+      (size_t)B * H * chunks * (D + 2) > cur().apart_elems)
     return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   return FLASHSVD_OK;
 }
@@ -85,9 +135,9 @@ int attn_fits(int B, int H, int D, int S_max) {
 GvParams gv_base() {
   GvParams p;
   memset(&p, 0, sizeof(p));
-  p.part = g_ctx.part;
-  p.counters = g_ctx.counters;
-  p.part_cap = (long long)g_ctx.part_elems;
+  p.part = cur().part;
+  p.counters = cur().counters;
+  p.part_cap = (long long)cur().part_elems;
   p.counters_cap = kCountersN;
   return p;
 }
@@ -96,7 +146,7 @@ GvParams gv_base() {
 int gv_fits(int K, int tiles) {
   const long long splits_max = ((long long)target_ctas() / tiles) + ceil_div(K, 512) + 1;
   if (tiles > kCountersN) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
-  if ((long long)tiles * splits_max * 512 > (long long)g_ctx.part_elems)
+  if ((long long)tiles * splits_max * 512 > (long long)cur().part_elems)
     return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   return FLASHSVD_OK;
 }
@@ -116,9 +166,9 @@ int decode_stage1(int pro, const bf16* x, long long ldx, const bf16* norm_g,
     off += N[i];
     tiles += gemv_tiles_for(MAP_PLAIN, N[i], 64);
   }
-  if ((size_t)M * off > g_ctx.z_elems) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  if ((size_t)M * off > cur().z_elems) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   FSVD_TRY(gv_fits(K, tiles));
-  p.out32 = g_ctx.z; p.ldo32 = off;
+  p.out32 = cur().z; p.ldo32 = off;
   return gemv_launch(p, pro, EPI_F32, MAP_PLAIN, M, target_ctas(), s);
 }
 
@@ -131,7 +181,7 @@ int decode_linear(const bf16* x, const bf16* U, const bf16* V, const bf16* bias,
   GvParams p = gv_base();
   p.K = r; p.nprob = 1;
   p.prob[0].W = V; p.prob[0].ldw = n; p.prob[0].N = n;
-  p.a32 = g_ctx.z; p.lda = r;
+  p.a32 = cur().z; p.lda = r;
   p.out16 = y; p.ldo16 = n; p.bias = bias; p.resid = resid; p.ldr = n;
   FSVD_TRY(gv_fits(r, gemv_tiles_for(MAP_PLAIN, n, 64)));
   return gemv_launch(p, PRO_F32, EPI_BF16, MAP_PLAIN, M, target_ctas(), s);
@@ -148,14 +198,14 @@ int decode_gateup(const bf16* x, const bf16* U_gu, const bf16* V_gu, bf16* h,
   p.K = r_f; p.nprob = 1;
   p.prob[0].W = V_gu; p.prob[0].ldw = f; p.prob[0].N = f;
   p.prob[0].a_col = 0; p.prob[0].a_col2 = r_f; p.prob[0].w_row2 = r_f;
-  p.a32 = g_ctx.z; p.lda = 2 * r_f;
+  p.a32 = cur().z; p.lda = 2 * r_f;
   p.out16 = h; p.ldo16 = f;
   FSVD_TRY(gv_fits(r_f, gemv_tiles_for(MAP_SWIGLU, f, 64)));
   return gemv_launch(p, PRO_F32, EPI_SWIGLU, MAP_SWIGLU, M, target_ctas(), s);
 }
 
 int ensure_scratch(int rows, int hidden, int ffn) {
-  if (rows > g_ctx.rows || hidden > g_ctx.max_hidden || ffn > g_ctx.max_ffn)
+  if (rows > cur().rows || hidden > cur().max_hidden || ffn > cur().max_ffn)
     return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   return FLASHSVD_OK;
 }
@@ -166,9 +216,16 @@ int check_factor(const flashsvd_factor& F, int d_in, int d_out, bool bias_ok) {
   if (!bias_ok && F.bias) return FLASHSVD_ERR_INVALID_ARG;
   FSVD_TRY(check_opt_ptr(F.bias));
   FSVD_TRY(check_w8(F.r));
-  if (F.r > g_ctx.max_rank) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  if (F.r > cur().max_rank) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   (void)d_in; (void)d_out;
   return FLASHSVD_OK;
+}
+
+// Whether the streamed low-rank FFN kernel covers an encoder FFN of these
+// shapes (d -> f at rank r1, f -> d at rank r2).
+bool ffn_stream_covers(int d, int r1, int f, int r2) {
+  return d % 64 == 0 && r1 % 64 == 0 && r2 % 64 == 0 && r1 >= 64 && r2 >= 64 &&
+         r1 <= kFfnStreamMaxRank && r2 <= kFfnStreamMaxRank && f % 8 == 0;
 }
 
 int check_layer(const flashsvd_layer* L) {
@@ -178,8 +235,11 @@ int check_layer(const flashsvd_layer* L) {
   FSVD_TRY(check_w8(L->f));
   if (L->H <= 0 || L->D <= 0 || L->H * L->D != L->d) return FLASHSVD_ERR_INVALID_ARG;
   if (L->D != 64 && L->D != 128) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
-  if (L->d > g_ctx.max_hidden || L->f > g_ctx.max_ffn) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   const bool enc = L->kind == FLASHSVD_ENCODER;
+  // a streamed encoder FFN keeps its [M x f] activation on chip: f is not
+  // bounded by the workspace
+  const bool streamed = enc && ffn_stream_covers(L->d, L->up.r, L->f, L->down.r);
+  if (L->d > cur().max_hidden || (L->f > cur().max_ffn && !streamed)) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   FSVD_TRY(check_factor(L->q, L->d, L->d, enc));
   FSVD_TRY(check_factor(L->k, L->d, L->d, enc));
   FSVD_TRY(check_factor(L->v, L->d, L->d, enc));
@@ -195,7 +255,7 @@ int check_layer(const flashsvd_layer* L) {
     FSVD_TRY(check_ptr(L->U_gu));
     FSVD_TRY(check_ptr(L->V_gu));
     FSVD_TRY(check_w8(L->r_f));
-    if (2 * L->r_f > g_ctx.max_rank * 2) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+    if (2 * L->r_f > cur().max_rank * 2) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
     FSVD_TRY(check_ptr(L->rope_cos));
     FSVD_TRY(check_ptr(L->rope_sin));
   }
@@ -209,9 +269,9 @@ PfLinear pf_base(const bf16* x, long long ldx, const flashsvd_factor& F, int M,
   p.x = x; p.ldx = ldx; p.U = cb(F.U); p.V = cb(F.V); p.bias = cb(F.bias);
   p.y = y; p.ldy = ldy; p.M = M; p.d = d; p.r = F.r; p.n = n;
   p.epi = PF_EPI_BF16;
-  p.z = g_ctx.zb;
-  p.zcnt = g_ctx.zcnt;
-  p.status = g_ctx.status;
+  p.z = cur().zb;
+  p.zcnt = cur().zcnt;
+  p.status = cur().status;
   return p;
 }
 
@@ -221,18 +281,18 @@ PfLinear pf_base(const bf16* x, long long ldx, const flashsvd_factor& F, int M,
 bool qkv_stage1_grouped(const bf16* x, int d, int M, const flashsvd_factor* const* F, bf16** z,
                         cudaStream_t s, int* st) {
   const long long need = (long long)M * (F[0]->r + F[1]->r + F[2]->r);
-  if (need > (long long)g_ctx.rows * 2 * g_ctx.max_rank) return false;
+  if (need > (long long)cur().rows * 2 * cur().max_rank) return false;
   const bf16* U[3];
   int r[3];
   long long off = 0;
   for (int i = 0; i < 3; ++i) {
     U[i] = cb(F[i]->U);
     r[i] = F[i]->r;
-    z[i] = g_ctx.zb + off;
+    z[i] = cur().zb + off;
     off += (long long)M * r[i];
     if (!aligned16(z[i]) || r[i] % 8) return false;
   }
-  *st = prefill_stage1_grouped(x, d, d, M, 3, U, r, z, g_ctx.status, s);
+  *st = prefill_stage1_grouped(x, d, d, M, 3, U, r, z, cur().status, s);
   return true;
 }
 
@@ -265,12 +325,12 @@ int layer_decode(const flashsvd_layer* L, bf16* x, bf16* kc, bf16* vc,
                  const int* seqlens, int B, int S_max, cudaStream_t s) {
   const int d = L->d, r = L->q.r;
   const bool same_r = L->k.r == r && L->v.r == r;
-  if (g_fused_decode && L->decode_pack && pack_shapes_ok(L) && g_ctx.sm_count <= 148 &&
+  if (g_fused_decode && L->decode_pack && pack_shapes_ok(L) && cur().sm_count <= 148 &&
       decode_fused_supported(B, d, L->D, r, L->r_f)) {
     const DecodeLayerDesc D = decode_desc(L);
-    const int st = decode_fused_launch(D, x, kc, vc, seqlens, B, S_max, g_ctx.xn, g_ctx.df_part,
-                                       kFusedPartFloats, g_ctx.df_cnt, g_ctx.df_cnt + 32, g_ctx.status,
-                                       g_ctx.sm_count, s);
+    const int st = decode_fused_launch(D, x, kc, vc, seqlens, B, S_max, cur().xn, cur().df_part,
+                                       kFusedPartFloats, cur().df_cnt, cur().df_cnt + 32, cur().status,
+                                       cur().sm_count, s);
     if (st != FLASHSVD_ERR_UNSUPPORTED_SHAPE) return st;
   }
   // 1) z_qkv = rmsnorm(x) . [U_q | U_k | U_v]
@@ -289,8 +349,8 @@ int layer_decode(const flashsvd_layer* L, bf16* x, bf16* kc, bf16* vc,
       p.prob[i].W = Vs[i]; p.prob[i].ldw = d; p.prob[i].N = d;
       p.prob[i].a_col = i * r; p.prob[i].kind = i;
     }
-    p.a32 = g_ctx.z; p.lda = 3 * r;
-    p.out16 = g_ctx.q; p.ldo16 = d;
+    p.a32 = cur().z; p.lda = 3 * r;
+    p.out16 = cur().q; p.ldo16 = d;
     p.k_cache = kc; p.v_cache = vc; p.seqlens = seqlens; p.S_max = S_max;
     p.HD = d; p.D = L->D;
     p.rope_cos = L->rope_cos; p.rope_sin = L->rope_sin;
@@ -301,34 +361,34 @@ int layer_decode(const flashsvd_layer* L, bf16* x, bf16* kc, bf16* vc,
   {
     AttnDecParams a;
     memset(&a, 0, sizeof(a));
-    a.q = g_ctx.q; a.k_cache = kc; a.v_cache = vc; a.seqlens = seqlens; a.out = g_ctx.att;
+    a.q = cur().q; a.k_cache = kc; a.v_cache = vc; a.seqlens = seqlens; a.out = cur().att;
     a.B = B; a.H = L->H; a.D = L->D; a.S_max = S_max;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)L->D);
-    a.part = g_ctx.apart; a.counters = g_ctx.acounters;
+    a.part = cur().apart; a.counters = cur().acounters;
     FSVD_TRY(attn_decode_launch(a, target_ctas(), s));
   }
   // 4-5) x = x + (att . U_o) . V_o
-  FSVD_TRY(decode_linear(g_ctx.att, cb(L->o.U), cb(L->o.V), nullptr, x, x, B, d, L->o.r, d, nullptr, 0.f, s));
+  FSVD_TRY(decode_linear(cur().att, cb(L->o.U), cb(L->o.V), nullptr, x, x, B, d, L->o.r, d, nullptr, 0.f, s));
   // 6-7) h = SiLU(gate) * up of rmsnorm(x)
-  FSVD_TRY(decode_gateup(x, cb(L->U_gu), cb(L->V_gu), g_ctx.h, B, d, L->r_f, L->f,
+  FSVD_TRY(decode_gateup(x, cb(L->U_gu), cb(L->V_gu), cur().h, B, d, L->r_f, L->f,
                          (const bf16*)L->norm2_g, L->norm_eps, s));
   // 8-9) x = x + (h . U_dn) . V_dn
-  return decode_linear(g_ctx.h, cb(L->down.U), cb(L->down.V), nullptr, x, x, B, L->f, L->down.r, d, nullptr, 0.f, s);
+  return decode_linear(cur().h, cb(L->down.U), cb(L->down.V), nullptr, x, x, B, L->f, L->down.r, d, nullptr, 0.f, s);
 }
 
 // ------------------------------------------------------ layer: prefill ----
 int layer_prefill(const flashsvd_layer* L, bf16* x, bf16* kc, bf16* vc,
                   int B, int S, int S_max, cudaStream_t s) {
   const int d = L->d, M = B * S;
-  FSVD_TRY(rmsnorm_launch(x, cb(L->norm1_g), g_ctx.xn, M, d, L->norm_eps, s));
+  FSVD_TRY(rmsnorm_launch(x, cb(L->norm1_g), cur().xn, M, d, L->norm_eps, s));
   const flashsvd_factor* F[3] = {&L->q, &L->k, &L->v};
-  bf16* dst[3] = {g_ctx.q, kc, vc};
+  bf16* dst[3] = {cur().q, kc, vc};
   bf16* zg[3];
   int gst = FLASHSVD_OK;
-  const bool grouped = qkv_stage1_grouped(g_ctx.xn, d, M, F, zg, s, &gst);
+  const bool grouped = qkv_stage1_grouped(cur().xn, d, M, F, zg, s, &gst);
   FSVD_TRY(gst);
   for (int i = 0; i < 3; ++i) {
-    PfLinear p = pf_base(g_ctx.xn, d, *F[i], M, d, d, g_ctx.q, d);
+    PfLinear p = pf_base(cur().xn, d, *F[i], M, d, d, cur().q, d);
     if (grouped) { p.z = zg[i]; p.z_ready = 1; }
     p.epi = PF_EPI_QKV; p.kind = i; p.cache = dst[i]; p.S = S; p.S_max = S_max;
     p.HD = d; p.D = L->D;
@@ -337,26 +397,38 @@ int layer_prefill(const flashsvd_layer* L, bf16* x, bf16* kc, bf16* vc,
   }
   AttnPfParams a;
   memset(&a, 0, sizeof(a));
-  a.q = g_ctx.q; a.k = kc; a.v = vc; a.out = g_ctx.att;
+  a.q = cur().q; a.k = kc; a.v = vc; a.out = cur().att;
   a.B = B; a.S = S; a.H = L->H; a.D = L->D; a.S_max = S_max; a.causal = 1;
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)L->D);
-  a.status = g_ctx.status;
+  a.status = cur().status;
   FSVD_TRY(attn_prefill_launch(a, s));
   {
-    PfLinear p = pf_base(g_ctx.att, d, L->o, M, d, d, x, d);
+    PfLinear p = pf_base(cur().att, d, L->o, M, d, d, x, d);
     p.resid = x; p.ldr = d;
     FSVD_TRY(prefill_linear_launch(p, s));
   }
-  FSVD_TRY(rmsnorm_launch(x, cb(L->norm2_g), g_ctx.xn, M, d, L->norm_eps, s));
+  FSVD_TRY(rmsnorm_launch(x, cb(L->norm2_g), cur().xn, M, d, L->norm_eps, s));
   {
     flashsvd_factor gu = {L->U_gu, L->V_gu, nullptr, 2 * L->r_f};
-    PfLinear p = pf_base(g_ctx.xn, d, gu, M, d, L->f, g_ctx.h, L->f);
+    PfLinear p = pf_base(cur().xn, d, gu, M, d, L->f, cur().h, L->f);
     p.epi = PF_EPI_SWIGLU;
     FSVD_TRY(prefill_linear_launch(p, s));
   }
-  PfLinear p = pf_base(g_ctx.h, L->f, L->down, M, L->f, d, x, d);
+  PfLinear p = pf_base(cur().h, L->f, L->down, M, L->f, d, x, d);
   p.resid = x; p.ldr = d;
   return prefill_linear_launch(p, s);
+}
+
+// Streamed low-rank FFN: z1 = x . U1 (tcgen05 stage 1 into the rank
+// scratch), then y = GELU(z1 . V1 + b1) . U2 . V2 + b2 + resid in one
+// kernel that keeps the [M x f] activation on chip.
+int lowrank_ffn(const bf16* x, const bf16* U1, const bf16* V1, const bf16* b1, const bf16* U2,
+                const bf16* V2, const bf16* b2, const bf16* resid, bf16* y, int M, int d, int r1, int f,
+                int r2, cudaStream_t s) {
+  bf16* z = cur().zb;
+  FSVD_TRY(prefill_stage1(x, d, d, M, U1, r1, z, cur().status, s));
+  return ffn_stream_launch(z, r1, V1, b1, U2, V2, b2, resid, y, M, f, r1, r2, d, cur().status,
+                           cur().sm_count, s);
 }
 
 // ------------------------------------------------------ layer: encoder ----
@@ -364,13 +436,13 @@ int layer_encoder(const flashsvd_layer* L, bf16* x, bf16* kc, bf16* vc,
                   int B, int S, int S_max, cudaStream_t s) {
   const int d = L->d, M = B * S;
   const flashsvd_factor* F[3] = {&L->q, &L->k, &L->v};
-  bf16* dst[3] = {g_ctx.q, kc, vc};
+  bf16* dst[3] = {cur().q, kc, vc};
   bf16* zg[3];
   int gst = FLASHSVD_OK;
   const bool grouped = qkv_stage1_grouped(x, d, M, F, zg, s, &gst);
   FSVD_TRY(gst);
   for (int i = 0; i < 3; ++i) {
-    PfLinear p = pf_base(x, d, *F[i], M, d, d, g_ctx.q, d);
+    PfLinear p = pf_base(x, d, *F[i], M, d, d, cur().q, d);
     if (grouped) { p.z = zg[i]; p.z_ready = 1; }
     p.epi = PF_EPI_QKV; p.kind = i; p.cache = dst[i]; p.S = S; p.S_max = S_max;
     p.HD = d; p.D = L->D;
@@ -378,28 +450,32 @@ int layer_encoder(const flashsvd_layer* L, bf16* x, bf16* kc, bf16* vc,
   }
   AttnPfParams a;
   memset(&a, 0, sizeof(a));
-  a.q = g_ctx.q; a.k = kc; a.v = vc; a.out = g_ctx.att;
+  a.q = cur().q; a.k = kc; a.v = vc; a.out = cur().att;
   a.B = B; a.S = S; a.H = L->H; a.D = L->D; a.S_max = S_max; a.causal = 0;
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)L->D);
-  a.status = g_ctx.status;
+  a.status = cur().status;
   FSVD_TRY(attn_prefill_launch(a, s));
   {
-    PfLinear p = pf_base(g_ctx.att, d, L->o, M, d, d, g_ctx.xn, d);
+    PfLinear p = pf_base(cur().att, d, L->o, M, d, d, cur().xn, d);
     p.resid = x; p.ldr = d;
     FSVD_TRY(prefill_linear_launch(p, s));
   }
-  FSVD_TRY(layernorm_launch(g_ctx.xn, cb(L->norm1_g), cb(L->norm1_b), x, M, d, L->norm_eps, s));
-  {
-    PfLinear p = pf_base(x, d, L->up, M, d, L->f, g_ctx.h, L->f);
-    p.epi = PF_EPI_GELU;
-    FSVD_TRY(prefill_linear_launch(p, s));
-  }
-  {
-    PfLinear p = pf_base(g_ctx.h, L->f, L->down, M, L->f, d, g_ctx.xn, d);
+  FSVD_TRY(layernorm_launch(cur().xn, cb(L->norm1_g), cb(L->norm1_b), x, M, d, L->norm_eps, s));
+  if (ffn_stream_covers(d, L->up.r, L->f, L->down.r)) {
+    // the FFN streamed over f-tiles: GELU(up(x)) never leaves the SM
+    FSVD_TRY(lowrank_ffn(x, cb(L->up.U), cb(L->up.V), cb(L->up.bias), cb(L->down.U), cb(L->down.V),
+                         cb(L->down.bias), x, cur().xn, M, d, L->up.r, L->f, L->down.r, s));
+  } else {
+    {
+      PfLinear p = pf_base(x, d, L->up, M, d, L->f, cur().h, L->f);
+      p.epi = PF_EPI_GELU;
+      FSVD_TRY(prefill_linear_launch(p, s));
+    }
+    PfLinear p = pf_base(cur().h, L->f, L->down, M, L->f, d, cur().xn, d);
     p.resid = x; p.ldr = d;
     FSVD_TRY(prefill_linear_launch(p, s));
   }
-  return layernorm_launch(g_ctx.xn, cb(L->norm2_g), cb(L->norm2_b), x, M, d, L->norm_eps, s);
+  return layernorm_launch(cur().xn, cb(L->norm2_g), cb(L->norm2_b), x, M, d, L->norm_eps, s);
 }
 
 }  // namespace
@@ -521,7 +597,7 @@ int flashsvd_decode_plan_create(const flashsvd_layer* layers, int n_layers, flas
   if (!layers || n_layers <= 0 || !k_caches || !v_caches || !plan || B <= 0 || S_max <= 0)
     return FLASHSVD_ERR_INVALID_ARG;
   if (capturing(nullptr)) return FLASHSVD_ERR_CAPTURE_UNSAFE;
-  if (!g_fused_decode || g_ctx.sm_count > 148) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  if (!g_fused_decode || cur().sm_count > 148) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   std::vector<DecodeLayerDesc> descs((size_t)n_layers);
   std::vector<bf16*> kc((size_t)n_layers), vc((size_t)n_layers);
   for (int i = 0; i < n_layers; ++i) {
@@ -535,10 +611,10 @@ int flashsvd_decode_plan_create(const flashsvd_layer* layers, int n_layers, flas
     vc[i] = reinterpret_cast<bf16*>(v_caches[i]);
   }
   DecodePlan* impl = nullptr;
-  FSVD_TRY(decode_plan_create(descs.data(), n_layers, kc.data(), vc.data(), B, S_max, g_ctx.sm_count, &impl));
+  FSVD_TRY(decode_plan_create(descs.data(), n_layers, kc.data(), vc.data(), B, S_max, cur().sm_count, &impl));
   flashsvd_decode_plan* out = new flashsvd_decode_plan();
   out->impl = impl;
-  out->device = g_ctx.device;
+  out->device = cur().device;
   out->B = B;
   out->d = layers[0].d;
   *plan = out;
@@ -549,11 +625,11 @@ int flashsvd_decode_plan_forward(const flashsvd_decode_plan* plan, flashsvd_bf16
                                  const int32_t* cache_seqlens, flashsvd_stream stream) {
   FSVD_TRY(need_init());
   if (!plan || !x_inout || !cache_seqlens) return FLASHSVD_ERR_INVALID_ARG;
-  if (plan->device != g_ctx.device) return FLASHSVD_ERR_INVALID_ARG;
+  if (plan->device != cur().device) return FLASHSVD_ERR_INVALID_ARG;
   if (!aligned16(x_inout)) return FLASHSVD_ERR_MISALIGNED;
-  if (plan->d > g_ctx.max_hidden) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
-  return decode_plan_launch(plan->impl, reinterpret_cast<bf16*>(x_inout), cache_seqlens, g_ctx.xn, g_ctx.df_part,
-                            kFusedPartFloats, g_ctx.df_cnt, g_ctx.df_cnt + 32, g_ctx.status,
+  if (plan->d > cur().max_hidden) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  return decode_plan_launch(plan->impl, reinterpret_cast<bf16*>(x_inout), cache_seqlens, cur().xn, cur().df_part,
+                            kFusedPartFloats, cur().df_cnt, cur().df_cnt + 32, cur().status,
                             (cudaStream_t)stream);
 }
 
@@ -570,63 +646,68 @@ int flashsvd_init(int device, int max_tokens, int max_rank, int max_hidden,
   if (device < 0 || max_tokens <= 0 || max_rank <= 0 || max_hidden <= 0 || max_ffn <= 0)
     return FLASHSVD_ERR_INVALID_ARG;
   if (capturing(nullptr)) return FLASHSVD_ERR_CAPTURE_UNSAFE;
-  if (g_ctx.device == device && max_tokens <= g_ctx.max_tokens && max_rank <= g_ctx.max_rank &&
-      max_hidden <= g_ctx.max_hidden && max_ffn <= g_ctx.max_ffn)
+  Ctx& d = g_default;
+  if (d.device == device && max_tokens <= d.max_tokens && max_rank <= d.max_rank &&
+      max_hidden <= d.max_hidden && max_ffn <= d.max_ffn)
     return FLASHSVD_OK;
   FSVD_CUDA(cudaSetDevice(device));
-  if (g_ctx.device >= 0) {
+  if (d.device >= 0) {
     cudaDeviceSynchronize();
-    free_ctx(g_ctx);
+    free_ctx(d);
   }
   Ctx c;
-  c.device = device;
-  c.max_tokens = max_tokens; c.max_rank = max_rank;
-  c.max_hidden = max_hidden; c.max_ffn = max_ffn;
-  cudaDeviceGetAttribute(&c.sm_count, cudaDevAttrMultiProcessorCount, device);
-  c.rows = max_tokens > DECODE_MAX_ROWS ? max_tokens : DECODE_MAX_ROWS;
-  const int wide = max_ffn > max_hidden ? max_ffn : max_hidden;
-  c.z_elems = (size_t)DECODE_MAX_ROWS * 3 * (max_rank > wide / 2 ? max_rank : wide / 2) + 4096;
-  c.part_elems = (size_t)16 << 20;
-  c.apart_elems = (size_t)16 << 20;  // split-sequence partials of decode attention
-  cudaError_t e = cudaSuccess;
-#define FSVD_ALLOC(ptr, bytes) \
-  if (e == cudaSuccess) e = cudaMalloc((void**)&(ptr), (bytes));
-  FSVD_ALLOC(c.z, c.z_elems * sizeof(float));
-  FSVD_ALLOC(c.part, c.part_elems * sizeof(float));
-  FSVD_ALLOC(c.counters, kCountersN * sizeof(int));
-  FSVD_ALLOC(c.apart, c.apart_elems * sizeof(float));
-  FSVD_ALLOC(c.acounters, kCountersN * sizeof(int));
-  FSVD_ALLOC(c.status, 64 * sizeof(int));
-  FSVD_ALLOC(c.xn, (size_t)c.rows * max_hidden * sizeof(bf16));
-  FSVD_ALLOC(c.q, (size_t)c.rows * max_hidden * sizeof(bf16));
-  FSVD_ALLOC(c.att, (size_t)c.rows * max_hidden * sizeof(bf16));
-  FSVD_ALLOC(c.h, (size_t)c.rows * max_ffn * sizeof(bf16));
-  FSVD_ALLOC(c.zb, (size_t)c.rows * 2 * max_rank * sizeof(bf16));
-  FSVD_ALLOC(c.df_part, (size_t)kFusedPartFloats * sizeof(float));
-  FSVD_ALLOC(c.df_cnt, (size_t)(4096 + 64) * sizeof(int));
-  FSVD_ALLOC(c.zcnt, (size_t)(c.rows / 128 + 1) * sizeof(int));
-#undef FSVD_ALLOC
-  if (e == cudaSuccess) e = cudaMemset(c.counters, 0, kCountersN * sizeof(int));
-  if (e == cudaSuccess) e = cudaMemset(c.acounters, 0, kCountersN * sizeof(int));
-  if (e == cudaSuccess) e = cudaMemset(c.status, 0, 64 * sizeof(int));
-  if (e == cudaSuccess) e = cudaMemset(c.df_cnt, 0, (4096 + 64) * sizeof(int));
-  if (e == cudaSuccess) e = cudaMemset(c.zcnt, 0, (c.rows / 128 + 1) * sizeof(int));
-  if (e == cudaSuccess) e = cudaDeviceSynchronize();
-  if (e != cudaSuccess) {
-    free_ctx(c);
-    g_last_cuda_error = (int)e;
-    return e == cudaErrorMemoryAllocation ? FLASHSVD_ERR_NO_MEMORY : FLASHSVD_ERR_CUDA;
-  }
-  g_ctx = c;
+  FSVD_TRY(alloc_ctx(c, device, max_tokens, max_rank, max_hidden, max_ffn));
+  d = c;
   return FLASHSVD_OK;
 }
 
 int flashsvd_shutdown(void) {
   std::lock_guard<std::mutex> lock(g_mu);
-  if (g_ctx.device < 0) return FLASHSVD_OK;
-  cudaSetDevice(g_ctx.device);
+  if (g_default.device < 0) return FLASHSVD_OK;
+  cudaSetDevice(g_default.device);
   cudaDeviceSynchronize();
-  free_ctx(g_ctx);
+  free_ctx(g_default);
+  return FLASHSVD_OK;
+}
+
+struct flashsvd_ctx {
+  Ctx c;
+};
+
+int flashsvd_ctx_create(int device, int max_tokens, int max_rank, int max_hidden, int max_ffn,
+                        flashsvd_ctx** ctx) {
+  if (!ctx || device < 0 || max_tokens <= 0 || max_rank <= 0 || max_hidden <= 0 || max_ffn <= 0)
+    return FLASHSVD_ERR_INVALID_ARG;
+  if (capturing(nullptr)) return FLASHSVD_ERR_CAPTURE_UNSAFE;
+  int prev = -1;
+  FSVD_CUDA(cudaGetDevice(&prev));
+  FSVD_CUDA(cudaSetDevice(device));
+  Ctx c;
+  const int st = alloc_ctx(c, device, max_tokens, max_rank, max_hidden, max_ffn);
+  cudaSetDevice(prev);
+  if (st != FLASHSVD_OK) return st;
+  flashsvd_ctx* out = new flashsvd_ctx();
+  out->c = c;
+  *ctx = out;
+  return FLASHSVD_OK;
+}
+
+int flashsvd_ctx_destroy(flashsvd_ctx* ctx) {
+  if (!ctx) return FLASHSVD_ERR_INVALID_ARG;
+  if (t_ctx == &ctx->c) t_ctx = nullptr;
+  int prev = -1;
+  cudaGetDevice(&prev);
+  cudaSetDevice(ctx->c.device);
+  cudaDeviceSynchronize();
+  free_ctx(ctx->c);
+  if (prev >= 0) cudaSetDevice(prev);
+  delete ctx;
+  return FLASHSVD_OK;
+}
+
+int flashsvd_ctx_bind(flashsvd_ctx* ctx) {
+  if (ctx) FSVD_CUDA(cudaSetDevice(ctx->c.device));
+  t_ctx = ctx ? &ctx->c : nullptr;
   return FLASHSVD_OK;
 }
 
@@ -635,13 +716,13 @@ int flashsvd_check_device_status(flashsvd_stream stream) {
   if (capturing(stream)) return FLASHSVD_ERR_CAPTURE_UNSAFE;
   FSVD_CUDA(cudaStreamSynchronize(stream));
   int word = 0;
-  FSVD_CUDA(cudaMemcpy(&word, g_ctx.status, sizeof(int), cudaMemcpyDeviceToHost));
+  FSVD_CUDA(cudaMemcpy(&word, cur().status, sizeof(int), cudaMemcpyDeviceToHost));
   if (word != DEV_STATUS_OK) {
-    FSVD_CUDA(cudaMemset(g_ctx.status, 0, sizeof(int)));
-    FSVD_CUDA(cudaMemset(g_ctx.df_cnt, 0, (4096 + 64) * sizeof(int)));
-    FSVD_CUDA(cudaMemset(g_ctx.counters, 0, kCountersN * sizeof(int)));
-    FSVD_CUDA(cudaMemset(g_ctx.acounters, 0, kCountersN * sizeof(int)));
-    FSVD_CUDA(cudaMemset(g_ctx.zcnt, 0, (g_ctx.rows / 128 + 1) * sizeof(int)));
+    FSVD_CUDA(cudaMemset(cur().status, 0, sizeof(int)));
+    FSVD_CUDA(cudaMemset(cur().df_cnt, 0, (4096 + 64) * sizeof(int)));
+    FSVD_CUDA(cudaMemset(cur().counters, 0, kCountersN * sizeof(int)));
+    FSVD_CUDA(cudaMemset(cur().acounters, 0, kCountersN * sizeof(int)));
+    FSVD_CUDA(cudaMemset(cur().zcnt, 0, (cur().rows / 128 + 1) * sizeof(int)));
     return word == DEV_STATUS_SCHEDULE ? FLASHSVD_ERR_UNSUPPORTED_SHAPE : FLASHSVD_ERR_TIMEOUT;
   }
   return FLASHSVD_OK;
@@ -657,7 +738,7 @@ int flashsvd_lowrank_linear(const flashsvd_bf16* x, const flashsvd_bf16* U,
   if (M < 0) return FLASHSVD_ERR_INVALID_ARG;
   FSVD_TRY(check_w8(d)); FSVD_TRY(check_w8(r)); FSVD_TRY(check_w8(n));
   if (M == 0) return FLASHSVD_OK;
-  if (M > g_ctx.rows || r > g_ctx.max_rank) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  if (M > cur().rows || r > cur().max_rank) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   if (M <= DECODE_MAX_ROWS)
     return decode_linear((const bf16*)x, (const bf16*)U, (const bf16*)V, (const bf16*)bias,
                          nullptr, (bf16*)y, M, d, r, n, nullptr, 0.f, stream);
@@ -674,7 +755,7 @@ int flashsvd_dense_linear_f32(const flashsvd_bf16* x, const flashsvd_bf16* W,
   if (M < 0) return FLASHSVD_ERR_INVALID_ARG;
   FSVD_TRY(check_w8(d)); FSVD_TRY(check_w8(n));
   if (M == 0) return FLASHSVD_OK;
-  if (M > g_ctx.rows) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  if (M > cur().rows) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   if (M <= DECODE_MAX_ROWS) {
     GvParams p = gv_base();
     p.K = d; p.nprob = 1;
@@ -687,7 +768,7 @@ int flashsvd_dense_linear_f32(const flashsvd_bf16* x, const flashsvd_bf16* W,
   PfLinear p;
   memset(&p, 0, sizeof(p));
   p.x = (const bf16*)x; p.ldx = d; p.V = (const bf16*)W; p.y32 = y; p.ldy = n;
-  p.M = M; p.d = d; p.r = d; p.n = n; p.epi = PF_EPI_F32; p.status = g_ctx.status;
+  p.M = M; p.d = d; p.r = d; p.n = n; p.epi = PF_EPI_F32; p.status = cur().status;
   return prefill_dense_launch(p, stream);
 }
 
@@ -700,7 +781,7 @@ int flashsvd_gateup_swiglu(const flashsvd_bf16* x, const flashsvd_bf16* U_gu,
   if (M < 0) return FLASHSVD_ERR_INVALID_ARG;
   FSVD_TRY(check_w8(d)); FSVD_TRY(check_w8(r_f)); FSVD_TRY(check_w8(f));
   if (M == 0) return FLASHSVD_OK;
-  if (M > g_ctx.rows || r_f > g_ctx.max_rank) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  if (M > cur().rows || r_f > cur().max_rank) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   if (M <= DECODE_MAX_ROWS)
     return decode_gateup((const bf16*)x, (const bf16*)U_gu, (const bf16*)V_gu, (bf16*)h, M, d, r_f, f,
                          nullptr, 0.f, stream);
@@ -720,16 +801,34 @@ int flashsvd_packed_gateup_mlp(const flashsvd_bf16* x,
   FSVD_TRY(need_init());
   FSVD_TRY(check_ptr(U_dn)); FSVD_TRY(check_ptr(V_dn)); FSVD_TRY(check_ptr(y));
   FSVD_TRY(check_w8(r_dn));
-  if (M > 0 && (M > g_ctx.rows || f > g_ctx.max_ffn || r_dn > g_ctx.max_rank))
+  if (M > 0 && (M > cur().rows || f > cur().max_ffn || r_dn > cur().max_rank))
     return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
-  FSVD_TRY(flashsvd_gateup_swiglu(x, U_gu, V_gu, (flashsvd_bf16*)g_ctx.h, M, d, r_f, f, stream));
+  FSVD_TRY(flashsvd_gateup_swiglu(x, U_gu, V_gu, (flashsvd_bf16*)cur().h, M, d, r_f, f, stream));
   if (M == 0) return FLASHSVD_OK;
   if (M <= DECODE_MAX_ROWS)
-    return decode_linear(g_ctx.h, (const bf16*)U_dn, (const bf16*)V_dn, nullptr, nullptr, (bf16*)y,
+    return decode_linear(cur().h, (const bf16*)U_dn, (const bf16*)V_dn, nullptr, nullptr, (bf16*)y,
                          M, f, r_dn, d, nullptr, 0.f, stream);
   flashsvd_factor dn = {U_dn, V_dn, nullptr, r_dn};
-  PfLinear p = pf_base(g_ctx.h, f, dn, M, f, d, (bf16*)y, d);
+  PfLinear p = pf_base(cur().h, f, dn, M, f, d, (bf16*)y, d);
   return prefill_linear_launch(p, stream);
+}
+
+int flashsvd_lowrank_ffn(const flashsvd_bf16* x, const flashsvd_bf16* U_up, const flashsvd_bf16* V_up,
+                         const flashsvd_bf16* b_up, const flashsvd_bf16* U_dn, const flashsvd_bf16* V_dn,
+                         const flashsvd_bf16* b_dn, const flashsvd_bf16* resid, flashsvd_bf16* y, int M,
+                         int d, int r_up, int f, int r_dn, flashsvd_stream stream) {
+  FSVD_TRY(need_init());
+  FSVD_TRY(check_ptr(x)); FSVD_TRY(check_ptr(U_up)); FSVD_TRY(check_ptr(V_up));
+  FSVD_TRY(check_ptr(U_dn)); FSVD_TRY(check_ptr(V_dn)); FSVD_TRY(check_ptr(y));
+  FSVD_TRY(check_opt_ptr(b_up)); FSVD_TRY(check_opt_ptr(b_dn)); FSVD_TRY(check_opt_ptr(resid));
+  if (M < 0) return FLASHSVD_ERR_INVALID_ARG;
+  FSVD_TRY(check_w8(d)); FSVD_TRY(check_w8(r_up)); FSVD_TRY(check_w8(f)); FSVD_TRY(check_w8(r_dn));
+  if (M == 0) return FLASHSVD_OK;
+  if (!ffn_stream_covers(d, r_up, f, r_dn)) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  if (M > cur().rows || (long long)M * r_up > (long long)cur().rows * 2 * cur().max_rank)
+    return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  return lowrank_ffn(cb(x), cb(U_up), cb(V_up), cb(b_up), cb(U_dn), cb(V_dn), cb(b_dn), cb(resid),
+                     (bf16*)y, M, d, r_up, f, r_dn, stream);
 }
 
 int flashsvd_dense_kv_decode_attn(const flashsvd_bf16* q,
@@ -757,7 +856,7 @@ int flashsvd_dense_kv_decode_attn(const flashsvd_bf16* q,
   a.k_cache = (bf16*)k_cache; a.v_cache = (bf16*)v_cache; a.seqlens = cache_seqlens;
   a.out = (bf16*)out; a.B = B; a.H = H; a.D = D; a.S_max = S_max;
   a.scale_log2 = scale * 1.4426950408889634f;
-  a.part = g_ctx.apart; a.counters = g_ctx.acounters;
+  a.part = cur().apart; a.counters = cur().acounters;
   return attn_decode_launch(a, target_ctas(), stream);
 }
 
@@ -776,7 +875,7 @@ int flashsvd_prefill_attn(const flashsvd_bf16* q, const flashsvd_bf16* k_cache,
   a.q = (const bf16*)q; a.k = (const bf16*)k_cache; a.v = (const bf16*)v_cache; a.out = (bf16*)out;
   a.B = B; a.S = S; a.H = H; a.D = D; a.S_max = S_max; a.causal = causal ? 1 : 0;
   a.scale_log2 = scale * 1.4426950408889634f;
-  a.status = g_ctx.status;
+  a.status = cur().status;
   return attn_prefill_launch(a, stream);
 }
 
@@ -844,11 +943,14 @@ int flashsvd_layer_forward(const flashsvd_layer* L, flashsvd_bf16* x_inout,
   if (mode == FLASHSVD_DECODE) {
     if (L->kind != FLASHSVD_DECODER || S != 1 || !cache_seqlens) return FLASHSVD_ERR_INVALID_ARG;
     if (B > DECODE_MAX_ROWS) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
-    if (3 * L->q.r > 3 * g_ctx.max_rank) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+    if (3 * L->q.r > 3 * cur().max_rank) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
     return layer_decode(L, x, kc, vc, cache_seqlens, B, S_max, stream);
   }
   if (S > S_max) return FLASHSVD_ERR_INVALID_ARG;
-  FSVD_TRY(ensure_scratch(B * S, L->d, L->f));
+  {
+    const bool streamed = L->kind == FLASHSVD_ENCODER && ffn_stream_covers(L->d, L->up.r, L->f, L->down.r);
+    FSVD_TRY(ensure_scratch(B * S, L->d, streamed ? 0 : L->f));
+  }
   if (mode == FLASHSVD_PREFILL_CAUSAL) {
     if (L->kind != FLASHSVD_DECODER) return FLASHSVD_ERR_INVALID_ARG;
     return layer_prefill(L, x, kc, vc, B, S, S_max, stream);

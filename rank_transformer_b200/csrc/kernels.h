@@ -107,6 +107,18 @@ int prefill_linear_launch(const PfLinear& p, cudaStream_t stream);
 int prefill_stage1_grouped(const bf16* x, long long ldx, int d, int M, int n, const bf16* const* U,
                            const int* r, bf16* const* z, int* status, cudaStream_t stream);
 int prefill_dense_launch(const PfLinear& p, cudaStream_t stream);
+// Stage 1 of one factorized linear: z [M x r] (row stride r) = x . U, bf16.
+int prefill_stage1(const bf16* x, long long ldx, int d, int M, const bf16* U, int r, bf16* z, int* status,
+                   cudaStream_t stream);
+
+// Streamed low-rank FFN (ffn_stream.cu): y = GELU(z1 . V1 + b1) . U2 . V2 + b2
+// + resid with z1 = x . U1 given [M x r1] (row stride ldz); the [M x f]
+// activation stays on chip.  r1, r2 multiples of 64 in [64, 256]; b1, b2,
+// resid may be null; resid may alias y.
+constexpr int kFfnStreamMaxRank = 256;
+int ffn_stream_launch(const bf16* z1, long long ldz, const bf16* V1, const bf16* b1, const bf16* U2,
+                      const bf16* V2, const bf16* b2, const bf16* resid, bf16* y, int M, int f, int r1,
+                      int r2, int d, int* status, int sms, cudaStream_t stream);
 
 // --------------------------------------------- fused decode layer ---------
 struct DecodeLayerDesc {

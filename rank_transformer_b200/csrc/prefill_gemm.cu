@@ -582,6 +582,16 @@ int prefill_stage1_grouped(const bf16* x, long long ldx, int d, int M, int n, co
                                                "tc_stage1_xu_grouped", stream);
 }
 
+int prefill_stage1(const bf16* x, long long ldx, int d, int M, const bf16* U, int r, bf16* z, int* status,
+                   cudaStream_t stream) {
+  TcArgs a;
+  memset(&a, 0, sizeof(a));
+  a.M = M; a.N = r; a.K = d;
+  a.y = z; a.ldy = r;
+  a.status = status;
+  return gemm(x, ldx, d, U, r, d, a, PF_EPI_BF16, false, "tc_stage1_xu", stream);
+}
+
 int prefill_linear_launch(const PfLinear& p, cudaStream_t stream) {
   if (!p.z) return FLASHSVD_ERR_NOT_INITIALIZED;
   const bool dual = p.epi == PF_EPI_SWIGLU;

@@ -70,6 +70,9 @@ _SIGS = {
     "flashsvd_init": ([_i, _i, _i, _i, _i], _i),
     "flashsvd_shutdown": ([], _i),
     "flashsvd_check_device_status": ([_p], _i),
+    "flashsvd_ctx_create": ([_i, _i, _i, _i, _i, C.POINTER(_p)], _i),
+    "flashsvd_ctx_bind": ([_p], _i),
+    "flashsvd_ctx_destroy": ([_p], _i),
     "flashsvd_launch_count": ([], C.c_int64),
     "flashsvd_set_decode_path": ([_i], _i),
     "flashsvd_decode_pack_bytes": ([_p, C.POINTER(C.c_size_t)], _i),
@@ -84,6 +87,7 @@ _SIGS = {
     "flashsvd_dense_linear_f32": ([_p, _p, _p, _i, _i, _i, _p], _i),
     "flashsvd_packed_gateup_mlp": ([_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p], _i),
     "flashsvd_gateup_swiglu": ([_p, _p, _p, _p, _i, _i, _i, _i, _p], _i),
+    "flashsvd_lowrank_ffn": ([_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p], _i),
     "flashsvd_dense_kv_decode_attn": ([_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _f, _p], _i),
     "flashsvd_prefill_attn": ([_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p], _i),
     "flashsvd_rmsnorm": ([_p, _p, _p, _i, _i, _f, _p], _i),
@@ -141,6 +145,39 @@ def init(device: int = 0, max_tokens: int = 8192, max_rank: int = 4096,
 
 def shutdown() -> None:
     _call("flashsvd_shutdown")
+
+
+class Context:
+    """A workspace of its own (flashsvd_ctx_create).  ``with ctx:`` binds it
+    to the calling thread for the block (flashsvd_ctx_bind) and restores the
+    default context afterwards."""
+
+    def __init__(self, device: int = 0, max_tokens: int = 8192, max_rank: int = 4096,
+                 max_hidden: int = 4096, max_ffn: int = 11008):
+        h = _p()
+        _call("flashsvd_ctx_create", device, max_tokens, max_rank, max_hidden, max_ffn,
+              C.byref(h))
+        self.handle = h.value
+
+    def bind(self) -> None:
+        _call("flashsvd_ctx_bind", self.handle)
+
+    @staticmethod
+    def unbind() -> None:
+        _call("flashsvd_ctx_bind", None)
+
+    def __enter__(self):
+        self.bind()
+        return self
+
+    def __exit__(self, *exc):
+        self.unbind()
+        return False
+
+    def destroy(self) -> None:
+        if self.handle:
+            _call("flashsvd_ctx_destroy", self.handle)
+            self.handle = None
 
 
 def check_device_status(stream=None) -> None:
@@ -213,6 +250,12 @@ def packed_gateup_mlp(x, U_gu, V_gu, U_dn, V_dn, y, M, d, r_f, f, r_dn, stream=N
 def gateup_swiglu(x, U_gu, V_gu, h, M, d, r_f, f, stream=None):
     _call("flashsvd_gateup_swiglu", ptr(x), ptr(U_gu), ptr(V_gu), ptr(h), M, d,
           r_f, f, stream_handle(stream))
+
+
+def lowrank_ffn(x, U_up, V_up, b_up, U_dn, V_dn, b_dn, resid, y, M, d, r_up, f, r_dn,
+                stream=None):
+    _call("flashsvd_lowrank_ffn", ptr(x), ptr(U_up), ptr(V_up), ptr(b_up), ptr(U_dn), ptr(V_dn),
+          ptr(b_dn), ptr(resid), ptr(y), M, d, r_up, f, r_dn, stream_handle(stream))
 
 
 def dense_kv_decode_attn(q, k_new, v_new, k_cache, v_cache, cache_seqlens, out,

@@ -82,6 +82,12 @@ def test_argument_errors_before_any_launch(fs):
     assert L.flashsvd_graph_compose(None, 0, C.byref(h)) == 1
     assert L.flashsvd_init(-1, 1, 1, 1, 1) == 1
     assert L.flashsvd_init(0, 0, 1, 1, 1) == 1
+    # contexts: bad arguments rejected before any allocation
+    assert L.flashsvd_ctx_create(-1, 1, 1, 1, 1, C.byref(h)) == 1
+    assert L.flashsvd_ctx_create(0, 0, 1, 1, 1, C.byref(h)) == 1
+    assert L.flashsvd_ctx_create(0, 1, 1, 1, 1, None) == 1
+    assert L.flashsvd_ctx_destroy(None) == 1
+    assert L.flashsvd_ctx_bind(None) == 0          # back to the default context
 
 
 def test_binding_raises_on_error(fs):

@@ -380,6 +380,24 @@ def pin_bert_layer_closed_form(o):
     _close(o.bert_layer(x, w, H), y, 1e-10)
 
 
+def pin_encoder_ffn(o):
+    # U_up = I, V_up = diag(a), U_dn = V_dn = I: y = GELU(a x + b_up) + b_dn
+    # elementwise, GELU(t) = t Phi(t).  With a rank-3 pair and zero biases,
+    # y = GELU(x (U_up V_up)) (U_dn V_dn) with the products formed first.
+    rng = _rng(15)
+    d = 6
+    I = np.eye(d)
+    a, b_up, b_dn = (rng.standard_normal(d) for _ in range(3))
+    x = rng.standard_normal((4, d))
+    t = a * x + b_up
+    _close(o.lowrank_gelu_ffn(x, I, np.diag(a), b_up, I, I, b_dn), t * norm.cdf(t) + b_dn)
+    f, r = 10, 3
+    U1, V1 = rng.standard_normal((d, r)), rng.standard_normal((r, f))
+    U2, V2 = rng.standard_normal((f, r)), rng.standard_normal((r, d))
+    h = x @ (U1 @ V1)
+    _close(o.lowrank_gelu_ffn(x, U1, V1, None, U2, V2, None), (h * norm.cdf(h)) @ (U2 @ V2), 1e-11)
+
+
 def pin_model_and_head(o):
     # Output head with a square, non-symmetric W (a transposed W changes the
     # result): rows of mean square 1, g = 1, eps = 0 give logits = x W.
@@ -414,7 +432,7 @@ PINS = [pin_lowrank_worked_example, pin_lowrank_associativity,
         pin_layernorm, pin_rope, pin_attention, pin_decode_matches_prefill,
         pin_decoder_layer_special_cases, pin_bert_layer, pin_head_and_greedy,
         pin_from_bf16, pin_decoder_layer_worked_example, pin_decoder_mlp_branch,
-        pin_bert_layer_closed_form, pin_model_and_head]
+        pin_bert_layer_closed_form, pin_model_and_head, pin_encoder_ffn]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
