@@ -42,7 +42,7 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=["decode7b", "linear-sweep", "bert", "mixed-rank",
-                                           "long-decode"],
+                                           "long-decode", "prefill-attn"],
                     default="decode7b",
                     help="decode7b (default): the headline line; the others print one JSON "
                          "line per measured case of the isolated-linear sweep, the BERT-shaped "
@@ -658,6 +658,78 @@ def run_bert(args):
     return 0
 
 
+def run_prefill_attn(args):
+    """Where forming the query inside the attention kernel pays: one
+    Llama-2-7B-shaped decoder layer (hidden 4096, 32 heads of 128, SwiGLU
+    11008 at rank 1792) over a 2048-token prompt, with the attention ranks
+    (q, k, v, o) swept, prefilled with the dense q projection (mode 0) and
+    with the query formed in the attention kernel (mode 1).  Times are CUDA
+    events over 10 layer prefills; the attention and q/k/v second-stage
+    kernels' shares come from the profiler (events around each launch)."""
+    import torch
+    sys.path.insert(0, ROOT)
+    from rank_transformer_b200 import flashsvd as fs
+    from rank_transformer_b200.model import _bf16_normal
+    torch.cuda.set_device(0)
+    d, H, D, f, r_f, S = 4096, 32, 128, 11008, 1792, 2048
+    fs.init(0, max_tokens=S, max_rank=4096, max_hidden=d, max_ffn=f)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(7)
+    stream = torch.cuda.Stream()
+    cos_t = torch.empty((S, D // 2), dtype=torch.float32, device="cuda")
+    sin_t = torch.empty_like(cos_t)
+    fs.rope_table(cos_t, sin_t, S, D, 10000.0)
+    x0 = _bf16_normal((S, d), 1.0, gen, "cuda")
+    kc = torch.zeros((1, S, H, D), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    for r in (128, 256, 512, 832, 1216):
+        w = {}
+        for n in ("q", "k", "v", "o"):
+            w["U_" + n] = _bf16_normal((d, r), d ** -0.5, gen, "cuda")
+            w["V_" + n] = _bf16_normal((r, d), r ** -0.5, gen, "cuda")
+        w["U_gu"] = _bf16_normal((d, 2 * r_f), d ** -0.5, gen, "cuda")
+        w["V_gu"] = _bf16_normal((2 * r_f, f), r_f ** -0.5, gen, "cuda")
+        w["U_dn"] = _bf16_normal((f, r_f), f ** -0.5, gen, "cuda")
+        w["V_dn"] = _bf16_normal((r_f, d), r_f ** -0.5, gen, "cuda")
+        w["g1"] = torch.ones(d, dtype=torch.bfloat16, device="cuda")
+        w["g2"] = torch.ones(d, dtype=torch.bfloat16, device="cuda")
+        L = fs.Layer()
+        L.kind, L.d, L.H, L.D, L.f, L.norm_eps = fs.DECODER, d, H, D, f, 1e-5
+        L.norm1_g, L.norm2_g = w["g1"].data_ptr(), w["g2"].data_ptr()
+        for n in ("q", "k", "v", "o"):
+            F = getattr(L, n)
+            F.U, F.V, F.bias, F.r = w["U_" + n].data_ptr(), w["V_" + n].data_ptr(), None, r
+        L.U_gu, L.V_gu, L.r_f = w["U_gu"].data_ptr(), w["V_gu"].data_ptr(), r_f
+        L.down.U, L.down.V, L.down.bias, L.down.r = w["U_dn"].data_ptr(), w["V_dn"].data_ptr(), None, r_f
+        L.rope_cos, L.rope_sin = cos_t.data_ptr(), sin_t.data_ptr()
+        out = {"workload": "prefill-attn", "layer": "7b-shaped decoder", "S": S, "rank_qkvo": r}
+        for mode in (0, 1):
+            fs.set_prefill_attention(mode)
+            x = x0.clone()
+
+            def one(i):
+                fs.layer_forward(L, x, kc, vc, None, 1, S, S, fs.PREFILL_CAUSAL, stream)
+            with torch.cuda.stream(stream):
+                for i in range(3):
+                    one(i)
+                ms = _event_ms(one, 10, stream)
+                fs.profile_enable(True)
+                one(0)
+                prof = fs.profile_report(reset=True)
+                fs.profile_enable(False)
+            fs.check_device_status(stream)
+            key = "factorized_q" if mode else "dense_q"
+            out[key] = {"layer_ms": round(ms, 4),
+                        "attention_ms": round(sum(v["ms"] for k, v in prof.items()
+                                                  if k.startswith("attn_prefill")), 4),
+                        "qkv_stage2_ms": round(prof.get("tc_stage2_qkv_rope", {}).get("ms", 0.0), 4)}
+        fs.set_prefill_attention(0)
+        out["factorized_faster"] = out["factorized_q"]["layer_ms"] < out["dense_q"]["layer_ms"]
+        print(json.dumps(out), flush=True)
+        del w
+    return 0
+
+
 def run_mixed(args):
     """Same 7B-shaped model with one retention ratio per layer drawn from
     {0.4, 0.6, 0.8}: prefill B=4 x 2048 (tcgen05 path), then 256 greedy
@@ -784,6 +856,8 @@ def main():
         return run_mixed(args)
     if args.workload == "long-decode":
         return run_long_decode(args)
+    if args.workload == "prefill-attn":
+        return run_prefill_attn(args)
     return run_ours(args)
 
 

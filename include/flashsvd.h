@@ -131,6 +131,19 @@ FLASHSVD_API int flashsvd_check_device_status(flashsvd_stream stream);
  * launch per stage.  Both give the same result within rounding. */
 FLASHSVD_API int flashsvd_set_decode_path(int fused);
 
+/* Prefill attention of DECODER layers (PREFILL_CAUSAL): mode 1 forms each
+ * query tile inside the attention kernel from the query's rank activation
+ * (flashsvd_prefill_attn_factorized: dense q never exists); mode 0, the
+ * default, runs the query's second-stage projection (dense q, RoPE in its
+ * epilogue) and the plain prefill attention.  Both give the same result
+ * within rounding.  Mode 0 is the faster one on B200 at every query rank
+ * measured (128 to 1216, 7B-shaped layer, 2048 tokens): in mode 1 each
+ * (query tile, head) item first waits for its own query tile (the operands
+ * of z_q V_q through the kernel's two-stage ring, the product, then RoPE),
+ * which the plain kernel loads ahead while the previous item finishes.
+ * Other modes return FLASHSVD_ERR_INVALID_ARG. */
+FLASHSVD_API int flashsvd_set_prefill_attention(int mode);
+
 /* Number of kernels this library has launched since load: eager launches
  * plus the kernel nodes of every replayed graph. */
 FLASHSVD_API int64_t flashsvd_launch_count(void);
@@ -248,6 +261,26 @@ FLASHSVD_API int flashsvd_prefill_attn(const flashsvd_bf16* q, const flashsvd_bf
                           const flashsvd_bf16* v_cache, flashsvd_bf16* out,
                           int B, int S, int H, int D, int S_max, int causal,
                           float scale, flashsvd_stream stream);
+
+/* Factorized prefill attention, [v1.5] Methodology 2, "Prefill" (prefill
+ * keeps a dedicated factorized attention kernel so that dense activations
+ * are not materialised): the query of every row is formed inside the
+ * kernel from the rank activation of the query projection,
+ *   q[b, s, h] = rope(z_q[b*S + s] . V_q[:, h*D .. h*D + D), position s),
+ *   out[b, s, h] = softmax(q . K[b, 0..S)^T * scale (causal: keys <= s)) . V
+ * so dense q is neither written nor read.  z_q [B*S x r] bf16 (row stride
+ * r), V_q [r x H*D], rotary tables [>= S x D/2] fp32 (flashsvd_rope_table),
+ * keys and values rows 0..S-1 of k_cache / v_cache [B, S_max, H, D]; out
+ * [B, S, H, D].  r a multiple of 64, D in {64, 128}.  With
+ * flashsvd_set_prefill_attention(1) the DECODER layer's PREFILL_CAUSAL mode
+ * uses it with the z_q of its q/k/v stage 1 (and drops that z_q from L2
+ * after its last head has read it). */
+FLASHSVD_API int flashsvd_prefill_attn_factorized(const flashsvd_bf16* z_q, const flashsvd_bf16* V_q,
+                                                  const float* rope_cos, const float* rope_sin,
+                                                  const flashsvd_bf16* k_cache,
+                                                  const flashsvd_bf16* v_cache, flashsvd_bf16* out,
+                                                  int B, int S, int H, int D, int S_max, int r,
+                                                  int causal, float scale, flashsvd_stream stream);
 
 /* --------------------------------------------------------------- glue ----
  * RMSNorm y = x * g / sqrt(mean(x^2) + eps); LayerNorm

@@ -35,6 +35,7 @@ struct Ctx {
   float* df_part = nullptr;    // fused decode: per-CTA partial slots
   int* df_cnt = nullptr;       // fused decode: tile counters, stage barriers, done counter
   int* zcnt = nullptr;         // prefill: per 128-row block counters of the z discard
+  long long zcnt_elems = 0;
   int rows = 0;                // rows of the scratch above
 };
 
@@ -83,13 +84,16 @@ int alloc_ctx(Ctx& c, int device, int max_tokens, int max_rank, int max_hidden, 
   FSVD_ALLOC(c.zb, (size_t)c.rows * 2 * max_rank * sizeof(bf16));
   FSVD_ALLOC(c.df_part, (size_t)kFusedPartFloats * sizeof(float));
   FSVD_ALLOC(c.df_cnt, (size_t)(4096 + 64) * sizeof(int));
-  FSVD_ALLOC(c.zcnt, (size_t)(c.rows / 128 + 1) * sizeof(int));
+  // (the factorized attention counts per batch row and query tile: at most
+  // rows / 128 + batch rows of them)
+  c.zcnt_elems = (long long)(c.rows / 128 + 1) + (c.rows < (1 << 16) ? c.rows : (1 << 16));
+  FSVD_ALLOC(c.zcnt, (size_t)c.zcnt_elems * sizeof(int));
 #undef FSVD_ALLOC
   if (e == cudaSuccess) e = cudaMemset(c.counters, 0, kCountersN * sizeof(int));
   if (e == cudaSuccess) e = cudaMemset(c.acounters, 0, kCountersN * sizeof(int));
   if (e == cudaSuccess) e = cudaMemset(c.status, 0, 64 * sizeof(int));
   if (e == cudaSuccess) e = cudaMemset(c.df_cnt, 0, (4096 + 64) * sizeof(int));
-  if (e == cudaSuccess) e = cudaMemset(c.zcnt, 0, (c.rows / 128 + 1) * sizeof(int));
+  if (e == cudaSuccess) e = cudaMemset(c.zcnt, 0, (size_t)c.zcnt_elems * sizeof(int));
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
     free_ctx(c);
@@ -297,6 +301,10 @@ bool qkv_stage1_grouped(const bf16* x, int d, int M, const flashsvd_factor* cons
 }
 
 bool g_fused_decode = true;
+// Prefill attention of decoder layers: query formed inside the attention
+// kernel (1) or from the dense q projection (0, the default: measured faster
+// at every query rank from 128 to 1216 on the 7B-shaped layer).
+int g_prefill_qf = 0;
 
 // Whether the fused decode layer (and hence a decode pack) covers L's shapes.
 bool pack_shapes_ok(const flashsvd_layer* L) {
@@ -387,7 +395,12 @@ int layer_prefill(const flashsvd_layer* L, bf16* x, bf16* kc, bf16* vc,
   int gst = FLASHSVD_OK;
   const bool grouped = qkv_stage1_grouped(cur().xn, d, M, F, zg, s, &gst);
   FSVD_TRY(gst);
-  for (int i = 0; i < 3; ++i) {
+  // Factorized attention ([v1.5] Methodology 2, "Prefill"): with z_q kept
+  // from the grouped stage 1, the attention kernel forms q = rope(z_q V_q)
+  // itself, so q's stage 2 is not run and dense q is never materialised.
+  // k and v still go through stage 2: decode reads them from the cache.
+  const bool fact_q = grouped && L->q.r % 64 == 0 && g_prefill_qf == 1;
+  for (int i = fact_q ? 1 : 0; i < 3; ++i) {
     PfLinear p = pf_base(cur().xn, d, *F[i], M, d, d, cur().q, d);
     if (grouped) { p.z = zg[i]; p.z_ready = 1; }
     p.epi = PF_EPI_QKV; p.kind = i; p.cache = dst[i]; p.S = S; p.S_max = S_max;
@@ -397,10 +410,17 @@ int layer_prefill(const flashsvd_layer* L, bf16* x, bf16* kc, bf16* vc,
   }
   AttnPfParams a;
   memset(&a, 0, sizeof(a));
-  a.q = cur().q; a.k = kc; a.v = vc; a.out = cur().att;
+  a.k = kc; a.v = vc; a.out = cur().att;
   a.B = B; a.S = S; a.H = L->H; a.D = L->D; a.S_max = S_max; a.causal = 1;
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)L->D);
   a.status = cur().status;
+  if (fact_q) {
+    a.zq = zg[0]; a.ldz = L->q.r; a.r = L->q.r; a.Vq = cb(L->q.V);
+    a.rope_cos = L->rope_cos; a.rope_sin = L->rope_sin;
+    a.zcnt = cur().zcnt; a.zcnt_cap = cur().zcnt_elems;
+  } else {
+    a.q = cur().q;
+  }
   FSVD_TRY(attn_prefill_launch(a, s));
   {
     PfLinear p = pf_base(cur().att, d, L->o, M, d, d, x, d);
@@ -549,6 +569,12 @@ const char* flashsvd_status_string(int status) {
 
 int flashsvd_last_cuda_error(void) { return g_last_cuda_error; }
 int flashsvd_version(void) { return 100; }
+
+int flashsvd_set_prefill_attention(int mode) {
+  if (mode < 0 || mode > 1) return FLASHSVD_ERR_INVALID_ARG;
+  g_prefill_qf = mode;
+  return FLASHSVD_OK;
+}
 
 int flashsvd_set_decode_path(int fused) {
   g_fused_decode = fused != 0;
@@ -722,7 +748,7 @@ int flashsvd_check_device_status(flashsvd_stream stream) {
     FSVD_CUDA(cudaMemset(cur().df_cnt, 0, (4096 + 64) * sizeof(int)));
     FSVD_CUDA(cudaMemset(cur().counters, 0, kCountersN * sizeof(int)));
     FSVD_CUDA(cudaMemset(cur().acounters, 0, kCountersN * sizeof(int)));
-    FSVD_CUDA(cudaMemset(cur().zcnt, 0, (cur().rows / 128 + 1) * sizeof(int)));
+    FSVD_CUDA(cudaMemset(cur().zcnt, 0, (size_t)cur().zcnt_elems * sizeof(int)));
     return word == DEV_STATUS_SCHEDULE ? FLASHSVD_ERR_UNSUPPORTED_SHAPE : FLASHSVD_ERR_TIMEOUT;
   }
   return FLASHSVD_OK;
@@ -876,6 +902,30 @@ int flashsvd_prefill_attn(const flashsvd_bf16* q, const flashsvd_bf16* k_cache,
   a.B = B; a.S = S; a.H = H; a.D = D; a.S_max = S_max; a.causal = causal ? 1 : 0;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.status = cur().status;
+  return attn_prefill_launch(a, stream);
+}
+
+int flashsvd_prefill_attn_factorized(const flashsvd_bf16* z_q, const flashsvd_bf16* V_q,
+                                     const float* rope_cos, const float* rope_sin,
+                                     const flashsvd_bf16* k_cache, const flashsvd_bf16* v_cache,
+                                     flashsvd_bf16* out, int B, int S, int H, int D, int S_max, int r,
+                                     int causal, float scale, flashsvd_stream stream) {
+  FSVD_TRY(need_init());
+  FSVD_TRY(check_ptr(z_q)); FSVD_TRY(check_ptr(V_q)); FSVD_TRY(check_ptr(k_cache));
+  FSVD_TRY(check_ptr(v_cache)); FSVD_TRY(check_ptr(out));
+  FSVD_TRY(check_ptr(rope_cos)); FSVD_TRY(check_ptr(rope_sin));
+  if (B < 0 || S < 0 || H <= 0 || r <= 0 || S_max < S || !(scale > 0.f)) return FLASHSVD_ERR_INVALID_ARG;
+  if ((D != 64 && D != 128) || r % 64) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0 || S == 0) return FLASHSVD_OK;
+  AttnPfParams a;
+  memset(&a, 0, sizeof(a));
+  a.k = (const bf16*)k_cache; a.v = (const bf16*)v_cache; a.out = (bf16*)out;
+  a.B = B; a.S = S; a.H = H; a.D = D; a.S_max = S_max; a.causal = causal ? 1 : 0;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.status = cur().status;
+  a.zq = (const bf16*)z_q; a.ldz = r; a.r = r; a.Vq = (const bf16*)V_q;
+  a.rope_cos = rope_cos; a.rope_sin = rope_sin;
+  // the caller's z_q is an input: it is not discarded from L2
   return attn_prefill_launch(a, stream);
 }
 

@@ -157,6 +157,14 @@ struct AttnPfParams {
   int B, S, H, D, S_max, causal;
   float scale_log2;
   int* status;       // device status word (bounded waits)
+  // Factorized query (zq non-null; q unused): q = rope(z_q V_q) is formed in
+  // the kernel from z_q [B*S x r] (row stride ldz) and V_q [r x H*D], with
+  // the rotary tables [S x D/2] at positions 0..S-1; r a multiple of 64.
+  // zcnt: zero counters (zcnt_cap of them) for discarding z_q from L2 after
+  // use, or null.
+  const bf16* zq; long long ldz; int r; const bf16* Vq;
+  const float* rope_cos; const float* rope_sin;
+  int* zcnt; long long zcnt_cap;
 };
 int attn_prefill_launch(const AttnPfParams& p, cudaStream_t stream);
 

@@ -75,6 +75,7 @@ _SIGS = {
     "flashsvd_ctx_destroy": ([_p], _i),
     "flashsvd_launch_count": ([], C.c_int64),
     "flashsvd_set_decode_path": ([_i], _i),
+    "flashsvd_set_prefill_attention": ([_i], _i),
     "flashsvd_decode_pack_bytes": ([_p, C.POINTER(C.c_size_t)], _i),
     "flashsvd_decode_pack": ([_p, _p, C.c_size_t, _p], _i),
     "flashsvd_decode_plan_create": ([_p, _i, _p, _p, _i, _i, _p], _i),
@@ -90,6 +91,8 @@ _SIGS = {
     "flashsvd_lowrank_ffn": ([_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p], _i),
     "flashsvd_dense_kv_decode_attn": ([_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _f, _p], _i),
     "flashsvd_prefill_attn": ([_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p], _i),
+    "flashsvd_prefill_attn_factorized": ([_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i,
+                                          _f, _p], _i),
     "flashsvd_rmsnorm": ([_p, _p, _p, _i, _i, _f, _p], _i),
     "flashsvd_layernorm": ([_p, _p, _p, _p, _i, _i, _f, _p], _i),
     "flashsvd_rope_table": ([_p, _p, _i, _i, _f, _p], _i),
@@ -184,6 +187,12 @@ def check_device_status(stream=None) -> None:
     _call("flashsvd_check_device_status", stream_handle(stream))
 
 
+def set_prefill_attention(mode: int) -> None:
+    """1: query formed inside the attention kernel; 0: dense q projection
+    (the default)."""
+    _call("flashsvd_set_prefill_attention", mode)
+
+
 def set_decode_path(fused: bool) -> None:
     _call("flashsvd_set_decode_path", int(fused))
 
@@ -269,6 +278,13 @@ def prefill_attn(q, k_cache, v_cache, out, B, S, H, D, S_max, causal, scale,
                  stream=None):
     _call("flashsvd_prefill_attn", ptr(q), ptr(k_cache), ptr(v_cache), ptr(out),
           B, S, H, D, S_max, int(causal), scale, stream_handle(stream))
+
+
+def prefill_attn_factorized(z_q, V_q, rope_cos, rope_sin, k_cache, v_cache, out, B, S, H, D,
+                            S_max, r, causal, scale, stream=None):
+    _call("flashsvd_prefill_attn_factorized", ptr(z_q), ptr(V_q), ptr(rope_cos), ptr(rope_sin),
+          ptr(k_cache), ptr(v_cache), ptr(out), B, S, H, D, S_max, r, int(causal), scale,
+          stream_handle(stream))
 
 
 def rmsnorm(x, g, y, M, d, eps, stream=None):

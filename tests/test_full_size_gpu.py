@@ -206,9 +206,12 @@ def test_prefill_attention_2048_causal(fs):
         assert_parity(got[0, :, h], ref, f"causal attention S=2048 h={h}")
 
 
-def test_decoder_prefill_layer_7b_512(fs):
+@pytest.mark.parametrize("qf", [0, 1])
+def test_decoder_prefill_layer_7b_512(fs, qf):
     """One Llama-2-7B-shaped low-rank decoder layer (ranks 1216 / 1792)
-    over a 512-token prompt: output rows and the cache rows it writes."""
+    over a 512-token prompt: output rows and the cache rows it writes, with
+    the query projected densely (0) or formed inside the attention kernel
+    (1)."""
     from tests.test_decode_gpu import _layer_struct
     d, H, D, f, r, r_f, S = 4096, 32, 128, 11008, 1216, 1792, 512
     rng = synth.rng_for(7200)
@@ -221,11 +224,15 @@ def test_decoder_prefill_layer_7b_512(fs):
     x = dev_bf16(xs)
     kc = torch.zeros((1, S, H, D), dtype=torch.bfloat16, device="cuda")
     vc = torch.zeros_like(kc)
-    fs.layer_forward(L, x, kc, vc, None, 1, S, S, fs.PREFILL_CAUSAL)
-    torch.cuda.synchronize()
+    fs.set_prefill_attention(qf)
+    try:
+        fs.layer_forward(L, x, kc, vc, None, 1, S, S, fs.PREFILL_CAUSAL)
+        torch.cuda.synchronize()
+    finally:
+        fs.set_prefill_attention(0)
     fs.check_device_status()
     y, k, v = oracle.decoder_layer_prefill(oracle.from_bf16(xs), oracle.widen_layer(w), H)
-    assert_parity(host_f64(x), y, "7B prefill layer S=512")
+    assert_parity(host_f64(x), y, f"7B prefill layer S=512 qf={qf}")
     assert_parity(host_f64(kc)[0], k, "7B prefill k cache")
     assert_parity(host_f64(vc)[0], v, "7B prefill v cache")
 
