@@ -42,7 +42,7 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=["decode7b", "linear-sweep", "bert", "mixed-rank",
-                                           "long-decode", "prefill-attn"],
+                                           "long-decode", "prefill-attn", "retention", "shared-basis"],
                     default="decode7b",
                     help="decode7b (default): the headline line; the others print one JSON "
                          "line per measured case of the isolated-linear sweep, the BERT-shaped "
@@ -730,6 +730,185 @@ def run_prefill_attn(args):
     return 0
 
 
+def _dense_decode_step(B, ctx, device, gen):
+    """A dense Llama-2-7B-shaped decode step in plain PyTorch (the reference
+    point of the retention curve): 32 pre-norm layers with dense bf16
+    q/k/v/o [4096 x 4096], gate/up [4096 x 11008] and down [11008 x 4096]
+    (cuBLAS), RoPE-free attention by scaled_dot_product_attention over a
+    fixed 'ctx'-key bf16 cache, the 4096 x 32000 head and an argmax; the
+    whole step captured as one CUDA graph.  Returns (graph, weight bytes,
+    cache bytes read per step)."""
+    import torch
+    import torch.nn.functional as F
+    d, H, D, f, V, nl = 4096, 32, 128, 11008, 32000, 32
+
+    def w(*shape):
+        return (torch.randn(*shape, device=device, generator=gen) * shape[0] ** -0.5).to(torch.bfloat16)
+    layers = [dict(qkv=w(d, 3 * d), o=w(d, d), gu=w(d, 2 * f), dn=w(f, d)) for _ in range(nl)]
+    kc = [torch.randn(B, H, ctx, D, device=device, generator=gen).to(torch.bfloat16) for _ in range(nl)]
+    vc = [torch.randn(B, H, ctx, D, device=device, generator=gen).to(torch.bfloat16) for _ in range(nl)]
+    W_lm = w(d, V)
+    x = torch.randn(B, d, device=device, generator=gen).to(torch.bfloat16)
+    tok = torch.zeros(B, dtype=torch.int64, device=device)
+
+    def step():
+        h = x
+        for L, k_, v_ in zip(layers, kc, vc):
+            n = F.rms_norm(h, (d,))
+            q, _, _ = (n @ L["qkv"]).split(d, dim=1)
+            a = F.scaled_dot_product_attention(q.view(B, H, 1, D), k_, v_).reshape(B, d)
+            h = h + a @ L["o"]
+            g, u = (F.rms_norm(h, (d,)) @ L["gu"]).split(f, dim=1)
+            h = h + (F.silu(g) * u) @ L["dn"]
+        tok.copy_(torch.argmax(F.rms_norm(h, (d,)) @ W_lm, dim=1))
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(2):
+            step()
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    wbytes = 2 * (nl * (3 * d * d + d * d + 2 * d * f + f * d) + d * V)
+    return g, wbytes, 2 * 2 * nl * B * ctx * d
+
+
+def run_retention(args):
+    """Decode speed against retention (FlashSVD v1.5 explainer, Results,
+    Robustness: speedups shrink as the model approaches dense): the
+    Llama-2-7B-shaped low-rank decoder at retention 0.2 / 0.4 / 0.6 / 0.8
+    (ranks by parameter retention), B = 1, contexts 2048 and 8192 (caches of
+    random history), 64 graph-replayed decode steps per point, beside a
+    dense decode step of the same shapes in plain PyTorch (cuBLAS GEMVs,
+    scaled_dot_product_attention, CUDA graph) at the same context.  Each
+    point also gives its fraction of the HBM roofline (algorithmic bytes:
+    factors or dense weights, head, K/V history)."""
+    import dataclasses
+    import torch
+    sys.path.insert(0, ROOT)
+    from rank_transformer_b200 import flashsvd as fs
+    from rank_transformer_b200.model import LLAMA7B, DecoderModel
+    torch.cuda.set_device(0)
+    peaks = measured_peaks()
+    fs.init(0, max_tokens=256, max_rank=4096, max_hidden=4096, max_ffn=11008)
+    stream = torch.cuda.Stream()
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(51)
+    steps = 64
+    for ctx in (2048, 8192):
+        g, wb, kvb = _dense_decode_step(1, ctx, "cuda", gen)
+        for _ in range(3):
+            g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            g.replay()
+        e1.record()
+        e1.synchronize()
+        dense_ms = e0.elapsed_time(e1) / steps
+        dense_gbs = (wb + kvb) / (dense_ms / 1e3) / 1e9
+        del g
+        torch.cuda.empty_cache()
+        print(json.dumps({"workload": "retention", "model": "dense (torch, cuBLAS, CUDA graph)",
+                          "context": ctx, "ms_per_step": round(dense_ms, 4),
+                          "tok_s": round(1e3 / dense_ms, 1), "weight_bytes": wb,
+                          "frac_of_hbm": round(dense_gbs / peaks["hbm_gbs"], 3)}), flush=True)
+        for rho in (0.2, 0.4, 0.6, 0.8):
+            cfg = dataclasses.replace(LLAMA7B, rho=(rho,))
+            m = DecoderModel(cfg, 1, ctx + steps + 8, seed=61)
+            with torch.cuda.stream(stream):
+                for kc_, vc_ in zip(m.k_cache, m.v_cache):
+                    kc_.normal_(generator=gen)
+                    vc_.normal_(generator=gen)
+            m.capture(stream)
+            with torch.cuda.stream(stream):
+                m.seqlens.fill_(ctx)
+                for _ in range(3):
+                    m.decode_step(stream)
+                m.seqlens.fill_(ctx)
+                ms = _event_ms(lambda i: m.decode_step(stream), steps, stream)
+            fs.check_device_status(stream)
+            byts = m.decode_step_bytes(ctx + steps // 2)
+            r_a, r_f = cfg.ranks(0)
+            print(json.dumps({
+                "workload": "retention", "rho": rho, "ranks": [r_a, r_f], "context": ctx,
+                "ms_per_step": round(ms, 4), "tok_s": round(1e3 / ms, 1),
+                "speedup_vs_dense": round(dense_ms / ms, 3),
+                "frac_of_hbm": round(byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 3),
+                "decode_path": "decode plan" if m.plan is not None else "per-stage"}), flush=True)
+            m.release_graphs()
+            del m
+            torch.cuda.empty_cache()
+    return 0
+
+
+def run_shared_basis(args):
+    """Shared bases (FlashSVD v1.5 explainer, Methodology 1, Basis Sharing:
+    one physical copy of a basis used by several layers): the
+    Llama-2-7B-shaped low-rank decoder (retention 0.6) whose input-side
+    factors U_q, U_k, U_v, U_o, U_gu, U_dn are shared by groups of 1 (no
+    sharing), 4 and 32 consecutive layers.  The decode plan reads a shared
+    factor from one pack with an L2 evict-last hint, so after the group's
+    first layer it comes from L2.  B = 1, context 2048, 64 graph-replayed
+    steps; algorithmic bytes count a shared factor once per step."""
+    import dataclasses
+    import torch
+    sys.path.insert(0, ROOT)
+    from rank_transformer_b200 import flashsvd as fs
+    from rank_transformer_b200.model import LLAMA7B, DecoderModel, _bf16_normal
+    torch.cuda.set_device(0)
+    peaks = measured_peaks()
+    cfg = LLAMA7B
+    fs.init(0, max_tokens=256, max_rank=2368, max_hidden=cfg.d, max_ffn=cfg.f)
+    stream = torch.cuda.Stream()
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(71)
+    ctx, steps = 2048, 64
+    d, f = cfg.d, cfg.f
+    r_a, r_f = cfg.ranks(0)
+    shapes = {"U_q": (d, r_a), "U_k": (d, r_a), "U_v": (d, r_a), "U_o": (d, r_a),
+              "U_gu": (d, 2 * r_f), "U_dn": (f, r_f)}
+    for group in (1, 4, 32):
+        layers, base = [], None
+        for i in range(cfg.layers):
+            w = {}
+            if i % group == 0:
+                base = {k: _bf16_normal(sh, sh[0] ** -0.5, gen, "cuda") for k, sh in shapes.items()}
+            w.update(base)
+            for n in ("q", "k", "v", "o"):
+                w["V_" + n] = _bf16_normal((r_a, d), r_a ** -0.5, gen, "cuda")
+            w["V_gu"] = _bf16_normal((2 * r_f, f), r_f ** -0.5, gen, "cuda")
+            w["V_dn"] = _bf16_normal((r_f, d), r_f ** -0.5, gen, "cuda")
+            w["g1"] = torch.ones(d, dtype=torch.bfloat16, device="cuda")
+            w["g2"] = torch.ones(d, dtype=torch.bfloat16, device="cuda")
+            layers.append(w)
+        m = DecoderModel(cfg, 1, ctx + steps + 8, seed=72, weights=layers)
+        with torch.cuda.stream(stream):
+            for kc_, vc_ in zip(m.k_cache, m.v_cache):
+                kc_.normal_(generator=gen)
+                vc_.normal_(generator=gen)
+        m.capture(stream)
+        with torch.cuda.stream(stream):
+            m.seqlens.fill_(ctx)
+            for _ in range(3):
+                m.decode_step(stream)
+            m.seqlens.fill_(ctx)
+            ms = _event_ms(lambda i: m.decode_step(stream), steps, stream)
+        fs.check_device_status(stream)
+        byts = m.decode_step_bytes(ctx + steps // 2)
+        print(json.dumps({
+            "workload": "shared-basis", "layers_per_shared_basis": group, "context": ctx,
+            "ms_per_step": round(ms, 4), "tok_s": round(1e3 / ms, 1),
+            "algorithmic_bytes_per_step": int(byts),
+            "frac_of_hbm": round(byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 3),
+            "decode_path": "decode plan" if m.plan is not None else "per-stage"}), flush=True)
+        m.release_graphs()
+        del m, layers, base
+        torch.cuda.empty_cache()
+    return 0
+
+
 def run_mixed(args):
     """Same 7B-shaped model with one retention ratio per layer drawn from
     {0.4, 0.6, 0.8}: prefill B=4 x 2048 (tcgen05 path), then 256 greedy
@@ -858,6 +1037,10 @@ def main():
         return run_long_decode(args)
     if args.workload == "prefill-attn":
         return run_prefill_attn(args)
+    if args.workload == "retention":
+        return run_retention(args)
+    if args.workload == "shared-basis":
+        return run_shared_basis(args)
     return run_ours(args)
 
 

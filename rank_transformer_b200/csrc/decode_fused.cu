@@ -110,8 +110,11 @@ struct DfPhase {
   int T, K, nk;
   int N[3];
   int a_col2;          // SwiGLU stage: offset of the up half in the previous output
-  long long pack_off;  // byte offset of this stage's entries in the pack
+  long long pack_off;  // byte offset of this stage's entries from the layer's pack
+                       // (a shared factor's entries live in an earlier layer's pack)
   const bf16* norm_g;
+  int shared;          // entries read by several layers: loaded with an L2 evict-last hint
+  int pad_[3];
 };
 
 // Per (stage, CTA) schedule record, built on the host with the pack: the
@@ -170,7 +173,7 @@ struct DfCfg {
   static constexpr int SCR_BYTES = (64 + CW * 128) * 4;
   static constexpr int MISC_BYTES = 6656;  // two schedule records, rstd, attention schedule
   static constexpr int BAR_BYTES = 512;
-  static constexpr int PH_BYTES = 2 * 768;  // two copies of a layer's record tail (stage table)
+  static constexpr int PH_BYTES = 2 * 896;  // two copies of a layer's record tail (stage table)
   static constexpr int SMEM = 1024 + NSLOT * SLOT + ABUF_BYTES + RED_BYTES + SCR_BYTES + MISC_BYTES +
                               BAR_BYTES + PH_BYTES;
   static_assert(SMEM <= 232448, "shared memory budget");
@@ -180,6 +183,25 @@ template <int N>
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(N) : "memory"); }
 __device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+// Bulk copies and L2 prefetches with an L2 cache policy (evict-last for
+// factors that several layers read: shared bases).
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void prefetch_l2_bulk_hint(const void* src, uint32_t bytes, uint64_t pol) {
+  asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;" ::"l"(src), "r"(bytes), "l"(pol)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                              uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          tc::smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(tc::smem_u32(bar)), "l"(pol)
+      : "memory");
 }
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
@@ -580,6 +602,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
     if (lane == 0) {
       // L2 prefetch cursor (layer, stage, entry), PF pack entries ahead
       constexpr int PF = 2;
+      const uint64_t pol_last = policy_evict_last();
       int pf_l = 0, pf_s = -1, pf_c = 0, pf_c1 = 0;
       auto pf_step = [&]() {
         while (pf_c >= pf_c1) {
@@ -596,8 +619,11 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
         const DfPhase& q = Lq->ph[pf_s];
         const int t = pf_c / q.nk, kc = pf_c - t * q.nk;
         const int kn = min(DF_KC, q.K - kc * DF_KC);
-        prefetch_l2_bulk(Lq->pack + q.pack_off + (long long)t * q.K * 128 + (long long)kc * 32768,
-                         (uint32_t)kn * 128u);
+        const uint8_t* pe = Lq->pack + q.pack_off + (long long)t * q.K * 128 + (long long)kc * 32768;
+        if (q.shared)
+          prefetch_l2_bulk_hint(pe, (uint32_t)kn * 128u, pol_last);
+        else
+          prefetch_l2_bulk(pe, (uint32_t)kn * 128u);
         ++pf_c;
       };
       for (int i = 0; i < PF; ++i) pf_step();
@@ -662,7 +688,10 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
             const uint32_t bytes = (uint32_t)min(DF_KC, ph.K - kc * DF_KC) * 128u;
             const uint8_t* e = Ly->pack + ph.pack_off + (long long)t * ph.K * 128 + (long long)kc * 32768;
             tc::mbar_expect_tx(full + slot, bytes);
-            bulk_g2s(slots + slot * C::SLOT, e, bytes, full + slot);
+            if (ph.shared)
+              bulk_g2s_hint(slots + slot * C::SLOT, e, bytes, full + slot, pol_last);
+            else
+              bulk_g2s(slots + slot * C::SLOT, e, bytes, full + slot);
             pf_step();
           }
         }
@@ -1673,6 +1702,33 @@ int decode_plan_create(const DecodeLayerDesc* layers, int n, bf16* const* k_cach
     long long b = 0;
     FSVD_TRY(fill_layer(L, k_caches[i], v_caches[i], B, S_max, G, &host[i], &b));
     bytes += (double)b;
+  }
+  // Shared bases ([v1.5] Methodology 1, Basis Sharing): a U stage whose
+  // factor pointers equal those of an earlier layer (same stage shape)
+  // reads that layer's pack entries, so every layer of the plan streams the
+  // same bytes, which an L2 evict-last hint keeps on chip after the first;
+  // their bytes count once per step.
+  for (int i = 1; i < n; ++i) {
+    const int ustage[4] = {0, 3, 5, 7};
+    for (int u = 0; u < 4; ++u) {
+      const int st = ustage[u];
+      for (int j = 0; j < i; ++j) {
+        const DecodeLayerDesc &A = layers[i], &Bj = layers[j];
+        bool same = false;
+        if (st == 0) same = A.U[0] == Bj.U[0] && A.U[1] == Bj.U[1] && A.U[2] == Bj.U[2] && A.r == Bj.r;
+        if (st == 3) same = A.U_o == Bj.U_o && A.r == Bj.r;
+        if (st == 5) same = A.U_gu == Bj.U_gu && A.r_f == Bj.r_f;
+        if (st == 7) same = A.U_dn == Bj.U_dn && A.r_f == Bj.r_f;
+        const DfPhase &pi = host[i].ph[st], &pj = host[j].ph[st];
+        if (!same || pi.K != pj.K || pi.nk != pj.nk || pi.T != pj.T || pi.nprob != pj.nprob) continue;
+        // pj.pack_off is relative to layer j's pack (itself maybe shared)
+        host[i].ph[st].pack_off = (long long)((host[j].pack + pj.pack_off) - host[i].pack);
+        host[i].ph[st].shared = 1;
+        host[j].ph[st].shared = 1;
+        bytes -= 2.0 * (double)pi.K * (pi.T * 64);
+        break;
+      }
+    }
   }
   DecodePlan* plan = new DecodePlan();
   if (cudaMalloc(&plan->dev, sizeof(DfLayer) * n) != cudaSuccess) {

@@ -149,9 +149,19 @@ class DecoderModel:
         L.rope_cos, L.rope_sin = self.rope_cos.data_ptr(), self.rope_sin.data_ptr()
         return L
 
+    def _unique_params(self) -> int:
+        """Elements of the layers' weights, a tensor shared by several
+        layers (shared bases) counted once."""
+        seen, n = set(), 0
+        for w in self.layers:
+            for t in w.values():
+                if t.data_ptr() not in seen:
+                    seen.add(t.data_ptr())
+                    n += t.numel()
+        return n
+
     def weight_bytes(self) -> int:
-        n = sum(t.numel() for w in self.layers for t in w.values())
-        return 2 * (n + self.W_lm.numel())
+        return 2 * (self._unique_params() + self.W_lm.numel())
 
     # ---------------------------------------------------------- prefill --
     def prefill(self, prompt, stream=None):
@@ -258,7 +268,7 @@ class DecoderModel:
         gains once, its K/V history at cache length ``context`` plus the new
         rows, and the activations in and out."""
         cfg = self.cfg
-        n = sum(t.numel() for w in self.layers for k, t in w.items())
+        n = self._unique_params()
         kv = 2 * cfg.layers * (context + 1) * cfg.d * 2 * self.B
         act = self.B * cfg.d * 2 * 2 * cfg.layers
         return 2 * n + kv + act
