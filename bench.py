@@ -50,9 +50,14 @@ def parse():
                          "(1 GPU)")
     ap.add_argument("--layers", type=int, default=32,
                     help="decoder layers (default 32; fewer only for small profiling cases)")
+    ap.add_argument("--no-l2-discard", action="store_true",
+                    help="leave prefill rank activations to the normal L2 write-back (control "
+                         "for measuring what discarding them saves)")
     ap.add_argument("--profile-step", action="store_true",
-                    help="after warm-up, run one prefill and two decode steps inside an NVTX "
-                         "range 'profile_step' (for an ncu launch list) and exit")
+                    help="after warm-up, run the workload's unit of work once inside an NVTX "
+                         "range 'profile_step' (for an ncu capture) and exit: decode7b one "
+                         "prefill and two decode steps, bert one forward, prefill-attn one "
+                         "rank-1216 layer prefill with the query formed in the attention kernel")
     return ap.parse_args()
 
 
@@ -74,27 +79,33 @@ def whole_job_rate(units_per_rank: float, world: int, ms: float) -> float:
     return world * units_per_rank / (ms / 1e3)
 
 
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "ncu_traffic_decode_layers_fused.txt")
+
+
 def ncu_traffic(kernel: str, layers: int):
-    """DRAM bytes per launch of the fused decode kernel from the committed
-    ncu capture (profiles/decode_layers_fused_*.md: per-layer traffic of a
-    2-layer launch, scaled to `layers`); None when the kernel source has
-    changed since that capture or for other kernels."""
+    """DRAM bytes per launch of the fused decode kernel from the committed ncu
+    record (key: value lines: the kernel source's sha1, the layers the
+    captured launch covered, dram__bytes_read.sum and dram__bytes_write.sum),
+    scaled per layer to `layers`; None for other kernels or when the kernel
+    source has changed since the capture."""
     import hashlib
-    import re as _re
     if kernel != "decode_layers_fused":
         return None
-    prof = os.path.join(ROOT, "profiles", "decode_layers_fused_llama7b_2layers_b1_ctx2048.md")
     src = os.path.join(ROOT, "rank_transformer_b200", "csrc", "decode_fused.cu")
     try:
-        text = open(prof).read()
+        rec = {}
+        for line in open(TRAFFIC_RECORD):
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                rec[k.strip()] = v.strip()
         sha = hashlib.sha1(open(src, "rb").read()).hexdigest()
-    except OSError:
+        if rec.get("kernel_source_sha1") != sha:
+            return None
+        per_layer = (float(rec["dram__bytes_read.sum"]) + float(rec["dram__bytes_write.sum"])) / \
+            float(rec["layers_launched"])
+    except (OSError, KeyError, ValueError):
         return None
-    m = _re.search(r"sha1 \(rank_transformer_b200/csrc/decode_fused.cu\): ([0-9a-f]{40})", text)
-    t = _re.search(r"= ([0-9.]+) MB per layer", text)
-    if not m or not t or m.group(1) != sha:
-        return None
-    return float(t.group(1)) * 1e6 * layers
+    return per_layer * layers
 
 
 def measured_peaks():
@@ -259,6 +270,8 @@ def run_ours(args):
     cfg = dataclasses.replace(LLAMA7B, layers=args.layers)
     S_max = PROMPT + DECODE_STEPS
     fs.init(local, max_tokens=B * PROMPT, max_rank=2368, max_hidden=cfg.d, max_ffn=cfg.f)
+    if args.no_l2_discard:
+        fs.set_l2_discard(False)
     model = DecoderModel(cfg, B, S_max, seed=1234 + rank)
     gen = torch.Generator(device="cuda")
     gen.manual_seed(99 + rank)
@@ -423,9 +436,8 @@ def run_ours(args):
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / peaks["hbm_gbs"],
                          "traffic": ncu_traffic(top, cfg.layers),
-                         "traffic_source": "ncu dram__bytes_read+write of a 2-layer launch, "
-                                           "scaled per layer (profiles/decode_layers_fused_"
-                                           "llama7b_2layers_b1_ctx2048.md)",
+                         "traffic_source": "ncu dram__bytes_read+write of a 2-layer launch of "
+                                           "the same kernel source, scaled per layer",
                          "launches_timed": tp["launches"],
                          "peak_source": peaks["source"] + " (burst copy)"},
             "kernel_times_ms": {k: round(v["ms"], 4) for k, v in sorted(prof.items())},
@@ -572,6 +584,8 @@ def run_bert(args):
         return free0 - free1
     ws_full, ws_small = ws_bytes(M), ws_bytes(32)
     fs.init(0, max_tokens=M, max_rank=r, max_hidden=d, max_ffn=8)
+    if args.no_l2_discard:
+        fs.set_l2_discard(False)
     before = torch.cuda.memory_allocated()
     m = EncoderModel(layers=nl, B=B, S=S, seed=3)
     model_bytes = torch.cuda.memory_allocated() - before   # weights + K/V buffers
@@ -581,6 +595,17 @@ def run_bert(args):
     x0 = torch.randn(M, d, device="cuda", generator=gen).to(torch.bfloat16)
     x = x0.clone()
     stream = torch.cuda.Stream()
+    if args.profile_step:
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                m.forward(x, stream)
+            stream.synchronize()
+            torch.cuda.nvtx.range_push("profile_step")
+            m.forward(x, stream)
+            stream.synchronize()
+            torch.cuda.nvtx.range_pop()
+        print(json.dumps({"profile_step": "done", "workload": "bert"}))
+        return 0
     with torch.cuda.stream(stream):
         for _ in range(3):
             x.copy_(x0)
@@ -682,7 +707,7 @@ def run_prefill_attn(args):
     x0 = _bf16_normal((S, d), 1.0, gen, "cuda")
     kc = torch.zeros((1, S, H, D), dtype=torch.bfloat16, device="cuda")
     vc = torch.zeros_like(kc)
-    for r in (128, 256, 512, 832, 1216):
+    for r in ((1216,) if args.profile_step else (128, 256, 512, 832, 1216)):
         w = {}
         for n in ("q", "k", "v", "o"):
             w["U_" + n] = _bf16_normal((d, r), d ** -0.5, gen, "cuda")
@@ -703,6 +728,19 @@ def run_prefill_attn(args):
         L.down.U, L.down.V, L.down.bias, L.down.r = w["U_dn"].data_ptr(), w["V_dn"].data_ptr(), None, r_f
         L.rope_cos, L.rope_sin = cos_t.data_ptr(), sin_t.data_ptr()
         out = {"workload": "prefill-attn", "layer": "7b-shaped decoder", "S": S, "rank_qkvo": r}
+        if args.profile_step:
+            fs.set_prefill_attention(1)
+            x = x0.clone()
+            with torch.cuda.stream(stream):
+                fs.layer_forward(L, x, kc, vc, None, 1, S, S, fs.PREFILL_CAUSAL, stream)
+                stream.synchronize()
+                torch.cuda.nvtx.range_push("profile_step")
+                fs.layer_forward(L, x, kc, vc, None, 1, S, S, fs.PREFILL_CAUSAL, stream)
+                stream.synchronize()
+                torch.cuda.nvtx.range_pop()
+            fs.set_prefill_attention(0)
+            print(json.dumps({"profile_step": "done", "workload": "prefill-attn", "rank_qkvo": r}))
+            return 0
         for mode in (0, 1):
             fs.set_prefill_attention(mode)
             x = x0.clone()

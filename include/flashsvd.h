@@ -144,6 +144,15 @@ FLASHSVD_API int flashsvd_set_decode_path(int fused);
  * Other modes return FLASHSVD_ERR_INVALID_ARG. */
 FLASHSVD_API int flashsvd_set_prefill_attention(int mode);
 
+/* Prefill rank activations (z of the factorized linears, z1 of the streamed
+ * FFN, z_q of the factorized attention) live in a workspace that stays in
+ * L2 between the two kernels of a linear; on != 0 (default) the kernel that
+ * reads a block of z last drops its L2 lines without write-back
+ * (discard.global.L2), so z never reaches HBM.  on = 0 leaves the lines to
+ * the normal write-back: a control for measuring what the discard saves.
+ * Results are identical either way. */
+FLASHSVD_API int flashsvd_set_l2_discard(int on);
+
 /* Number of kernels this library has launched since load: eager launches
  * plus the kernel nodes of every replayed graph. */
 FLASHSVD_API int64_t flashsvd_launch_count(void);

@@ -47,6 +47,10 @@ std::mutex g_mu;
 
 inline Ctx& cur() { return t_ctx ? *t_ctx : g_default; }
 
+// Whether prefill kernels drop a rank activation's L2 lines after its last
+// use (discard.global.L2: no write-back to HBM).  On by default.
+bool g_l2_discard = true;
+
 void free_ctx(Ctx& c) {
   void* ptrs[] = {c.z, c.part, c.counters, c.apart, c.acounters, c.status,
                   c.xn, c.q, c.att, c.h, c.zb, c.df_part, c.df_cnt, c.zcnt};
@@ -274,7 +278,7 @@ PfLinear pf_base(const bf16* x, long long ldx, const flashsvd_factor& F, int M,
   p.y = y; p.ldy = ldy; p.M = M; p.d = d; p.r = F.r; p.n = n;
   p.epi = PF_EPI_BF16;
   p.z = cur().zb;
-  p.zcnt = cur().zcnt;
+  p.zcnt = g_l2_discard ? cur().zcnt : nullptr;
   p.status = cur().status;
   return p;
 }
@@ -417,7 +421,7 @@ int layer_prefill(const flashsvd_layer* L, bf16* x, bf16* kc, bf16* vc,
   if (fact_q) {
     a.zq = zg[0]; a.ldz = L->q.r; a.r = L->q.r; a.Vq = cb(L->q.V);
     a.rope_cos = L->rope_cos; a.rope_sin = L->rope_sin;
-    a.zcnt = cur().zcnt; a.zcnt_cap = cur().zcnt_elems;
+    a.zcnt = g_l2_discard ? cur().zcnt : nullptr; a.zcnt_cap = cur().zcnt_elems;
   } else {
     a.q = cur().q;
   }
@@ -448,7 +452,7 @@ int lowrank_ffn(const bf16* x, const bf16* U1, const bf16* V1, const bf16* b1, c
   bf16* z = cur().zb;
   FSVD_TRY(prefill_stage1(x, d, d, M, U1, r1, z, cur().status, s));
   return ffn_stream_launch(z, r1, V1, b1, U2, V2, b2, resid, y, M, f, r1, r2, d, cur().status,
-                           cur().sm_count, s);
+                           cur().sm_count, g_l2_discard, s);
 }
 
 // ------------------------------------------------------ layer: encoder ----
@@ -569,6 +573,11 @@ const char* flashsvd_status_string(int status) {
 
 int flashsvd_last_cuda_error(void) { return g_last_cuda_error; }
 int flashsvd_version(void) { return 100; }
+
+int flashsvd_set_l2_discard(int on) {
+  g_l2_discard = on != 0;
+  return FLASHSVD_OK;
+}
 
 int flashsvd_set_prefill_attention(int mode) {
   if (mode < 0 || mode > 1) return FLASHSVD_ERR_INVALID_ARG;

@@ -43,6 +43,7 @@ constexpr uint32_t FS_TMEM_COLS = 512;   // S[2] 0..255 (Y reuses them), acc2 25
 struct FsArgs {
   int M, f, r1, r2, d;
   const bf16* z1; long long ldz;  // rank activations (their L2 lines are discarded after use)
+  int discard;
   const bf16* b1;      // [f] or null
   const bf16* b2;      // [d] or null
   const bf16* resid;   // [M x d] or null (may alias y)
@@ -389,7 +390,7 @@ ffn_stream_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(z2_full);
-      if (q == 0 && part == 0) {
+      if (a.discard && q == 0 && part == 0) {
         // every MMA that read this tile's z1 has completed (acc_full), and
         // no other tile reads these rows: drop their L2 lines without
         // write-back (whole 128-byte lines inside the tile's rows only)
@@ -452,7 +453,7 @@ ffn_stream_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant
 // V2 [r2 x d], b2 [d] (or null), resid [M x d] (or null, may alias y).
 int ffn_stream_launch(const bf16* z1, long long ldz, const bf16* V1, const bf16* b1, const bf16* U2,
                       const bf16* V2, const bf16* b2, const bf16* resid, bf16* y, int M, int f, int r1,
-                      int r2, int d, int* status, int sms, cudaStream_t stream) {
+                      int r2, int d, int* status, int sms, bool discard, cudaStream_t stream) {
   if (M <= 0 || f <= 0 || d <= 0) return FLASHSVD_ERR_INVALID_ARG;
   if (r1 % 64 || r2 % 64 || r1 < 64 || r2 < 64 || r1 > FS_RMAX || r2 > FS_RMAX || f % 8 || d % 8)
     return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
@@ -465,7 +466,7 @@ int ffn_stream_launch(const bf16* z1, long long ldz, const bf16* V1, const bf16*
   FSVD_TRY(set_smem_once(smem_once, ffn_stream_kernel, FS_SMEM));
   FsArgs a;
   a.M = M; a.f = f; a.r1 = r1; a.r2 = r2; a.d = d;
-  a.z1 = z1; a.ldz = ldz;
+  a.z1 = z1; a.ldz = ldz; a.discard = discard ? 1 : 0;
   a.b1 = b1; a.b2 = b2; a.resid = resid; a.y = y; a.status = status;
   const int tiles = (M + 127) / 128;
   const int grid = tiles < sms ? tiles : sms;

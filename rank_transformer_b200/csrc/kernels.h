@@ -118,7 +118,7 @@ int prefill_stage1(const bf16* x, long long ldx, int d, int M, const bf16* U, in
 constexpr int kFfnStreamMaxRank = 256;
 int ffn_stream_launch(const bf16* z1, long long ldz, const bf16* V1, const bf16* b1, const bf16* U2,
                       const bf16* V2, const bf16* b2, const bf16* resid, bf16* y, int M, int f, int r1,
-                      int r2, int d, int* status, int sms, cudaStream_t stream);
+                      int r2, int d, int* status, int sms, bool discard, cudaStream_t stream);
 
 // --------------------------------------------- fused decode layer ---------
 struct DecodeLayerDesc {

@@ -76,6 +76,7 @@ _SIGS = {
     "flashsvd_launch_count": ([], C.c_int64),
     "flashsvd_set_decode_path": ([_i], _i),
     "flashsvd_set_prefill_attention": ([_i], _i),
+    "flashsvd_set_l2_discard": ([_i], _i),
     "flashsvd_decode_pack_bytes": ([_p, C.POINTER(C.c_size_t)], _i),
     "flashsvd_decode_pack": ([_p, _p, C.c_size_t, _p], _i),
     "flashsvd_decode_plan_create": ([_p, _i, _p, _p, _i, _i, _p], _i),
@@ -191,6 +192,10 @@ def set_prefill_attention(mode: int) -> None:
     """1: query formed inside the attention kernel; 0: dense q projection
     (the default)."""
     _call("flashsvd_set_prefill_attention", mode)
+
+
+def set_l2_discard(on: bool) -> None:
+    _call("flashsvd_set_l2_discard", int(on))
 
 
 def set_decode_path(fused: bool) -> None:
