@@ -85,7 +85,7 @@ int alloc_ctx(Ctx& c, int device, int max_tokens, int max_rank, int max_hidden, 
   FSVD_ALLOC(c.q, (size_t)c.rows * max_hidden * sizeof(bf16));
   FSVD_ALLOC(c.att, (size_t)c.rows * max_hidden * sizeof(bf16));
   FSVD_ALLOC(c.h, (size_t)c.rows * max_ffn * sizeof(bf16));
-  FSVD_ALLOC(c.zb, (size_t)c.rows * 2 * max_rank * sizeof(bf16));
+  FSVD_ALLOC(c.zb, (size_t)c.rows * 3 * max_rank * sizeof(bf16));  // grouped q/k/v stage 1: 3 ranks
   FSVD_ALLOC(c.df_part, (size_t)kFusedPartFloats * sizeof(float));
   FSVD_ALLOC(c.df_cnt, (size_t)(4096 + 64) * sizeof(int));
   // (the factorized attention counts per batch row and query tile: at most
@@ -289,7 +289,7 @@ PfLinear pf_base(const bf16* x, long long ldx, const flashsvd_factor& F, int M,
 bool qkv_stage1_grouped(const bf16* x, int d, int M, const flashsvd_factor* const* F, bf16** z,
                         cudaStream_t s, int* st) {
   const long long need = (long long)M * (F[0]->r + F[1]->r + F[2]->r);
-  if (need > (long long)cur().rows * 2 * cur().max_rank) return false;
+  if (need > (long long)cur().rows * 3 * cur().max_rank) return false;
   const bf16* U[3];
   int r[3];
   long long off = 0;
@@ -302,6 +302,30 @@ bool qkv_stage1_grouped(const bf16* x, int d, int M, const flashsvd_factor* cons
   }
   *st = prefill_stage1_grouped(x, d, d, M, 3, U, r, z, cur().status, s);
   return true;
+}
+
+// Stage 2 of the q, k, v projections (those of `first` .. 2) as one grouped
+// tcgen05 launch over the rank activations that the grouped stage 1 left
+// stacked in the scratch (equal ranks): q to the q buffer, k and v (k with
+// RoPE when the tables are given) into the caches.
+int qkv_stage2_grouped(const flashsvd_factor* const* F, bf16* const* z, int first, int M, int d, int D, int S,
+                       int S_max, bf16* q_out, bf16* kc, bf16* vc, const float* cos_t, const float* sin_t,
+                       cudaStream_t s) {
+  QkvGroup g;
+  memset(&g, 0, sizeof(g));
+  bf16* dst[3] = {nullptr, kc, vc};
+  for (int i = first; i < 3; ++i) {
+    g.row[g.n] = (int)((z[i] - z[0]) / F[0]->r);
+    g.V[g.n] = cb(F[i]->V); g.bias[g.n] = cb(F[i]->bias); g.kind[g.n] = i; g.cache[g.n] = dst[i];
+    ++g.n;
+  }
+  g.M = M; g.r = F[0]->r; g.z = z[0];
+  g.q = q_out; g.ldq = d;
+  g.S = S; g.S_max = S_max; g.HD = d; g.D = D;
+  g.rope_cos = cos_t; g.rope_sin = sin_t;
+  g.zcnt = g_l2_discard ? cur().zcnt : nullptr;
+  g.status = cur().status;
+  return prefill_qkv_stage2_grouped(g, s);
 }
 
 bool g_fused_decode = true;
@@ -404,13 +428,18 @@ int layer_prefill(const flashsvd_layer* L, bf16* x, bf16* kc, bf16* vc,
   // itself, so q's stage 2 is not run and dense q is never materialised.
   // k and v still go through stage 2: decode reads them from the cache.
   const bool fact_q = grouped && L->q.r % 64 == 0 && g_prefill_qf == 1;
-  for (int i = fact_q ? 1 : 0; i < 3; ++i) {
-    PfLinear p = pf_base(cur().xn, d, *F[i], M, d, d, cur().q, d);
-    if (grouped) { p.z = zg[i]; p.z_ready = 1; }
-    p.epi = PF_EPI_QKV; p.kind = i; p.cache = dst[i]; p.S = S; p.S_max = S_max;
-    p.HD = d; p.D = L->D;
-    if (i < 2) { p.rope_cos = L->rope_cos; p.rope_sin = L->rope_sin; }
-    FSVD_TRY(prefill_linear_launch(p, s));
+  if (grouped && L->k.r == L->q.r && L->v.r == L->q.r) {
+    FSVD_TRY(qkv_stage2_grouped(F, zg, fact_q ? 1 : 0, M, d, L->D, S, S_max, cur().q, kc, vc, L->rope_cos,
+                                L->rope_sin, s));
+  } else {
+    for (int i = fact_q ? 1 : 0; i < 3; ++i) {
+      PfLinear p = pf_base(cur().xn, d, *F[i], M, d, d, cur().q, d);
+      if (grouped) { p.z = zg[i]; p.z_ready = 1; }
+      p.epi = PF_EPI_QKV; p.kind = i; p.cache = dst[i]; p.S = S; p.S_max = S_max;
+      p.HD = d; p.D = L->D;
+      if (i < 2) { p.rope_cos = L->rope_cos; p.rope_sin = L->rope_sin; }
+      FSVD_TRY(prefill_linear_launch(p, s));
+    }
   }
   AttnPfParams a;
   memset(&a, 0, sizeof(a));
@@ -465,12 +494,16 @@ int layer_encoder(const flashsvd_layer* L, bf16* x, bf16* kc, bf16* vc,
   int gst = FLASHSVD_OK;
   const bool grouped = qkv_stage1_grouped(x, d, M, F, zg, s, &gst);
   FSVD_TRY(gst);
-  for (int i = 0; i < 3; ++i) {
-    PfLinear p = pf_base(x, d, *F[i], M, d, d, cur().q, d);
-    if (grouped) { p.z = zg[i]; p.z_ready = 1; }
-    p.epi = PF_EPI_QKV; p.kind = i; p.cache = dst[i]; p.S = S; p.S_max = S_max;
-    p.HD = d; p.D = L->D;
-    FSVD_TRY(prefill_linear_launch(p, s));
+  if (grouped && L->k.r == L->q.r && L->v.r == L->q.r) {
+    FSVD_TRY(qkv_stage2_grouped(F, zg, 0, M, d, L->D, S, S_max, cur().q, kc, vc, nullptr, nullptr, s));
+  } else {
+    for (int i = 0; i < 3; ++i) {
+      PfLinear p = pf_base(x, d, *F[i], M, d, d, cur().q, d);
+      if (grouped) { p.z = zg[i]; p.z_ready = 1; }
+      p.epi = PF_EPI_QKV; p.kind = i; p.cache = dst[i]; p.S = S; p.S_max = S_max;
+      p.HD = d; p.D = L->D;
+      FSVD_TRY(prefill_linear_launch(p, s));
+    }
   }
   AttnPfParams a;
   memset(&a, 0, sizeof(a));
@@ -860,7 +893,7 @@ int flashsvd_lowrank_ffn(const flashsvd_bf16* x, const flashsvd_bf16* U_up, cons
   FSVD_TRY(check_w8(d)); FSVD_TRY(check_w8(r_up)); FSVD_TRY(check_w8(f)); FSVD_TRY(check_w8(r_dn));
   if (M == 0) return FLASHSVD_OK;
   if (!ffn_stream_covers(d, r_up, f, r_dn)) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
-  if (M > cur().rows || (long long)M * r_up > (long long)cur().rows * 2 * cur().max_rank)
+  if (M > cur().rows || (long long)M * r_up > (long long)cur().rows * 3 * cur().max_rank)
     return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   return lowrank_ffn(cb(x), cb(U_up), cb(V_up), cb(b_up), cb(U_dn), cb(V_dn), cb(b_dn), cb(resid),
                      (bf16*)y, M, d, r_up, f, r_dn, stream);

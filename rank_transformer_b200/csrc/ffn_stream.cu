@@ -12,8 +12,8 @@
 //   z2 = bf16(acc2) -> smem (over z1's area)
 //   y[:, 256 p ..] = z2 . V2[:, 256 p ..] + b2 + resid   (TMEM cols 0..255)
 // The MMA of chunk c + 1 overlaps the epilogue of chunk c (two S and two H
-// buffers).  Warps: 0 TMA producer, 1 MMA issuer, 2..9 epilogue (two per
-// TMEM lane quadrant).  All B operands stream through one ring of 32 KB
+// buffers).  Warps: 0 TMA producer, 1 MMA issuer, 2..17 epilogue (four per
+// TMEM lane quadrant, a quarter of the chunk's columns each).  All B operands stream through one ring of 32 KB
 // slots in the order the MMA warp consumes them.  z1 is read once per tile
 // from the rank scratch and its L2 lines are discarded after use, so z1 is
 // never written back to HBM either.
@@ -27,7 +27,10 @@
 namespace fsvd {
 namespace {
 
-constexpr int FS_THREADS = 320;
+constexpr int FS_NPART = 4;                // epilogue warps per TMEM lane quadrant
+constexpr int FS_EPI = 4 * FS_NPART;       // epilogue warps
+constexpr int FS_THREADS = 32 * (2 + FS_EPI);
+constexpr int FS_CPW = 128 / FS_NPART;     // chunk columns per epilogue warp
 constexpr int FS_STAGES = 3;
 constexpr int FS_SLOT = 32768;           // one 64-row k-block of B, up to 256 columns
 constexpr int FS_RMAX = 256;             // r1, r2 <= 256 (multiples of 64)
@@ -141,14 +144,14 @@ ffn_stream_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant
     tc::mbar_init(z_empty, 1);
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(s_full + b, 1);
-      tc::mbar_init(s_empty + b, 8);
-      tc::mbar_init(h_full + b, 8);
+      tc::mbar_init(s_empty + b, FS_EPI);
+      tc::mbar_init(h_full + b, FS_EPI);
       tc::mbar_init(h_empty + b, 1);
     }
     tc::mbar_init(acc_full, 1);
-    tc::mbar_init(z2_full, 8);
+    tc::mbar_init(z2_full, FS_EPI);
     tc::mbar_init(y_full, 1);
-    tc::mbar_init(y_empty, 8);
+    tc::mbar_init(y_empty, FS_EPI);
     tc::mbar_init(drain, 1);
     *abort_flag = 0;
     tc::fence_barrier_init();
@@ -307,9 +310,9 @@ ffn_stream_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant
   } else {
     // --------------------------------------------------------- epilogue --
     // Warp w reads TMEM lanes 32 (w % 4) .. + 31 (its 32 rows of the tile);
-    // the two warps of a lane quadrant take the two column halves.
+    // the four warps of a lane quadrant take a quarter of the columns each.
     const int q = warp & 3;
-    const int part = (warp - 2) >> 2;
+    const int part = (warp - 2) >> 2;   // 0 .. FS_NPART - 1
     const int row = q * 32 + lane;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     // tcgen05.ld is warp-collective: every wait result is made warp-uniform
@@ -328,36 +331,50 @@ ffn_stream_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant
         const uint32_t k = (uint32_t)(u >> 1) & 1u;
         if (!wwait(s_full + b, k)) { ok = false; break; }
         tc::fence_after_sync();
-        uint32_t r[64];
-        const uint32_t sc = tmem_base + lane_base + (uint32_t)(b * 128 + part * 64);
+        uint32_t r[FS_CPW];
+        const uint32_t sc = tmem_base + lane_base + (uint32_t)(b * 128 + part * FS_CPW);
         tc::tmem_ld32(sc, r);
-        tc::tmem_ld32(sc + 32, r + 32);
         tc::tmem_ld_wait();
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(s_empty + b);  // S[b] may be overwritten now
         // + b1, GELU (columns past f: S = 0 from the zero-filled V1 and no
         // bias, so H = GELU(0) = 0 there)
-        const int col0 = c * 128 + part * 64;
-        float x[64];
+        const int col0 = c * 128 + part * FS_CPW;
+        float x[FS_CPW];
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          const int col = col0 + j;
-          x[j] = __uint_as_float(r[j]) + ((a.b1 && col < a.f) ? bf2f(a.b1[col]) : 0.f);
+        for (int j = 0; j < FS_CPW; ++j) x[j] = __uint_as_float(r[j]);
+        if (a.b1) {
+          // 8 bias values per 16-byte load (f is a multiple of 8)
+#pragma unroll
+          for (int g8 = 0; g8 < FS_CPW / 8; ++g8) {
+            const int col = col0 + 8 * g8;
+            if (col < a.f) {
+              const uint4 bb = __ldg(reinterpret_cast<const uint4*>(a.b1 + col));
+              x[8 * g8 + 0] += bf_lo(bb.x); x[8 * g8 + 1] += bf_hi(bb.x);
+              x[8 * g8 + 2] += bf_lo(bb.y); x[8 * g8 + 3] += bf_hi(bb.y);
+              x[8 * g8 + 4] += bf_lo(bb.z); x[8 * g8 + 5] += bf_hi(bb.z);
+              x[8 * g8 + 6] += bf_lo(bb.w); x[8 * g8 + 7] += bf_hi(bb.w);
+            }
+          }
         }
 #pragma unroll
-        for (int j = 0; j < 64; j += 2) gelu_erf2(x[j], x[j + 1]);
+        for (int j = 0; j < FS_CPW; j += 2) gelu_erf2(x[j], x[j + 1]);
         // H[b] must have been consumed by the MMA of chunk u - 2
         if (!wwait(h_empty + b, k ^ 1u)) { ok = false; break; }
-        uint8_t* hblk = smem + FS_H_OFF + (b * 2 + part) * FS_BLK;
+        // columns part * FS_CPW .. of the chunk: A block (col >> 6), 16-byte
+        // chunks ((col & 63) >> 3) .. of the 128-byte swizzled row
+        const int hc0 = part * FS_CPW;
+        uint8_t* hblk = smem + FS_H_OFF + (b * 2 + (hc0 >> 6)) * FS_BLK;
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
+        for (int ch = 0; ch < FS_CPW / 8; ++ch) {
           uint4 w;
           w.x = pack2(x[ch * 8 + 0], x[ch * 8 + 1]);
           w.y = pack2(x[ch * 8 + 2], x[ch * 8 + 3]);
           w.z = pack2(x[ch * 8 + 4], x[ch * 8 + 5]);
           w.w = pack2(x[ch * 8 + 6], x[ch * 8 + 7]);
-          *reinterpret_cast<uint4*>(hblk + row * 128 + ((ch ^ (row & 7)) << 4)) = w;
+          const int c16 = ((hc0 & 63) >> 3) + ch;
+          *reinterpret_cast<uint4*>(hblk + row * 128 + ((c16 ^ (row & 7)) << 4)) = w;
         }
         tc::fence_proxy_async_smem();  // H is read by the tensor cores
         __syncwarp();
@@ -368,8 +385,8 @@ ffn_stream_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant
       // z1 has completed once acc_full fires) ----
       if (!wwait(acc_full, (uint32_t)it & 1u)) { ok = false; break; }
       tc::fence_after_sync();
-      // 32-column groups g = part, part + 2, ... (r2 / 32 groups in all)
-      for (int g = part; g < 2 * KB2; g += 2) {
+      // 32-column groups g = part, part + FS_NPART, ... (r2 / 32 groups in all)
+      for (int g = part; g < 2 * KB2; g += FS_NPART) {
         uint32_t r[32];
         tc::tmem_ld32(tmem_base + lane_base + 256u + (uint32_t)(32 * g), r);
         tc::tmem_ld_wait();
@@ -406,11 +423,12 @@ ffn_stream_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant
       for (int p = 0; p < NP && ok; ++p, ++v) {
         if (!wwait(y_full, (uint32_t)(v & 1))) { ok = false; break; }
         tc::fence_after_sync();
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < 256 / (32 * FS_NPART); ++j) {
           uint32_t r[32];
-          tc::tmem_ld32(tmem_base + lane_base + (uint32_t)(part * 128 + 32 * j), r);
+          const int pc = part * (256 / FS_NPART) + 32 * j;   // column within the pass
+          tc::tmem_ld32(tmem_base + lane_base + (uint32_t)pc, r);
           tc::tmem_ld_wait();
-          const int col0 = p * 256 + part * 128 + 32 * j;
+          const int col0 = p * 256 + pc;
           if (!mok) continue;
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
@@ -420,8 +438,9 @@ ffn_stream_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant
 #pragma unroll
             for (int i = 0; i < 8; ++i) o[i] = __uint_as_float(r[e + i]);
             if (a.b2) {
-#pragma unroll
-              for (int i = 0; i < 8; ++i) o[i] += bf2f(a.b2[col + i]);
+              const uint4 bb = __ldg(reinterpret_cast<const uint4*>(a.b2 + col));
+              o[0] += bf_lo(bb.x); o[1] += bf_hi(bb.x); o[2] += bf_lo(bb.y); o[3] += bf_hi(bb.y);
+              o[4] += bf_lo(bb.z); o[5] += bf_hi(bb.z); o[6] += bf_lo(bb.w); o[7] += bf_hi(bb.w);
             }
             if (a.resid) {
               const uint4 rr = *reinterpret_cast<const uint4*>(a.resid + (long long)m * a.d + col);

@@ -107,6 +107,23 @@ int prefill_linear_launch(const PfLinear& p, cudaStream_t stream);
 int prefill_stage1_grouped(const bf16* x, long long ldx, int d, int M, int n, const bf16* const* U,
                            const int* r, bf16* const* z, int* status, cudaStream_t stream);
 int prefill_dense_launch(const PfLinear& p, cudaStream_t stream);
+// Stage 2 of n <= 3 of the q, k, v projections in one tcgen05 launch.  The
+// rank activations are stacked in one buffer z (row stride r, equal ranks):
+// problem i reads rows row[i] .. row[i] + M; kind[i] 0 = q (to q, row stride
+// ldq), 1 = k, 2 = v (to cache[i] [B, S_max, H, D] rows 0..S-1, as the
+// single-problem QKV epilogue); bias[i] may be null; RoPE on q and k when
+// the tables are given.  zcnt (3 x ceil(M / 128) zero counters) or null:
+// each problem's z rows are discarded from L2 after their last use.
+struct QkvGroup {
+  int n, M, r;
+  const bf16* z; int row[3];
+  const bf16* V[3]; const bf16* bias[3]; int kind[3];
+  bf16* cache[3]; bf16* q; long long ldq;
+  int S, S_max, HD, D;
+  const float* rope_cos; const float* rope_sin;
+  int* zcnt; int* status;
+};
+int prefill_qkv_stage2_grouped(const QkvGroup& g, cudaStream_t stream);
 // Stage 1 of one factorized linear: z [M x r] (row stride r) = x . U, bf16.
 int prefill_stage1(const bf16* x, long long ldx, int d, int M, const bf16* U, int r, bf16* z, int* status,
                    cudaStream_t stream);

@@ -93,6 +93,11 @@ struct TcArgs {
   // stride gldy[i]) and width gN[i].  nprob <= 1: a.y, a.ldy, a.N.
   int nprob; int pt[3];
   bf16* gy[3]; long long gldy[3]; int gN[3];
+  // Grouped q/k/v stage 2 (QKV epilogue): problem i reads A rows from
+  // grow[i] (the rank activations stacked in one buffer), has epilogue kind
+  // gkind[i] (0 q -> gy[i], 1 k, 2 v -> gcache[i]), bias gbias[i] and RoPE
+  // when grope[i].
+  int grow[3]; int gkind[3]; bf16* gcache[3]; const bf16* gbias[3]; int grope[3];
 };
 
 // Problem of global column tile gn of a grouped launch, and its first tile.
@@ -252,7 +257,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           const int kr = (second ? a.b2 : 0) + kk * BK;
           uint8_t* sA = smem + stage * L::STAGE_BYTES;
           uint8_t* sB = sA + L::A_BYTES;
-          tc::tma_load_2d(sA, &tmA, full + stage, ka, m0);
+          tc::tma_load_2d(sA, &tmA, full + stage, ka, m0 + (a.nprob > 1 ? a.grow[gp] : 0));
 #pragma unroll
           for (int j = 0; j < BN / 64; ++j) tc::tma_load_2d(sB + j * 8192, mB, full + stage, n0 + 64 * j, kr);
           ++issued;
@@ -338,6 +343,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const int half = a.D >> 1;
         const int hc = half >> 5;  // chunks per half head
         const int bq = mok ? m / a.S : 0, tq = mok ? m - bq * a.S : 0;
+        // this tile's problem (grouped q/k/v: its kind, cache, bias, RoPE)
+        const bool grp = a.nprob > 1;
+        const int kind = grp ? a.gkind[gp] : a.kind;
+        bf16* const cache = grp ? a.gcache[gp] : a.cache;
+        const bf16* const bias = grp ? a.gbias[gp] : a.bias;
+        const bool rope = grp ? (a.grope[gp] != 0) : (a.rope_cos != nullptr);
         int pair = 0;
         for (int c = 0; c < BN / 32; ++c) {
           if ((c % (2 * hc)) >= hc) continue;  // second-half chunks ride along
@@ -351,17 +362,17 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           float lo[32], hi[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) { lo[j] = __uint_as_float(r0[j]); hi[j] = __uint_as_float(r1[j]); }
-          if (a.bias) {
+          if (bias) {
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
               float b0[8], b1[8];
-              load8(a.bias + n + 8 * g, b0);
-              load8(a.bias + n + half + 8 * g, b1);
+              load8(bias + n + 8 * g, b0);
+              load8(bias + n + half + 8 * g, b1);
 #pragma unroll
               for (int j = 0; j < 8; ++j) { lo[8 * g + j] += b0[j]; hi[8 * g + j] += b1[j]; }
             }
           }
-          if (a.rope_cos) {
+          if (rope) {
             // 32 consecutive angles of this row's position: 16-byte loads.
             const int i0 = n % a.D;
             const float4* cs = reinterpret_cast<const float4*>(a.rope_cos + (long long)tq * half + i0);
@@ -379,8 +390,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
               }
             }
           }
-          bf16* dst = a.kind == 0 ? a.y + (long long)m * a.ldy
-                                  : a.cache + ((long long)bq * a.S_max + tq) * a.HD;
+          bf16* dst = kind == 0 ? ty + (long long)m * tldy
+                                : cache + ((long long)bq * a.S_max + tq) * a.HD;
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
             store8(dst + n + 8 * g, lo + 8 * g);
@@ -463,17 +474,21 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         // done.  One warp counts the block's finished column tiles; the last
         // CTA's warp discards the block's z lines (whole 128-byte lines
         // inside rows [m0, m0 + 128) only).
-        const int mb = t % a.tiles_m;
+        // (grouped: counters and rows per problem, whose A rows start at
+        // grow[gp] and whose column tiles are pt[gp] .. pt[gp + 1])
+        const int gtn = a.nprob > 1 ? (gp + 1 < a.nprob ? a.pt[gp + 1] : a.tiles_n) - a.pt[gp] : a.tiles_n;
+        const int mb = (a.nprob > 1 ? gp * a.tiles_m : 0) + t % a.tiles_m;
+        const long long zr = a.nprob > 1 ? a.grow[gp] : 0;
         const unsigned act = __activemask();
         int last = 0;
         if (lane == 0) {
-          last = atomicAdd(a.zcnt + mb, 1) == a.tiles_n - 1;
+          last = atomicAdd(a.zcnt + mb, 1) == gtn - 1;
           if (last) a.zcnt[mb] = 0;
         }
         last = __shfl_sync(act, last, __ffs(act) - 1);
         if (last) {
-          const long long b0 = (long long)m0 * a.zld * 2;
-          const long long b1 = (long long)min(m0 + BM, a.M) * a.zld * 2;
+          const long long b0 = (zr + m0) * a.zld * 2;
+          const long long b1 = (zr + min(m0 + BM, a.M)) * a.zld * 2;
           const uintptr_t base = reinterpret_cast<uintptr_t>(a.zdrop);
           const uintptr_t l0 = (base + b0 + 127) & ~(uintptr_t)127, l1 = (base + b1) & ~(uintptr_t)127;
           for (uintptr_t ln = l0 + (uintptr_t)lane * 128; ln < l1; ln += 32 * 128)
@@ -590,6 +605,32 @@ int prefill_stage1(const bf16* x, long long ldx, int d, int M, const bf16* U, in
   a.y = z; a.ldy = r;
   a.status = status;
   return gemm(x, ldx, d, U, r, d, a, PF_EPI_BF16, false, "tc_stage1_xu", stream);
+}
+
+int prefill_qkv_stage2_grouped(const QkvGroup& g, cudaStream_t stream) {
+  if (g.n < 1 || g.n > 3) return FLASHSVD_ERR_INVALID_ARG;
+  if (g.D % 64 != 0 || 256 % g.D != 0) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  TcArgs a;
+  memset(&a, 0, sizeof(a));
+  a.M = g.M; a.K = g.r;
+  a.status = g.status;
+  a.nprob = g.n;
+  a.S = g.S; a.S_max = g.S_max; a.HD = g.HD; a.D = g.D;
+  a.rope_cos = g.rope_cos; a.rope_sin = g.rope_sin;
+  int rows = 0;
+  CUtensorMap mb[3];
+  for (int i = 0; i < g.n; ++i) {
+    FSVD_TRY(make_map(&mb[i], g.V[i], g.r, g.HD, g.HD, BK));
+    a.gN[i] = g.HD; a.gy[i] = g.q; a.gldy[i] = g.ldq;
+    a.grow[i] = g.row[i]; a.gkind[i] = g.kind[i]; a.gcache[i] = g.cache[i]; a.gbias[i] = g.bias[i];
+    a.grope[i] = (g.kind[i] < 2 && g.rope_cos) ? 1 : 0;
+    rows = max(rows, g.row[i] + g.M);
+  }
+  CUtensorMap ma;
+  FSVD_TRY(make_map(&ma, g.z, rows, g.r, g.r, BM));
+  if (g.zcnt) { a.zdrop = g.z; a.zld = g.r; a.zcnt = g.zcnt; }
+  return launch_tc<256, 4, false, PF_EPI_QKV>(ma, mb[0], mb[g.n > 1 ? 1 : 0], mb[g.n > 2 ? 2 : 0], a,
+                                              "tc_stage2_qkv_grouped", stream);
 }
 
 int prefill_linear_launch(const PfLinear& p, cudaStream_t stream) {
