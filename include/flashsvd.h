@@ -127,8 +127,11 @@ FLASHSVD_API int flashsvd_check_device_status(flashsvd_stream stream);
 /* Decode implementation used by flashsvd_layer_forward(DECODE): fused != 0
  * (default) runs the whole layer as one persistent kernel (one CTA per SM,
  * factor tiles streamed through a TMA ring across all nine stages, stages
- * separated by bounded grid barriers) when B <= 8; fused == 0 runs one
- * launch per stage.  Both give the same result within rounding. */
+ * separated by bounded grid barriers) when B <= 4; fused == 0 runs one
+ * launch per stage.  Both give the same result within rounding.  The fused
+ * kernel is launched cooperatively (all of its CTAs resident at once, or the
+ * launch fails with FLASHSVD_ERR_CUDA), since its CTAs wait on one
+ * another. */
 FLASHSVD_API int flashsvd_set_decode_path(int fused);
 
 /* Prefill attention of DECODER layers (PREFILL_CAUSAL): mode 1 forms each
@@ -152,6 +155,19 @@ FLASHSVD_API int flashsvd_set_prefill_attention(int mode);
  * the normal write-back: a control for measuring what the discard saves.
  * Results are identical either way. */
 FLASHSVD_API int flashsvd_set_l2_discard(int on);
+
+/* Failure-detection test hook.  Arms a one-shot fault: the next launch of
+ * the fused decode kernel (a DECODE-mode flashsvd_layer_forward over a
+ * decode pack, or flashsvd_decode_plan_forward) takes it, and its CTA 0
+ * does not arrive at the kernel's first grid barrier.  The other CTAs'
+ * bounded waits then expire (after about two seconds of SM cycles); every
+ * CTA abandons the step, the launch completes, and
+ * flashsvd_check_device_status returns FLASHSVD_ERR_TIMEOUT.  The kernel's
+ * stage counters are reset at the end of that launch, so the next launch
+ * runs normally.  No GPU fault is involved.  The hook is read when the
+ * launch is issued (not during stream capture: a captured launch keeps the
+ * value it had). */
+FLASHSVD_API int flashsvd_debug_drop_barrier_arrival(void);
 
 /* Number of kernels this library has launched since load: eager launches
  * plus the kernel nodes of every replayed graph. */

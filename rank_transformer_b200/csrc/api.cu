@@ -607,6 +607,11 @@ const char* flashsvd_status_string(int status) {
 int flashsvd_last_cuda_error(void) { return g_last_cuda_error; }
 int flashsvd_version(void) { return 100; }
 
+int flashsvd_debug_drop_barrier_arrival(void) {
+  g_df_drop_arrival.store(1);
+  return FLASHSVD_OK;
+}
+
 int flashsvd_set_l2_discard(int on) {
   g_l2_discard = on != 0;
   return FLASHSVD_OK;

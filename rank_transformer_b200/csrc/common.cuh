@@ -97,6 +97,61 @@ inline int set_smem_once(SmemAttrOnce& once, Kern kernel, int bytes) {
   return FLASHSVD_OK;
 }
 
+// The same launch as launch_pdl, as a cooperative launch: every CTA of the
+// grid is resident at once (the launch fails otherwise), which kernels whose
+// CTAs wait on one another (grid barriers) rely on.
+template <typename... KArgs, typename... Args>
+inline int launch_pdl_coop(const LaunchTag& tag, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                           cudaStream_t stream, Args&&... args) {
+  const bool prof = prof_active(stream);
+  if (prof) prof_begin(stream);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess) return cuda_status(e);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (prof) prof_end(tag, stream);
+  return FLASHSVD_OK;
+}
+
+// The same launch as launch_pdl with the grid in clusters of `cluster_x`
+// CTAs along x (CTA pairs of the 2-SM tensor-core kernels).
+template <typename... KArgs, typename... Args>
+inline int launch_pdl_cluster(const LaunchTag& tag, int cluster_x, void (*kernel)(KArgs...), dim3 grid,
+                              dim3 block, size_t smem, cudaStream_t stream, Args&&... args) {
+  const bool prof = prof_active(stream);
+  if (prof) prof_begin(stream);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster_x;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess) return cuda_status(e);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (prof) prof_end(tag, stream);
+  return FLASHSVD_OK;
+}
+
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 inline int round_up(int a, int b) { return ceil_div(a, b) * b; }
 inline bool aligned16(const void* p) { return (((uintptr_t)p) & 15u) == 0; }

@@ -159,6 +159,7 @@ struct DfParams {
   int* bar;       // [DF_NPHASE] arrivals per stage, accumulated over the layers
   int* done;
   int* status;
+  int drop_arrival;  // test hook: CTA 0 does not arrive at the first grid barrier
 };
 
 template <int MT>
@@ -1276,7 +1277,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
       DF_TRACE(l, ph_i, 3);
       // (the CTA barrier above orders every consumer's writes before this
       // thread's release, which is cumulative over them)
-      if (tid == 0) red_release_add(p.bar + ph_i, 1);
+      if (tid == 0 && !(p.drop_arrival && g == 0 && l == 0 && ph_i == 0)) red_release_add(p.bar + ph_i, 1);
     }
     }  // layers
     // ---- final pass: x = x' + z V_dn of the last layer, this CTA's tiles ----
@@ -1645,7 +1646,14 @@ void fill_common(DfParams& p, const DecodeLayerDesc& L, int B, int S_max, const 
   p.x = x; p.xm = xm;
   p.rope_cos = L.rope_cos; p.rope_sin = L.rope_sin;
   p.part = part; p.bar = bar; p.done = done; p.status = status;
+  p.drop_arrival = g_df_drop_arrival.exchange(0);
 }
+
+}  // namespace
+
+std::atomic<int> g_df_drop_arrival{0};
+
+namespace {
 
 int launch_df(const DfParams& p, int G, double bytes, cudaStream_t stream) {
   const LaunchTag tag{p.nlayer > 1 ? "decode_layers_fused" : "decode_layer_fused", bytes, 0.0};
@@ -1654,7 +1662,7 @@ int launch_df(const DfParams& p, int G, double bytes, cudaStream_t stream) {
     auto kern = decode_layer_kernel<MT_>;                                                            \
     static SmemAttrOnce smem_once;                                                                   \
     FSVD_TRY(set_smem_once(smem_once, kern, DfCfg<MT_>::SMEM));                                      \
-    return launch_pdl(tag, kern, dim3(G), dim3(DfCfg<MT_>::THREADS), (size_t)DfCfg<MT_>::SMEM, stream, p); \
+    return launch_pdl_coop(tag, kern, dim3(G), dim3(DfCfg<MT_>::THREADS), (size_t)DfCfg<MT_>::SMEM, stream, p); \
   }
   if (p.B <= 1) FSVD_DF_LAUNCH(1)
   if (p.B <= 2) FSVD_DF_LAUNCH(2)

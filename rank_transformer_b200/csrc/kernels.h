@@ -166,7 +166,11 @@ int decode_plan_launch(const DecodePlan* plan, bf16* x, const int* seqlens, bf16
 void decode_plan_destroy(DecodePlan* plan);
 int encode_map(CUtensorMap* map, const void* base, long long rows, long long cols, long long ld,
                int box_cols, int box_rows, bool swizzle128);
-constexpr int kFusedPartFloats = 2 * 148 * 16 * 640;  // two halves; per SM 16 slots of 640 floats
+constexpr int kFusedPartFloats = 2 * 148 * 16 * 640;
+// Test hook (flashsvd_debug_drop_barrier_arrival): when set, the next fused
+// decode launch takes it (resetting it) and its CTA 0 skips its first
+// grid-barrier arrival, so that the other CTAs' bounded waits expire.
+extern std::atomic<int> g_df_drop_arrival;  // two halves; per SM 16 slots of 640 floats
 
 // ------------------------------------------------ prefill attention -------
 struct AttnPfParams {

@@ -172,10 +172,12 @@ __device__ __forceinline__ void load8(const bf16* p, float* v) {
   v[4] = bf_lo(u.z); v[5] = bf_hi(u.z); v[6] = bf_lo(u.w); v[7] = bf_hi(u.w);
 }
 
-template <int BN, int STAGES, bool DUAL>
+// PAIR: one CTA of a 2-SM pair, which holds half of the tile's BN columns
+// of B (the other CTA the other half) and its own 128 rows of A.
+template <int BN, int STAGES, bool DUAL, bool PAIR = false>
 struct Layout {
   static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BK * BN * 2;
+  static constexpr int B_BYTES = BK * (PAIR ? BN / 2 : BN) * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
   static constexpr int SMEM = 1024 + BAR_OFF + 256;  // + alignment slack
@@ -184,12 +186,18 @@ struct Layout {
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "tensor memory allocation must be a power of 2");
 };
 
-template <int BN, int STAGES, bool DUAL, int EPI>
+// PAIR: launched in clusters of 2; each pair computes a 256 x BN tile with
+// the 2-SM MMA (cta_group::2): the leader (rank 0) issues it and owns the
+// operand-full barriers, both CTAs load their halves of A and B (for the
+// dual form, half of the gate columns and half of the up columns) and run
+// the epilogue of their 128 rows.  Tiles are counted per pair (a.tiles_m =
+// ceil(M / 256)).
+template <int BN, int STAGES, bool DUAL, int EPI, bool PAIR = false>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
                const __grid_constant__ TcArgs a) {
-  using L = Layout<BN, STAGES, DUAL>;
+  using L = Layout<BN, STAGES, DUAL, PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
@@ -204,7 +212,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int tiles = a.tiles_m * a.tiles_n;
   const int nkb = (a.K + BK - 1) / BK;
   const int kb_total = DUAL ? 2 * nkb : nkb;
-  constexpr uint32_t IDESC = tc::idesc_bf16(BN, true);
+  constexpr uint32_t IDESC = tc::idesc_bf16(BN, true, PAIR ? 256 : 128);
+  // pair: rank in the pair, the pair's index and count
+  const uint32_t rank = PAIR ? tc::cluster_ctarank() : 0u;
+  const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  constexpr int TM = PAIR ? 2 * BM : BM;   // rows per tile
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -213,7 +226,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(tfull + b, 1);
-      tc::mbar_init(tempty + b, 8);
+      tc::mbar_init(tempty + b, PAIR ? 16 : 8);   // the epilogue warps of both CTAs
     }
     tc::mbar_init(drain, 1);
     *abort_flag = 0;
@@ -226,11 +239,19 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     if (a.nprob > 2) tc::tma_prefetch_desc(&tmB2);
   }
   if (warp == 1) {
-    tc::tmem_alloc(tmem_holder, L::TMEM_COLS);
-    tc::tmem_relinquish();
+    if (PAIR) {
+      tc::tmem_alloc_pair(tmem_holder, L::TMEM_COLS);
+      tc::tmem_relinquish_pair();
+    } else {
+      tc::tmem_alloc(tmem_holder, L::TMEM_COLS);
+      tc::tmem_relinquish();
+    }
     tc::fence_before_sync();
   }
   __syncthreads();
+  // pair: the peer's loads signal the leader's barriers and the leader's
+  // MMAs write the peer's tensor memory: both must be set up first
+  if (PAIR) tc::cluster_sync();
   tc::fence_after_sync();
   const uint32_t tmem_base = *tmem_holder;
 
@@ -244,29 +265,43 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       uint32_t phase = 0;
       int issued = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+      for (int t = unit; t < tiles && ok; t += units) {
         const int gn = t / a.tiles_m, gp = group_of(a, gn);
-        const int m0 = (t % a.tiles_m) * BM, n0 = (gn - (gp ? a.pt[gp] : 0)) * BN;
+        const int m0 = (t % a.tiles_m) * TM + (int)rank * BM, n0 = (gn - (gp ? a.pt[gp] : 0)) * BN;
         const CUtensorMap* mB = gp == 0 ? &tmB : (gp == 1 ? &tmB1 : &tmB2);
         for (int kb = 0; kb < kb_total; ++kb) {
           if (!tc::mbar_wait(empty + stage, phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
-          tc::mbar_expect_tx(full + stage, L::STAGE_BYTES);
           const bool second = DUAL && kb >= nkb;
           const int kk = second ? kb - nkb : kb;
           const int ka = (second ? a.a2 : 0) + kk * BK;
           const int kr = (second ? a.b2 : 0) + kk * BK;
           uint8_t* sA = smem + stage * L::STAGE_BYTES;
           uint8_t* sB = sA + L::A_BYTES;
-          tc::tma_load_2d(sA, &tmA, full + stage, ka, m0 + (a.nprob > 1 ? a.grow[gp] : 0));
+          const int arow = m0 + (a.nprob > 1 ? a.grow[gp] : 0);
+          if (PAIR) {
+            // both halves complete on the leader's barrier, which expects
+            // the bytes of both CTAs
+            const uint32_t fb = tc::mapa_shared(tc::smem_u32(full + stage), 0);
+            if (rank == 0) tc::mbar_expect_tx(full + stage, 2 * L::STAGE_BYTES);
+            tc::tma_load_2d_pair(sA, &tmA, fb, ka, arow);
 #pragma unroll
-          for (int j = 0; j < BN / 64; ++j) tc::tma_load_2d(sB + j * 8192, mB, full + stage, n0 + 64 * j, kr);
+            for (int j = 0; j < BN / 128; ++j)
+              tc::tma_load_2d_pair(sB + j * 8192, mB, fb, n0 + (int)rank * (BN / 2) + 64 * j, kr);
+          } else {
+            tc::mbar_expect_tx(full + stage, L::STAGE_BYTES);
+            tc::tma_load_2d(sA, &tmA, full + stage, ka, arow);
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j) tc::tma_load_2d(sB + j * 8192, mB, full + stage, n0 + 64 * j, kr);
+          }
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
-      if (!ok) {
+      if (!ok && rank == 0) {
         // Winding down: let this CTA's copies that are still in flight land
-        // before shared memory is released (bounded, ignores the flag).
+        // before shared memory is released (bounded, ignores the flag).  A
+        // pair's copies all complete on the leader's barriers; the peer is
+        // held by the final cluster barrier instead.
         const int outstanding = issued < STAGES ? issued : STAGES;
         for (int i = 1; i <= outstanding; ++i) {
           int s = stage - i;
@@ -279,12 +314,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer --
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++it) {
+      for (int t = unit; t < tiles && ok; t += units, ++it) {
         const int buf = it & 1;
         const uint32_t tph = (uint32_t)(it >> 1) & 1u;
         if (!tc::mbar_wait(tempty + buf, tph ^ 1u, abort_flag, a.status)) { ok = false; break; }
@@ -302,15 +337,30 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t ad = tc::sdesc_sw128(sa + k * 32, 16, 1024);
             const uint64_t bd = tc::sdesc_sw128(sb + k * 2048, 8192, 1024);
-            tc::mma_bf16(d, ad, bd, IDESC, (first && k == 0) ? 0u : 1u);
+            if (PAIR)
+              tc::mma_bf16_pair(d, ad, bd, IDESC, (first && k == 0) ? 0u : 1u);
+            else
+              tc::mma_bf16(d, ad, bd, IDESC, (first && k == 0) ? 0u : 1u);
           }
-          tc::mma_commit(empty + stage);
+          // the stage is free in both CTAs of a pair
+          if (PAIR)
+            tc::mma_commit_pair_mc(empty + stage, (uint16_t)3);
+          else
+            tc::mma_commit(empty + stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
-        if (ok) tc::mma_commit(tfull + buf);
+        if (ok) {
+          if (PAIR)
+            tc::mma_commit_pair_mc(tfull + buf, (uint16_t)3);
+          else
+            tc::mma_commit(tfull + buf);
+        }
       }
       // Every MMA this thread issued has completed once `drain` fires.
-      tc::mma_commit(drain);
+      if (PAIR)
+        tc::mma_commit_pair(drain);
+      else
+        tc::mma_commit(drain);
       const long long t0 = clock64();
       while (!tc::mbar_try_wait(drain, 0) && clock64() - t0 < tc::kWaitCycles) {}
     }
@@ -322,13 +372,13 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const int part = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     int it = 0;
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
+    for (int t = unit; t < tiles; t += units, ++it) {
       const int buf = it & 1;
       const uint32_t tph = (uint32_t)(it >> 1) & 1u;
       if (!tc::mbar_wait(tfull + buf, tph, abort_flag, a.status)) break;
       tc::fence_after_sync();
       const int gn = t / a.tiles_m, gp = group_of(a, gn);
-      const int m0 = (t % a.tiles_m) * BM, n0 = (gn - (gp ? a.pt[gp] : 0)) * BN;
+      const int m0 = (t % a.tiles_m) * TM + (int)rank * BM, n0 = (gn - (gp ? a.pt[gp] : 0)) * BN;
       // this tile's output (grouped launches: its problem's)
       bf16* const ty = a.nprob > 1 ? a.gy[gp] : a.y;
       const long long tldy = a.nprob > 1 ? a.gldy[gp] : a.ldy;
@@ -440,10 +490,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
               continue;
             }
             if (DUAL) {
+              // SiLU(g) * u = g u / (1 + 2^(-g log2 e)): hardware exp2
+              // approximation and reciprocal (relative error ~2^-22, far
+              // below the bf16 rounding of the output)
 #pragma unroll
               for (int j = 0; j < 8; ++j) {
                 const float u = __uint_as_float(r1[8 * g + j]);
-                v[j] = v[j] / (1.f + expf(-v[j])) * u;
+                float e, rc;
+                asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(v[j] * -1.4426950408889634f));
+                asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rc) : "f"(1.f + e));
+                v[j] = v[j] * rc * u;
               }
             } else {
               const int gi = PLAIN ? g : 0;
@@ -468,7 +524,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       }
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(tempty + buf);
+      if (lane == 0) {
+        if (PAIR)   // the accumulator buffer spans both CTAs: release it at the leader
+          tc::mbar_arrive_cluster(tc::mapa_shared(tc::smem_u32(tempty + buf), 0));
+        else
+          tc::mbar_arrive(tempty + buf);
+      }
       if (a.zdrop && q == 0 && part == 0) {
         // This tile's MMAs are complete: every TMA read of its z rows is
         // done.  One warp counts the block's finished column tiles; the last
@@ -477,7 +538,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         // (grouped: counters and rows per problem, whose A rows start at
         // grow[gp] and whose column tiles are pt[gp] .. pt[gp + 1])
         const int gtn = a.nprob > 1 ? (gp + 1 < a.nprob ? a.pt[gp + 1] : a.tiles_n) - a.pt[gp] : a.tiles_n;
-        const int mb = (a.nprob > 1 ? gp * a.tiles_m : 0) + t % a.tiles_m;
+        const int mb = (a.nprob > 1 ? gp * a.tiles_m * (TM / BM) : 0) + m0 / BM;
         const long long zr = a.nprob > 1 ? a.grow[gp] : 0;
         const unsigned act = __activemask();
         int last = 0;
@@ -499,9 +560,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   }
 
   __syncthreads();
+  // pair: the leader's MMAs have drained and both epilogues have read their
+  // tensor memory before either CTA frees it
+  if (PAIR) tc::cluster_sync();
   if (warp == 1) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tmem_base, L::TMEM_COLS);
+    if (PAIR)
+      tc::tmem_dealloc_pair(tmem_base, L::TMEM_COLS);
+    else
+      tc::tmem_dealloc(tmem_base, L::TMEM_COLS);
   }
 }
 
@@ -529,14 +596,14 @@ double gemm_bytes(const TcArgs& a, bool dual) {
   return 2.0 * ((double)a.M * a.K * halves + (double)a.K * a.N * halves + (double)a.M * a.N);
 }
 
-template <int BN, int STAGES, bool DUAL, int EPI>
+template <int BN, int STAGES, bool DUAL, int EPI, bool PAIR = false>
 int launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb1, const CUtensorMap& mb2,
               TcArgs a, const char* name, cudaStream_t stream) {
-  using L = Layout<BN, STAGES, DUAL>;
-  auto kern = tc_gemm_kernel<BN, STAGES, DUAL, EPI>;
+  using L = Layout<BN, STAGES, DUAL, PAIR>;
+  auto kern = tc_gemm_kernel<BN, STAGES, DUAL, EPI, PAIR>;
   static SmemAttrOnce smem_once;
   FSVD_TRY(set_smem_once(smem_once, kern, L::SMEM));
-  a.tiles_m = ceil_div(a.M, BM);
+  a.tiles_m = ceil_div(a.M, PAIR ? 2 * BM : BM);
   if (a.nprob > 1) {
     // grouped: problem i's column tiles start at pt[i]; a.N = total width
     int nt = 0;
@@ -551,10 +618,28 @@ int launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& m
     a.tiles_n = ceil_div(a.N, BN);
   }
   const int tiles = a.tiles_m * a.tiles_n;
-  const int grid = tiles < sm_count() ? tiles : sm_count();
   const double flops = 2.0 * a.M * (double)a.N * a.K * (DUAL ? 2.0 : 1.0);
   const LaunchTag tag{name, gemm_bytes(a, DUAL), flops};
+  if (PAIR) {
+    const int pairs = sm_count() / 2;
+    const int grid = 2 * (tiles < pairs ? tiles : pairs);
+    return launch_pdl_cluster(tag, 2, kern, dim3(grid), dim3(TC_THREADS), (size_t)L::SMEM, stream, ma, mb, mb1,
+                              mb2, a);
+  }
+  const int grid = tiles < sm_count() ? tiles : sm_count();
   return launch_pdl(tag, kern, dim3(grid), dim3(TC_THREADS), (size_t)L::SMEM, stream, ma, mb, mb1, mb2, a);
+}
+
+// Whether BN = 256 GEMMs of at least 256 rows run as 2-SM CTA pairs
+// (cta_group::2: each CTA loads half of B, so the operand traffic into an
+// SM per FLOP drops by a third).
+constexpr bool kGemmPairs = true;
+
+template <int EPI>
+int launch_wide(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb1, const CUtensorMap& mb2,
+                const TcArgs& a, const char* name, cudaStream_t stream) {
+  if (kGemmPairs && a.M >= 2 * BM) return launch_tc<256, 6, false, EPI, true>(ma, mb, mb1, mb2, a, name, stream);
+  return launch_tc<256, 4, false, EPI>(ma, mb, mb1, mb2, a, name, stream);
 }
 
 // One tensor-core GEMM C = A . B with the given epilogue.
@@ -564,14 +649,15 @@ int gemm(const bf16* A, long long lda, long long a_cols, const bf16* B, long lon
   FSVD_TRY(make_map(&ma, A, a.M, a_cols, lda, BM));
   if (dual) {
     FSVD_TRY(make_map(&mb, B, b_rows, a.N, ldb, BK));
+    // (single CTAs: as a 2-SM pair this dual form measured slower)
     return launch_tc<128, 6, true, PF_EPI_SWIGLU>(ma, mb, mb, mb, a, name, stream);
   }
   FSVD_TRY(make_map(&mb, B, b_rows, a.N, ldb, BK));
   switch (epi) {
-    case PF_EPI_BF16: return launch_tc<256, 4, false, PF_EPI_BF16>(ma, mb, mb, mb, a, name, stream);
-    case PF_EPI_GELU: return launch_tc<256, 4, false, PF_EPI_GELU>(ma, mb, mb, mb, a, name, stream);
-    case PF_EPI_QKV: return launch_tc<256, 4, false, PF_EPI_QKV>(ma, mb, mb, mb, a, name, stream);
-    case PF_EPI_F32: return launch_tc<256, 4, false, PF_EPI_F32>(ma, mb, mb, mb, a, name, stream);
+    case PF_EPI_BF16: return launch_wide<PF_EPI_BF16>(ma, mb, mb, mb, a, name, stream);
+    case PF_EPI_GELU: return launch_wide<PF_EPI_GELU>(ma, mb, mb, mb, a, name, stream);
+    case PF_EPI_QKV: return launch_wide<PF_EPI_QKV>(ma, mb, mb, mb, a, name, stream);
+    case PF_EPI_F32: return launch_wide<PF_EPI_F32>(ma, mb, mb, mb, a, name, stream);
     default: return FLASHSVD_ERR_INVALID_ARG;
   }
 }
@@ -593,7 +679,7 @@ int prefill_stage1_grouped(const bf16* x, long long ldx, int d, int M, int n, co
     a.gy[i] = z[i]; a.gldy[i] = r[i]; a.gN[i] = r[i];
   }
   a.y = z[0]; a.ldy = r[0];
-  return launch_tc<256, 4, false, PF_EPI_BF16>(ma, mb[0], mb[n > 1 ? 1 : 0], mb[n > 2 ? 2 : 0], a,
+  return launch_wide<PF_EPI_BF16>(ma, mb[0], mb[n > 1 ? 1 : 0], mb[n > 2 ? 2 : 0], a,
                                                "tc_stage1_xu_grouped", stream);
 }
 
@@ -629,7 +715,7 @@ int prefill_qkv_stage2_grouped(const QkvGroup& g, cudaStream_t stream) {
   CUtensorMap ma;
   FSVD_TRY(make_map(&ma, g.z, rows, g.r, g.r, BM));
   if (g.zcnt) { a.zdrop = g.z; a.zld = g.r; a.zcnt = g.zcnt; }
-  return launch_tc<256, 4, false, PF_EPI_QKV>(ma, mb[0], mb[g.n > 1 ? 1 : 0], mb[g.n > 2 ? 2 : 0], a,
+  return launch_wide<PF_EPI_QKV>(ma, mb[0], mb[g.n > 1 ? 1 : 0], mb[g.n > 2 ? 2 : 0], a,
                                               "tc_stage2_qkv_grouped", stream);
 }
 

@@ -77,6 +77,7 @@ _SIGS = {
     "flashsvd_set_decode_path": ([_i], _i),
     "flashsvd_set_prefill_attention": ([_i], _i),
     "flashsvd_set_l2_discard": ([_i], _i),
+    "flashsvd_debug_drop_barrier_arrival": ([], _i),
     "flashsvd_decode_pack_bytes": ([_p, C.POINTER(C.c_size_t)], _i),
     "flashsvd_decode_pack": ([_p, _p, C.c_size_t, _p], _i),
     "flashsvd_decode_plan_create": ([_p, _i, _p, _p, _i, _i, _p], _i),

@@ -102,7 +102,7 @@ def test_decoder_prefill_forms_q_in_attention(fs):
     # algorithmic FLOPs are those of two d-wide products, not three)
     g = prof.get("tc_stage2_qkv_grouped", {})
     assert g.get("launches") == 1, prof
-    assert g.get("flops") == 2.0 * S * (2 * d) * r, prof
+    assert abs(g.get("flops", 0.0) / (2.0 * S * (2 * d) * r) - 1.0) < 1e-6, prof
     assert prof.get("tc_stage2_qkv_rope", {}).get("launches", 0) == 0, prof
     y, k, v = oracle.decoder_layer_prefill(oracle.from_bf16(xs), oracle.widen_layer(w), H)
     assert_parity(host_f64(x), y, "layer prefill with in-kernel q")
