@@ -64,7 +64,11 @@ constexpr int DF_KC = 256;            // rows per ring entry
 constexpr int DF_MAX_SU = 16;         // tiles (or attention pairs) per CTA and stage
 constexpr int DF_PART_STRIDE = 640;   // floats per partial slot (>= 4 x 64, >= 4 + 128)
 constexpr int DF_NPHASE = 9;
-constexpr int DF_ABUF_COLS = 4096;    // floats per row of the stage-input buffer
+constexpr int DF_ABUF_COLS = 4096;    // floats per row of the stage-input buffer at MT = 1
+constexpr int DF_ABUF_WIDE = 5120;    // ... at MT >= 2 (a SwiGLU stage of r_f up to 2560)
+// Stage-input row width of the MT-row kernel (the MT = 1 kernel has no
+// shared memory left beside its six-slot ring for the wider buffer).
+__host__ __device__ constexpr int df_acols(int MT) { return MT == 1 ? DF_ABUF_COLS : DF_ABUF_WIDE; }
 constexpr int DF_MAX_PAIRS = 8;       // attention (batch, head) pairs per CTA
 constexpr int DF_MAX_NK = 64;         // 256-row chunks per factor (K <= 16384)
 constexpr int DF_CMAX = 15;           // contributing CTAs per tile (or pair) read
@@ -114,8 +118,17 @@ struct DfPhase {
                        // (a shared factor's entries live in an earlier layer's pack)
   const bf16* norm_g;
   int shared;          // entries read by several layers: loaded with an L2 evict-last hint
-  int pad_[3];
+  int ustride;         // SRC_PART stages: unit-table slots per (input chunk, segment)
+  int pad_[2];
 };
+
+// A 256-row input chunk of a SRC_PART stage spans 4 previous-stage column
+// tiles of 64 when it starts on a tile boundary (always for one segment;
+// for the SwiGLU stage's second segment when the up half's offset r_f is a
+// multiple of 64), else 5.
+inline int part_ustride(const DfPhase& ph) {
+  return (ph.map == MAP_SWIGLU && ph.a_col2 % 64) ? 5 : 4;
+}
 
 // Per (stage, CTA) schedule record, built on the host with the pack: the
 // input chunks (problem << 8 | 256-row chunk) of the CTA's entries in
@@ -169,7 +182,8 @@ struct DfCfg {
   static constexpr int THREADS = CT + 32;            // + the producer warp
   static constexpr int SLOT = 32768;
   static constexpr int NSLOT = MT == 1 ? 6 : (MT == 2 ? 5 : 4);
-  static constexpr int ABUF_BYTES = MT * DF_ABUF_COLS * 4;
+  static constexpr int ACOLS = df_acols(MT);
+  static constexpr int ABUF_BYTES = MT * ACOLS * 4;
   static constexpr int RED_BYTES = 512;              // per-warp sums of squares (RMSNorm)
   static constexpr int SCR_BYTES = (64 + CW * 128) * 4;
   static constexpr int MISC_BYTES = 6656;  // two schedule records, rstd, attention schedule
@@ -473,7 +487,7 @@ __device__ __forceinline__ void ffma2(float& a0, float& a1, float x, float y0, f
 // ring entry.  w points at the warp's region of the entry: 16-byte pieces
 // (rows 2p and 2p + 1 of the warp's 4 columns), piece p = 32 i + lane, so
 // every load of the warp reads 512 consecutive bytes.  a points at the
-// entry's input chunk (row m at m * DF_ABUF_COLS).  FULL: all 256 rows are
+// entry's input chunk (row m at m * df_acols(MT)).  FULL: all 256 rows are
 // valid; else pieces at or beyond kn / 2 are skipped (kn is even).
 template <int MT, bool FULL>
 __device__ __forceinline__ void entry_mac(float (&acc)[MT][4], const uint8_t* w, const float* a, int kn,
@@ -487,7 +501,7 @@ __device__ __forceinline__ void entry_mac(float (&acc)[MT][4], const uint8_t* w,
     u[i] = valid ? *reinterpret_cast<const uint4*>(w + pc * 16) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
     for (int m = 0; m < MT; ++m)
-      av[i][m] = valid ? *reinterpret_cast<const float2*>(a + m * DF_ABUF_COLS + 2 * pc) : make_float2(0.f, 0.f);
+      av[i][m] = valid ? *reinterpret_cast<const float2*>(a + m * df_acols(MT) + 2 * pc) : make_float2(0.f, 0.f);
   }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -552,7 +566,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* slots = smem;
-  float* abuf = reinterpret_cast<float*>(smem + C::NSLOT * C::SLOT);   // [MT][DF_ABUF_COLS]
+  float* abuf = reinterpret_cast<float*>(smem + C::NSLOT * C::SLOT);   // [MT][C::ACOLS]
   float* red = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(abuf) + C::ABUF_BYTES);
   float* scr = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(red) + C::RED_BYTES);
   uint8_t* misc = reinterpret_cast<uint8_t*>(scr) + C::SCR_BYTES;
@@ -828,7 +842,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
                 if (ph.norm) v = gain4(v, ph.norm_g, j);
               }
             }
-            *reinterpret_cast<float4*>(abuf + m * DF_ABUF_COLS + j) = v;
+            *reinterpret_cast<float4*>(abuf + m * C::ACOLS + j) = v;
           }
         }
         if (ph.norm) {
@@ -859,7 +873,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
             for (int k2 = 0; k2 < 2; ++k2) {
               if (k2 == 1 && !h1) continue;
               const int m = k2 ? m1 : m0, j = k2 ? j1 : j0;
-              float4* a4 = reinterpret_cast<float4*>(abuf + m * DF_ABUF_COLS + j);
+              float4* a4 = reinterpret_cast<float4*>(abuf + m * C::ACOLS + j);
               float4 v;
               if (src == SRC_XMID) {
                 v = *a4;
@@ -894,7 +908,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
               v = round4(make_float4(gv.x / (1.f + expf(-gv.x)) * uv.x, gv.y / (1.f + expf(-gv.y)) * uv.y,
                                      gv.z / (1.f + expf(-gv.z)) * uv.z, gv.w / (1.f + expf(-gv.w)) * uv.w));
             }
-            *reinterpret_cast<float4*>(abuf + m * DF_ABUF_COLS + ci * 256 + i) = v;
+            *reinterpret_cast<float4*>(abuf + m * C::ACOLS + ci * 256 + i) = v;
           }
         } else if (src == SRC_ATT) {
           // attention output: dims k % D .. + 3 of head k / D of row m
@@ -905,7 +919,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
             if (m < p.B && k < ph.K && nunits)
               v = round4(attn_gather4(part_prev, utab + ((ci * MT + m) * hpc + i / p.D) * 16, k % p.D));
-            *reinterpret_cast<float4*>(abuf + m * DF_ABUF_COLS + ci * 256 + i) = v;
+            *reinterpret_cast<float4*>(abuf + m * C::ACOLS + ci * 256 + i) = v;
           }
         } else if (src == SRC_PART) {
           // fp32 rank activations z (plain column tiles of 64)
@@ -924,10 +938,10 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
               float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
               if (m < p.B && k < ph.K && nunits) {
                 const int col = seg * ph.a_col2 + k, col0 = seg * ph.a_col2 + kc * DF_KC;
-                v = gather4_one(part_prev, utab + ((ci * nseg + seg) * 5 + (col >> 6) - (col0 >> 6)) * 16,
+                v = gather4_one(part_prev, utab + ((ci * nseg + seg) * ph.ustride + (col >> 6) - (col0 >> 6)) * 16,
                                 m * 64 + (col & 63));
               }
-              *reinterpret_cast<float4*>(abuf + m * DF_ABUF_COLS + ci * 256 * nseg + seg * 256 + i) = v;
+              *reinterpret_cast<float4*>(abuf + m * C::ACOLS + ci * 256 * nseg + seg * 256 + i) = v;
             }
           } else
           for (int e0 = tid; e0 < tot; e0 += 2 * C::CT) {
@@ -946,13 +960,13 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
               const int kc = clist[ci < n ? ci : 0] & 255;
               const int k = kc * DF_KC + i;
               ok[k2] = e < tot && m < p.B && k < ph.K && nunits;
-              dst[k2] = e < tot ? m * DF_ABUF_COLS + ci * 256 * nseg + seg * 256 + i : -1;
+              dst[k2] = e < tot ? m * C::ACOLS + ci * 256 * nseg + seg * 256 + i : -1;
               uu[k2] = utab;
               ww[k2] = nullptr;
               idx[k2] = 0;
               if (!ok[k2]) continue;
               const int col = seg * ph.a_col2 + k, col0 = seg * ph.a_col2 + kc * DF_KC;
-              uu[k2] = utab + ((ci * nseg + seg) * 5 + (col >> 6) - (col0 >> 6)) * 16;
+              uu[k2] = utab + ((ci * nseg + seg) * ph.ustride + (col >> 6) - (col0 >> 6)) * 16;
               idx[k2] = m * 64 + (col & 63);
             }
             float4 sv[2];
@@ -1414,6 +1428,7 @@ long long build_stages(const DecodeLayerDesc& L, DfPhase* P, PackStage* Q) {
     for (int j = ph.nprob; j < 4; ++j) ph.tile_start[j] = T;
     ph.T = T;
     ph.pack_off = off;
+    ph.ustride = part_ustride(ph);
     if (Q) {
       PackStage& q = Q[i];
       q.off = off; q.K = K; q.T = T; q.map = map; q.nprob = ph.nprob;
@@ -1479,7 +1494,7 @@ bool build_sched(const DfPhase* P, int G, int d, SchedRec* R) {
           int ci = 0;
           while (ci < r.n && r.clist[ci] != key) ++ci;
           if (ci == r.n) {
-            if (r.n == 16 || (r.n + 1) * 256 * nseg > DF_ABUF_COLS) return false;
+            if (r.n == 16 || (r.n + 1) * 256 * nseg > DF_ABUF_WIDE) return false;
             r.clist[r.n++] = key;
           }
           r.chunk_of[c - c0] = (uint8_t)ci;
@@ -1491,9 +1506,10 @@ bool build_sched(const DfPhase* P, int G, int d, SchedRec* R) {
         for (int t = 0; t < r.nunits; ++t)
           if (!tile_slots(P[4], t, G, r.utab[t])) return false;
       } else if (ph.src == SRC_PART) {
-        r.nunits = r.n * nseg * 5;
+        const int us = ph.ustride;
+        r.nunits = r.n * nseg * us;
         for (int ui = 0; ui < r.nunits; ++ui) {
-          const int j = ui % 5, cs = ui / 5, seg = cs % nseg, ci = cs / nseg;
+          const int j = ui % us, cs = ui / us, seg = cs % nseg, ci = cs / nseg;
           const int pi = r.clist[ci] >> 8, kc = r.clist[ci] & 255;
           const int col0 = seg * ph.a_col2 + kc * DF_KC;
           const int kn = std::min(DF_KC, ph.K - kc * DF_KC);
@@ -1557,9 +1573,9 @@ bool stages_fit(const DfPhase* P, int G, int MT, int D) {
           if (t >= ph.tile_start[j]) pi = j;
         if (!seen[pi][kc]) { seen[pi][kc] = true; ++n; }
       }
-      if (n * 256 * nseg > DF_ABUF_COLS) return false;
+      if (n * 256 * nseg > df_acols(MT)) return false;
       int units = 0;
-      if (ph.src == SRC_PART) units = n * nseg * 5;
+      if (ph.src == SRC_PART) units = n * nseg * ph.ustride;
       else if (ph.src == SRC_SWIGLU) units = n * 8;
       else if (ph.src == SRC_ATT) units = n * MT * (DF_KC / D);
       if (units > DF_MAX_UNITS) return false;

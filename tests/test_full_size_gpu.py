@@ -298,3 +298,40 @@ def test_decoder_model_teacher_forced(fs):
         assert_parity(logits[t + 1], ref, f"logits after decode step {t}")
         agree += int(np.argmax(ref) == toks[t + 1])
     print(f"greedy token agreement with the oracle: {agree}/{steps + 1}")
+
+
+@pytest.mark.parametrize("B", [1, 2, 4])
+def test_decode_layer_rank_2368(fs, B):
+    """A retention-0.8 7B-shaped layer (ranks 1664 / 2368: the SwiGLU stage
+    input is 2 x 2368 values) decoding at context 1024.  At B = 2 and 4 the
+    fused kernel takes it (its wider stage-input buffer); at B = 1 the layer
+    runs the per-stage kernels.  Both against the oracle."""
+    from tests.test_decode_gpu import _layer_struct
+    d, H, D, f, r, r_f, P = 4096, 32, 128, 11008, 1664, 2368, 1024
+    S_max = P + 4
+    rng = synth.rng_for(9900 + B)
+    w = synth.decoder_layer_weights(rng, d, f, r, r_f, gain_jitter=0.1)
+    cos_t = torch.empty((S_max, D // 2), dtype=torch.float32, device="cuda")
+    sin_t = torch.empty_like(cos_t)
+    fs.rope_table(cos_t, sin_t, S_max, D, 10000.0)
+    L, dev = _layer_struct(fs, w, d, H, D, f, r, r_f, cos_t, sin_t)
+    kc0 = synth.normal_bf16(rng, (B, S_max, H, D))
+    vc0 = synth.normal_bf16(rng, (B, S_max, H, D))
+    xt = synth.normal_bf16(rng, (B, d))
+    kc, vc = dev_bf16(kc0), dev_bf16(vc0)
+    seq = torch.full((B,), P, dtype=torch.int32, device="cuda")
+    x = dev_bf16(xt)
+    torch.cuda.synchronize()
+    fs.profile_enable(True)
+    try:
+        fs.layer_forward(L, x, kc, vc, seq, B, 1, S_max, fs.DECODE)
+        prof = fs.profile_report(reset=True)
+    finally:
+        fs.profile_enable(False)
+    fs.check_device_status()
+    fused = prof.get("decode_layer_fused", {}).get("launches", 0) == 1
+    assert fused == (B > 1), prof
+    y, kn, vn = oracle.decoder_layer_decode(oracle.from_bf16(xt), oracle.widen_layer(w), H,
+                                            oracle.from_bf16(kc0), oracle.from_bf16(vc0), [P] * B)
+    assert_parity(host_f64(x), y, f"rank-2368 decode layer B={B}")
+    assert_parity(host_f64(kc)[:, P], kn, f"rank-2368 appended k B={B}")
