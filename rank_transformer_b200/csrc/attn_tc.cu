@@ -7,16 +7,21 @@
 //
 // Persistent CTAs (one per SM) walk the (128-query tile, batch row, head)
 // items, heaviest first; 10 warps:
-//   warp 0  TMA: Q once, then 128-key K and V tiles into a 2-stage ring;
+//   warp 0  TMA: Q once, then 128-key K and V tiles into two rings of their
+//           own (K one tile ahead of V), so a K tile waits only for the S
+//           MMA that read its slot and a V tile for the P V MMA;
 //   warp 1  TMEM owner and MMA issuer: S = Q K^T into one of two 128-column
-//           TMEM buffers, then O += P V into a D-column TMEM accumulator;
+//           TMEM buffers, then O += P V into a D-column TMEM accumulator,
+//           with P read from TMEM (the A operand of a TMEM-A MMA);
 //   warps 2-9  two threads per query row (each half of the keys and of O):
-//           load S from TMEM, mask, online softmax (exp2 domain, the row max
-//           exchanged through shared memory), rescale O in TMEM when the
-//           row's reference max moves, write P (bf16) into 128-byte-swizzled
-//           shared memory as the next MMA's A operand; at the end O / l.
-// All operand tiles are 128-byte swizzled; S of tile j+1 is computed while
-// the softmax of tile j runs.  Every wait is bounded.
+//           load the row of S from TMEM (both halves, so each thread has
+//           the row max without an exchange), mask, online softmax (exp2
+//           domain), rescale O in TMEM when the row's reference max moves,
+//           write P (bf16 pairs) into one of two 64-column TMEM buffers; at
+//           the end O / l.
+// S of tile j+1 and P V of tile j-1 run on the tensor cores while the
+// softmax of tile j runs: the softmax waits for P V only when it rescales O
+// or reuses a P buffer.  Every wait is bounded.
 //
 // Factorized form (QF, FlashSVD v1.5 explainer, Methodology 2, "Prefill":
 // a dedicated factorized attention kernel avoids dense materialisation):
@@ -44,6 +49,46 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// (x0, x1) -> (2^x0, 2^x1) on the FMA and integer pipes, leaving the
+// special-function unit (16 results per clock per SM, the softmax's limit)
+// to the other elements.  Range reduction x = j + f with j = round(x) (adding
+// 1.5 * 2^23 leaves j in the low mantissa bits) and f in [-1/2, 1/2]; 2^f by
+// a cubic fitted to it on that interval (relative error below 7.5e-5, well
+// under the bf16 rounding of P); 2^j by adding j to the exponent field.
+// Inputs are clamped at -125, so the result stays a normal number: a masked
+// key (-inf) gives 2^-125 instead of 0, below every fp32 rounding step of l
+// and of O.
+__device__ __forceinline__ void ex2_poly2(float& x0, float& x1) {
+  constexpr float C0 = 0.99992806f, C1 = 0.69326097f, C2 = 0.24261113f, C3 = 0.05517165f;
+  x0 = fmaxf(x0, -125.f);
+  x1 = fmaxf(x1, -125.f);
+  uint32_t t0, t1;
+  asm("{\n\t.reg .b64 xx, tt, jj, ff, pp, cc;\n\t"
+      "mov.b64 xx, {%2, %3};\n\t"
+      "mov.b64 cc, {%4, %4};\n\t"
+      "add.rn.f32x2 tt, xx, cc;\n\t"           // t = x + 1.5 * 2^23
+      "mov.b64 cc, {%5, %5};\n\t"
+      "add.rn.f32x2 jj, tt, cc;\n\t"           // j = t - 1.5 * 2^23 (exact)
+      "mov.b64 cc, {%6, %6};\n\t"
+      "fma.rn.f32x2 ff, jj, cc, xx;\n\t"       // f = x - j (exact)
+      "mov.b64 pp, {%7, %7};\n\t"
+      "mov.b64 cc, {%8, %8};\n\t"
+      "fma.rn.f32x2 pp, pp, ff, cc;\n\t"
+      "mov.b64 cc, {%9, %9};\n\t"
+      "fma.rn.f32x2 pp, pp, ff, cc;\n\t"
+      "mov.b64 cc, {%10, %10};\n\t"
+      "fma.rn.f32x2 pp, pp, ff, cc;\n\t"
+      "mov.b64 {%0, %1}, pp;\n\t"
+      "mov.b64 {%2, %3}, tt;\n\t}"
+      : "=r"(t0), "=r"(t1), "+f"(x0), "+f"(x1)
+      : "f"(12582912.f), "f"(-12582912.f), "f"(-1.f), "f"(C3), "f"(C2), "f"(C1), "f"(C0));
+  // t0, t1: 2^f bits; x0, x1: the bits of t, whose low 9 bits are j
+  x0 = __uint_as_float(t0 + (__float_as_uint(x0) << 23));
+  x1 = __uint_as_float(t1 + (__float_as_uint(x1) << 23));
+}
+// Of every 4 element pairs of a row's P, this many take ex2_poly2.
+constexpr int AT_EMU = 1;
+
 // max(a, b, c) in one instruction.
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
@@ -76,15 +121,21 @@ template <int D>
 struct AtLayout {
   static constexpr int KB = D / 64;              // 64-column blocks of a head
   static constexpr int TILE = AT_BN * 128;       // one [128 x 64] bf16 block, 16 KB
+  static constexpr int NST = D == 64 ? 4 : 3;    // stages of the K ring and of the V ring
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + KB * TILE;
-  static constexpr int V_OFF = K_OFF + 2 * KB * TILE;
-  static constexpr int P_OFF = V_OFF + 2 * KB * TILE;
-  static constexpr int BAR_OFF = P_OFF + 2 * TILE;
-  static constexpr int X_OFF = BAR_OFF + 256;     // [2 tiles][2 halves][128] row partials
-  static constexpr int SMEM = 1024 + X_OFF + 2 * 2 * 128 * 4;
+  static constexpr int V_OFF = K_OFF + NST * KB * TILE;
+  static constexpr int BAR_OFF = V_OFF + NST * KB * TILE;
+  static constexpr int X_OFF = BAR_OFF + 512;     // [2 halves][128] row sums l
+  static constexpr int SMEM = 1024 + X_OFF + 2 * 128 * 4;
   static_assert(SMEM <= 232448, "shared memory budget");
 };
+// TMEM columns: S buffers [0, 128) and [128, 256), O [256, 256 + D), P
+// buffers (bf16 pairs, 64 columns each) [384, 448) and [448, 512); the
+// factorized form accumulates Q in [384, 384 + D), over the P buffers,
+// between the previous item's last P V and the item's first P.
+constexpr uint32_t AT_TM_O = 256;
+constexpr uint32_t AT_TM_P = 384;
 
 struct AtParams {
   int B, S, H, S_max;
@@ -107,14 +158,17 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   using L = AtLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  constexpr int NST = L::NST;
   uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
-  uint64_t* kv_full = q_full + 1;    // [2]
-  uint64_t* kv_empty = kv_full + 2;  // [2]
-  uint64_t* s_full = kv_empty + 2;   // [2]
+  uint64_t* k_full = q_full + 1;     // [NST]
+  uint64_t* k_empty = k_full + NST;  // [NST]
+  uint64_t* v_full = k_empty + NST;  // [NST]
+  uint64_t* v_empty = v_full + NST;  // [NST]
+  uint64_t* s_full = v_empty + NST;  // [2]
   uint64_t* s_empty = s_full + 2;    // [2]
-  uint64_t* p_full = s_empty + 2;
-  uint64_t* o_done = p_full + 1;
-  uint64_t* drain = o_done + 1;
+  uint64_t* p_full = s_empty + 2;    // [2] P buffer written (count 8)
+  uint64_t* o_done = p_full + 2;     // [2] P V of a tile using that P buffer done
+  uint64_t* drain = o_done + 2;
   uint64_t* q_empty = drain + 1;     // the item's S MMAs are done: Q may be reloaded
   uint64_t* o_free = q_empty + 1;    // the epilogue has read O (count 8)
   uint64_t* qacc_full = o_free + 1;  // QF: the item's Q = z_q V_q is in TMEM
@@ -124,12 +178,21 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Persistent: work item k = (query tile, batch row, head), heaviest
-  // (longest causal) query tiles first; CTA c takes items c, c + G, ...
+  // (longest causal) query tiles first.  CTA c of G takes one item per round
+  // of G, in snake order (round i: item i G + c, or i G + G - 1 - c when i
+  // is odd), which pairs heavy causal tiles with light ones: at 16 query
+  // tiles x 32 heads on 148 CTAs the longest CTA walks 31 key tiles (the
+  // mean is 29.4) instead of 38 with a plain stride.
   // Barrier phases run on across items: T counts this CTA's key tiles, I
   // its items.
   const int qtiles = (p.S + AT_BM - 1) / AT_BM;
   const int BH = p.B * p.H;
   const int NW = qtiles * BH;
+  const int G = gridDim.x, cta = blockIdx.x;
+  const int full_rounds = NW / G, rem = NW - full_rounds * G;
+  const int n_items =
+      full_rounds + ((rem > 0 && ((full_rounds & 1) ? (G - 1 - cta) < rem : cta < rem)) ? 1 : 0);
+  auto item_k = [&](int i) { return i * G + ((i & 1) ? G - 1 - cta : cta); };
   const int nt_all = (p.S + AT_BN - 1) / AT_BN;
   struct Item { int b, h, m0, nt; };
   auto item_of = [&](int k) {
@@ -148,14 +211,18 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     tc::mbar_init(q_full, QF ? 8 : 1);
     tc::mbar_init(qacc_full, 1);
     tc::mbar_init(qacc_free, 8);
+    for (int i = 0; i < NST; ++i) {
+      tc::mbar_init(k_full + i, 1);
+      tc::mbar_init(k_empty + i, 1);
+      tc::mbar_init(v_full + i, 1);
+      tc::mbar_init(v_empty + i, 1);
+    }
     for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(kv_full + i, 1);
-      tc::mbar_init(kv_empty + i, 1);
       tc::mbar_init(s_full + i, 1);
       tc::mbar_init(s_empty + i, 8);
+      tc::mbar_init(p_full + i, 8);
+      tc::mbar_init(o_done + i, 1);
     }
-    tc::mbar_init(p_full, 8);
-    tc::mbar_init(o_done, 1);
     tc::mbar_init(drain, 1);
     tc::mbar_init(q_empty, 1);
     tc::mbar_init(o_free, 8);
@@ -169,7 +236,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     if (QF) tc::tma_prefetch_desc(&tmVq);
   }
   if (warp == 1) {
-    tc::tmem_alloc(tmem_holder, 512);  // S0 [0,128), S1 [128,256), O [256, 256 + D), QF: Q [384, 384 + D)
+    tc::tmem_alloc(tmem_holder, 512);
     tc::tmem_relinquish();
     tc::fence_before_sync();
   }
@@ -183,10 +250,13 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA --
     if (lane == 0) {
-      int R = 0;  // ring uses of this CTA (K/V tiles, and QF's z_q / V_q k-blocks)
+      // R counts this CTA's ring uses; the K and V rings advance together
+      // (a QF k-block stage fills both, a key tile one of each).
+      int R = 0;
       bool ok = true;
-      for (int k = blockIdx.x, I = 0; k < NW && ok; k += gridDim.x, ++I) {
-        const Item it = item_of(k);
+      auto ring_ph = [](int rr) { return ((uint32_t)(rr / NST) & 1u) ^ 1u; };
+      for (int I = 0; I < n_items && ok; ++I) {
+        const Item it = item_of(item_k(I));
         const int hx = it.h * D;
         if (!QF) {
           if (!(ok = tc::mbar_wait(q_empty, ((uint32_t)I & 1u) ^ 1u, abort_flag, p.status))) break;
@@ -194,34 +264,51 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           for (int kb = 0; kb < L::KB; ++kb)
             tc::tma_load_2d(smem + L::Q_OFF + kb * L::TILE, &tmQ, q_full, hx + 64 * kb, it.b * p.S + it.m0);
         } else {
-          // z_q rows of the tile (K region) and V_q[:, head] (V region), KB
-          // k-blocks of 64 per ring stage
+          // z_q rows of the tile (K ring) and V_q[:, head] (V ring), KB
+          // k-blocks of 64 per stage
           for (int sq = 0; sq < nqs && ok; ++sq) {
-            const int rr = R + sq, st = rr & 1;
-            if (!(ok = tc::mbar_wait(kv_empty + st, ((uint32_t)(rr >> 1) & 1u) ^ 1u, abort_flag, p.status))) break;
+            const int rr = R + sq, st = rr % NST;
+            if (!(ok = tc::mbar_wait(k_empty + st, ring_ph(rr), abort_flag, p.status))) break;
+            if (!(ok = tc::mbar_wait(v_empty + st, ring_ph(rr), abort_flag, p.status))) break;
             const int nb = min(L::KB, p.nq - sq * L::KB);
-            tc::mbar_expect_tx(kv_full + st, (uint32_t)(nb * (L::TILE + L::KB * 8192)));
+            tc::mbar_expect_tx(k_full + st, (uint32_t)(nb * L::TILE));
+            tc::mbar_expect_tx(v_full + st, (uint32_t)(nb * L::KB * 8192));
             for (int kb = 0; kb < nb; ++kb) {
               const int kq = sq * L::KB + kb;
-              tc::tma_load_2d(smem + L::K_OFF + (st * L::KB + kb) * L::TILE, &tmQ, kv_full + st, kq * 64,
+              tc::tma_load_2d(smem + L::K_OFF + (st * L::KB + kb) * L::TILE, &tmQ, k_full + st, kq * 64,
                               it.b * p.S + it.m0);
               uint8_t* vdst = smem + L::V_OFF + st * L::KB * L::TILE + kb * L::KB * 8192;
               for (int j = 0; j < L::KB; ++j)
-                tc::tma_load_2d(vdst + j * 8192, &tmVq, kv_full + st, hx + 64 * j, kq * 64);
+                tc::tma_load_2d(vdst + j * 8192, &tmVq, v_full + st, hx + 64 * j, kq * 64);
             }
           }
           if (!ok) break;
           R += nqs;
         }
-        for (int j = 0; j < it.nt; ++j) {
-          const int t = R + j, st = t & 1;
-          if (!(ok = tc::mbar_wait(kv_empty + st, ((uint32_t)(t >> 1) & 1u) ^ 1u, abort_flag, p.status))) break;
-          tc::mbar_expect_tx(kv_full + st, (uint32_t)(2 * L::KB * L::TILE));
-          const int row = it.b * p.S_max + j * AT_BN;
-          for (int kb = 0; kb < L::KB; ++kb) {
-            tc::tma_load_2d(smem + L::K_OFF + (st * L::KB + kb) * L::TILE, &tmK, kv_full + st, hx + 64 * kb, row);
-            tc::tma_load_2d(smem + L::V_OFF + (st * L::KB + kb) * L::TILE, &tmV, kv_full + st, hx + 64 * kb, row);
-          }
+        // key tiles: K(0), then K(j + 1) before V(j)
+        const int row0 = it.b * p.S_max;
+        auto load_k = [&](int j) {
+          const int rr = R + j, st = rr % NST;
+          if (!tc::mbar_wait(k_empty + st, ring_ph(rr), abort_flag, p.status)) return false;
+          tc::mbar_expect_tx(k_full + st, (uint32_t)(L::KB * L::TILE));
+          for (int kb = 0; kb < L::KB; ++kb)
+            tc::tma_load_2d(smem + L::K_OFF + (st * L::KB + kb) * L::TILE, &tmK, k_full + st, hx + 64 * kb,
+                            row0 + j * AT_BN);
+          return true;
+        };
+        auto load_v = [&](int j) {
+          const int rr = R + j, st = rr % NST;
+          if (!tc::mbar_wait(v_empty + st, ring_ph(rr), abort_flag, p.status)) return false;
+          tc::mbar_expect_tx(v_full + st, (uint32_t)(L::KB * L::TILE));
+          for (int kb = 0; kb < L::KB; ++kb)
+            tc::tma_load_2d(smem + L::V_OFF + (st * L::KB + kb) * L::TILE, &tmV, v_full + st, hx + 64 * kb,
+                            row0 + j * AT_BN);
+          return true;
+        };
+        if (it.nt > 0) ok = load_k(0);
+        for (int j = 0; j < it.nt && ok; ++j) {
+          if (j + 1 < it.nt) ok = load_k(j + 1);
+          ok = ok && load_v(j);
         }
         R += it.nt;
       }
@@ -232,51 +319,59 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       constexpr uint32_t IDESC_S = tc::idesc_bf16(AT_BN, false);  // B = K rows, K-major
       constexpr uint32_t IDESC_O = tc::idesc_bf16(D, true);       // B = V rows, MN-major
       const uint32_t sq = tc::smem_u32(smem + L::Q_OFF);
-      const uint32_t sp = tc::smem_u32(smem + L::P_OFF);
       bool ok = true;
-      int T = 0;  // S tiles of this CTA (S buffers, P, O barriers)
+      int T = 0;  // S tiles of this CTA (S and P buffers, their barriers)
       int R = 0;  // ring uses of this CTA
-      for (int k = blockIdx.x, I = 0; k < NW && ok; k += gridDim.x, ++I) {
-        const Item it = item_of(k);
+      auto ring_ph = [](int rr) { return (uint32_t)(rr / NST) & 1u; };
+      for (int I = 0; I < n_items && ok; ++I) {
+        const Item it = item_of(item_k(I));
         // O (+)= P_t V_t once the softmax has written P_t (and rescaled O);
         // an item's first P V overwrites O, so the previous item's epilogue
-        // must have read it.  V_t sits in ring stage rr & 1.
+        // must have read it.  V_t sits in V ring stage rr % NST.
         auto issue_pv = [&](int t, int rr, bool first) {
-          if (!tc::mbar_wait(p_full, (uint32_t)t & 1u, abort_flag, p.status)) return false;
+          const int pb = t & 1, st = rr % NST;
+          if (!tc::mbar_wait(p_full + pb, (uint32_t)(t >> 1) & 1u, abort_flag, p.status)) return false;
+          if (!tc::mbar_wait(v_full + st, ring_ph(rr), abort_flag, p.status)) return false;
           if (first && !tc::mbar_wait(o_free, ((uint32_t)I & 1u) ^ 1u, abort_flag, p.status)) return false;
           tc::fence_after_sync();
-          const uint32_t sv = tc::smem_u32(smem + L::V_OFF + (rr & 1) * L::KB * L::TILE);
+          const uint32_t sv = tc::smem_u32(smem + L::V_OFF + st * L::KB * L::TILE);
 #pragma unroll
           for (int kk = 0; kk < AT_BN / 16; ++kk) {
-            const uint64_t ad = tc::sdesc_sw128(sp + (kk >> 2) * L::TILE + (kk & 3) * 32, 16, 1024);
             const uint64_t bd = tc::sdesc_sw128(sv + kk * 2048, L::TILE, 1024);
-            tc::mma_bf16(tmem + 256, ad, bd, IDESC_O, (!first || kk > 0) ? 1u : 0u);
+            tc::mma_bf16_ts(tmem + AT_TM_O, tmem + AT_TM_P + pb * 64 + kk * 8, bd, IDESC_O,
+                            (!first || kk > 0) ? 1u : 0u);
           }
-          tc::mma_commit(o_done);
-          tc::mma_commit(kv_empty + (rr & 1));
+          tc::mma_commit(o_done + pb);
+          tc::mma_commit(v_empty + st);
           return true;
         };
         if (QF) {
-          // Q = z_q V_q[:, head] into TMEM columns 384.. once the softmax
-          // warps have read the previous item's Q
+          // Q = z_q V_q[:, head] into TMEM columns 384.. (over the P
+          // buffers) once the softmax warps have read the previous item's Q
+          // and the previous item's last P V has read its P
           if (!(ok = tc::mbar_wait(qacc_free, ((uint32_t)I & 1u) ^ 1u, abort_flag, p.status))) break;
-          for (int sq = 0; sq < nqs && ok; ++sq) {
-            const int rr = R + sq, st = rr & 1;
-            if (!(ok = tc::mbar_wait(kv_full + st, (uint32_t)(rr >> 1) & 1u, abort_flag, p.status))) break;
+          if (T > 0 && !(ok = tc::mbar_wait(o_done + ((T - 1) & 1), (uint32_t)((T - 1) >> 1) & 1u, abort_flag,
+                                            p.status)))
+            break;
+          for (int sq2 = 0; sq2 < nqs && ok; ++sq2) {
+            const int rr = R + sq2, st = rr % NST;
+            if (!(ok = tc::mbar_wait(k_full + st, ring_ph(rr), abort_flag, p.status))) break;
+            if (!(ok = tc::mbar_wait(v_full + st, ring_ph(rr), abort_flag, p.status))) break;
             tc::fence_after_sync();
-            const int nb = min(L::KB, p.nq - sq * L::KB);
+            const int nb = min(L::KB, p.nq - sq2 * L::KB);
             for (int kb = 0; kb < nb; ++kb) {
-              const int kq = sq * L::KB + kb;
+              const int kq = sq2 * L::KB + kb;
               const uint32_t sz = tc::smem_u32(smem + L::K_OFF + (st * L::KB + kb) * L::TILE);
               const uint32_t svq = tc::smem_u32(smem + L::V_OFF + st * L::KB * L::TILE + kb * L::KB * 8192);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
                 const uint64_t ad = tc::sdesc_sw128(sz + kk * 32, 16, 1024);
                 const uint64_t bd = tc::sdesc_sw128(svq + kk * 2048, 8192, 1024);
-                tc::mma_bf16(tmem + 384, ad, bd, IDESC_O, (kq > 0 || kk > 0) ? 1u : 0u);
+                tc::mma_bf16(tmem + AT_TM_P, ad, bd, IDESC_O, (kq > 0 || kk > 0) ? 1u : 0u);
               }
             }
-            tc::mma_commit(kv_empty + st);
+            tc::mma_commit(k_empty + st);
+            tc::mma_commit(v_empty + st);
           }
           if (!ok) break;
           R += nqs;
@@ -284,19 +379,20 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         }
         if (!(ok = tc::mbar_wait(q_full, (uint32_t)I & 1u, abort_flag, p.status))) break;
         for (int j = 0; j < it.nt && ok; ++j) {
-          const int t = T + j, st = t & 1;
-          const int rr = R + j, sr = rr & 1;
-          if (!(ok = tc::mbar_wait(kv_full + sr, (uint32_t)(rr >> 1) & 1u, abort_flag, p.status))) break;
-          if (!(ok = tc::mbar_wait(s_empty + st, ((uint32_t)(t >> 1) & 1u) ^ 1u, abort_flag, p.status))) break;
+          const int t = T + j, sb = t & 1;
+          const int rr = R + j, st = rr % NST;
+          if (!(ok = tc::mbar_wait(k_full + st, ring_ph(rr), abort_flag, p.status))) break;
+          if (!(ok = tc::mbar_wait(s_empty + sb, ((uint32_t)(t >> 1) & 1u) ^ 1u, abort_flag, p.status))) break;
           tc::fence_after_sync();
-          const uint32_t sk = tc::smem_u32(smem + L::K_OFF + sr * L::KB * L::TILE);
+          const uint32_t sk = tc::smem_u32(smem + L::K_OFF + st * L::KB * L::TILE);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t ad = tc::sdesc_sw128(sq + (kk >> 2) * L::TILE + (kk & 3) * 32, 16, 1024);
             const uint64_t bd = tc::sdesc_sw128(sk + (kk >> 2) * L::TILE + (kk & 3) * 32, 16, 1024);
-            tc::mma_bf16(tmem + st * AT_BN, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+            tc::mma_bf16(tmem + sb * AT_BN, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
           }
-          tc::mma_commit(s_full + st);
+          tc::mma_commit(s_full + sb);
+          tc::mma_commit(k_empty + st);
           if (j > 0) ok = issue_pv(t - 1, rr - 1, j == 1);
         }
         if (!ok) break;
@@ -314,20 +410,21 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     // ------------------------------------------------- softmax, epilogue --
     // Warp w (2..9) reads TMEM lanes 32 (w % 4) .. + 31; warps 2-5 take keys
     // [0, 64) of a tile and O columns [0, D/2), warps 6-9 the other halves.
+    // Both threads of a row read the whole row of S, so they take the same
+    // row max (and the same rescale decisions) without an exchange.
     const int quad = warp & 3;
     const int hf = (warp - 2) >> 2;
     const int r = quad * 32 + lane;       // query row within the tile
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-    float* xr = reinterpret_cast<float*>(smem + L::X_OFF);  // [2][2][128]
+    float* xr = reinterpret_cast<float*>(smem + L::X_OFF);  // [2 halves][128]
     const float sc = p.scale_log2;
     float m, l;                           // m: reference max, scaled units
-    uint8_t* sP = smem + L::P_OFF;
     constexpr int HC = AT_BN / 2;         // keys per thread
     constexpr int OC = D / 2;             // O columns per thread
     // tcgen05.ld / st are warp-collective: wait results are made
-    // warp-uniform.  The 8 softmax warps meet at a named barrier every tile,
-    // so the loop never exits early: after a failed wait it runs on without
-    // touching tensor memory.
+    // warp-uniform.  The 8 softmax warps meet at a named barrier every
+    // item, so the loop never exits early: after a failed wait it runs on
+    // without touching tensor memory.
     auto wwait = [&](uint64_t* bar, uint32_t par) {
       return __all_sync(0xffffffffu, tc::mbar_wait(bar, par, abort_flag, p.status)) != 0;
     };
@@ -336,8 +433,8 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     int T = 0;
     // (every item and tile is visited even after a failed wait, so that the
     // named barriers stay matched)
-    for (int k = blockIdx.x, I = 0; k < NW; k += gridDim.x, ++I) {
-    const Item it = item_of(k);
+    for (int I = 0; I < n_items; ++I) {
+    const Item it = item_of(item_k(I));
     const int m0 = it.m0, nt = it.nt, b = it.b, h = it.h;
     const int q = m0 + r;                 // query position
     m = -INFINITY;
@@ -352,9 +449,11 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       uint32_t qa[32], qb[32];
       if (ok) {
         tc::fence_after_sync();
-        tc::tmem_ld32(tmem + lane_base + 384 + base0, qa);
-        tc::tmem_ld32(tmem + lane_base + 384 + base0 + D / 2, qb);
+        tc::tmem_ld32(tmem + lane_base + AT_TM_P + base0, qa);
+        tc::tmem_ld32(tmem + lane_base + AT_TM_P + base0 + D / 2, qb);
         tc::tmem_ld_wait();
+        tc::reg_fence<32>(qa);
+        tc::reg_fence<32>(qb);
         if (p.zcnt && warp == 2) {
           // every Q MMA of this item has completed, so every TMA read of
           // its z_q rows is done; the last of the H heads' items drops the
@@ -418,43 +517,55 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       }
     }
     for (int j = 0; j < nt; ++j) {
-      const int t = T + j, st = t & 1;
-      ok = ok && wwait(s_full + st, (uint32_t)(t >> 1) & 1u);
-      float s[HC];
+      const int t = T + j, sb = t & 1;
+      // the P V of tile t - 2 must have read P buffer sb (checked first: it
+      // has normally long completed)
+      if (t >= 2) ok = ok && wwait(o_done + sb, (uint32_t)((t - 2) >> 1) & 1u);
+      ok = ok && wwait(s_full + sb, (uint32_t)(t >> 1) & 1u);
+      float s[HC], so[HC];  // this thread's half of the keys, the other half
+      const bool masked = j * AT_BN + AT_BN > p.S || (CAUSAL && j * AT_BN + AT_BN - 1 > m0);
+      const int n0 = j * AT_BN + hf * HC, n1 = j * AT_BN + (1 - hf) * HC;
+      float mx8[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) mx8[c] = -INFINITY;
       if (ok) {
         tc::fence_after_sync();
+        const uint32_t sa = tmem + lane_base + sb * AT_BN;
+        // this thread's half first; its max runs while the other half loads
+#pragma unroll
+        for (int c = 0; c < HC / 32; ++c) tc::tmem_ld32(sa + hf * HC + c * 32, reinterpret_cast<uint32_t*>(s + c * 32));
+        tc::tmem_ld_wait();
+        tc::reg_fence<HC>(s);
 #pragma unroll
         for (int c = 0; c < HC / 32; ++c)
-          tc::tmem_ld32(tmem + lane_base + st * AT_BN + hf * HC + c * 32, reinterpret_cast<uint32_t*>(s + c * 32));
+          tc::tmem_ld32(sa + (1 - hf) * HC + c * 32, reinterpret_cast<uint32_t*>(so + c * 32));
+        // mask (raw scores: the scale is positive) and row max
+        if (masked) {
+#pragma unroll
+          for (int c = 0; c < HC; ++c)
+            if (n0 + c >= p.S || (CAUSAL && n0 + c > q)) s[c] = -INFINITY;
+        }
+#pragma unroll
+        for (int c = 0; c < HC; c += 2) mx8[(c >> 1) & 3] = max3(mx8[(c >> 1) & 3], s[c], s[c + 1]);
         tc::tmem_ld_wait();
+        tc::reg_fence<HC>(so);
       } else {
 #pragma unroll
-        for (int c = 0; c < HC; ++c) s[c] = -INFINITY;
+        for (int c = 0; c < HC; ++c) s[c] = so[c] = -INFINITY;
       }
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(s_empty + st);
-      // mask (raw scores: the scale is positive) and partial row max
-      const int n0 = j * AT_BN + hf * HC;
-      const bool need_mask = n0 + HC > p.S || (CAUSAL && n0 + HC - 1 > m0);
-      if (need_mask) {
+      if (lane == 0) tc::mbar_arrive(s_empty + sb);
+      if (masked) {
 #pragma unroll
-        for (int c = 0; c < HC; ++c) {
-          const int key = n0 + c;
-          if (key >= p.S || (CAUSAL && key > q)) s[c] = -INFINITY;
-        }
+        for (int c = 0; c < HC; ++c)
+          if (n1 + c >= p.S || (CAUSAL && n1 + c > q)) so[c] = -INFINITY;
       }
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c = 0; c < HC; c += 2) mx4[(c >> 1) & 3] = max3(mx4[(c >> 1) & 3], s[c], s[c + 1]);
-      float* xt = xr + st * 256;
-      xt[hf * 128 + r] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-      sm_sync();
-      const float rawmax = fmaxf(xt[r], xt[128 + r]);
+      for (int c = 0; c < HC; c += 2) mx8[4 + ((c >> 1) & 3)] = max3(mx8[4 + ((c >> 1) & 3)], so[c], so[c + 1]);
+      const float rawmax = fmaxf(fmaxf(max3(mx8[0], mx8[1], mx8[2]), max3(mx8[3], mx8[4], mx8[5])),
+                                 fmaxf(mx8[6], mx8[7]));
       const float mx = rawmax == -INFINITY ? -INFINITY : rawmax * sc;
-      // PV of tile j-1 must be complete before O is rescaled or P rewritten
-      if (j > 0) ok = ok && wwait(o_done, (uint32_t)(t - 1) & 1u);
-      tc::fence_after_sync();
       // The row's reference m (P = 2^(s sc - m)) moves up only when the tile
       // max exceeds it by more than 8: P stays <= 2^8 (exact enough in bf16
       // and in the fp32 sums), O and l keep the same reference, and O is
@@ -463,52 +574,60 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       const float m_new = raise ? fmaxf(mx, m) : m;
       const bool grow = j > 0 && raise && m != -INFINITY;
       if (ok && __any_sync(0xffffffffu, grow)) {
-        const float corr = grow ? exp2f(m - m_new) : 1.f;
-        l *= corr;
+        // every P V so far (they complete in order) must be done
+        ok = wwait(o_done + ((t - 1) & 1), (uint32_t)((t - 1) >> 1) & 1u);
+        if (ok) {
+          tc::fence_after_sync();
+          const float corr = grow ? exp2f(m - m_new) : 1.f;
+          l *= corr;
 #pragma unroll
-        for (int c = 0; c < OC / 32; ++c) {
-          uint32_t o[32];
-          tc::tmem_ld32(tmem + lane_base + 256 + hf * OC + c * 32, o);
-          tc::tmem_ld_wait();
+          for (int c = 0; c < OC / 32; ++c) {
+            uint32_t o[32];
+            tc::tmem_ld32(tmem + lane_base + AT_TM_O + hf * OC + c * 32, o);
+            tc::tmem_ld_wait();
+            tc::reg_fence<32>(o);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
-          tc::tmem_st32(tmem + lane_base + 256 + hf * OC + c * 32, o);
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
+            tc::tmem_st32(tmem + lane_base + AT_TM_O + hf * OC + c * 32, o);
+          }
+          tc::tmem_st_wait();
         }
-        tc::tmem_st_wait();
       }
       m = m_new;
-      // P = 2^(s sc - m), bf16, this half of row r of the swizzled A operand
+      // P = 2^(s sc - m) as bf16 pairs into this half of P buffer sb
       const float mneg = m == -INFINITY ? 0.f : -m;
       float l4[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[HC / 2];
 #pragma unroll
-      for (int ch = 0; ch < HC / 8; ++ch) {
-        float pv[8];
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          float x0 = s[ch * 8 + e], x1 = s[ch * 8 + e + 1];
-          fma2_sc(x0, x1, sc, mneg);  // masked keys: -inf, and 2^-inf = 0
-          pv[e] = ex2_approx(x0);
-          pv[e + 1] = ex2_approx(x1);
-          add2(l4[e & 3], l4[(e + 1) & 3], pv[e], pv[e + 1]);
+      for (int e = 0; e < HC; e += 2) {
+        float x0 = s[e], x1 = s[e + 1];
+        fma2_sc(x0, x1, sc, mneg);  // masked keys: -inf, and 2^-inf = 0
+        if (((e >> 1) & 3) < AT_EMU) {
+          ex2_poly2(x0, x1);
+        } else {
+          x0 = ex2_approx(x0);
+          x1 = ex2_approx(x1);
         }
-        uint4 u;
-        u.x = pack_bf2(pv[0], pv[1]); u.y = pack_bf2(pv[2], pv[3]);
-        u.z = pack_bf2(pv[4], pv[5]); u.w = pack_bf2(pv[6], pv[7]);
-        *reinterpret_cast<uint4*>(sP + hf * L::TILE + r * 128 + ((ch ^ (r & 7)) << 4)) = u;
+        const float p0 = x0, p1 = x1;
+        add2(l4[e & 3], l4[(e + 1) & 3], p0, p1);
+        pk[e >> 1] = pack_bf2(p0, p1);
       }
       l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-      tc::fence_proxy_async_smem();   // P is read by the tensor cores
-      tc::fence_before_sync();        // O rows rewritten in TMEM above
+      if (ok) {
+        tc::tmem_st32(tmem + lane_base + AT_TM_P + sb * 64 + hf * 32, pk);
+        tc::tmem_st_wait();
+      }
+      tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(p_full);
+      if (lane == 0) tc::mbar_arrive(p_full + sb);
     }
     // ---- O / l -> bf16 ----
-    const bool fin = ok && nt > 0 && wwait(o_done, (uint32_t)(T + nt - 1) & 1u);
-    sm_sync();  // every partner has read the last tile's row maxima
+    const int tl = T + nt - 1;
+    const bool fin = ok && nt > 0 && wwait(o_done + (tl & 1), (uint32_t)(tl >> 1) & 1u);
     xr[hf * 128 + r] = l;
     sm_sync();
     const float lt = xr[r] + xr[128 + r];
-    sm_sync();  // both halves have read l before the next item's maxima reuse xr
+    sm_sync();  // both halves have read l before the next item rewrites xr
     if (fin) {
       tc::fence_after_sync();
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
@@ -517,8 +636,9 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 #pragma unroll
       for (int c = 0; c < OC / 32; ++c) {
         uint32_t o[32];
-        tc::tmem_ld32(tmem + lane_base + 256 + hf * OC + c * 32, o);
+        tc::tmem_ld32(tmem + lane_base + AT_TM_O + hf * OC + c * 32, o);
         tc::tmem_ld_wait();
+        tc::reg_fence<32>(o);
         if (q < p.S) {
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {

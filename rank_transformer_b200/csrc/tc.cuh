@@ -124,6 +124,18 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D[tmem] (+)= A[tmem] x B[smem desc]; kind::f16.  A is M = 128 lanes (row i
+// in lane i), K along the columns, two bf16 per 32-bit column (the lower
+// half holds the even k).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrive (once) on `bar` when every MMA issued so far by this thread is done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -145,6 +157,15 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
       : "memory");
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Registers filled by tcgen05.ld are written asynchronously; passing them
+// through an empty volatile asm after tmem_ld_wait() makes every later use
+// depend on a statement ordered after the wait (the compiler may otherwise
+// move a register-only consumer above it).
+template <int N, typename T>
+__device__ __forceinline__ void reg_fence(T* r) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(*reinterpret_cast<uint32_t*>(r + i)));
+}
 // 32 lanes x 32 consecutive 32-bit columns from registers: thread i writes
 // lane (base + i).
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
