@@ -40,9 +40,8 @@
 // Roles per CTA (CW consumer warps + 1 producer warp):
 //   warp CW   producer: fills every ring entry in order -- one bulk copy
 //             per pack entry for the GEMV stages (prefetched two entries
-//             ahead into L2), TMA loads of 64-key cache chunks for attention
-//             (a layer's chunks of this CTA are prefetched into L2 at its
-//             stage 1); it never waits for activations.
+//             ahead into L2), TMA loads of 64-key cache chunks for attention;
+//             it never waits for activations.
 //   consumers multiply-accumulate ring entries against the stage input
 //             built in shared memory, and run attention with per-warp
 //             online-softmax state.  The next GEMV stage's schedule record
@@ -547,11 +546,6 @@ __device__ __forceinline__ int scatter_index(int lane) {
   return idx;
 }
 
-__device__ __forceinline__ void prefetch_l2_2d(const CUtensorMap* tm, int c0, int c1) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(tm), "r"(c0), "r"(c1)
-               : "memory");
-}
-
 // Asynchronous 16-byte global -> shared copy (completion: cp_async_wait).
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(dst)), "l"(src) : "memory");
@@ -652,8 +646,11 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
         for (int ph_i = 0; ph_i < DF_NPHASE && ok && !*abort_flag; ++ph_i) {
           const DfPhase& ph = Ly->ph[ph_i];
           if (ph_i == 1) {
-            // History rows are fixed for this step: pull this layer's cache
-            // chunks of this CTA into L2 ahead of its attention stage.
+            // History lengths are fixed for this step: the attention
+            // schedule (and this CTA's share of it) once the previous
+            // kernel is done.  The cache chunks are not prefetched into L2
+            // here: that extra HBM traffic during the q/k/v stage slowed
+            // the stage more than it sped up the attention stage.
             if (!waited) {
               pdl_wait();
               waited = true;
@@ -662,15 +659,6 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
             }
             tc::tma_prefetch_desc(&Ly->kmap);
             tc::tma_prefetch_desc(&Ly->vmap);
-            for (int c = a0; c < a1; ++c) {
-              int b, h, kc;
-              attn_entry(s, c, b, h, kc);
-              if (kc >= s.nk[b]) continue;  // padding
-              for (int bx = 0; bx < NB; ++bx) {
-                prefetch_l2_2d(&Ly->kmap, h * p.D + 64 * bx, b * p.S_max + kc * 64);
-                prefetch_l2_2d(&Ly->vmap, h * p.D + 64 * bx, b * p.S_max + kc * 64);
-              }
-            }
           }
           if (ph.type == DF_ATTN) {
             // K/V chunks of the dense cache (rows before the current position
@@ -829,13 +817,16 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
         for (int m = 0; m < MT; ++m) ssq[m] = 0.f;
         if (xin) {
           // x (the layer input, complete before this stage) into the input
-          // rows; zero rows past B (SRC_XOUT: x is built after the barrier)
+          // rows; zero rows past B.  SRC_XOUT: the previous layer's x'
+          // (stored at its stage 5, several barriers ago), to which the
+          // partials of z V_dn are added after the barrier.
           const int d4 = p.d >> 2;
+          const bf16* xsrc = src == SRC_XOUT ? p.xm : p.x;
           for (int e = tid; e < MT * d4; e += C::CT) {
             const int m = e / d4, j = (e - m * d4) * 4;
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (m < p.B && src != SRC_XOUT) {
-              const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(p.x + (long long)m * p.d + j));
+            if (m < p.B) {
+              const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(xsrc + (long long)m * p.d + j));
               v = make_float4(bf_lo(raw.x), bf_hi(raw.x), bf_lo(raw.y), bf_hi(raw.y));
               if (src == SRC_X) {
                 add_sq<MT>(ssq, m, v);
@@ -874,13 +865,7 @@ decode_layer_kernel(const __grid_constant__ DfParams p) {
               if (k2 == 1 && !h1) continue;
               const int m = k2 ? m1 : m0, j = k2 ? j1 : j0;
               float4* a4 = reinterpret_cast<float4*>(abuf + m * C::ACOLS + j);
-              float4 v;
-              if (src == SRC_XMID) {
-                v = *a4;
-              } else {
-                const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(p.xm + (long long)m * p.d + j));
-                v = make_float4(bf_lo(raw.x), bf_hi(raw.x), bf_lo(raw.y), bf_hi(raw.y));
-              }
+              float4 v = *a4;  // x (SRC_XMID) or the previous layer's x' (SRC_XOUT)
               add4(v, sp[k2]);
               v = round4(v);
               add_sq<MT>(ssq, m, v);
