@@ -37,6 +37,7 @@
 #ifndef FLASHSVD_H
 #define FLASHSVD_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -210,6 +211,25 @@ FLASHSVD_API int flashsvd_lowrank_linear(const flashsvd_bf16* x, const flashsvd_
 FLASHSVD_API int flashsvd_dense_linear_f32(const flashsvd_bf16* x, const flashsvd_bf16* W,
                               float* y, int M, int d, int n,
                               flashsvd_stream stream);
+
+/* -------------------------------------------------------------- head --
+ * The decode step's output head (dense, not factorized; part of the
+ * per-step replay unit of [v1.5] Methodology 4) with the final RMSNorm
+ * folded into the same split-K GEMV:
+ *   logits[M x n] = rmsnorm(x) . W   (fp32),   W [d x n] row-major bf16.
+ * x [M x d] bf16 (row stride d); g [d] bf16 RMSNorm gain, or NULL for no
+ * norm (logits = x . W); eps >= 0; logits [M x n] fp32 (row stride n).
+ * 1 <= M <= 32 (and <= max_tokens), d and n multiples of 8.  Each CTA sums
+ * the squares of its slice of x; the CTA that completes a column tile
+ * scales its sums by rstd(x) (x . g is not rounded to bf16 first, unlike a
+ * separate flashsvd_rmsnorm).  Errors: FLASHSVD_ERR_INVALID_ARG (null
+ * pointer, M < 0, eps < 0 with a gain), FLASHSVD_ERR_MISALIGNED,
+ * FLASHSVD_ERR_UNSUPPORTED_SHAPE (M > 32, widths, workspace too small for
+ * the split partials).  Allocates nothing; safe during capture.
+ */
+FLASHSVD_API int flashsvd_head_logits(const flashsvd_bf16* x, const flashsvd_bf16* g, float eps,
+                                      const flashsvd_bf16* W, float* logits, int M, int d,
+                                      int n, flashsvd_stream stream);
 
 /* -------------------------------------------------- packed gate|up MLP --
  * [v1.5] Methodology 3 (Packed MLP Execution): the input-side gate and up

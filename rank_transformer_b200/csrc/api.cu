@@ -845,6 +845,26 @@ int flashsvd_dense_linear_f32(const flashsvd_bf16* x, const flashsvd_bf16* W,
   return prefill_dense_launch(p, stream);
 }
 
+int flashsvd_head_logits(const flashsvd_bf16* x, const flashsvd_bf16* g, float eps,
+                         const flashsvd_bf16* W, float* logits, int M, int d, int n,
+                         flashsvd_stream stream) {
+  FSVD_TRY(need_init());
+  FSVD_TRY(check_ptr(x)); FSVD_TRY(check_opt_ptr(g)); FSVD_TRY(check_ptr(W));
+  FSVD_TRY(check_ptr(logits));
+  if (M < 0 || (g && !(eps >= 0.f))) return FLASHSVD_ERR_INVALID_ARG;
+  FSVD_TRY(check_w8(d)); FSVD_TRY(check_w8(n));
+  if (M == 0) return FLASHSVD_OK;
+  if (M > DECODE_MAX_ROWS || M > cur().rows) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
+  GvParams p = gv_base();
+  p.K = d; p.nprob = 1;
+  p.prob[0].W = (const bf16*)W; p.prob[0].ldw = n; p.prob[0].N = n;
+  p.x = (const bf16*)x; p.ldx = d;
+  p.norm_g = (const bf16*)g; p.eps = eps;
+  p.out32 = logits; p.ldo32 = n;
+  FSVD_TRY(gv_fits(d, gemv_tiles_for(MAP_PLAIN, n, 64)));
+  return gemv_launch(p, g ? PRO_RMSNORM : PRO_BF16, EPI_F32, MAP_PLAIN, M, target_ctas(), stream);
+}
+
 int flashsvd_gateup_swiglu(const flashsvd_bf16* x, const flashsvd_bf16* U_gu,
                            const flashsvd_bf16* V_gu, flashsvd_bf16* h, int M,
                            int d, int r_f, int f, flashsvd_stream stream) {

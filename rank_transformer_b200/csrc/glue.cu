@@ -25,6 +25,10 @@ __device__ __forceinline__ void ld8(const bf16* p, float* v) {
   v[0] = bf_lo(u.x); v[1] = bf_hi(u.x); v[2] = bf_lo(u.y); v[3] = bf_hi(u.y);
   v[4] = bf_lo(u.z); v[5] = bf_hi(u.z); v[6] = bf_lo(u.w); v[7] = bf_hi(u.w);
 }
+__device__ __forceinline__ void unpack8(const uint4& u, float* v) {
+  v[0] = bf_lo(u.x); v[1] = bf_hi(u.x); v[2] = bf_lo(u.y); v[3] = bf_hi(u.y);
+  v[4] = bf_lo(u.z); v[5] = bf_hi(u.z); v[6] = bf_lo(u.w); v[7] = bf_hi(u.w);
+}
 __device__ __forceinline__ void st8(bf16* p, const float* v) {
   uint4 u;
   u.x = pack_bf2(v[0], v[1]); u.y = pack_bf2(v[2], v[3]);
@@ -32,35 +36,49 @@ __device__ __forceinline__ void st8(bf16* p, const float* v) {
   *reinterpret_cast<uint4*>(p) = u;
 }
 
-// Rows of up to 32 * 256 = 8192 elements are held in registers.
+// Rows of up to ROW_VEC * 8 * blockDim.x elements (8192 at 256 threads) are
+// held in registers; the launcher gives rows of up to 4096 elements 128
+// threads, so that every row of a 2048-row norm is resident in one wave
+// (16 CTAs per SM).  The gains (and LayerNorm's bias) do not depend on the
+// previous kernel: they are loaded before the programmatic-launch wait.
 constexpr int ROW_VEC = 4;  // 16-byte vectors per thread
 
 __global__ void __launch_bounds__(NT)
 rmsnorm_kernel(const bf16* x, const bf16* g, bf16* y, int d, float eps) {
   __shared__ float sh[NT / 32];
   pdl_launch_dependents();
+  const int nt = blockDim.x;
+  // x and g stay packed (bf16) in registers between the two passes
+  uint4 graw[ROW_VEC], xraw[ROW_VEC];
+#pragma unroll
+  for (int i = 0; i < ROW_VEC; ++i) {
+    const int c = (threadIdx.x + i * nt) * 8;
+    if (c < d) graw[i] = *reinterpret_cast<const uint4*>(g + c);
+  }
   pdl_wait();
   const long long row = blockIdx.x;
-  float v[ROW_VEC][8];
   float ss = 0.f;
 #pragma unroll
   for (int i = 0; i < ROW_VEC; ++i) {
-    const int c = (threadIdx.x + i * NT) * 8;
+    const int c = (threadIdx.x + i * nt) * 8;
     if (c < d) {
-      ld8(x + row * d + c, v[i]);
+      xraw[i] = *reinterpret_cast<const uint4*>(x + row * d + c);
+      float v[8];
+      unpack8(xraw[i], v);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) ss = fmaf(v[i][j], v[i][j], ss);
+      for (int j = 0; j < 8; ++j) ss = fmaf(v[j], v[j], ss);
     }
   }
   const float rs = rsqrtf(block_sum(ss, sh) / (float)d + eps);
 #pragma unroll
   for (int i = 0; i < ROW_VEC; ++i) {
-    const int c = (threadIdx.x + i * NT) * 8;
+    const int c = (threadIdx.x + i * nt) * 8;
     if (c < d) {
-      float gg[8], o[8];
-      ld8(g + c, gg);
+      float v[8], gg[8], o[8];
+      unpack8(xraw[i], v);
+      unpack8(graw[i], gg);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) o[j] = v[i][j] * rs * gg[j];
+      for (int j = 0; j < 8; ++j) o[j] = v[j] * rs * gg[j];
       st8(y + row * d + c, o);
     }
   }
@@ -71,28 +89,41 @@ layernorm_kernel(const bf16* x, const bf16* g, const bf16* b, bf16* y, int d,
                  float eps) {
   __shared__ float sh[NT / 32];
   pdl_launch_dependents();
+  const int nt = blockDim.x;
+  uint4 graw[ROW_VEC], braw[ROW_VEC], xraw[ROW_VEC];
+#pragma unroll
+  for (int i = 0; i < ROW_VEC; ++i) {
+    const int c = (threadIdx.x + i * nt) * 8;
+    if (c < d) {
+      graw[i] = *reinterpret_cast<const uint4*>(g + c);
+      braw[i] = *reinterpret_cast<const uint4*>(b + c);
+    }
+  }
   pdl_wait();
   const long long row = blockIdx.x;
-  float v[ROW_VEC][8];
   float s = 0.f;
 #pragma unroll
   for (int i = 0; i < ROW_VEC; ++i) {
-    const int c = (threadIdx.x + i * NT) * 8;
+    const int c = (threadIdx.x + i * nt) * 8;
     if (c < d) {
-      ld8(x + row * d + c, v[i]);
+      xraw[i] = *reinterpret_cast<const uint4*>(x + row * d + c);
+      float v[8];
+      unpack8(xraw[i], v);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) s += v[i][j];
+      for (int j = 0; j < 8; ++j) s += v[j];
     }
   }
   const float mean = block_sum(s, sh) / (float)d;
   float q = 0.f;
 #pragma unroll
   for (int i = 0; i < ROW_VEC; ++i) {
-    const int c = (threadIdx.x + i * NT) * 8;
+    const int c = (threadIdx.x + i * nt) * 8;
     if (c < d) {
+      float v[8];
+      unpack8(xraw[i], v);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const float t = v[i][j] - mean;
+        const float t = v[j] - mean;
         q = fmaf(t, t, q);
       }
     }
@@ -100,13 +131,14 @@ layernorm_kernel(const bf16* x, const bf16* g, const bf16* b, bf16* y, int d,
   const float rs = rsqrtf(block_sum(q, sh) / (float)d + eps);
 #pragma unroll
   for (int i = 0; i < ROW_VEC; ++i) {
-    const int c = (threadIdx.x + i * NT) * 8;
+    const int c = (threadIdx.x + i * nt) * 8;
     if (c < d) {
-      float gg[8], bb[8], o[8];
-      ld8(g + c, gg);
-      ld8(b + c, bb);
+      float v[8], gg[8], bb[8], o[8];
+      unpack8(xraw[i], v);
+      unpack8(graw[i], gg);
+      unpack8(braw[i], bb);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) o[j] = (v[i][j] - mean) * rs * gg[j] + bb[j];
+      for (int j = 0; j < 8; ++j) o[j] = (v[j] - mean) * rs * gg[j] + bb[j];
       st8(y + row * d + c, o);
     }
   }
@@ -237,6 +269,9 @@ norm_warp_kernel(const bf16* x, const bf16* g, const bf16* b, bf16* y, int M, in
   }
 }
 
+// Threads of the one-CTA-per-row norms: 128 up to 4096 elements, else NT.
+inline int norm_threads(int d) { return d <= 128 * ROW_VEC * 8 ? 128 : NT; }
+
 template <bool LN>
 int norm_warp_launch(const bf16* x, const bf16* g, const bf16* b, bf16* y, int M, int d, float eps,
                      cudaStream_t s) {
@@ -259,7 +294,8 @@ int rmsnorm_launch(const bf16* x, const bf16* g, bf16* y, int M, int d,
   if (d > NT * ROW_VEC * 8) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return FLASHSVD_OK;
   if (d <= 2048) return norm_warp_launch<false>(x, g, nullptr, y, M, d, eps, s);
-  return launch_pdl(LaunchTag{"rmsnorm", 4.0 * M * d, 0.0}, rmsnorm_kernel, dim3(M), dim3(NT), 0, s, x, g, y, d, eps);
+  return launch_pdl(LaunchTag{"rmsnorm", 4.0 * M * d, 0.0}, rmsnorm_kernel, dim3(M), dim3(norm_threads(d)), 0, s,
+                    x, g, y, d, eps);
 }
 
 int layernorm_launch(const bf16* x, const bf16* g, const bf16* b, bf16* y,
@@ -267,7 +303,8 @@ int layernorm_launch(const bf16* x, const bf16* g, const bf16* b, bf16* y,
   if (d > NT * ROW_VEC * 8) return FLASHSVD_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return FLASHSVD_OK;
   if (d <= 2048) return norm_warp_launch<true>(x, g, b, y, M, d, eps, s);
-  return launch_pdl(LaunchTag{"layernorm", 4.0 * M * d, 0.0}, layernorm_kernel, dim3(M), dim3(NT), 0, s, x, g, b, y, d, eps);
+  return launch_pdl(LaunchTag{"layernorm", 4.0 * M * d, 0.0}, layernorm_kernel, dim3(M), dim3(norm_threads(d)), 0,
+                    s, x, g, b, y, d, eps);
 }
 
 int rope_table_launch(float* c, float* sn, int S_max, int D, float base,

@@ -88,6 +88,7 @@ _SIGS = {
     "flashsvd_lowrank_linear": ([_p, _p, _p, _p, _p, _i, _i, _i, _i, _p], _i),
     "flashsvd_lowrank_linear_noalloc": ([_p, _p, _p, _p, _p, _i, _i, _i, _i, _p], _i),
     "flashsvd_dense_linear_f32": ([_p, _p, _p, _i, _i, _i, _p], _i),
+    "flashsvd_head_logits": ([_p, _p, _f, _p, _p, _i, _i, _i, _p], _i),
     "flashsvd_packed_gateup_mlp": ([_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p], _i),
     "flashsvd_gateup_swiglu": ([_p, _p, _p, _p, _i, _i, _i, _i, _p], _i),
     "flashsvd_lowrank_ffn": ([_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p], _i),
@@ -278,6 +279,14 @@ def dense_kv_decode_attn(q, k_new, v_new, k_cache, v_cache, cache_seqlens, out,
     _call("flashsvd_dense_kv_decode_attn", ptr(q), ptr(k_new), ptr(v_new),
           ptr(k_cache), ptr(v_cache), ptr(cache_seqlens), ptr(out), B, H, D,
           S_max, scale, stream_handle(stream))
+
+
+HEAD_MAX_ROWS = 32  # flashsvd_head_logits takes 1..32 rows
+
+
+def head_logits(x, g, eps, W, logits, M, d, n, stream=None):
+    _call("flashsvd_head_logits", ptr(x), ptr(g), eps, ptr(W), ptr(logits), M, d, n,
+          stream_handle(stream))
 
 
 def prefill_attn(q, k_cache, v_cache, out, B, S, H, D, S_max, causal, scale,

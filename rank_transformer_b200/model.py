@@ -178,7 +178,10 @@ class DecoderModel:
         last = x.view(B, S, cfg.d)[:, S - 1]
         for b in range(B):
             fs.rmsnorm(last[b], self.g_final, self.xn[b], 1, cfg.d, cfg.eps, stream)
-        fs.dense_linear_f32(self.xn, self.W_lm, self.logits, B, cfg.d, cfg.vocab, stream)
+        if B <= fs.HEAD_MAX_ROWS:
+            fs.head_logits(self.xn, None, 0.0, self.W_lm, self.logits, B, cfg.d, cfg.vocab, stream)
+        else:
+            fs.dense_linear_f32(self.xn, self.W_lm, self.logits, B, cfg.d, cfg.vocab, stream)
         fs.greedy(self.logits, self.tokens, B, cfg.vocab, stream)
         self.seqlens.fill_(S)
         return x
@@ -186,8 +189,13 @@ class DecoderModel:
     # ----------------------------------------------------------- decode --
     def _head(self, stream):
         cfg = self.cfg
-        fs.rmsnorm(self.x, self.g_final, self.xn, self.B, cfg.d, cfg.eps, stream)
-        fs.dense_linear_f32(self.xn, self.W_lm, self.logits, self.B, cfg.d, cfg.vocab, stream)
+        if self.B <= fs.HEAD_MAX_ROWS:
+            # final RMSNorm folded into the head GEMV
+            fs.head_logits(self.x, self.g_final, cfg.eps, self.W_lm, self.logits, self.B, cfg.d,
+                           cfg.vocab, stream)
+        else:
+            fs.rmsnorm(self.x, self.g_final, self.xn, self.B, cfg.d, cfg.eps, stream)
+            fs.dense_linear_f32(self.xn, self.W_lm, self.logits, self.B, cfg.d, cfg.vocab, stream)
         fs.greedy(self.logits, self.tokens, self.B, cfg.vocab, stream)
         fs.advance_seqlens(self.seqlens, self.B, stream)
 

@@ -63,6 +63,7 @@ def test_argument_errors_before_any_launch(fs):
             != 4:
         pytest.skip("library already initialised in this process")
     assert L.flashsvd_layer_forward(None, aligned, aligned, aligned, None, 1, 1, 8, 1, None) == 4
+    assert L.flashsvd_head_logits(aligned, None, 0.0, aligned, aligned, 1, 64, 64, None) == 4
     # null / misaligned / width not a multiple of 8 / negative sizes
     assert L.flashsvd_rmsnorm(None, aligned, aligned, 1, 64, 1e-5, None) == 1
     assert L.flashsvd_rmsnorm(misaligned, aligned, aligned, 1, 64, 1e-5, None) == 2

@@ -121,6 +121,28 @@ def test_dense_kv_decode_attention(fs, D, append):
     assert_parity(host_f64(out), ref, f"decode attn D={D} append={append}")
 
 
+@pytest.mark.parametrize("d", [768, 2056, 4096, 4104, 8192])
+@pytest.mark.parametrize("M", [1, 3, 2048])
+def test_norm_widths(fs, d, M):
+    """RMSNorm and LayerNorm across the three launch shapes: one warp per
+    row (d <= 2048), one 128-thread CTA per row (d <= 4096) and one
+    256-thread CTA per row (up to 8192), with ragged vector counts."""
+    if M == 2048 and d not in (4096, 8192):
+        pytest.skip("many rows checked at the 7B width and the maximum")
+    rng = synth.rng_for(4100 + d + M)
+    x = synth.normal_bf16(rng, (M, d))
+    g = synth.normal_bf16(rng, (d,), 0.1, 1.0)
+    b = synth.normal_bf16(rng, (d,), 0.1)
+    y = torch.empty((M, d), dtype=torch.bfloat16, device="cuda")
+    X, G, Bb = oracle.from_bf16(x), oracle.from_bf16(g), oracle.from_bf16(b)
+    fs.rmsnorm(dev_bf16(x), dev_bf16(g), y, M, d, 1e-5)
+    torch.cuda.synchronize()
+    assert_parity(host_f64(y), oracle.rmsnorm(X, G, 1e-5), f"rmsnorm d={d} M={M}")
+    fs.layernorm(dev_bf16(x), dev_bf16(g), dev_bf16(b), y, M, d, 1e-12)
+    torch.cuda.synchronize()
+    assert_parity(host_f64(y), oracle.layernorm(X, G, Bb, 1e-12), f"layernorm d={d} M={M}")
+
+
 def test_glue_kernels(fs):
     rng = synth.rng_for(4000)
     M, d = 5, 768
