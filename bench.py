@@ -760,7 +760,8 @@ def run_prefill_attn(args):
             out[key] = {"layer_ms": round(ms, 4),
                         "attention_ms": round(sum(v["ms"] for k, v in prof.items()
                                                   if k.startswith("attn_prefill")), 4),
-                        "qkv_stage2_ms": round(prof.get("tc_stage2_qkv_rope", {}).get("ms", 0.0), 4)}
+                        "qkv_stage2_ms": round(sum(prof.get(k, {}).get("ms", 0.0)
+                                                   for k in ("tc_stage2_qkv_grouped", "tc_stage2_qkv_rope")), 4)}
         fs.set_prefill_attention(0)
         out["factorized_faster"] = out["factorized_q"]["layer_ms"] < out["dense_q"]["layer_ms"]
         print(json.dumps(out), flush=True)
