@@ -182,7 +182,10 @@ struct Layout {
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
   static constexpr int SMEM = 1024 + BAR_OFF + 256;  // + alignment slack
   static constexpr int ACC_COLS = DUAL ? 2 * BN : BN;
-  static constexpr int TMEM_COLS = 2 * ACC_COLS;
+  // accumulator buffers: two (the epilogue of a tile overlaps the next
+  // tile's main loop) unless one accumulator fills the 512 columns
+  static constexpr int NBUF = 2 * ACC_COLS <= 512 ? 2 : 1;
+  static constexpr int TMEM_COLS = NBUF * ACC_COLS;
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "tensor memory allocation must be a power of 2");
 };
 
@@ -320,8 +323,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       int it = 0;
       bool ok = true;
       for (int t = unit; t < tiles && ok; t += units, ++it) {
-        const int buf = it & 1;
-        const uint32_t tph = (uint32_t)(it >> 1) & 1u;
+        const int buf = it % L::NBUF;
+        const uint32_t tph = (uint32_t)(it / L::NBUF) & 1u;
         if (!tc::mbar_wait(tempty + buf, tph ^ 1u, abort_flag, a.status)) { ok = false; break; }
         tc::fence_after_sync();
         const uint32_t d0 = tmem_base + (uint32_t)(buf * L::ACC_COLS);
@@ -373,8 +376,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const int row = q * 32 + lane;
     int it = 0;
     for (int t = unit; t < tiles; t += units, ++it) {
-      const int buf = it & 1;
-      const uint32_t tph = (uint32_t)(it >> 1) & 1u;
+      const int buf = it % L::NBUF;
+      const uint32_t tph = (uint32_t)(it / L::NBUF) & 1u;
       if (!tc::mbar_wait(tfull + buf, tph, abort_flag, a.status)) break;
       tc::fence_after_sync();
       const int gn = t / a.tiles_m, gp = group_of(a, gn);
@@ -649,8 +652,15 @@ int gemm(const bf16* A, long long lda, long long a_cols, const bf16* B, long lon
   FSVD_TRY(make_map(&ma, A, a.M, a_cols, lda, BM));
   if (dual) {
     FSVD_TRY(make_map(&mb, B, b_rows, a.N, ldb, BK));
-    // (single CTAs: as a 2-SM pair this dual form measured slower)
-    return launch_tc<128, 6, true, PF_EPI_SWIGLU>(ma, mb, mb, mb, a, name, stream);
+    // 256-wide gate and up accumulators fill the 512 TMEM columns, so the
+    // accumulator is single-buffered (the epilogue does not overlap the
+    // next tile's main loop); 128-wide tiles with a double-buffered
+    // accumulator ran their MMAs at about 57 % of the tensor-core rate and
+    // took 6.1 ms per 7B prefill against 4.5 (single CTAs) and 4.2 ms
+    // (2-SM pairs) for 256-wide ones.
+    if (kGemmPairs && a.M >= 2 * BM)
+      return launch_tc<256, 6, true, PF_EPI_SWIGLU, true>(ma, mb, mb, mb, a, name, stream);
+    return launch_tc<256, 4, true, PF_EPI_SWIGLU>(ma, mb, mb, mb, a, name, stream);
   }
   FSVD_TRY(make_map(&mb, B, b_rows, a.N, ldb, BK));
   switch (epi) {
