@@ -657,10 +657,15 @@ int gemm(const bf16* A, long long lda, long long a_cols, const bf16* B, long lon
     // next tile's main loop); 128-wide tiles with a double-buffered
     // accumulator ran their MMAs at about 57 % of the tensor-core rate and
     // took 6.1 ms per 7B prefill against 4.5 (single CTAs) and 4.2 ms
-    // (2-SM pairs) for 256-wide ones.
-    if (kGemmPairs && a.M >= 2 * BM)
-      return launch_tc<256, 6, true, PF_EPI_SWIGLU, true>(ma, mb, mb, mb, a, name, stream);
-    return launch_tc<256, 4, true, PF_EPI_SWIGLU>(ma, mb, mb, mb, a, name, stream);
+    // (2-SM pairs) for 256-wide ones.  With a short K (r_f < 1024: 2 x 16
+    // k-blocks or fewer per tile) the exposed epilogue outweighs that and
+    // the double-buffered 128-wide tiles stay ahead.
+    if (a.K >= 1024) {
+      if (kGemmPairs && a.M >= 2 * BM)
+        return launch_tc<256, 6, true, PF_EPI_SWIGLU, true>(ma, mb, mb, mb, a, name, stream);
+      return launch_tc<256, 4, true, PF_EPI_SWIGLU>(ma, mb, mb, mb, a, name, stream);
+    }
+    return launch_tc<128, 6, true, PF_EPI_SWIGLU>(ma, mb, mb, mb, a, name, stream);
   }
   FSVD_TRY(make_map(&mb, B, b_rows, a.N, ldb, BK));
   switch (epi) {
