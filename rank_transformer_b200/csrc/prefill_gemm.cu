@@ -186,7 +186,9 @@ struct Layout {
   // tile's main loop) unless one accumulator fills the 512 columns
   static constexpr int NBUF = 2 * ACC_COLS <= 512 ? 2 : 1;
   static constexpr int TMEM_COLS = NBUF * ACC_COLS;
-  static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "tensor memory allocation must be a power of 2");
+  // allocations are powers of 2 of at least 32 columns
+  static constexpr int TMEM_ALLOC = TMEM_COLS <= 256 ? 256 : 512;
+  static_assert(TMEM_COLS <= 512, "tensor memory: 512 columns");
 };
 
 // PAIR: launched in clusters of 2; each pair computes a 256 x BN tile with
@@ -243,10 +245,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   }
   if (warp == 1) {
     if (PAIR) {
-      tc::tmem_alloc_pair(tmem_holder, L::TMEM_COLS);
+      tc::tmem_alloc_pair(tmem_holder, L::TMEM_ALLOC);
       tc::tmem_relinquish_pair();
     } else {
-      tc::tmem_alloc(tmem_holder, L::TMEM_COLS);
+      tc::tmem_alloc(tmem_holder, L::TMEM_ALLOC);
       tc::tmem_relinquish();
     }
     tc::fence_before_sync();
@@ -569,9 +571,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   if (warp == 1) {
     tc::fence_after_sync();
     if (PAIR)
-      tc::tmem_dealloc_pair(tmem_base, L::TMEM_COLS);
+      tc::tmem_dealloc_pair(tmem_base, L::TMEM_ALLOC);
     else
-      tc::tmem_dealloc(tmem_base, L::TMEM_COLS);
+      tc::tmem_dealloc(tmem_base, L::TMEM_ALLOC);
   }
 }
 
@@ -641,6 +643,21 @@ constexpr bool kGemmPairs = true;
 template <int EPI>
 int launch_wide(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb1, const CUtensorMap& mb2,
                 const TcArgs& a, const char* name, cudaStream_t stream) {
+  // Widths that 192-column tiles cover with less padding than 256-column
+  // ones (rank-192 projections: a quarter of a 256-wide tile is empty) run
+  // 192-wide single-CTA tiles (a 2-SM pair would split them into 96-column
+  // halves, below the 64-column TMA box granularity).  Not for the q/k/v
+  // epilogue, whose RoPE pairs columns within a head that a 192-column tile
+  // may split.
+  if constexpr (EPI != PF_EPI_QKV) {
+    bool narrow = true;
+    const int np = a.nprob > 1 ? a.nprob : 1;
+    for (int i = 0; i < np; ++i) {
+      const int n = a.nprob > 1 ? a.gN[i] : a.N;
+      if (ceil_div(n, 192) * 192 >= ceil_div(n, 256) * 256) narrow = false;
+    }
+    if (narrow) return launch_tc<192, 5, false, EPI>(ma, mb, mb1, mb2, a, name, stream);
+  }
   if (kGemmPairs && a.M >= 2 * BM) return launch_tc<256, 6, false, EPI, true>(ma, mb, mb1, mb2, a, name, stream);
   return launch_tc<256, 4, false, EPI>(ma, mb, mb1, mb2, a, name, stream);
 }
